@@ -1,0 +1,343 @@
+"""Float64 CPU oracle of the SparseSAM encoder-block hot path.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or execute this module: only
+the tests, the smoke check and the benchmark's CPU-baseline / reference legs do. It shares no code
+with the CUDA library and imports nothing from it.
+
+What it computes, step by step, as the SparseSAM pages describe it (the pages give prose only; each
+open choice takes the plainest reading, listed beside each function):
+
+  S1 score  -- SparseSAM technical summary (Dutch), "Methodologie" 1, "Op Gradiënten Gebaseerde
+               Ordening"; Japanese summary "手法" 1, 勾配に基づく順序付け: a parameter-free Sobel
+               operator gives the local gradient magnitude of each token.
+  S2 perm   -- same sections, "Stripe-Sort Permutatie": sort the tokens by that score, treat the
+               sorted list as a matrix, transpose it and flatten it.
+  S3 attn   -- same sections, "Statisch Sparsiteitspatroon": the permutation splits the N x N
+               attention matrix into a 4 x 4 mosaic of sub-maps, each banded around its diagonal,
+               plus a small global keep-set; SparseSAM README, "apply_sam(..., ratio=0.5)  # density
+               50%": the knob is the computed fraction.
+  S4 rcmlp  -- Dutch summary "Methodologie" 2, "Residual-Consistency MLP": the MLP runs on the top-K
+               keep-set only; the residual set passes through unchanged.
+
+Pins (tests/test_oracle_pins.py): closed forms, invariants, library routines and brute force.
+The pattern's constants -- block-size rule, one global offset block, the nearest-density band width --
+are a reading of silent pages: their implementation is pinned by hand-derived counts, but against the
+pages themselves they are parity unpinned (the pages print no worked example).
+
+All arithmetic is IEEE float64. S1 uses one RN operation per step in a fixed order (numpy never fuses
+multiply-add), so its results are bit-reproducible.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+from scipy.special import erf
+
+STRIPES = 4          # "4 x 4 mosaic" (Dutch summary, Statisch Sparsiteitspatroon); group_size=4 (README, PE example)
+MAX_BLOCK = 64       # reading: block size is the largest divisor of L that is <= 64 with >= 4 blocks
+GLOBAL_BLOCKS = 1    # reading: the global keep-set is offset block 0 of every stripe
+
+
+# ---------------------------------------------------------------------------------------------
+# S1: Sobel score
+# ---------------------------------------------------------------------------------------------
+def sobel_score(lum: np.ndarray) -> np.ndarray:
+    """Squared Sobel gradient magnitude per token, float64 [B, Hg*Wg] in raster order.
+
+    Reading: replicate (clamp-to-edge) border, so a constant image scores exactly 0; the squared
+    magnitude gx^2 + gy^2 orders tokens as the magnitude does, so no square root; no normalisation.
+    Operation order (each a single float64 RN op):
+      gx = ((l[y-1,x+1] - l[y-1,x-1]) + 2*(l[y,x+1] - l[y,x-1])) + (l[y+1,x+1] - l[y+1,x-1])
+      gy = ((l[y+1,x-1] - l[y-1,x-1]) + 2*(l[y+1,x] - l[y-1,x])) + (l[y+1,x+1] - l[y-1,x+1])
+      s  = gx*gx + gy*gy
+    """
+    lum = np.asarray(lum)
+    assert lum.ndim == 3
+    B, H, W = lum.shape
+    l = lum.astype(np.float64)
+    out = np.empty((B, H * W), dtype=np.float64)
+    for b in range(B):
+        img = l[b]
+
+        def at(dy, dx):
+            ys = np.clip(np.arange(H) + dy, 0, H - 1)
+            xs = np.clip(np.arange(W) + dx, 0, W - 1)
+            return img[ys][:, xs]
+
+        gx = ((at(-1, 1) - at(-1, -1)) + 2.0 * (at(0, 1) - at(0, -1))) + (at(1, 1) - at(1, -1))
+        gy = ((at(1, -1) - at(-1, -1)) + 2.0 * (at(1, 0) - at(-1, 0))) + (at(1, 1) - at(-1, 1))
+        out[b] = (gx * gx + gy * gy).reshape(-1)
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# Units: which tokens an attention unit holds, in its enumeration (raster) order
+# ---------------------------------------------------------------------------------------------
+@dataclass(frozen=True)
+class Geometry:
+    batch: int
+    grid_h: int
+    grid_w: int
+    mode: str = "global"      # "global" | "window"
+    window: int = 14
+
+    @property
+    def padded(self):
+        if self.mode == "global":
+            return self.grid_h, self.grid_w
+        ws = self.window
+        return -(-self.grid_h // ws) * ws, -(-self.grid_w // ws) * ws
+
+    @property
+    def windows(self) -> int:
+        if self.mode == "global":
+            return 1
+        hp, wp = self.padded
+        return (hp // self.window) * (wp // self.window)
+
+    @property
+    def units(self) -> int:
+        return self.batch * self.windows
+
+    @property
+    def unit_tokens(self) -> int:
+        return self.grid_h * self.grid_w if self.mode == "global" else self.window ** 2
+
+
+def unit_members(geo: Geometry):
+    """For every unit, (image index, array of raster token ids of the image or -1 for a pad token).
+
+    Global mode: the whole image in row-major order. Window mode (SAM's windowed blocks): the grid
+    is padded bottom/right to a multiple of the window and cut into windows in row-major window
+    order; a window enumerates its tokens row-major.
+    """
+    units = []
+    if geo.mode == "global":
+        for b in range(geo.batch):
+            units.append((b, np.arange(geo.grid_h * geo.grid_w)))
+        return units
+    ws = geo.window
+    hp, wp = geo.padded
+    for b in range(geo.batch):
+        for wy in range(hp // ws):
+            for wx in range(wp // ws):
+                ids = np.full(ws * ws, -1, dtype=np.int64)
+                for r in range(ws):
+                    for c in range(ws):
+                        y, x = wy * ws + r, wx * ws + c
+                        if y < geo.grid_h and x < geo.grid_w:
+                            ids[r * ws + c] = y * geo.grid_w + x
+                units.append((b, ids))
+    return units
+
+
+def unit_scores(score: np.ndarray, geo: Geometry) -> np.ndarray:
+    """[U, N] float64 scores of each unit's tokens in enumeration order; pad tokens score +0.0."""
+    out = np.zeros((geo.units, geo.unit_tokens), dtype=np.float64)
+    for u, (b, ids) in enumerate(unit_members(geo)):
+        real = ids >= 0
+        out[u, real] = score[b, ids[real]]
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# S2: stable sort and stripe transpose
+# ---------------------------------------------------------------------------------------------
+def ranked_order(s: np.ndarray) -> np.ndarray:
+    """Enumeration indices sorted by score, descending; equal scores keep lower index first.
+
+    Reading: descending (the keep-set is the "top-K"); a stable sort on the raster enumeration.
+    """
+    s = np.asarray(s, dtype=np.float64)
+    return np.argsort(-s, kind="stable")
+
+
+def stripe_transpose(ranked: np.ndarray, stripes: int = STRIPES):
+    """Stripe-sort permutation from a ranked list.
+
+    The ranked list is read row-major as an (L, S) matrix, transposed to (S, L) and flattened, so
+    position p = j*L + k holds rank S*k + j. Returns (perm, inv): perm[p] = enumeration index at
+    permuted position p, inv[perm[p]] = p.
+    """
+    n = ranked.shape[0]
+    assert n % stripes == 0, "token count must be a multiple of the stripe count"
+    L = n // stripes
+    perm = ranked.reshape(L, stripes).T.reshape(-1).copy()
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(n)
+    return perm.astype(np.int32), inv.astype(np.int32)
+
+
+def stripe_sort(score: np.ndarray, geo: Geometry):
+    """perm, inv int32 [U, N] for every attention unit (S2)."""
+    us = unit_scores(score, geo)
+    perms = np.empty(us.shape, dtype=np.int32)
+    invs = np.empty(us.shape, dtype=np.int32)
+    for u in range(us.shape[0]):
+        perms[u], invs[u] = stripe_transpose(ranked_order(us[u]))
+    return perms, invs
+
+
+# ---------------------------------------------------------------------------------------------
+# S3: static pattern
+# ---------------------------------------------------------------------------------------------
+def block_size(L: int) -> int:
+    """Largest divisor b of L with b <= 64 and L/b >= 4 (reading of the unstated block size)."""
+    for b in range(min(MAX_BLOCK, L), 0, -1):
+        if L % b == 0 and L // b >= 4:
+            return b
+    raise ValueError(f"stripe length {L} too short for a 4-block pattern")
+
+
+def band_start(a: int, W: int, nb: int) -> int:
+    """First offset block of the width-W band of row a: the window is shifted inward at the edges."""
+    return min(max(a - (W - 1) // 2, 0), nb - W)
+
+
+def kept_offset_blocks(a: int, W: int, nb: int, g: int = GLOBAL_BLOCKS) -> list[int]:
+    """Key offset blocks a' kept for query offset block a: Band_W(a) united with [0, g)."""
+    s = band_start(a, W, nb)
+    return sorted(set(range(s, s + W)) | set(range(g)))
+
+
+def density_of(W: int, nb: int, g: int = GLOBAL_BLOCKS) -> float:
+    return sum(len(kept_offset_blocks(a, W, nb, g)) for a in range(nb)) / float(nb * nb)
+
+
+@dataclass(frozen=True)
+class Pattern:
+    N: int
+    L: int
+    b: int
+    nb: int
+    W: int
+    g: int
+    rho: float
+    row_ptr: np.ndarray   # CSR over query offset blocks a: kept key offset blocks
+    col_idx: np.ndarray
+
+
+def pattern(N: int, density: float) -> Pattern:
+    """The static pattern for an N-token unit at the requested density.
+
+    The band width W in [1, nb] is the one whose realised density is nearest to the request; a tie
+    goes to the smaller W. The same offset-block pattern holds in all 16 sub-maps of the mosaic.
+    """
+    if not (0.0 < density <= 1.0):
+        raise ValueError("density must lie in (0, 1]")
+    assert N % STRIPES == 0
+    L = N // STRIPES
+    b = block_size(L)
+    nb = L // b
+    best_W, best_err = None, None
+    for W in range(1, nb + 1):
+        err = abs(density_of(W, nb) - density)
+        if best_err is None or err < best_err:
+            best_W, best_err = W, err
+    W = best_W
+    rows = [kept_offset_blocks(a, W, nb) for a in range(nb)]
+    row_ptr = np.zeros(nb + 1, dtype=np.int32)
+    row_ptr[1:] = np.cumsum([len(r) for r in rows])
+    col_idx = np.array([c for r in rows for c in r], dtype=np.int32)
+    return Pattern(N, L, b, nb, W, GLOBAL_BLOCKS, density_of(W, nb), row_ptr, col_idx)
+
+
+def position_offset_block(N: int, b: int) -> np.ndarray:
+    """Offset block a of every permuted position p = j*L + a*b + r."""
+    L = N // STRIPES
+    return (np.arange(N) % L) // b
+
+
+def attention(q, k, v, perm, density: float) -> np.ndarray:
+    """Stripe-Sort attention, float64 [U, N, heads, dh].
+
+    Qp = Q[perm], Kp = K[perm], Vp = V[perm]; each permuted query row takes a softmax (with its max
+    subtracted, summed in float64, no online rescaling) of Qp.Kp/sqrt(dh) over its kept keys only,
+    then out[perm[p]] = Op[p].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    U, N, H, D = q.shape
+    pat = pattern(N, density)
+    blk = position_offset_block(N, pat.b)
+    scale = 1.0 / math.sqrt(D)
+    out = np.empty((U, N, H, D), dtype=np.float64)
+    for u in range(U):
+        pm = perm[u]
+        qp = q[u][pm].transpose(1, 0, 2)   # [H, N, D]
+        kp = k[u][pm].transpose(1, 0, 2)
+        vp = v[u][pm].transpose(1, 0, 2)
+        for a in range(pat.nb):
+            rows = np.nonzero(blk == a)[0]
+            kept = pat.col_idx[pat.row_ptr[a]:pat.row_ptr[a + 1]]
+            keys = np.nonzero(np.isin(blk, kept))[0]
+            s = np.matmul(qp[:, rows], kp[:, keys].transpose(0, 2, 1)) * scale
+            s = s - s.max(axis=2, keepdims=True)
+            e = np.exp(s)
+            p = e / e.sum(axis=2, keepdims=True)
+            o = np.matmul(p, vp[:, keys])                # [H, rows, D]
+            out[u, pm[rows]] = o.transpose(1, 0, 2)
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# S4: Residual-Consistency MLP
+# ---------------------------------------------------------------------------------------------
+def keep_count(density: float, tokens: int) -> int:
+    """K = ceil(d*N - 1e-9) in float64: the top-K keep-set size over an image's real tokens."""
+    if not (0.0 < density <= 1.0):
+        raise ValueError("density must lie in (0, 1]")
+    return int(math.ceil(density * tokens - 1e-9))
+
+
+def keep_list(score: np.ndarray, density: float) -> np.ndarray:
+    """int32 [B, K]: the K highest-scoring tokens of each image, in rank order (per-image sort)."""
+    B, T = score.shape
+    K = keep_count(density, T)
+    out = np.empty((B, K), dtype=np.int32)
+    for b in range(B):
+        out[b] = ranked_order(score[b])[:K]
+    return out
+
+
+def gelu(z: np.ndarray) -> np.ndarray:
+    """Exact (erf) GELU: z/2 * (1 + erf(z/sqrt(2)))."""
+    return 0.5 * z * (1.0 + erf(z / math.sqrt(2.0)))
+
+
+def rcmlp(x, w1, b1, w2, b2, keep) -> np.ndarray:
+    """y = x; y[t] = x[t] + (W2 GELU(W1 x[t] + b1) + b2) for every kept token t of each image.
+
+    x [B, T, C]; w1 [hidden, C]; w2 [C, hidden]; b1/b2 may be None (zero). Rows outside the keep
+    set are copied unchanged.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    w1 = np.asarray(w1, dtype=np.float64)
+    w2 = np.asarray(w2, dtype=np.float64)
+    b1 = np.zeros(w1.shape[0]) if b1 is None else np.asarray(b1, dtype=np.float64)
+    b2 = np.zeros(w2.shape[0]) if b2 is None else np.asarray(b2, dtype=np.float64)
+    y = x.copy()
+    for b in range(x.shape[0]):
+        rows = np.asarray(keep[b], dtype=np.int64)
+        if rows.size == 0:
+            continue
+        xs = x[b, rows]
+        h = gelu(xs @ w1.T + b1)
+        y[b, rows] = xs + (h @ w2.T + b2)
+    return y
+
+
+# ---------------------------------------------------------------------------------------------
+# The whole block, for the smoke check and the CPU baseline
+# ---------------------------------------------------------------------------------------------
+def hot_path(lum, q, k, v, x, w1, b1, w2, b2, geo: Geometry, density: float):
+    """S1..S4 in order; returns (score, perm, inv, keep, attn_out, mlp_out)."""
+    score = sobel_score(lum)
+    perm, inv = stripe_sort(score, geo)
+    keep = keep_list(score, density)
+    out = attention(q, k, v, perm, density)
+    y = rcmlp(x, w1, b1, w2, b2, keep)
+    return score, perm, inv, keep, out, y

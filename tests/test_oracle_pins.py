@@ -1,0 +1,405 @@
+"""Pins of the float64 oracle against facts fixed outside it.
+
+Each pin is a closed form, an invariant, a library routine (scipy / torch, float64) or a brute-force
+count on a tiny input -- never the oracle's own formula retyped. The mutation tests at the end plant
+a plausible mistake in the oracle (on the CPU) and check that some pin catches it.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.ndimage
+import torch
+import torch.nn.functional as F
+
+from oracle import sparsesam_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ------------------------------------------------------------------------------------------------
+# S1 score
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("shape", [(1, 1, 1), (2, 5, 7), (1, 16, 16)])
+@pytest.mark.parametrize("c", [0.0, 0.37, -3.5])
+def test_sobel_constant_is_zero(shape, c):
+    s = O.sobel_score(np.full(shape, c, np.float32))
+    assert np.all(s == 0.0) and not np.any(np.signbit(s))
+
+
+def test_sobel_ramp_closed_form():
+    # l = a*x + b*y with dyadic a, b: every float64 step is exact. Interior: gx = 8a, gy = 8b.
+    # At a clamped border column the two-sided difference becomes one-sided: gx = 4a (same for y).
+    H, W, a, b = 9, 11, 0.25, -0.125
+    yy, xx = np.meshgrid(np.arange(H), np.arange(W), indexing="ij")
+    lum = (a * xx + b * yy).astype(np.float32)[None]
+    s = O.sobel_score(lum).reshape(H, W)
+    gx = np.where((xx == 0) | (xx == W - 1), 4 * a, 8 * a)
+    gy = np.where((yy == 0) | (yy == H - 1), 4 * b, 8 * b)
+    assert np.array_equal(s, gx * gx + gy * gy)
+
+
+def test_sobel_matches_scipy_nearest():
+    g = np.random.default_rng(11)
+    lum = g.random((3, 13, 10)).astype(np.float32)
+    s = O.sobel_score(lum)
+    for i in range(3):
+        img = lum[i].astype(np.float64)
+        sx = scipy.ndimage.sobel(img, axis=1, mode="nearest")
+        sy = scipy.ndimage.sobel(img, axis=0, mode="nearest")
+        np.testing.assert_allclose(s[i], (sx * sx + sy * sy).reshape(-1), rtol=1e-12, atol=1e-14)
+
+
+def test_sobel_brute_force_4x4():
+    g = np.random.default_rng(3)
+    lum = g.random((1, 4, 4)).astype(np.float32)
+    l = lum[0].astype(np.float64)
+    kx = np.array([[-1, 0, 1], [-2, 0, 2], [-1, 0, 1]], np.float64)
+    want = np.zeros((4, 4))
+    for y in range(4):
+        for x in range(4):
+            gx = gy = 0.0
+            for dy in (-1, 0, 1):
+                for dx in (-1, 0, 1):
+                    v = l[min(max(y + dy, 0), 3), min(max(x + dx, 0), 3)]
+                    gx += kx[dy + 1, dx + 1] * v
+                    gy += kx[dx + 1, dy + 1] * v
+            want[y, x] = gx * gx + gy * gy
+    np.testing.assert_allclose(O.sobel_score(lum).reshape(4, 4), want, rtol=1e-12, atol=1e-15)
+
+
+def test_sobel_rotation_and_transpose_invariant():
+    # gx^2+gy^2 is invariant under a 90-degree rotation and a transpose of the grid.
+    g = np.random.default_rng(5)
+    lum = g.random((1, 8, 8)).astype(np.float32)
+    s = O.sobel_score(lum).reshape(8, 8)
+    st = O.sobel_score(np.ascontiguousarray(lum[0].T)[None]).reshape(8, 8)
+    sr = O.sobel_score(np.ascontiguousarray(np.rot90(lum[0]))[None]).reshape(8, 8)
+    assert np.array_equal(st, s.T)
+    assert np.array_equal(sr, np.rot90(s))
+
+
+# ------------------------------------------------------------------------------------------------
+# S2 permutation
+# ------------------------------------------------------------------------------------------------
+def _geo(h, w, mode="global", batch=1):
+    return O.Geometry(batch, h, w, mode, 14)
+
+
+def test_perm_flat_image_closed_form():
+    # All scores equal: the stable sort is the identity, so pi[j*L + k] = 4k + j.
+    geo = _geo(16, 16)
+    perm, inv = O.stripe_sort(np.zeros((1, 256)), geo)
+    L = 64
+    want = np.array([4 * k + j for j in range(4) for k in range(L)])
+    assert np.array_equal(perm[0], want)
+    assert np.array_equal(inv[0][perm[0]], np.arange(256))
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_perm_is_bijection_and_inverse(seed):
+    g = np.random.default_rng(seed)
+    geo = _geo(16, 12, batch=2)
+    score = O.sobel_score(g.random((2, 16, 12)).astype(np.float32))
+    perm, inv = O.stripe_sort(score, geo)
+    for u in range(2):
+        assert np.array_equal(np.sort(perm[u]), np.arange(192))
+        assert np.array_equal(inv[u][perm[u]], np.arange(192))
+        assert np.array_equal(perm[u][inv[u]], np.arange(192))
+
+
+def test_perm_brute_force_rank_count_with_ties():
+    # rank(t) = #{u : s_u > s_t or (s_u == s_t and u < t)}; position of rank r is (r%4)*L + r//4.
+    g = np.random.default_rng(7)
+    for trial in range(20):
+        n = 8 * (1 + trial % 3)
+        s = g.integers(0, 3, size=n).astype(np.float64)      # many ties
+        perm, inv = O.stripe_transpose(O.ranked_order(s))
+        L = n // 4
+        for t in range(n):
+            r = sum(1 for u in range(n) if s[u] > s[t] or (s[u] == s[t] and u < t))
+            assert perm[(r % 4) * L + r // 4] == t
+            assert inv[t] == (r % 4) * L + r // 4
+
+
+def test_perm_rank_order_independent_of_enumeration():
+    g = np.random.default_rng(9)
+    s = g.random(64)
+    fwd = O.ranked_order(s)
+    rev = O.ranked_order(s[::-1])
+    assert np.array_equal(fwd, (63 - rev))
+
+
+def test_perm_stripes_interleave_ranks():
+    # Stripe j holds ranks j, j+4, j+8, ...: every stripe spans the whole score range.
+    g = np.random.default_rng(4)
+    s = g.random(256)
+    perm, _ = O.stripe_transpose(O.ranked_order(s))
+    ranked = list(O.ranked_order(s))
+    rank_of = {t: r for r, t in enumerate(ranked)}
+    for j in range(4):
+        ranks = [rank_of[t] for t in perm[j * 64:(j + 1) * 64]]
+        assert ranks == list(range(j, 256, 4))
+        assert s[perm[j * 64]] >= s[perm[j * 64 + 63]]
+
+
+def test_window_geometry_and_pads():
+    geo = O.Geometry(2, 64, 64, "window", 14)
+    assert geo.padded == (70, 70) and geo.windows == 25 and geo.units == 50 and geo.unit_tokens == 196
+    members = O.unit_members(geo)
+    for b in range(2):
+        ids = np.concatenate([m[1] for m in members if m[0] == b])
+        real = ids[ids >= 0]
+        assert np.array_equal(np.sort(real), np.arange(4096))
+        assert (ids < 0).sum() == 25 * 196 - 4096
+    # Pads score +0.0 and sort after every real token of positive score, in raster order.
+    score = np.random.default_rng(1).random((2, 4096)) + 0.5
+    us = O.unit_scores(score, geo)
+    perm, _ = O.stripe_sort(score, geo)
+    u = 24                                           # bottom-right window: 8x8 real, 132 pads
+    ranked = O.ranked_order(us[u])
+    pads = [t for t in range(196) if members[u][1][t] < 0]
+    assert len(pads) == 132 and list(ranked[-132:]) == pads
+    assert sorted(perm[u]) == list(range(196))
+
+
+# ------------------------------------------------------------------------------------------------
+# Pattern
+# ------------------------------------------------------------------------------------------------
+def _golden_patterns():
+    rows = []
+    with open(os.path.join(GOLDEN, "pattern_table.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                N, d, L, b, nb, W, nnz = line.split()
+                rows.append((int(N), float(d), int(L), int(b), int(nb), int(W), int(nnz)))
+    return rows
+
+
+@pytest.mark.parametrize("row", _golden_patterns())
+def test_pattern_hand_derived_table(row):
+    N, d, L, b, nb, W, nnz = row
+    p = O.pattern(N, d)
+    assert (p.L, p.b, p.nb, p.W) == (L, b, nb, W)
+    assert p.row_ptr[-1] == nnz
+    assert p.rho == nnz / (nb * nb)
+
+
+@pytest.mark.parametrize("N,d", [(4096, 0.4), (4096, 0.3), (196, 0.3), (256, 0.4), (64, 0.5)])
+def test_pattern_structure(N, d):
+    p = O.pattern(N, d)
+    for a in range(p.nb):
+        kept = list(p.col_idx[p.row_ptr[a]:p.row_ptr[a + 1]])
+        assert a in kept                   # diagonal (local interactions)
+        assert 0 in kept                   # global keep-set
+        band = [c for c in kept if c != 0] if a - (p.W - 1) // 2 > 0 and p.nb > p.W else kept
+        assert band == list(range(band[0], band[0] + len(band)))   # one contiguous band
+    # a larger W never lowers the density
+    rhos = [O.density_of(W, p.nb) for W in range(1, p.nb + 1)]
+    assert rhos == sorted(rhos) and rhos[-1] == 1.0
+
+
+def test_pattern_density_one_is_dense():
+    for N in (64, 196, 256, 4096):
+        p = O.pattern(N, 1.0)
+        assert p.rho == 1.0 and p.row_ptr[-1] == p.nb * p.nb
+
+
+def test_pattern_rejects_bad_density():
+    for d in (0.0, -0.1, 1.5):
+        with pytest.raises(ValueError):
+            O.pattern(256, d)
+
+
+# ------------------------------------------------------------------------------------------------
+# S3 attention
+# ------------------------------------------------------------------------------------------------
+def _sdpa64(q, k, v, mask=None):
+    # torch's own float64 attention: q,k,v [N, H, D] -> [N, H, D]
+    qt, kt, vt = (torch.from_numpy(np.ascontiguousarray(a.transpose(1, 0, 2))) for a in (q, k, v))
+    m = None if mask is None else torch.from_numpy(mask)
+    o = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=m)
+    return o.numpy().transpose(1, 0, 2)
+
+
+def _rand_qkv(U, N, H, D, seed):
+    g = np.random.default_rng(seed)
+    return [g.standard_normal((U, N, H, D)) for _ in range(3)]
+
+
+def test_attention_dense_equals_sdpa_and_is_perm_invariant():
+    U, N, H, D = 2, 64, 2, 16
+    q, k, v = _rand_qkv(U, N, H, D, 0)
+    g = np.random.default_rng(1)
+    perm = np.stack([g.permutation(N) for _ in range(U)]).astype(np.int32)
+    ident = np.stack([np.arange(N)] * U).astype(np.int32)
+    o1 = O.attention(q, k, v, perm, 1.0)
+    o2 = O.attention(q, k, v, ident, 1.0)
+    for u in range(U):
+        np.testing.assert_allclose(o1[u], _sdpa64(q[u], k[u], v[u]), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(o1, o2, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("N,d", [(64, 0.5), (256, 0.4), (196, 0.3)])
+def test_attention_matches_masked_brute_force(N, d):
+    # Dense attention with a -inf mask built position by position from the block description:
+    # permuted position p = j*L + a*b + r belongs to offset block a; key p' is kept for query p iff
+    # its offset block is in p's kept list.
+    U, H, D = 1, 2, 8
+    q, k, v = _rand_qkv(U, N, H, D, 2)
+    g = np.random.default_rng(3)
+    perm = g.permutation(N).astype(np.int32)[None]
+    p = O.pattern(N, d)
+    L = N // 4
+    mask = np.full((N, N), -np.inf)
+    for pq in range(N):
+        a = (pq % L) // p.b
+        kept = set(p.col_idx[p.row_ptr[a]:p.row_ptr[a + 1]])
+        for pk in range(N):
+            if (pk % L) // p.b in kept:
+                mask[pq, pk] = 0.0
+    assert abs((mask == 0).mean() - p.rho) < 1e-12
+    pm = perm[0]
+    op = _sdpa64(q[0][pm], k[0][pm], v[0][pm], mask)
+    want = np.empty_like(op)
+    want[pm] = op
+    np.testing.assert_allclose(O.attention(q, k, v, perm, d)[0], want, rtol=1e-10, atol=1e-12)
+
+
+def test_attention_constant_v_and_identical_keys():
+    U, N, H, D = 1, 256, 1, 8
+    q, k, v = _rand_qkv(U, N, H, D, 5)
+    perm = np.arange(N, dtype=np.int32)[None]
+    vc = np.broadcast_to(np.arange(D, dtype=np.float64), v.shape).copy()
+    np.testing.assert_allclose(O.attention(q, k, vc, perm, 0.4), vc, rtol=0, atol=1e-12)
+    # identical keys: uniform weights -> each query gets the mean of the V rows it keeps
+    k1 = np.broadcast_to(k[:, :1], k.shape).copy()
+    out = O.attention(q, k1, v, perm, 0.4)
+    L, b = 64, 16
+    for pq in (0, 17, 100, 255):
+        a = (pq % L) // b
+        kept_blocks = {0, a}                       # W = 1 at N=256, d=0.4: own block + global
+        keys = [pk for pk in range(N) if (pk % L) // b in kept_blocks]
+        np.testing.assert_allclose(out[0, pq, 0], v[0, keys, 0].mean(axis=0), rtol=1e-10, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------------------------
+# S4 RC-MLP
+# ------------------------------------------------------------------------------------------------
+def _mlp_inputs(B=2, T=48, C=16, Hd=32, seed=0, bias=True):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((B, T, C))
+    w1 = g.standard_normal((Hd, C)) * 0.2
+    w2 = g.standard_normal((C, Hd)) * 0.2
+    b1 = g.standard_normal(Hd) * 0.1 if bias else None
+    b2 = g.standard_normal(C) * 0.1 if bias else None
+    return x, w1, b1, w2, b2
+
+
+def test_keep_count_values():
+    assert O.keep_count(0.4, 4096) == 1639
+    assert O.keep_count(0.3, 4096) == 1229
+    assert O.keep_count(0.4, 256) == 103
+    assert O.keep_count(0.5, 4096) == 2048      # integral d*N is not rounded up
+    assert O.keep_count(1.0, 4096) == 4096
+    assert O.keep_count(0.25, 4) == 1
+
+
+def test_rcmlp_dense_equals_torch_mlp():
+    x, w1, b1, w2, b2 = _mlp_inputs()
+    keep = np.stack([np.random.default_rng(b).permutation(48) for b in range(2)])
+    y = O.rcmlp(x, w1, b1, w2, b2, keep)
+    lin1 = torch.nn.Linear(16, 32, dtype=torch.float64)
+    lin2 = torch.nn.Linear(32, 16, dtype=torch.float64)
+    with torch.no_grad():
+        lin1.weight.copy_(torch.from_numpy(w1)); lin1.bias.copy_(torch.from_numpy(b1))
+        lin2.weight.copy_(torch.from_numpy(w2)); lin2.bias.copy_(torch.from_numpy(b2))
+        xt = torch.from_numpy(x)
+        want = xt + lin2(F.gelu(lin1(xt), approximate="none"))
+    np.testing.assert_allclose(y, want.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_rcmlp_empty_keep_is_identity_and_residual_rows_untouched():
+    x, w1, b1, w2, b2 = _mlp_inputs(seed=1)
+    y0 = O.rcmlp(x, w1, b1, w2, b2, np.zeros((2, 0), np.int32))
+    assert np.array_equal(y0, x)
+    keep = np.array([[3, 0, 40], [47, 5, 6]])
+    y = O.rcmlp(x, w1, b1, w2, b2, keep)
+    for b in range(2):
+        rest = np.setdiff1d(np.arange(48), keep[b])
+        assert np.array_equal(y[b, rest], x[b, rest])
+        assert not np.allclose(y[b, keep[b]], x[b, keep[b]])
+
+
+def test_rcmlp_zero_w2_adds_b2():
+    x, w1, b1, w2, b2 = _mlp_inputs(seed=2)
+    keep = np.array([[1, 2, 3], [9, 8, 7]])
+    y = O.rcmlp(x, w1, b1, np.zeros_like(w2), b2, keep)
+    for b in range(2):
+        np.testing.assert_allclose(y[b, keep[b]], x[b, keep[b]] + b2, rtol=0, atol=0)
+
+
+def test_gelu_matches_torch():
+    z = np.linspace(-6, 6, 1001)
+    np.testing.assert_allclose(O.gelu(z), F.gelu(torch.from_numpy(z), approximate="none").numpy(),
+                               rtol=1e-14, atol=1e-15)
+
+
+def test_keep_list_is_top_k_brute_force():
+    g = np.random.default_rng(8)
+    score = g.integers(0, 5, size=(2, 40)).astype(np.float64)
+    keep = O.keep_list(score, 0.3)
+    K = O.keep_count(0.3, 40)
+    for b in range(2):
+        ranks = [sum(1 for u in range(40) if score[b, u] > score[b, t]
+                     or (score[b, u] == score[b, t] and u < t)) for t in range(40)]
+        want = [t for r in range(K) for t in range(40) if ranks[t] == r]
+        assert list(keep[b]) == want
+
+
+# ------------------------------------------------------------------------------------------------
+# Mutations: a planted mistake in the oracle must fail some pin above
+# ------------------------------------------------------------------------------------------------
+def test_mutation_untransposed_stripes_caught(monkeypatch):
+    def wrong(ranked, stripes=4):
+        perm = ranked.copy().astype(np.int32)
+        inv = np.empty_like(perm); inv[perm] = np.arange(len(perm))
+        return perm, inv
+    monkeypatch.setattr(O, "stripe_transpose", wrong)
+    with pytest.raises(AssertionError):
+        test_perm_flat_image_closed_form()
+
+
+def test_mutation_ascending_sort_caught(monkeypatch):
+    monkeypatch.setattr(O, "ranked_order", lambda s: np.argsort(np.asarray(s), kind="stable"))
+    with pytest.raises(AssertionError):
+        test_keep_list_is_top_k_brute_force()
+
+
+def test_mutation_sobel_sign_caught(monkeypatch):
+    real = O.sobel_score
+
+    def wrong(lum):   # gy computed with a dropped centre term: a plausible transcription slip
+        lum = np.asarray(lum).astype(np.float64)
+        B, H, W = lum.shape
+        out = np.empty((B, H * W))
+        for b in range(B):
+            img = lum[b]
+            at = lambda dy, dx: img[np.clip(np.arange(H) + dy, 0, H - 1)][:, np.clip(np.arange(W) + dx, 0, W - 1)]
+            gx = ((at(-1, 1) - at(-1, -1)) + 2.0 * (at(0, 1) - at(0, -1))) + (at(1, 1) - at(1, -1))
+            gy = (at(1, -1) - at(-1, -1)) + (at(1, 1) - at(-1, 1))
+            out[b] = (gx * gx + gy * gy).reshape(-1)
+        return out
+    monkeypatch.setattr(O, "sobel_score", wrong)
+    with pytest.raises(AssertionError):
+        test_sobel_matches_scipy_nearest()
+    monkeypatch.setattr(O, "sobel_score", real)
+
+
+def test_mutation_band_off_by_one_caught(monkeypatch):
+    monkeypatch.setattr(O, "band_start", lambda a, W, nb: min(max(a - W // 2, 0), nb - W))
+    with pytest.raises(AssertionError):
+        for row in _golden_patterns():
+            test_pattern_hand_derived_table(row)
