@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of one SparseSAM encoder block's hot path on B200.
+
+A step is one pass of the whole path -- Sobel score, stripe-sort permutation, Stripe-Sort sparse
+attention, Residual-Consistency MLP -- over one batch of the named synthetic workload (default:
+SAM ViT-B global block, 1 x 64x64 tokens, 12 heads x 64, density 0.4, MLP 768->3072->768).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1). The path has no exchange step: each rank runs an
+independent replica of the workload (weak scaling) and the job's throughput is all ranks' tokens
+over the slowest rank's device time. Rank 0 prints one JSON line.
+
+--impl reference times the float64 CPU oracle (the only reference this method has) on the host
+cores, on a bounded sample of the same workload, and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from structured_activation_sparsity_b200 import workloads  # noqa: E402
+
+METRIC = "Stripe-Sort attn + RC-MLP tokens/s per block; effective TFLOP/s vs bf16 peak"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one attention launch, from the ncu capture
+# summarised in profiles/ (None until captured for the current kernel).
+ATTN_TRAFFIC_BYTES = {}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["bf16_tflops"], d["bf16_tflops_sustained"], d["hbm_gbs"], "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.period, self.ok = [], period_s, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            props = torch.cuda.get_device_properties(device_index)
+            h = None
+            bus = getattr(props, "pci_bus_id", None)
+            if bus is not None:
+                dom = getattr(props, "pci_domain_id", 0)
+                dev = getattr(props, "pci_device_id", 0)
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08X}:{bus:02X}:{dev:02X}.0")
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv, self.h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report what we could not sample
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": getattr(self, "max_mhz", None), "reasons": [],
+                    "samples": 0, "note": getattr(self, "err", "no samples")}
+        mhz = [m for m, _ in self.samples]
+        seen = 0
+        for _, r in self.samples:
+            seen |= r
+        reasons = [k for k, bit in self.REASONS.items() if seen & bit and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle (the reference arm and the cpu_baseline leg)
+# ------------------------------------------------------------------------------------------------
+def cpu_sample(wl, min_seconds: float = 10.0):
+    """Time the float64 oracle on a bounded sample of the workload; return per-step seconds for
+    the full workload and a description. The sample: image 0's score, permutation and keep list;
+    attention of unit 0 for `hs` heads; the RC-MLP of image 0's kept rows. Per-step time is scaled
+    linearly to all units, heads and images."""
+    from oracle import sparsesam_oracle as O
+    from structured_activation_sparsity_b200 import synth
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    lum = synth.luminance(wl)[:1]
+    g = np.random.default_rng(wl.seed)
+    hs = min(wl.heads, 2)
+    shape = (1, wl.unit_tokens, hs, wl.head_dim)
+    q, k, v = (synth.bf16_to_f64(synth.to_bf16(g.standard_normal(shape, dtype=np.float32)))
+               for _ in range(3))
+    x, w1, b1, w2, b2 = synth.mlp_params(wl.with_(batch=1))
+    x, w1, w2 = (synth.bf16_to_f64(synth.to_bf16(a)) for a in (x, w1, w2))
+    geo = O.Geometry(1, wl.grid_h, wl.grid_w, wl.mode, wl.window)
+    reps, t_sp, t_at, t_mlp = 0, 0.0, 0.0, 0.0
+    t_begin = time.perf_counter()
+    while reps == 0 or time.perf_counter() - t_begin < min_seconds:
+        t0 = time.perf_counter()
+        score = O.sobel_score(lum)
+        perm, _ = O.stripe_sort(score, geo)
+        keep = O.keep_list(score, wl.density)
+        t1 = time.perf_counter()
+        O.attention(q, k, v, perm[:1], wl.density)
+        t2 = time.perf_counter()
+        O.rcmlp(x, w1, None, w2, None, keep)
+        t3 = time.perf_counter()
+        t_sp, t_at, t_mlp, reps = t_sp + t1 - t0, t_at + t2 - t1, t_mlp + t3 - t2, reps + 1
+    t_sp, t_at, t_mlp = t_sp / reps, t_at / reps, t_mlp / reps
+    step = (t_sp * wl.batch + t_at * wl.units * wl.heads / hs + t_mlp * wl.batch)
+    desc = (f"oracle on image 0 (score+perm+keep), unit 0 x {hs}/{wl.heads} heads (attention), "
+            f"image 0's {O.keep_count(wl.density, wl.tokens_per_image)} kept rows (MLP); "
+            f"{reps} reps, scaled linearly to {wl.batch} image(s), {wl.units} unit(s), "
+            f"{wl.heads} heads")
+    return step, desc, cores, reps * (t_sp + t_at + t_mlp)
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return
+    steps_t = []
+    desc = cores = None
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        cpu_sample(wl, min_seconds=0.0)
+    for _ in range(args.steps):
+        step, desc, cores, _ = cpu_sample(wl, min_seconds=0.0)
+        steps_t.append(step)
+    per_step = sum(steps_t) / len(steps_t)
+    value = wl.batch * wl.tokens_per_image / per_step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl, args, extra=None):
+    c = {"workload": wl.name, "batch": wl.batch, "grid": f"{wl.grid_h}x{wl.grid_w}",
+         "mode": wl.mode, "heads": wl.heads, "head_dim": wl.head_dim, "density": wl.density,
+         "mlp": f"{wl.dim}->{wl.hidden}->{wl.dim}", "parallelism": f"replicas x{args.gpus}"}
+    if wl.mode == "window":
+        c["window"] = wl.window
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+def make_sets(wl, n_sets, dev, density=None):
+    import torch
+    from structured_activation_sparsity_b200 import synth
+    from structured_activation_sparsity_b200.hotpath import HotPath
+
+    lum = torch.from_numpy(synth.luminance(wl))
+    q, k, v = (synth.to_bf16(a) for a in synth.qkv(wl))
+    mlp = [synth.to_bf16(a) for a in synth.mlp_params(wl)]
+    sets = []
+    for _ in range(n_sets):
+        hp = HotPath(wl, device=dev, density=density)
+        hp.load(lum, q, k, v, *mlp)
+        sets.append(hp)
+    return sets, (lum, q, k, v, mlp)
+
+
+def set_bytes(hp):
+    ts = [hp.lum, hp.score, hp.perm, hp.inv, hp.keep, hp.q, hp.k, hp.v, hp.out, hp.x, hp.w1,
+          hp.w2, hp.ws_attn, hp.ws_mlp]
+    return sum(t.numel() * t.element_size() for t in ts if t is not None)
+
+
+def time_steps(sets, steps, stream, dist=None):
+    import torch
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for i in range(steps):
+        sets[i % len(sets)].step(stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    return ev0.elapsed_time(ev1) / 1e3
+
+
+def max_over_ranks(x, dist, dev):
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args, wl, rank, world, local_rank, dist):
+    import torch
+    from structured_activation_sparsity_b200 import _lib as L
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    bf16_peak, bf16_sust, hbm_peak, peak_src = peaks()
+
+    probe, _ = make_sets(wl, 1, dev)
+    per_set = set_bytes(probe[0])
+    n_sets = max(2, math.ceil(3 * L2_BYTES / per_set))
+    sets = probe + make_sets(wl, n_sets - 1, dev)[0]
+    pat = sets[0].pattern
+    tokens_per_step = wl.batch * wl.tokens_per_image
+    attn_flops = workloads.attn_flops(wl.units, wl.unit_tokens, wl.heads, wl.head_dim, pat.rho)
+    mlp_flops = workloads.mlp_flops(wl.batch * pat.keep, wl.dim, wl.hidden)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            sets[i % n_sets].step(stream)
+    torch.cuda.synchronize()
+    if L.sparsesam_device_status(stream) != L.SS_OK:
+        raise RuntimeError("a device wait timed out during warm-up")
+
+    # ---- timed region: exactly K steps --------------------------------------------------------
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    n0 = L.sparsesam_launch_count()
+    t = time_steps(sets, args.steps, stream, dist)
+    launches = L.sparsesam_launch_count() - n0
+    clocks.stop()
+    t = max_over_ranks(t, dist, dev)
+    ms_per_step = t / args.steps * 1e3
+    value = world * tokens_per_step * args.steps / t
+
+    # ---- per-kernel durations: the same K steps again with launch tracing on ---------------------
+    L.sparsesam_trace_start(8 * args.steps + 16)
+    time_steps(sets, args.steps, stream, dist)
+    recs = L.sparsesam_trace_stop()
+    per_kernel = {}
+    for name, ms in recs:
+        per_kernel.setdefault(name, []).append(ms)
+    kernels = {n: {"launches": len(v), "avg_us": 1e3 * sum(v) / len(v)} for n, v in per_kernel.items()}
+    attn_us = kernels["attn"]["avg_us"]
+    achieved = attn_flops / (attn_us * 1e-6) / 1e12
+    traffic = ATTN_TRAFFIC_BYTES.get(wl.name)
+
+    # ---- dense comparison: the same kernels at density 1.0 -----------------------------------------
+    dense_sets = make_sets(wl, n_sets, dev, density=1.0)[0]
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            dense_sets[i % n_sets].step(stream)
+    td = max_over_ranks(time_steps(dense_sets, args.steps, stream, dist), dist, dev)
+    dense_value = world * tokens_per_step * args.steps / td
+    dpat = dense_sets[0].pattern
+    dense_flops = (workloads.attn_flops(wl.units, wl.unit_tokens, wl.heads, wl.head_dim, dpat.rho)
+                   + workloads.mlp_flops(wl.batch * dpat.keep, wl.dim, wl.hidden))
+    del dense_sets
+
+    # ---- end to end: pinned host inputs in, results out, through the same C-ABI calls ------------
+    hp = sets[0]
+    host_in = [t_.detach().to("cpu").pin_memory() for t_ in hp.input_tensors()]
+    host_out = [torch.empty(hp.out.shape, dtype=hp.out.dtype).pin_memory(),
+                torch.empty(hp.x.shape, dtype=hp.x.dtype).pin_memory()]
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = sum(x.numel() * x.element_size() for x in host_out)
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for dst, src in zip(hp.input_tensors(), host_in):
+                dst.copy_(src, non_blocking=True)
+            hp.step(stream)
+            host_out[0].copy_(hp.out, non_blocking=True)
+            host_out[1].copy_(hp.x, non_blocking=True)
+
+    for _ in range(max(3, args.warmup // 4)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    te = max_over_ranks(ev0.elapsed_time(ev1) / 1e3, dist, dev)
+    e2e_value = world * tokens_per_step * args.steps / te
+
+    if L.sparsesam_device_status(stream) != L.SS_OK:
+        raise RuntimeError("a device wait timed out during timing")
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(wl, args, {
+            "l2": f"{n_sets} rotating input sets of {per_set / 2**20:.0f} MiB (> 3x L2)",
+            "realised_density": pat.rho, "mlp_tokens_per_image": pat.keep}),
+        "clocks": clocks.summary(),
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "effective_tflops": (attn_flops + mlp_flops) * args.steps * world / t / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "attn", "achieved": achieved,
+                     "peak": bf16_peak, "unit": "TFLOP/s", "frac": achieved / bf16_peak,
+                     "traffic": traffic, "peak_source": f"{peak_src} bf16 burst",
+                     "algorithmic_flops_per_launch": attn_flops},
+        "kernels": kernels,
+        "dense": {"value": dense_value, "unit": UNIT, "ms_per_step": td / args.steps * 1e3,
+                  "effective_tflops": dense_flops * args.steps * world / td / 1e12,
+                  "sparse_speedup": value / dense_value},
+    }
+    if world == 1:
+        step_s, desc, cores, _ = cpu_sample(wl)
+        line["cpu_baseline"] = {"value": tokens_per_step / step_s, "unit": UNIT, "cores": cores,
+                                "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="vitb_global", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    wl = workloads.get(args.workload)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local_rank))
+        dist = tdist
+    try:
+        run_ours(args, wl, rank, world, local_rank, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,169 @@
+/*
+ * sparsesam.h -- C ABI of the SparseSAM encoder-block hot path on B200 (sm_100a).
+ *
+ * SparseSAM ("SparseSAM: Structured Sparsification of Activations in Segment Anything Models")
+ * accelerates SAM's ViT encoder with two training-free steps: Stripe-Sort attention and the
+ * Residual-Consistency MLP. This library runs the four steps of one encoder block's hot path:
+ *
+ *   sparsesam_score  S1  Sobel gradient score per token
+ *   sparsesam_perm   S2  stable sort by score + stripe transpose -> permutation; top-K keep list
+ *   sparsesam_attn   S3  static block-sparse attention over the permuted sequence
+ *   sparsesam_rcmlp  S4  fc1-GELU-fc2 on the kept tokens, added to the residual in place
+ *
+ * Conventions shared by every call
+ *   - Pointers marked (device) are device memory owned by the caller; nothing is allocated or
+ *     freed by these calls. Pointers marked (host) are host memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every GPU call is
+ *     asynchronous on it and never synchronises; results are ready when the stream is.
+ *   - Arguments are validated on the host before any launch. On a validation error nothing is
+ *     launched and the call returns a negative SS_E* code; sparsesam_strerror() names it.
+ *   - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
+ *   - A device-side wait that gives up (it never should) records SS_ETIMEOUT in a device status
+ *     word, makes the kernel return early and leaves the context usable; sparsesam_device_status()
+ *     reads and clears that word.
+ *
+ * Layouts (shared by the calls; U = attention units, N = tokens per unit)
+ *   global mode: U = batch, N = grid_h*grid_w (raster order).
+ *   window mode: the grid is padded bottom/right to a multiple of `window` and split into
+ *                windows in row-major window order; U = batch*windows, N = window^2, a window's
+ *                tokens in window-local raster order (pads included).
+ *   lum   fp32 [batch, grid_h, grid_w]
+ *   score fp64 [batch, grid_h*grid_w]               (pads are not stored; they score +0.0)
+ *   perm  int32 [U, N]  perm[u][p] = unit-local token at permuted position p
+ *   inv   int32 [U, N]  inv[u][perm[u][p]] = p
+ *   keep  int32 [batch, K]  image-raster token ids of the K top-ranked tokens, in rank order
+ *   q,k,v,out bf16 [U, N, heads, head_dim]
+ *   x     bf16 [batch, grid_h*grid_w, C]  (never padded)
+ */
+#ifndef SPARSESAM_H
+#define SPARSESAM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define SS_OK            0
+#define SS_EINVAL       (-1)  /* a null pointer, a non-positive size, density outside (0,1]      */
+#define SS_EUNSUPPORTED (-2)  /* a valid shape this build does not run (head_dim, N % 4, C % 64) */
+#define SS_EWORKSPACE   (-3)  /* workspace pointer null/misaligned or smaller than required     */
+#define SS_ECUDA        (-4)  /* a CUDA runtime/driver call failed (launch, tensor-map encode)   */
+#define SS_ETIMEOUT     (-5)  /* a device-side wait gave up (read via sparsesam_device_status)   */
+
+#define SS_GLOBAL 0
+#define SS_WINDOW 1
+
+/* One encoder block's shape. The SparseSAM README's registry call apply_sam(encoder, "sparsesam",
+ * ratio) takes the density as `ratio` ("ratio=0.5  # density 50%"); here it is `density`. */
+typedef struct {
+  int32_t batch;      /* images                                                   */
+  int32_t grid_h;     /* token grid rows of one image (64 for SAM at 1024 px)      */
+  int32_t grid_w;     /* token grid columns                                       */
+  int32_t mode;       /* SS_GLOBAL or SS_WINDOW                                    */
+  int32_t window;     /* window side in tokens (SAM: 14); ignored in global mode   */
+  int32_t heads;      /* attention heads                                          */
+  int32_t head_dim;   /* 64 or 80                                                  */
+  double  density;    /* fraction of attention and of MLP tokens computed, (0, 1]  */
+} ss_cfg;
+
+/* The static pattern a config implies (Stripe-Sort attention; SparseSAM Dutch technical summary,
+ * "Statisch Sparsiteitspatroon": a 4x4 mosaic of sub-maps, each with a banded diagonal, plus a small
+ * global keep-set). Offset block a of stripe j holds permuted positions j*L + a*b ... + b-1. */
+typedef struct {
+  int32_t units;        /* U                                                      */
+  int32_t unit_tokens;  /* N                                                      */
+  int32_t stripes;      /* 4                                                      */
+  int32_t L;            /* N / 4, the stripe length                               */
+  int32_t b;            /* block size: largest divisor of L with b <= 64, L/b >= 4 */
+  int32_t nb;           /* offset blocks per stripe, L / b                        */
+  int32_t W;            /* band width in offset blocks                            */
+  int32_t g;            /* global offset blocks (1)                               */
+  int32_t nnz;          /* kept (query offset block, key offset block) pairs      */
+  int32_t keep;         /* K = ceil(density * grid_h*grid_w - 1e-9), per image    */
+  double  rho;          /* realised attention density nnz / nb^2                 */
+} ss_pattern;
+
+/* Host only. Fills *out for cfg. Band width W is the one in [1, nb] whose density is nearest to
+ * cfg->density (ties: smaller W). Returns SS_OK or SS_EINVAL / SS_EUNSUPPORTED. */
+int sparsesam_pattern(const ss_cfg* cfg, ss_pattern* out);
+
+/* Host only. The kept key offset blocks of every query offset block as CSR: row_ptr[nb+1] and
+ * col_idx[nnz] (host, caller-owned, cap = capacity of col_idx). Row a lists, ascending, the
+ * offset blocks in [s, s+W) united with [0, g), s = clamp(a - (W-1)/2, 0, nb - W). All 16
+ * sub-maps (query stripe i, key stripe j) share this list. Returns SS_OK, SS_EINVAL (null / cap
+ * too small) or SS_EUNSUPPORTED. */
+int sparsesam_blocklist(const ss_cfg* cfg, int32_t* row_ptr, int32_t* col_idx, int32_t cap);
+
+/* S1 (SparseSAM Dutch technical summary, "Methodologie" 1, "Op Gradiënten Gebaseerde Ordening":
+ * a parameter-free Sobel operator's gradient magnitude as the information-density proxy).
+ * lum (device) fp32 [batch, grid_h, grid_w] -> score (device) fp64 [batch, grid_h*grid_w]:
+ *   gx = ((l[y-1,x+1]-l[y-1,x-1]) + 2*(l[y,x+1]-l[y,x-1])) + (l[y+1,x+1]-l[y+1,x-1])
+ *   gy = ((l[y+1,x-1]-l[y-1,x-1]) + 2*(l[y+1,x]-l[y-1,x])) + (l[y+1,x+1]-l[y-1,x+1])
+ *   score = gx*gx + gy*gy
+ * with clamp-to-edge borders, each step one fp64 round-to-nearest operation, no FMA. Bit-exact. */
+int sparsesam_score(const ss_cfg* cfg, const float* lum, double* score, void* stream);
+
+/* S2 (same summary, "Stripe-Sort Permutatie": sort the tokens by score, read the sorted list as a
+ * matrix, transpose it and flatten it). Per unit: stable sort descending by score (equal scores:
+ * lower enumeration index first) giving ranked tokens t_0..t_{N-1}; then perm[j*L + k] = t_{4k+j}.
+ * score (device) -> perm, inv (device) int32 [U, N]; keep (device) int32 [batch, K]: the first K
+ * tokens of each image's own ranking over its real tokens (window mode: per image, not per
+ * window). Any of perm/inv/keep may be NULL to skip it (not all three). Scores must not be NaN. */
+int sparsesam_perm(const ss_cfg* cfg, const double* score, int32_t* perm, int32_t* inv,
+                   int32_t* keep, void* stream);
+
+/* Bytes of device workspace sparsesam_attn needs for cfg (0 on an invalid cfg). */
+size_t sparsesam_attn_workspace(const ss_cfg* cfg);
+
+/* S3 (same summary, "Statisch Sparsiteitspatroon"; a FlashAttention-2-style kernel over a static
+ * pattern). For every unit and head: Qp = q[perm], Kp = k[perm], Vp = v[perm];
+ * Op[p] = softmax over the kept keys p' of (Qp[p].Kp[p'] / sqrt(head_dim)) applied to Vp;
+ * out[perm[p]] = Op[p]. q, k, v (device, read only), perm (device) from sparsesam_perm, out
+ * (device, may not alias q/k/v). bf16 operands, fp32 accumulation and softmax, probabilities rounded
+ * to bf16 before the second product. ws (device, 256-byte aligned) >= sparsesam_attn_workspace(cfg)
+ * bytes of scratch; its contents on entry do not matter. */
+int sparsesam_attn(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const int32_t* perm, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace sparsesam_rcmlp needs (0 on invalid arguments). */
+size_t sparsesam_rcmlp_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden);
+
+/* S4 (same summary, "Residual-Consistency MLP": only the top-K keep-set runs through the MLP; the
+ * residual set bypasses it unchanged). In place on x (device) bf16 [batch, grid_h*grid_w, C]:
+ * for each image b and kept token t = keep[b][r], r < K:
+ *   x[b,t,:] = bf16( x[b,t,:] + (w2 . GELU(w1 . x[b,t,:] + b1) + b2) ),  GELU(z) = z/2 (1+erf(z/sqrt2))
+ * every other row is left bit-for-bit untouched. w1 bf16 [hidden, C], w2 bf16 [C, hidden]
+ * (row-major, PyTorch nn.Linear weight layout); b1 [hidden], b2 [C] bf16 or NULL (zero). keep
+ * (device) int32 [batch, K] with distinct rows per image (as sparsesam_perm writes it).
+ * C and hidden must be multiples of 64. bf16 operands, fp32 accumulation; the hidden activation
+ * is rounded to bf16 between the two products. ws (device, 256-byte aligned) >=
+ * sparsesam_rcmlp_workspace bytes. */
+int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden,
+                    const uint16_t* w1, const uint16_t* b1, const uint16_t* w2, const uint16_t* b2,
+                    const int32_t* keep, void* ws, size_t ws_bytes, void* stream);
+
+/* Reads (and clears) the device status word that bounded device waits write. Synchronises the
+ * given stream. *status receives SS_OK or SS_ETIMEOUT. Returns SS_OK or SS_ECUDA. */
+int sparsesam_device_status(int32_t* status, void* stream);
+
+/* Kernel launches this library has issued since it was loaded (host counter). */
+uint64_t sparsesam_launch_count(void);
+
+/* Per-launch tracing. While enabled, each kernel launch is bracketed by two CUDA events on its
+ * stream (at most `capacity` launches are recorded). sparsesam_trace_stop synchronises the events,
+ * and sparsesam_trace_get(i, ...) returns the i-th launch's kernel name and duration in ms.
+ * Returns the number of records (stop) or SS_OK / SS_EINVAL / SS_ECUDA. */
+int sparsesam_trace_start(int32_t capacity);
+int sparsesam_trace_stop(void);
+int sparsesam_trace_get(int32_t i, const char** name, float* ms);
+
+/* Static text for a return code. */
+const char* sparsesam_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPARSESAM_H */

@@ -1,0 +1,189 @@
+"""ctypes binding of libsparsesam.so (the C ABI in include/sparsesam.h).
+
+Argument marshalling only: every step of the hot path runs in the library's sm_100a kernels. Tensor
+arguments may be torch tensors (their data_ptr() is passed) or raw integer addresses. There is no
+fallback: if the library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsparsesam.so")
+
+SS_OK = 0
+SS_EINVAL = -1
+SS_EUNSUPPORTED = -2
+SS_EWORKSPACE = -3
+SS_ECUDA = -4
+SS_ETIMEOUT = -5
+SS_GLOBAL = 0
+SS_WINDOW = 1
+
+
+class SsCfg(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+                ("mode", ctypes.c_int32), ("window", ctypes.c_int32), ("heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("density", ctypes.c_double)]
+
+
+class SsPattern(ctypes.Structure):
+    _fields_ = [("units", ctypes.c_int32), ("unit_tokens", ctypes.c_int32),
+                ("stripes", ctypes.c_int32), ("L", ctypes.c_int32), ("b", ctypes.c_int32),
+                ("nb", ctypes.c_int32), ("W", ctypes.c_int32), ("g", ctypes.c_int32),
+                ("nnz", ctypes.c_int32), ("keep", ctypes.c_int32), ("rho", ctypes.c_double)]
+
+
+class SparseSAMError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} failed: {code} ({strerror(code)})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m structured_activation_sparsity_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, SZ, VP = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_void_p
+    cfgp = ctypes.POINTER(SsCfg)
+    sig = {
+        "sparsesam_pattern": (ctypes.c_int, [cfgp, ctypes.POINTER(SsPattern)]),
+        "sparsesam_blocklist": (ctypes.c_int, [cfgp, P, P, I32]),
+        "sparsesam_score": (ctypes.c_int, [cfgp, P, P, VP]),
+        "sparsesam_perm": (ctypes.c_int, [cfgp, P, P, P, P, VP]),
+        "sparsesam_attn_workspace": (SZ, [cfgp]),
+        "sparsesam_attn": (ctypes.c_int, [cfgp, P, P, P, P, P, P, SZ, VP]),
+        "sparsesam_rcmlp_workspace": (SZ, [cfgp, I32, I32]),
+        "sparsesam_rcmlp": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, P, SZ, VP]),
+        "sparsesam_device_status": (ctypes.c_int, [ctypes.POINTER(I32), VP]),
+        "sparsesam_launch_count": (ctypes.c_uint64, []),
+        "sparsesam_trace_start": (ctypes.c_int, [I32]),
+        "sparsesam_trace_stop": (ctypes.c_int, []),
+        "sparsesam_trace_get": (ctypes.c_int, [I32, ctypes.POINTER(ctypes.c_char_p),
+                                               ctypes.POINTER(ctypes.c_float)]),
+        "sparsesam_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def strerror(code: int) -> str:
+    return lib.sparsesam_strerror(int(code)).decode()
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream  # torch.cuda.Stream
+
+
+def _check(fn: str, rc: int) -> int:
+    if rc != SS_OK:
+        raise SparseSAMError(fn, rc)
+    return rc
+
+
+def make_cfg(batch, grid_h, grid_w, mode="global", window=14, heads=1, head_dim=64,
+             density=1.0) -> SsCfg:
+    m = SS_GLOBAL if mode in ("global", SS_GLOBAL) else SS_WINDOW
+    return SsCfg(batch, grid_h, grid_w, m, window, heads, head_dim, float(density))
+
+
+def cfg_for(wl, density: float | None = None) -> SsCfg:
+    """SsCfg of a workloads.Workload."""
+    return make_cfg(wl.batch, wl.grid_h, wl.grid_w, wl.mode, wl.window, wl.heads, wl.head_dim,
+                    wl.density if density is None else density)
+
+
+def sparsesam_pattern(cfg: SsCfg) -> SsPattern:
+    p = SsPattern()
+    _check("sparsesam_pattern", lib.sparsesam_pattern(ctypes.byref(cfg), ctypes.byref(p)))
+    return p
+
+
+def sparsesam_blocklist(cfg: SsCfg):
+    """(row_ptr, col_idx) as Python int lists."""
+    p = sparsesam_pattern(cfg)
+    row_ptr = (ctypes.c_int32 * (p.nb + 1))()
+    col_idx = (ctypes.c_int32 * max(1, p.nnz))()
+    _check("sparsesam_blocklist",
+           lib.sparsesam_blocklist(ctypes.byref(cfg), ctypes.cast(row_ptr, ctypes.c_void_p),
+                                   ctypes.cast(col_idx, ctypes.c_void_p), p.nnz))
+    return list(row_ptr), list(col_idx)[:p.nnz]
+
+
+def sparsesam_score(cfg, lum, score, stream=None):
+    return _check("sparsesam_score",
+                  lib.sparsesam_score(ctypes.byref(cfg), _ptr(lum), _ptr(score), _stream(stream)))
+
+
+def sparsesam_perm(cfg, score, perm, inv, keep, stream=None):
+    return _check("sparsesam_perm",
+                  lib.sparsesam_perm(ctypes.byref(cfg), _ptr(score), _ptr(perm), _ptr(inv),
+                                     _ptr(keep), _stream(stream)))
+
+
+def sparsesam_attn_workspace(cfg) -> int:
+    return int(lib.sparsesam_attn_workspace(ctypes.byref(cfg)))
+
+
+def sparsesam_attn(cfg, q, k, v, perm, out, ws, ws_bytes, stream=None):
+    return _check("sparsesam_attn",
+                  lib.sparsesam_attn(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(perm),
+                                     _ptr(out), _ptr(ws), int(ws_bytes), _stream(stream)))
+
+
+def sparsesam_rcmlp_workspace(cfg, C: int, hidden: int) -> int:
+    return int(lib.sparsesam_rcmlp_workspace(ctypes.byref(cfg), int(C), int(hidden)))
+
+
+def sparsesam_rcmlp(cfg, x, C, hidden, w1, b1, w2, b2, keep, ws, ws_bytes, stream=None):
+    return _check("sparsesam_rcmlp",
+                  lib.sparsesam_rcmlp(ctypes.byref(cfg), _ptr(x), int(C), int(hidden), _ptr(w1),
+                                      _ptr(b1), _ptr(w2), _ptr(b2), _ptr(keep), _ptr(ws),
+                                      int(ws_bytes), _stream(stream)))
+
+
+def sparsesam_device_status(stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check("sparsesam_device_status", lib.sparsesam_device_status(ctypes.byref(v), _stream(stream)))
+    return v.value
+
+
+def sparsesam_launch_count() -> int:
+    return int(lib.sparsesam_launch_count())
+
+
+def sparsesam_trace_start(capacity: int):
+    return _check("sparsesam_trace_start", lib.sparsesam_trace_start(int(capacity)))
+
+
+def sparsesam_trace_stop():
+    """Returns [(kernel name, ms), ...] for the launches recorded since trace_start."""
+    n = lib.sparsesam_trace_stop()
+    if n < 0:
+        raise SparseSAMError("sparsesam_trace_stop", n)
+    out = []
+    for i in range(n):
+        name, ms = ctypes.c_char_p(), ctypes.c_float()
+        _check("sparsesam_trace_get", lib.sparsesam_trace_get(i, ctypes.byref(name), ctypes.byref(ms)))
+        out.append((name.value.decode(), float(ms.value)))
+    return out

@@ -1,0 +1,437 @@
+// Host side of the C ABI declared in include/sparsesam.h: argument validation, workspace carving,
+// TMA descriptor encoding, launch tracing and the status word. Every GPU step runs in this
+// library's kernels; nothing here computes on the host except the static pattern's integers.
+#include <math.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "kernels.h"
+
+namespace ss {
+
+// Device status word written by bounded device waits that give up (see sparsesam_device_status).
+__device__ int g_status = 0;
+
+namespace {
+
+std::mutex g_mu;
+std::atomic<uint64_t> g_launches{0};
+
+// ---- per-device address of the status word ----------------------------------------------------
+int* status_word() {
+  static int* addr[128] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
+// ---- launch tracing -----------------------------------------------------------------------------
+struct TraceRec {
+  const char* name;
+  cudaEvent_t e0, e1;
+  float ms;
+};
+std::vector<TraceRec> g_trace;
+int g_trace_used = 0;
+bool g_tracing = false;
+
+template <class F>
+cudaError_t traced(const char* name, cudaStream_t st, F&& f) {
+  TraceRec* rec = nullptr;
+  if (g_tracing && g_trace_used < (int)g_trace.size()) {
+    rec = &g_trace[g_trace_used++];
+    rec->name = name;
+    cudaEventRecord(rec->e0, st);
+  }
+  cudaError_t e = f();
+  if (rec) cudaEventRecord(rec->e1, st);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
+// ---- tensor maps --------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor of `mats` matrices [rows, inner] with rows `row_bytes` apart; box [box_rows, box_inner].
+// `rank` must match the dimensionality of the kernel's TMA instruction (2: one matrix, 3: a stack).
+bool encode_bf16(CUtensorMap* m, cuuint32_t rank, const void* base, uint64_t inner, uint64_t rows,
+                 uint64_t mats, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                 CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, mats};
+  cuuint64_t strides[2] = {row_bytes, row_bytes * rows};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (rank != 2 && rank != 3) return false;
+  if (rank == 2 && mats != 1) return false;
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---- geometry -----------------------------------------------------------------------------------
+struct Geo {
+  int B, Hg, Wg, T;      // images, grid, tokens per image
+  int window_mode, ws, wpr, windows;
+  int U, N;              // attention units, tokens per unit
+};
+
+int geometry(const ss_cfg* c, Geo* g) {
+  if (!c) return SS_EINVAL;
+  if (c->batch < 1 || c->grid_h < 1 || c->grid_w < 1) return SS_EINVAL;
+  if (c->mode != SS_GLOBAL && c->mode != SS_WINDOW) return SS_EINVAL;
+  if (c->mode == SS_WINDOW && c->window < 1) return SS_EINVAL;
+  if (!(c->density > 0.0 && c->density <= 1.0)) return SS_EINVAL;   // also rejects NaN
+  if ((int64_t)c->grid_h * c->grid_w > (1 << 24) || c->batch > (1 << 20)) return SS_EUNSUPPORTED;
+  g->B = c->batch;
+  g->Hg = c->grid_h;
+  g->Wg = c->grid_w;
+  g->T = c->grid_h * c->grid_w;
+  g->window_mode = c->mode == SS_WINDOW;
+  if (g->window_mode) {
+    g->ws = c->window;
+    g->wpr = (c->grid_w + c->window - 1) / c->window;
+    g->windows = g->wpr * ((c->grid_h + c->window - 1) / c->window);
+    g->N = c->window * c->window;
+  } else {
+    g->ws = 0;
+    g->wpr = 1;
+    g->windows = 1;
+    g->N = g->T;
+  }
+  if ((int64_t)g->B * g->windows > (1 << 24)) return SS_EUNSUPPORTED;
+  g->U = g->B * g->windows;
+  return SS_OK;
+}
+
+int pattern_of(const ss_cfg* c, const Geo& g, ss_pattern* p) {
+  if (g.N % kStripes != 0) return SS_EUNSUPPORTED;
+  const int L = g.N / kStripes;
+  const int b = block_size_for(L);
+  if (b == 0) return SS_EUNSUPPORTED;
+  const int nb = L / b;
+  const int W = choose_band(nb, kGlobalBlocks, c->density);
+  p->units = g.U;
+  p->unit_tokens = g.N;
+  p->stripes = kStripes;
+  p->L = L;
+  p->b = b;
+  p->nb = nb;
+  p->W = W;
+  p->g = kGlobalBlocks;
+  p->nnz = pattern_nnz(W, nb, kGlobalBlocks);
+  p->keep = keep_count(c->density, g.T);
+  p->rho = (double)p->nnz / (double)(nb * nb);
+  return SS_OK;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_err(cudaError_t e) { return e == cudaSuccess ? SS_OK : SS_ECUDA; }
+
+size_t attn_ws_bytes(const Geo& g, int heads, int dh) {
+  return 3 * align256((size_t)g.U * heads * g.N * dh * 2);
+}
+
+size_t rcmlp_ws_bytes(const Geo& g, int K, int C, int hidden) {
+  const size_t M = (size_t)g.B * K;
+  return align256(M * C * 2) + align256(M * hidden * 2);
+}
+
+int gemm_bn(int n) { return n % 256 == 0 && n >= 1024 ? 256 : (n % 128 == 0 ? 128 : 64); }
+
+}  // namespace
+}  // namespace ss
+
+using namespace ss;
+
+extern "C" {
+
+int sparsesam_pattern(const ss_cfg* cfg, ss_pattern* out) {
+  if (!out) return SS_EINVAL;
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  return pattern_of(cfg, g, out);
+}
+
+int sparsesam_blocklist(const ss_cfg* cfg, int32_t* row_ptr, int32_t* col_idx, int32_t cap) {
+  if (!row_ptr || !col_idx) return SS_EINVAL;
+  ss_pattern p;
+  int rc = sparsesam_pattern(cfg, &p);
+  if (rc) return rc;
+  if (cap < p.nnz) return SS_EINVAL;
+  int n = 0;
+  row_ptr[0] = 0;
+  for (int a = 0; a < p.nb; ++a) {
+    for (int ka = 0; ka < p.nb; ++ka)
+      if (block_kept(a, ka, p.W, p.nb, p.g)) col_idx[n++] = ka;
+    row_ptr[a + 1] = n;
+  }
+  return SS_OK;
+}
+
+int sparsesam_score(const ss_cfg* cfg, const float* lum, double* score, void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  if (!lum || !score) return SS_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_err(traced("sobel_score", st, [&] {
+    return launch_sobel_score(lum, score, g.B, g.Hg, g.Wg, st);
+  }));
+}
+
+int sparsesam_perm(const ss_cfg* cfg, const double* score, int32_t* perm, int32_t* inv,
+                   int32_t* keep, void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  if (!score || (!perm && !inv && !keep)) return SS_EINVAL;
+  ss_pattern p;
+  if ((perm || inv) && (rc = pattern_of(cfg, g, &p))) return rc;
+  if (g.N > kMaxRankTokens || g.T > kMaxRankTokens) return SS_EUNSUPPORTED;
+  if (g.U > 65535) return SS_EUNSUPPORTED;
+  const int K = keep_count(cfg->density, g.T);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!g.window_mode) {
+    return cuda_err(traced("stripe_rank", st, [&] {
+      return launch_stripe_rank(score, 0, g.B, g.Hg, g.Wg, 0, g.B, g.T, K, perm, inv, keep, st);
+    }));
+  }
+  if (perm || inv) {
+    rc = cuda_err(traced("stripe_rank_window", st, [&] {
+      return launch_stripe_rank(score, 1, g.B, g.Hg, g.Wg, g.ws, g.U, g.N, 0, perm, inv, nullptr,
+                                st);
+    }));
+    if (rc) return rc;
+  }
+  if (keep) {
+    rc = cuda_err(traced("keep_rank", st, [&] {
+      return launch_stripe_rank(score, 0, g.B, g.Hg, g.Wg, 0, g.B, g.T, K, nullptr, nullptr, keep,
+                                st);
+    }));
+  }
+  return rc;
+}
+
+size_t sparsesam_attn_workspace(const ss_cfg* cfg) {
+  Geo g;
+  if (geometry(cfg, &g) || cfg->heads < 1 || cfg->head_dim < 1) return 0;
+  return attn_ws_bytes(g, cfg->heads, cfg->head_dim);
+}
+
+int sparsesam_attn(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const int32_t* perm, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  if (cfg->heads < 1 || cfg->head_dim < 1) return SS_EINVAL;
+  if (!q || !k || !v || !perm || !out) return SS_EINVAL;
+  if (cfg->head_dim != 64 && cfg->head_dim != 80) return SS_EUNSUPPORTED;
+  ss_pattern p;
+  if ((rc = pattern_of(cfg, g, &p))) return rc;
+  const int heads = cfg->heads, dh = cfg->head_dim;
+  if ((int64_t)g.U * heads > 65535) return SS_EUNSUPPORTED;
+  if ((int64_t)g.U * g.N * heads * (dh / 8) >= (int64_t)1 << 31) return SS_EUNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return SS_EINVAL;
+  const size_t need = attn_ws_bytes(g, heads, dh);
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SS_EWORKSPACE;
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+
+  const size_t one = need / 3;
+  uint16_t* qp = static_cast<uint16_t*>(ws);
+  uint16_t* kp = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + one);
+  uint16_t* vp = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + 2 * one);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  rc = cuda_err(traced("gather_qkv", st, [&] {
+    return launch_gather_qkv(q, k, v, perm, qp, kp, vp, g.U, g.N, heads, dh, p.b, st);
+  }));
+  if (rc) return rc;
+
+  CUtensorMap tm[6];
+  const uint64_t mats = (uint64_t)g.U * heads;
+  const uint16_t* bufs[3] = {qp, kp, vp};
+  for (int i = 0; i < 3; ++i) {
+    if (!encode_bf16(&tm[i], 3, bufs[i], dh, g.N, mats, (uint64_t)dh * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return SS_ECUDA;
+    if (dh == 80 && !encode_bf16(&tm[3 + i], 3, bufs[i], dh, g.N, mats, (uint64_t)dh * 2, 16, 128,
+                                 CU_TENSOR_MAP_SWIZZLE_32B))
+      return SS_ECUDA;
+  }
+  AttnParams ap;
+  ap.perm = perm;
+  ap.out = out;
+  ap.U = g.U;
+  ap.N = g.N;
+  ap.heads = heads;
+  ap.L = p.L;
+  ap.b = p.b;
+  ap.nb = p.nb;
+  ap.W = p.W;
+  ap.g = p.g;
+  ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dh));
+  return cuda_err(traced("attn", st, [&] {
+    return launch_attn(&tm[0], &tm[1], &tm[2], &tm[3], &tm[4], &tm[5], ap, dh, status, st);
+  }));
+}
+
+size_t sparsesam_rcmlp_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden) {
+  Geo g;
+  if (geometry(cfg, &g) || C < 1 || hidden < 1) return 0;
+  return rcmlp_ws_bytes(g, keep_count(cfg->density, g.T), C, hidden);
+}
+
+int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, const uint16_t* w1,
+                    const uint16_t* b1, const uint16_t* w2, const uint16_t* b2,
+                    const int32_t* keep, void* ws, size_t ws_bytes, void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  if (!x || !w1 || !w2 || !keep || C < 1 || hidden < 1) return SS_EINVAL;
+  if (C % 64 != 0 || hidden % 64 != 0) return SS_EUNSUPPORTED;
+  if (!aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16)) return SS_EINVAL;
+  const int K = keep_count(cfg->density, g.T);
+  const int64_t M = (int64_t)g.B * K;
+  if (M * (hidden > C ? hidden : C) >= ((int64_t)1 << 31) || (M + 127) / 128 > 65535)
+    return SS_EUNSUPPORTED;
+  const size_t need = rcmlp_ws_bytes(g, K, C, hidden);
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SS_EWORKSPACE;
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+  uint16_t* xk = static_cast<uint16_t*>(ws);
+  uint16_t* hbuf =
+      reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + align256((size_t)M * C * 2));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  rc = cuda_err(traced("gather_rows", st, [&] {
+    return launch_gather_rows(x, keep, xk, g.B, g.T, K, C, st);
+  }));
+  if (rc) return rc;
+
+  const int bn1 = gemm_bn(hidden), bn2 = gemm_bn(C);
+  CUtensorMap ta1, tb1, ta2, tb2;
+  if (!encode_bf16(&ta1, 2, xk, C, M, 1, (uint64_t)C * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16(&tb1, 2, w1, C, hidden, 1, (uint64_t)C * 2, 64, bn1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16(&ta2, 2, hbuf, hidden, M, 1, (uint64_t)hidden * 2, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16(&tb2, 2, w2, hidden, C, 1, (uint64_t)hidden * 2, 64, bn2,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return SS_ECUDA;
+
+  GemmEpilogue e1 = {};
+  e1.kind = 0;
+  e1.bias = b1;
+  e1.out = hbuf;
+  rc = cuda_err(traced("rcmlp_fc1", st, [&] {
+    return launch_gemm(&ta1, &tb1, (int)M, hidden, C, bn1, e1, status, st);
+  }));
+  if (rc) return rc;
+  GemmEpilogue e2 = {};
+  e2.kind = 1;
+  e2.bias = b2;
+  e2.x = x;
+  e2.keep = keep;
+  e2.K_per_image = K;
+  e2.T = g.T;
+  return cuda_err(traced("rcmlp_fc2", st, [&] {
+    return launch_gemm(&ta2, &tb2, (int)M, C, hidden, bn2, e2, status, st);
+  }));
+}
+
+int sparsesam_device_status(int32_t* out, void* stream) {
+  if (!out) return SS_EINVAL;
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return SS_ECUDA;
+  *out = v;
+  return SS_OK;
+}
+
+uint64_t sparsesam_launch_count(void) { return g_launches.load(); }
+
+int sparsesam_trace_start(int32_t capacity) {
+  if (capacity < 1) return SS_EINVAL;
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (auto& r : g_trace) {
+    cudaEventDestroy(r.e0);
+    cudaEventDestroy(r.e1);
+  }
+  g_trace.assign(capacity, TraceRec{nullptr, nullptr, nullptr, 0.f});
+  for (auto& r : g_trace)
+    if (cudaEventCreate(&r.e0) != cudaSuccess || cudaEventCreate(&r.e1) != cudaSuccess)
+      return SS_ECUDA;
+  g_trace_used = 0;
+  g_tracing = true;
+  return SS_OK;
+}
+
+int sparsesam_trace_stop(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_tracing = false;
+  for (int i = 0; i < g_trace_used; ++i) {
+    TraceRec& r = g_trace[i];
+    if (cudaEventSynchronize(r.e1) != cudaSuccess ||
+        cudaEventElapsedTime(&r.ms, r.e0, r.e1) != cudaSuccess)
+      return SS_ECUDA;
+  }
+  return g_trace_used;
+}
+
+int sparsesam_trace_get(int32_t i, const char** name, float* ms) {
+  if (i < 0 || i >= g_trace_used || !name || !ms) return SS_EINVAL;
+  *name = g_trace[i].name;
+  *ms = g_trace[i].ms;
+  return SS_OK;
+}
+
+const char* sparsesam_strerror(int code) {
+  switch (code) {
+    case SS_OK: return "ok";
+    case SS_EINVAL: return "invalid argument";
+    case SS_EUNSUPPORTED: return "unsupported shape";
+    case SS_EWORKSPACE: return "workspace missing, misaligned or too small";
+    case SS_ECUDA: return "CUDA call failed";
+    case SS_ETIMEOUT: return "device wait timed out";
+  }
+  return "unknown error";
+}
+
+}  // extern "C"

@@ -1,0 +1,56 @@
+// Host-side launchers of the library's kernels (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pattern.h"
+#include "sparsesam.h"
+
+namespace ss {
+
+constexpr int kMaxRankTokens = 16384;   // tokens per unit the rank kernel holds in shared memory
+
+cudaError_t launch_sobel_score(const float* lum, double* score, int B, int H, int W,
+                               cudaStream_t st);
+
+cudaError_t launch_stripe_rank(const double* score, int window_mode, int B, int Hg, int Wg, int ws,
+                               int units, int N, int K, int32_t* perm, int32_t* inv,
+                               int32_t* keep, cudaStream_t st);
+
+// Gathers q, k, v [U, N, heads, dh] into the block-major permuted layout [U*heads, N, dh].
+cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                              const int32_t* perm, uint16_t* qp, uint16_t* kp, uint16_t* vp,
+                              int U, int N, int heads, int dh, int b, cudaStream_t st);
+
+struct AttnParams {
+  const int32_t* perm;   // [U, N]
+  uint16_t* out;         // [U, N, heads, dh]
+  int U, N, heads, L, b, nb, W, g;
+  float scale_log2;      // log2(e) / sqrt(dh)
+};
+// Block-sparse attention over the gathered sequences (tensor maps over [U*heads, N, dh]).
+cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                        const CUtensorMap* tq_tail, const CUtensorMap* tk_tail,
+                        const CUtensorMap* tv_tail, const AttnParams& p, int dh, int* status,
+                        cudaStream_t st);
+
+// Gathers the kept rows of x [B, T, C] into xk [B*K, C].
+cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* keep, uint16_t* xk, int B, int T,
+                               int K, int C, cudaStream_t st);
+
+struct GemmEpilogue {
+  int kind;                 // 0: out = bf16(GELU(acc + bias)) into out[M, N]
+                            // 1: x[b, keep[m], n] = bf16(x + acc + bias)
+  const uint16_t* bias;     // [N] or null
+  uint16_t* out;            // kind 0
+  uint16_t* x;              // kind 1: [B, T, N]
+  const int32_t* keep;      // kind 1: [B*K]
+  int K_per_image, T;       // kind 1
+};
+// C[M, N] = A[M, Kd] * B[N, Kd]^T on tcgen05 with the given epilogue.
+cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, int M, int N, int Kd,
+                        int BN, const GemmEpilogue& ep, int* status, cudaStream_t st);
+
+}  // namespace ss

@@ -1,0 +1,119 @@
+// S1 Sobel score and S2 stripe-sort permutation kernels.
+//
+// S1 follows the SparseSAM Dutch technical summary, "Op Gradiënten Gebaseerde Ordening" (a
+// parameter-free Sobel operator's gradient magnitude per token). S2 follows "Stripe-Sort
+// Permutatie" (sort by that score, read the sorted list as a matrix, transpose, flatten).
+//
+// The sort is done by rank counting rather than a comparison network: rank(t) = number of tokens
+// that come before t in the stable descending order. With N <= 16384 tokens per unit that is N^2
+// independent compares spread over the whole GPU (32 target tokens per CTA, 8 warps splitting the
+// other tokens), no synchronisation beyond one CTA-level reduction, and the result is the stable
+// order by construction. Each rank is scattered straight into perm, inv and the keep list.
+#include "kernels.h"
+
+namespace ss {
+
+__global__ void __launch_bounds__(256) k_sobel_score(const float* __restrict__ lum,
+                                                     double* __restrict__ score, int B, int H,
+                                                     int W) {
+  int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  int per = H * W;
+  if (idx >= B * per) return;
+  int b = idx / per;
+  int r = idx - b * per;
+  int y = r / W, x = r - (r / W) * W;
+  int ym = y > 0 ? y - 1 : 0, yp = y < H - 1 ? y + 1 : H - 1;
+  int xm = x > 0 ? x - 1 : 0, xp = x < W - 1 ? x + 1 : W - 1;
+  const float* img = lum + (size_t)b * per;
+  double l_mm = img[ym * W + xm], l_m0 = img[ym * W + x], l_mp = img[ym * W + xp];
+  double l_0m = img[y * W + xm], l_0p = img[y * W + xp];
+  double l_pm = img[yp * W + xm], l_p0 = img[yp * W + x], l_pp = img[yp * W + xp];
+  // Each step is one fp64 round-to-nearest operation, in a fixed order, never fused.
+  double gx = __dadd_rn(__dadd_rn(__dsub_rn(l_mp, l_mm), __dmul_rn(2.0, __dsub_rn(l_0p, l_0m))),
+                        __dsub_rn(l_pp, l_pm));
+  double gy = __dadd_rn(__dadd_rn(__dsub_rn(l_pm, l_mm), __dmul_rn(2.0, __dsub_rn(l_p0, l_m0))),
+                        __dsub_rn(l_pp, l_mp));
+  score[idx] = __dadd_rn(__dmul_rn(gx, gx), __dmul_rn(gy, gy));
+}
+
+// Unit-local token t -> its score key (bits of a non-negative double, which order like the value).
+struct UnitMap {
+  int window_mode;   // 0: unit = image, t = raster index; 1: unit = window, t = window raster
+  int Hg, Wg, ws, wpr, nwin;
+  __device__ __forceinline__ unsigned long long key(const double* score, int u, int t) const {
+    if (!window_mode) {
+      return (unsigned long long)__double_as_longlong(score[(size_t)u * Hg * Wg + t]);
+    }
+    int b = u / nwin, w = u - (u / nwin) * nwin;
+    int wy = w / wpr, wx = w - (w / wpr) * wpr;
+    int y = wy * ws + t / ws, x = wx * ws + t % ws;
+    if (y >= Hg || x >= Wg) return 0ull;   // pad token: +0.0
+    return (unsigned long long)__double_as_longlong(score[(size_t)b * Hg * Wg + y * Wg + x]);
+  }
+};
+
+// grid (ceil(N/32), units), block 256, dynamic smem N * 8 bytes.
+__global__ void __launch_bounds__(256) k_stripe_rank(const double* __restrict__ score, UnitMap m,
+                                                     int N, int K, int32_t* __restrict__ perm,
+                                                     int32_t* __restrict__ inv,
+                                                     int32_t* __restrict__ keep) {
+  extern __shared__ unsigned long long s_key[];
+  __shared__ int s_cnt[8][32];
+  const int u = blockIdx.y;
+  for (int t = threadIdx.x; t < N; t += blockDim.x) s_key[t] = m.key(score, u, t);
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 32 + lane;
+  const int tt = t < N ? t : N - 1;
+  const unsigned long long kt = s_key[tt];
+  const int chunk = (N + 7) / 8;
+  const int lo = warp * chunk, hi = min(N, lo + chunk);
+  int cnt = 0;
+  for (int o = lo; o < hi; ++o) {
+    unsigned long long ko = s_key[o];
+    cnt += (ko > kt) | ((ko == kt) & (o < tt));
+  }
+  s_cnt[warp][lane] = cnt;
+  __syncthreads();
+  if (warp == 0 && t < N) {
+    int r = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) r += s_cnt[w][lane];
+    const int L = N / kStripes;
+    const int pos = (r % kStripes) * L + r / kStripes;   // stripe transpose
+    if (perm) perm[(size_t)u * N + pos] = t;
+    if (inv) inv[(size_t)u * N + t] = pos;
+    if (keep && r < K) keep[(size_t)u * K + r] = t;
+  }
+}
+
+cudaError_t launch_sobel_score(const float* lum, double* score, int B, int H, int W,
+                               cudaStream_t st) {
+  int n = B * H * W;
+  k_sobel_score<<<(n + 255) / 256, 256, 0, st>>>(lum, score, B, H, W);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stripe_rank(const double* score, int window_mode, int B, int Hg, int Wg, int ws,
+                               int units, int N, int K, int32_t* perm, int32_t* inv,
+                               int32_t* keep, cudaStream_t st) {
+  UnitMap m;
+  m.window_mode = window_mode;
+  m.Hg = Hg;
+  m.Wg = Wg;
+  m.ws = ws;
+  m.wpr = window_mode ? (Wg + ws - 1) / ws : 1;
+  m.nwin = window_mode ? m.wpr * ((Hg + ws - 1) / ws) : 1;
+  size_t smem = (size_t)N * sizeof(unsigned long long);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_stripe_rank, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid((N + 31) / 32, units);
+  k_stripe_rank<<<grid, 256, smem, st>>>(score, m, N, K, perm, inv, keep);
+  return cudaGetLastError();
+}
+
+}  // namespace ss

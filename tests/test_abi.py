@@ -1,0 +1,132 @@
+"""CPU checks of the C-ABI library: it loads, exports every declared symbol, validates arguments on
+the host before touching a GPU, and its static pattern equals the oracle's bit for bit."""
+import ctypes
+import math
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle import sparsesam_oracle as O
+from structured_activation_sparsity_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sparsesam.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*[a-z_0-9 ]+\*?\s*\**\s*(sparsesam_\w+)\s*\(", text, re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 14
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(\w+)$", out, re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(L.lib, n)
+
+
+def test_no_launches_without_gpu_work():
+    assert L.sparsesam_launch_count() == 0
+
+
+def test_strerror():
+    assert L.strerror(0) == "ok"
+    for c in (-1, -2, -3, -4, -5):
+        assert L.strerror(c) != "unknown error"
+    assert L.strerror(-99) == "unknown error"
+
+
+# ---- pattern / blocklist equal the oracle ----------------------------------------------------
+CASES = [
+    (1, 16, 16, "global", 0.4), (1, 64, 64, "global", 0.4), (4, 64, 64, "global", 0.3),
+    (1, 64, 64, "global", 0.5), (1, 64, 64, "global", 1.0), (2, 64, 64, "window", 0.3),
+    (2, 64, 64, "window", 0.4), (2, 64, 64, "window", 0.5), (1, 32, 32, "global", 0.25),
+    (1, 8, 8, "global", 0.5), (1, 4, 4, "global", 0.6), (1, 6, 6, "global", 0.5),
+    (1, 16, 16, "window", 0.7), (1, 20, 28, "global", 0.33), (3, 128, 128, "global", 0.3),
+]
+
+
+@pytest.mark.parametrize("B,H,W,mode,d", CASES)
+def test_pattern_matches_oracle(B, H, W, mode, d):
+    ws = 14 if not (H == 16 and mode == "window") else 8
+    cfg = L.make_cfg(B, H, W, mode, ws, 2, 64, d)
+    p = L.sparsesam_pattern(cfg)
+    geo = O.Geometry(B, H, W, mode, ws)
+    op = O.pattern(geo.unit_tokens, d)
+    assert (p.units, p.unit_tokens) == (geo.units, geo.unit_tokens)
+    assert (p.L, p.b, p.nb, p.W, p.g) == (op.L, op.b, op.nb, op.W, op.g)
+    assert p.rho == op.rho
+    assert p.keep == O.keep_count(d, H * W)
+    row_ptr, col_idx = L.sparsesam_blocklist(cfg)
+    assert row_ptr == list(op.row_ptr) and col_idx == list(op.col_idx)
+
+
+@pytest.mark.parametrize("d", [x / 100 for x in range(1, 101, 3)] + [0.4, 0.3, 0.5, 1.0])
+def test_keep_count_and_band_choice_sweep(d):
+    for h, w in ((4, 4), (14, 14), (16, 16), (32, 32), (64, 64)):
+        T = h * w
+        cfg = L.make_cfg(1, h, w, "global", 14, 1, 64, d)
+        p = L.sparsesam_pattern(cfg)
+        assert p.keep == O.keep_count(d, T)
+        assert p.W == O.pattern(T, d).W
+
+
+# ---- host-side validation (no GPU is touched: every case fails before any CUDA call) ----------
+FAKE = 1 << 20      # an aligned, never-dereferenced address
+
+
+def test_validation_codes():
+    good = L.make_cfg(1, 16, 16, "global", 14, 1, 64, 0.4)
+    lib = L.lib
+    by = ctypes.byref
+    # bad density / shapes
+    for d in (0.0, -0.5, 1.5, float("nan")):
+        assert lib.sparsesam_pattern(by(L.make_cfg(1, 16, 16, density=d)), by(L.SsPattern())) == L.SS_EINVAL
+    assert lib.sparsesam_pattern(by(L.make_cfg(0, 16, 16, density=0.4)), by(L.SsPattern())) == L.SS_EINVAL
+    assert lib.sparsesam_pattern(by(L.make_cfg(1, 5, 5, density=0.4)), by(L.SsPattern())) == L.SS_EUNSUPPORTED
+    assert lib.sparsesam_pattern(by(L.make_cfg(1, 2, 2, density=0.4)), by(L.SsPattern())) == L.SS_EUNSUPPORTED
+    assert lib.sparsesam_pattern(None, by(L.SsPattern())) == L.SS_EINVAL
+    assert lib.sparsesam_pattern(by(L.make_cfg(1, 16, 16, "window", 0, density=0.4)), by(L.SsPattern())) == L.SS_EINVAL
+    # null pointers
+    assert lib.sparsesam_score(by(good), None, FAKE, None) == L.SS_EINVAL
+    assert lib.sparsesam_perm(by(good), FAKE, None, None, None, None) == L.SS_EINVAL
+    assert lib.sparsesam_attn(by(good), None, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == L.SS_EINVAL
+    # unsupported head_dim
+    bad_dh = L.make_cfg(1, 16, 16, "global", 14, 1, 96, 0.4)
+    assert lib.sparsesam_attn(by(bad_dh), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == L.SS_EUNSUPPORTED
+    # misaligned q
+    assert lib.sparsesam_attn(by(good), FAKE + 2, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == L.SS_EINVAL
+    # workspace too small / misaligned / missing
+    need = L.sparsesam_attn_workspace(good)
+    assert need == 3 * 256 * 64 * 2
+    assert lib.sparsesam_attn(by(good), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, None) == L.SS_EWORKSPACE
+    assert lib.sparsesam_attn(by(good), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 16, need, None) == L.SS_EWORKSPACE
+    assert lib.sparsesam_attn(by(good), FAKE, FAKE, FAKE, FAKE, FAKE, None, need, None) == L.SS_EWORKSPACE
+    # rcmlp: C not a multiple of 64, workspace
+    assert lib.sparsesam_rcmlp(by(good), FAKE, 48, 256, FAKE, None, FAKE, None, FAKE, FAKE, 1 << 30, None) == L.SS_EUNSUPPORTED
+    need_m = L.sparsesam_rcmlp_workspace(good, 64, 256)
+    K = O.keep_count(0.4, 256)
+    assert need_m == math.ceil(K * 64 * 2 / 256) * 256 + math.ceil(K * 256 * 2 / 256) * 256
+    assert lib.sparsesam_rcmlp(by(good), FAKE, 64, 256, FAKE, None, FAKE, None, FAKE, FAKE, need_m - 1, None) == L.SS_EWORKSPACE
+    # blocklist capacity
+    rp = (ctypes.c_int32 * 8)()
+    ci = (ctypes.c_int32 * 2)()
+    assert lib.sparsesam_blocklist(by(good), ctypes.cast(rp, ctypes.c_void_p), ctypes.cast(ci, ctypes.c_void_p), 2) == L.SS_EINVAL
+    # trace records outside the range
+    name, ms = ctypes.c_char_p(), ctypes.c_float()
+    assert lib.sparsesam_trace_get(0, by(name), by(ms)) == L.SS_EINVAL
+    assert L.sparsesam_launch_count() == 0
+
+
+def test_binding_raises_on_error():
+    with pytest.raises(L.SparseSAMError) as e:
+        L.sparsesam_pattern(L.make_cfg(1, 5, 5, density=0.4))
+    assert e.value.code == L.SS_EUNSUPPORTED
