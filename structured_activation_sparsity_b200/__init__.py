@@ -4,12 +4,25 @@ The four steps -- Sobel score, stripe-sort permutation, Stripe-Sort block-sparse
 Residual-Consistency MLP -- run in the C-ABI library libsparsesam.so (include/sparsesam.h). This
 package is its thin Python binding (`_lib`), plus the synthetic workload shapes and input
 generators used by the tests and the benchmark.
+
+Names of the binding are resolved on first use, so `python -m structured_activation_sparsity_b200.build`
+works before the library exists; using any of them without the built library raises ImportError.
 """
-from ._lib import (  # noqa: F401
-    SS_ECUDA, SS_EINVAL, SS_EUNSUPPORTED, SS_EWORKSPACE, SS_ETIMEOUT, SS_GLOBAL, SS_OK, SS_WINDOW,
-    SparseSAMError, SsCfg, SsPattern, cfg_for, make_cfg, sparsesam_attn, sparsesam_attn_workspace,
-    sparsesam_blocklist, sparsesam_device_status, sparsesam_launch_count, sparsesam_pattern,
-    sparsesam_perm, sparsesam_rcmlp, sparsesam_rcmlp_workspace, sparsesam_score,
-    sparsesam_trace_start, sparsesam_trace_stop, strerror,
-)
-from .hotpath import HotPath  # noqa: F401
+import importlib
+
+_LIB_NAMES = {
+    "SS_ECUDA", "SS_EINVAL", "SS_EUNSUPPORTED", "SS_EWORKSPACE", "SS_ETIMEOUT", "SS_GLOBAL",
+    "SS_OK", "SS_WINDOW", "SparseSAMError", "SsCfg", "SsPattern", "cfg_for", "make_cfg",
+    "sparsesam_attn", "sparsesam_attn_workspace", "sparsesam_blocklist",
+    "sparsesam_device_status", "sparsesam_launch_count", "sparsesam_pattern", "sparsesam_perm",
+    "sparsesam_rcmlp", "sparsesam_rcmlp_workspace", "sparsesam_score",
+    "sparsesam_trace_start", "sparsesam_trace_stop", "strerror",
+}
+
+
+def __getattr__(name):
+    if name in _LIB_NAMES:
+        return getattr(importlib.import_module("._lib", __name__), name)
+    if name == "HotPath":
+        return importlib.import_module(".hotpath", __name__).HotPath
+    raise AttributeError(name)
