@@ -145,6 +145,25 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden,
                     const uint16_t* w1, const uint16_t* b1, const uint16_t* w2, const uint16_t* b2,
                     const int32_t* keep, void* ws, size_t ws_bytes, void* stream);
 
+/* S4 without a caller-provided workspace. The SparseSAM pages have no counterpart to this call;
+ * it exists for callers that cannot allocate device memory where they run the block: code inside
+ * another runtime's stream capture (cudaMalloc is not allowed there), hosts whose allocator owns
+ * all device memory and gives plug-ins none, and latency-bound loops that must not pay cudaMalloc's
+ * implicit device-wide synchronisation. Same arguments, semantics and results as sparsesam_rcmlp,
+ * minus ws/ws_bytes: the scratch lives in a 16 MiB array inside this library (a file-scope
+ * __device__ array that every GPU loading the library holds until the process exits).
+ *   - Returns SS_EWORKSPACE, before any CUDA call, when sparsesam_rcmlp_workspace(cfg, C, hidden)
+ *     exceeds 16 MiB (e.g. the SAM ViT-B global block, 12.6 MB, fits; batch 4 does not).
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls on a device share the one array and leave their contents in it; nothing needs
+ *     clearing because each call writes every scratch byte before reading it. Calls whose GPU
+ *     execution overlaps (different streams, no ordering between them) race on the array. */
+int sparsesam_rcmlp_noalloc(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden,
+                            const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
+                            const uint16_t* b2, const int32_t* keep, void* stream);
+
 /* Reads (and clears) the device status word that bounded device waits write. Synchronises the
  * given stream. *status receives SS_OK or SS_ETIMEOUT. Returns SS_OK or SS_ECUDA. */
 int sparsesam_device_status(int32_t* status, void* stream);

@@ -57,6 +57,7 @@ def _load():
         "sparsesam_attn": (ctypes.c_int, [cfgp, P, P, P, P, P, P, SZ, VP]),
         "sparsesam_rcmlp_workspace": (SZ, [cfgp, I32, I32]),
         "sparsesam_rcmlp": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, P, SZ, VP]),
+        "sparsesam_rcmlp_noalloc": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, VP]),
         "sparsesam_device_status": (ctypes.c_int, [ctypes.POINTER(I32), VP]),
         "sparsesam_launch_count": (ctypes.c_uint64, []),
         "sparsesam_trace_start": (ctypes.c_int, [I32]),
@@ -160,6 +161,15 @@ def sparsesam_rcmlp(cfg, x, C, hidden, w1, b1, w2, b2, keep, ws, ws_bytes, strea
                   lib.sparsesam_rcmlp(ctypes.byref(cfg), _ptr(x), int(C), int(hidden), _ptr(w1),
                                       _ptr(b1), _ptr(w2), _ptr(b2), _ptr(keep), _ptr(ws),
                                       int(ws_bytes), _stream(stream)))
+
+
+def sparsesam_rcmlp_noalloc(cfg, x, C, hidden, w1, b1, w2, b2, keep, stream=None):
+    """sparsesam_rcmlp with its scratch in the library's fixed 16 MiB device array (no workspace
+    argument, nothing allocated). For callers that cannot allocate device memory."""
+    return _check("sparsesam_rcmlp_noalloc",
+                  lib.sparsesam_rcmlp_noalloc(ctypes.byref(cfg), _ptr(x), int(C), int(hidden),
+                                              _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(keep),
+                                              _stream(stream)))
 
 
 def sparsesam_device_status(stream=None) -> int:
