@@ -375,6 +375,33 @@ def run_ours(args, wl, rank, world, local_rank, dist):
     print(json.dumps(line), flush=True)
 
 
+def run_kernel_loop(args, wl, local_rank):
+    """One library call of the step in a loop (for ncu captures and isolated timings)."""
+    import torch
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    hp = make_sets(wl, 1, dev)[0][0]
+    with torch.cuda.stream(stream):
+        hp.score_step(stream)
+        hp.perm_step(stream)
+    fn = {"score": hp.score_step, "perm": hp.perm_step, "attn": hp.attn_step,
+          "rcmlp": hp.mlp_step}[args.kernel_loop]
+    for _ in range(args.warmup):
+        fn(stream)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        fn(stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel_loop": args.kernel_loop, "workload": wl.name,
+                      "avg_us_per_call": 1e3 * ev0.elapsed_time(ev1) / args.steps,
+                      "note": "inputs stay resident in L2 across calls"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -382,6 +409,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="vitb_global", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--kernel-loop", default=None, choices=["score", "perm", "attn", "rcmlp"],
+                    help="run only this library call in a loop (profiling aid; no bench line)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = workloads.get(args.workload)
@@ -391,6 +420,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, wl, rank)
+        return
+    if args.kernel_loop:
+        run_kernel_loop(args, wl, local_rank)
         return
     dist = None
     if world > 1:

@@ -67,10 +67,11 @@ cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16
 // ---------------------------------------------------------------------------------------------
 // Attention kernel
 // ---------------------------------------------------------------------------------------------
-constexpr int kBM = 128;       // query rows per CTA
-constexpr int kBN = 128;       // keys per tile
-constexpr int kStages = 2;     // K/V ring depth
-constexpr int kAttnThreads = 192;
+constexpr int kBM = 128;          // query rows per CTA
+constexpr int kBN = 128;          // keys per tile
+constexpr int kStages = 3;        // K/V ring depth
+constexpr int kAttnThreads = 320; // 10 warps
+constexpr float kLazyRescale = 8.f;   // log2 headroom before O and l are rescaled
 
 template <int DH>
 struct AttnSmem {
@@ -82,9 +83,10 @@ struct AttnSmem {
   static constexpr int kK = ((kQTail + kTailBytes + 1023) / 1024) * 1024;
   static constexpr int kStageBytes = ((kMain + kTailBytes + 1023) / 1024) * 1024;
   static constexpr int kV = kK + kStages * kStageBytes;
-  static constexpr int kP = kV + kStages * kStageBytes;
+  static constexpr int kP = kV + kStages * kStageBytes;  // two P buffers, one per softmax group
   static constexpr int kPBytes = kBM * kBN * 2;        // two 128B-swizzled atoms of 64 keys
-  static constexpr int kBar = kP + kPBytes;
+  static constexpr int kML = kP + 2 * kPBytes;         // float m[2][128], l[2][128]
+  static constexpr int kBar = kML + 4 * kBM * 4;
   static constexpr int kBytes = kBar + 256;
   static constexpr int kAlloc = kBytes + 1024;         // slack to align the base to 1024
 };
@@ -125,12 +127,16 @@ __device__ __forceinline__ bool tile_full(int q0, int q_last, int c0, const Attn
   return true;
 }
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
+// One CTA = one (unit, head, 128-row query tile). The key tiles are split between two softmax
+// warpgroups (tile n goes to group n % 2), so the MMA warp alternates between them: while one
+// group turns its S tile into probabilities, the tensor core runs the other group's P*V and the
+// next Q*K^T. Each group keeps its own running max m, sum l and accumulator O (in TMEM); at the
+// end the two partial results of every row are merged.
+//   warp 0      TMA producer (Q once, then K/V tiles into a 3-stage ring)
+//   warp 1      TMEM allocator and tcgen05.mma issuer
+//   warps 2-5   softmax group 0 (one thread per query row = TMEM lane)
+//   warps 6-9   softmax group 1
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256, 256+dh), O1 [384, 384+dh).
 template <int DH>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -142,16 +148,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
+  float* s_m = reinterpret_cast<float*>(smem + S::kML);   // [2][128]
+  float* s_l = s_m + 2 * kBM;                              // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;                 // [kStages]
   uint64_t* v_full = k_full + kStages;         // [kStages]
   uint64_t* kv_empty = v_full + kStages;       // [kStages]
-  uint64_t* s_full = kv_empty + kStages;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* o_full = p_full + 1;
-  uint64_t* o_empty = o_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 1);
+  uint64_t* s_full = kv_empty + kStages;       // [2]
+  uint64_t* p_full = s_full + 2;               // [2]
+  uint64_t* o_done = p_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -168,20 +175,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(v_full + i, 1);
       mbar_init(kv_empty + i, 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(o_full, 1);
-    mbar_init(o_empty, 128);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(s_full + w, 1);
+      mbar_init(p_full + w, 128);
+    }
+    mbar_init(o_done, 1);
     *abort = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 256);
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_s = tmem;          // columns [0, 128)
-  const uint32_t tmem_o = tmem + 128;    // columns [128, 128 + DH)
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -214,70 +220,85 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, 64, false, true);
       constexpr uint32_t idesc_pv_tail = idesc_bf16_f32(kBM, 16, false, true);
       const uint32_t q_addr = smem_u32(smem + S::kQ);
-      const uint32_t p_addr = smem_u32(smem + S::kP);
       bool ok = mbar_wait(q_full, 0, abort, status);
-      tc_fence_after();
-      for (int n = 0; ok && n < ntiles; ++n) {
+      // S_w = Q K_n^T for tile n (w = n % 2).
+      auto issue_qk = [&](int n) -> bool {
         const int st = n % kStages;
-        const uint32_t ph = (n / kStages) & 1;
-        const uint32_t k_addr = smem_u32(smem + S::kK + st * S::kStageBytes);
-        const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kStageBytes);
-        if (!(ok = mbar_wait(k_full + st, ph, abort, status))) break;
+        if (!mbar_wait(k_full + st, (n / kStages) & 1, abort, status)) return false;
         tc_fence_after();
-        // S = Q K^T over head_dim: 16-wide K steps inside the 128B atom, then the 16-col tail.
+        const uint32_t k_addr = smem_u32(smem + S::kK + st * S::kStageBytes);
+        const uint32_t d = tmem + (n & 1) * kBN;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_bf16_ss(tmem_s, smem_desc(q_addr + kk * 32, 16, 1024, kSwizzle128B),
+          umma_bf16_ss(d, smem_desc(q_addr + kk * 32, 16, 1024, kSwizzle128B),
                        smem_desc(k_addr + kk * 32, 16, 1024, kSwizzle128B), idesc_qk, kk > 0);
         if (kHasTail)
-          umma_bf16_ss(tmem_s, smem_desc(q_addr + S::kMain, 16, 256, kSwizzle32B),
+          umma_bf16_ss(d, smem_desc(q_addr + S::kMain, 16, 256, kSwizzle32B),
                        smem_desc(k_addr + S::kMain, 16, 256, kSwizzle32B), idesc_qk, 1);
-        umma_commit(s_full);
-        if (!(ok = mbar_wait(p_full, n & 1, abort, status))) break;
-        if (!(ok = mbar_wait(v_full + st, ph, abort, status))) break;
-        if (n > 0 && !(ok = mbar_wait(o_empty, (n - 1) & 1, abort, status))) break;
+        umma_commit(s_full + (n & 1));
+        return true;
+      };
+      // O_w (+)= P_w V_n once group w has written P_w for tile n.
+      auto issue_pv = [&](int n) -> bool {
+        const int st = n % kStages, w = n & 1;
+        if (!mbar_wait(p_full + w, (n >> 1) & 1, abort, status)) return false;
+        if (!mbar_wait(v_full + st, (n / kStages) & 1, abort, status)) return false;
         tc_fence_after();
-        // O_tile = P V: A = P (K-major, two 64-key atoms), B = V (MN-major over head_dim).
+        const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kStageBytes);
+        const uint32_t p_addr = smem_u32(smem + S::kP + w * S::kPBytes);
+        const uint32_t d = tmem + 256 + w * 128;
+        const uint32_t acc = n >= 2;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           const uint64_t a = smem_desc(p_addr + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024,
                                        kSwizzle128B);
-          umma_bf16_ss(tmem_o, a, smem_desc(v_addr + kk * 2048, kBN * 128, 1024, kSwizzle128B),
-                       idesc_pv, kk > 0);
+          umma_bf16_ss(d, a, smem_desc(v_addr + kk * 2048, kBN * 128, 1024, kSwizzle128B),
+                       idesc_pv, acc | (kk > 0));
           if (kHasTail)
-            umma_bf16_ss(tmem_o + 64, a,
+            umma_bf16_ss(d + 64, a,
                          smem_desc(v_addr + S::kMain + kk * 512, kBN * 32, 256, kSwizzle32B),
-                         idesc_pv_tail, kk > 0);
+                         idesc_pv_tail, acc | (kk > 0));
         }
-        umma_commit(o_full);
         umma_commit(kv_empty + st);
+        return true;
+      };
+      if (ok) tc_fence_after();
+      if (ok && ntiles > 0) ok = issue_qk(0);
+      if (ok && ntiles > 1) ok = issue_qk(1);
+      for (int n = 0; ok && n < ntiles; ++n) {
+        ok = issue_pv(n);
+        if (ok && n + 2 < ntiles) ok = issue_qk(n + 2);
       }
+      if (ok) umma_commit(o_done);
     }
   } else {
-    // ------------------------------ softmax warps -----------------------------
-    const int row = 32 * (warp & 3) + lane;      // TMEM lane == query row within the tile
+    // ------------------------------ softmax groups ----------------------------
+    const int grp = (warp - 2) >> 2;                    // 0 or 1
+    const int row = 32 * (warp & 3) + lane;             // TMEM lane == query row
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
+    const uint32_t t_s = tmem + grp * kBN + lane_off;
+    const uint32_t t_o = tmem + 256 + grp * 128 + lane_off;
     const int qrow = q0 + row;
     const int b4 = P.b * kStripes;
     const int a_q = min(qrow, P.N - 1) / b4;
     const int s_q = band_start(a_q, P.W, P.nb);
     const int band_lo = s_q * b4, band_hi = (s_q + P.W) * b4, glob_hi = P.g * b4;
-    const uint32_t p_row_addr = smem_u32(smem + S::kP);
-    float o[DH];
-#pragma unroll
-    for (int d = 0; d < DH; ++d) o[d] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f;
+    const uint32_t p_base = smem_u32(smem + S::kP + grp * S::kPBytes);
+    const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
+    float m_ref = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int n = 0; n < ntiles; ++n) {
-      if (!(ok = mbar_wait(s_full, n & 1, abort, status))) break;
+    int j = 0;
+    for (int n = grp; n < ntiles; n += 2, ++j) {
+      // Warp-collective wait: either every lane goes on to the .sync.aligned TMEM ops or none.
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full + grp, j & 1, abort, status));
+      if (!ok) break;
       tc_fence_after();
-      float s[kBN];
+      float sv[kBN];
+      {
+        uint32_t r[128];
+        tmem_ld128(t_s, r);
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_s + lane_off + c * 32, r);
-        #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+        for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(r[i]);
       }
       const int c0 = tiles.tile(n) * kBN;
       if (!tile_full(q0, q_last, c0, P)) {
@@ -285,16 +306,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int i = 0; i < kBN; ++i) {
           const int c = c0 + i;
           const bool kept = c < P.N && (c < glob_hi || (c >= band_lo && c < band_hi));
-          if (!kept) s[i] = -INFINITY;
+          if (!kept) sv[i] = -INFINITY;
         }
       }
-      float mx = -INFINITY;
+      // Row max: eight independent chains of 3-input max over elements k, k+8, k+16, ...
+      float mx[8];
 #pragma unroll
-      for (int i = 0; i < kBN; ++i) mx = fmaxf(mx, s[i]);
-      const float m_new = fmaxf(m_run, mx * P.scale_log2);
-      const float ref = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2(m_run - ref);
-      float rowsum = 0.f;
+      for (int k = 0; k < 8; ++k) mx[k] = fmax3(sv[k], sv[k + 8], sv[k + 16]);
+#pragma unroll
+      for (int t = 3; t + 1 < 16; t += 2)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv[k + 8 * t], sv[k + 8 * t + 8]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], sv[k + 8 * 15]);
+      const float x_max =
+          fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])), fmaxf(mx[6], mx[7])) *
+          P.scale_log2;
+      // Lazy rescale: the reference max moves only when the row max passes it by 2^8, so O in
+      // TMEM is rescaled on few tiles. The decision is warp-wide (TMEM ops are warp-collective);
+      // the rescale itself runs after P is written, when the S registers are free.
+      const bool grow = x_max > m_ref + kLazyRescale;
+      const bool rescale = __any_sync(0xffffffffu, grow);
+      float alpha = 1.f;
+      if (rescale) {
+        const float m_new = grow ? x_max : m_ref;
+        alpha = (m_ref == -INFINITY) ? 0.f : ex2_mufu(m_ref - m_new);
+        l_run *= alpha;
+        m_ref = m_new;
+      }
+      const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
+      const uint64_t nref2 = f2_pack(-ref, -ref);
+      uint64_t sum2a = 0, sum2b = 0;   // two packed partial sums (bit pattern 0 = +0.0f pair)
 #pragma unroll
       for (int at = 0; at < 2; ++at) {
 #pragma unroll
@@ -303,55 +345,78 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int i = at * 64 + cc * 8 + 2 * e;
-            const float p0 = ex2(fmaf(s[i], P.scale_log2, -ref));
-            const float p1 = ex2(fmaf(s[i + 1], P.scale_log2, -ref));
-            rowsum += p0 + p1;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), scale2, nref2), x0, x1);
+            const float p0 = ex2_mufu(x0), p1 = ex2_mufu(x1);
+            if (e & 1)
+              sum2b = f2_add(sum2b, f2_pack(p0, p1));
+            else
+              sum2a = f2_add(sum2a, f2_pack(p0, p1));
             w[e] = pack_bf16(p0, p1);
           }
-          st_shared_v4(p_row_addr + at * (kBM * 128) + sw128_offset(row, cc), w[0], w[1], w[2],
-                       w[3]);
+          st_shared_v4(p_base + at * (kBM * 128) + sw128_offset(row, cc), w[0], w[1], w[2], w[3]);
+        }
+      }
+      float sa0, sa1;
+      f2_unpack(f2_add(sum2a, sum2b), sa0, sa1);
+      l_run += sa0 + sa1;
+      if (rescale && j > 0) {
+        // O_w holds the group's earlier tiles: their P*V completed before this S was committed,
+        // and this tile's P*V is issued only after the arrive below.
+#pragma unroll 1
+        for (int c = 0; c < (DH + 31) / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(t_o + c * 32, o);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
-      l_run = l_run * alpha + rowsum;
-      m_run = m_new;
-#pragma unroll
-      for (int d = 0; d < DH; ++d) o[d] *= alpha;
-      if (!(ok = mbar_wait(o_full, n & 1, abort, status))) break;
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_o + lane_off + c * 32, r);
-        #pragma unroll
-        for (int i = 0; i < 32; ++i) o[c * 32 + i] += __uint_as_float(r[i]);
-      }
-      if (kHasTail) {
-        uint32_t r[16];
-        tmem_ld16(tmem_o + lane_off + 64, r);
-        #pragma unroll
-        for (int i = 0; i < 16; ++i) o[64 + (i & 15)] += __uint_as_float(r[i]);
-      }
-      tc_fence_before();
-      mbar_arrive(o_empty);
+      mbar_arrive(p_full + grp);
     }
-    // Epilogue: normalise and scatter the row back to its token: out[u, perm[p], h, :].
-    if (ok && qrow < P.N) {
-      const int u = uh / P.heads, h = uh - (uh / P.heads) * P.heads;
-      const int p = blockmajor_to_canonical(qrow, P.b, P.L);
-      const int t = min(max(__ldg(P.perm + (size_t)u * P.N + p), 0), P.N - 1);
-      const float inv_l = 1.f / l_run;
-      uint4* dst = reinterpret_cast<uint4*>(P.out + ((size_t)(u * P.N + t) * P.heads + h) * DH);
+    // ---- merge the two groups' partial rows and scatter them to out[u, perm[p], h, :] ----
+    s_m[grp * kBM + row] = m_ref;
+    s_l[grp * kBM + row] = l_run;
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, 0, abort, status));
+    tc_fence_after();
+    named_barrier(1, 256);
+    if (ok) {
+      const float m0 = s_m[row], m1 = s_m[kBM + row];
+      const float l0 = s_l[row], l1 = s_l[kBM + row];
+      const float mm = fmaxf(m0, m1);
+      const float a0 = (m0 == -INFINITY) ? 0.f : ex2_mufu(m0 - mm);
+      const float a1 = (m1 == -INFINITY) ? 0.f : ex2_mufu(m1 - mm);
+      const float L = l0 * a0 + l1 * a1;
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const float f0 = a0 * inv, f1 = a1 * inv;
+      const bool has0 = ntiles > 0, has1 = ntiles > 1;   // a group with no tile has no O
+      const bool store = qrow < P.N;
+      uint16_t* dst = nullptr;
+      if (store) {
+        const int u = uh / P.heads, h = uh - (uh / P.heads) * P.heads;
+        const int p = blockmajor_to_canonical(qrow, P.b, P.L);
+        const int t = min(max(__ldg(P.perm + (size_t)u * P.N + p), 0), P.N - 1);
+        dst = P.out + ((size_t)(u * P.N + t) * P.heads + h) * DH;
+      }
+      const uint32_t o0 = tmem + 256 + lane_off, o1 = tmem + 384 + lane_off;
+      constexpr int kChunks = DH / 8;            // 8 or 10 chunks of 8 columns
+      for (int c = grp; c < kChunks; c += 2) {    // the two groups split the columns
+        uint32_t x0[8], x1[8];
+        tmem_ld8(o0 + c * 8, x0);                 // every lane loads (warp-collective) ...
+        tmem_ld8(o1 + c * 8, x1);
+        float v[8];
 #pragma unroll
-      for (int c = 0; c < DH / 8; ++c) {
-        uint4 w;
-        w.x = pack_bf16(o[c * 8 + 0] * inv_l, o[c * 8 + 1] * inv_l);
-        w.y = pack_bf16(o[c * 8 + 2] * inv_l, o[c * 8 + 3] * inv_l);
-        w.z = pack_bf16(o[c * 8 + 4] * inv_l, o[c * 8 + 5] * inv_l);
-        w.w = pack_bf16(o[c * 8 + 6] * inv_l, o[c * 8 + 7] * inv_l);
-        dst[c] = w;
+        for (int i = 0; i < 8; ++i)
+          v[i] = (has0 ? __uint_as_float(x0[i]) * f0 : 0.f) +
+                 (has1 ? __uint_as_float(x1[i]) * f1 : 0.f);
+        uint4 wv;
+        wv.x = pack_bf16(v[0], v[1]);
+        wv.y = pack_bf16(v[2], v[3]);
+        wv.z = pack_bf16(v[4], v[5]);
+        wv.w = pack_bf16(v[6], v[7]);
+        if (store) reinterpret_cast<uint4*>(dst)[c] = wv;   // ... only rows < N store
       }
     }
   }
@@ -359,7 +424,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
