@@ -136,7 +136,8 @@ size_t sparsesam_rcmlp_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden);
  * for each image b and kept token t = keep[b][r], r < K:
  *   x[b,t,:] = bf16( x[b,t,:] + (w2 . GELU(w1 . x[b,t,:] + b1) + b2) ),  GELU(z) = z/2 (1+erf(z/sqrt2))
  * every other row is left bit-for-bit untouched. w1 bf16 [hidden, C], w2 bf16 [C, hidden]
- * (row-major, PyTorch nn.Linear weight layout); b1 [hidden], b2 [C] bf16 or NULL (zero). keep
+ * (row-major, PyTorch nn.Linear weight layout); b1 [hidden], b2 [C] bf16 or NULL (zero); x, w1,
+ * w2, b1 and b2 16-byte aligned. keep
  * (device) int32 [batch, K] with distinct rows per image (as sparsesam_perm writes it).
  * C and hidden must be multiples of 64. bf16 operands, fp32 accumulation; the hidden activation
  * is rounded to bf16 between the two products. ws (device, 256-byte aligned) >=
@@ -150,10 +151,10 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden,
  * another runtime's stream capture (cudaMalloc is not allowed there), hosts whose allocator owns
  * all device memory and gives plug-ins none, and latency-bound loops that must not pay cudaMalloc's
  * implicit device-wide synchronisation. Same arguments, semantics and results as sparsesam_rcmlp,
- * minus ws/ws_bytes: the scratch lives in a 16 MiB array inside this library (a file-scope
+ * minus ws/ws_bytes: the scratch lives in a 32 MiB array inside this library (a file-scope
  * __device__ array that every GPU loading the library holds until the process exits).
  *   - Returns SS_EWORKSPACE, before any CUDA call, when sparsesam_rcmlp_workspace(cfg, C, hidden)
- *     exceeds 16 MiB (e.g. the SAM ViT-B global block, 12.6 MB, fits; batch 4 does not).
+ *     exceeds 32 MiB (e.g. the SAM ViT-B global block, 28 MB, fits; batch 4 does not).
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
  *     that device current); make that first call before any stream capture.

@@ -164,7 +164,7 @@ def sparsesam_rcmlp(cfg, x, C, hidden, w1, b1, w2, b2, keep, ws, ws_bytes, strea
 
 
 def sparsesam_rcmlp_noalloc(cfg, x, C, hidden, w1, b1, w2, b2, keep, stream=None):
-    """sparsesam_rcmlp with its scratch in the library's fixed 16 MiB device array (no workspace
+    """sparsesam_rcmlp with its scratch in the library's fixed 32 MiB device array (no workspace
     argument, nothing allocated). For callers that cannot allocate device memory."""
     return _check("sparsesam_rcmlp_noalloc",
                   lib.sparsesam_rcmlp_noalloc(ctypes.byref(cfg), _ptr(x), int(C), int(hidden),

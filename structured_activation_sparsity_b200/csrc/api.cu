@@ -161,12 +161,53 @@ size_t attn_ws_bytes(const Geo& g, int heads, int dh) {
   return 3 * align256((size_t)g.U * heads * g.N * dh * 2);
 }
 
-size_t rcmlp_ws_bytes(const Geo& g, int K, int C, int hidden) {
-  const size_t M = (size_t)g.B * K;
-  return align256(M * C * 2) + align256(M * hidden * 2);
+// The GEMM work split is planned for the B200's 148 SMs, so the workspace size does not depend on
+// the device a call runs on; the launch uses min(units, the device's SMs) persistent CTAs.
+constexpr int kPlanSMs = 148;
+
+struct MlpPlan {
+  GemmPlan fc1, fc2;
+  size_t xk, h, partial, counters, total;   // byte offsets/sizes inside the workspace
+};
+
+MlpPlan mlp_plan(const Geo& g, int K, int C, int hidden) {
+  MlpPlan p;
+  const int M = g.B * K;
+  p.fc1 = gemm_plan(M, hidden, C, kPlanSMs);
+  p.fc2 = gemm_plan(M, C, hidden, kPlanSMs);
+  const size_t xk_bytes = align256((size_t)M * C * 2);
+  const size_t h_bytes = align256((size_t)M * hidden * 2);
+  const size_t part = align256(gemm_partial_bytes(p.fc1) > gemm_partial_bytes(p.fc2)
+                                   ? gemm_partial_bytes(p.fc1)
+                                   : gemm_partial_bytes(p.fc2));
+  const int tiles = (p.fc1.m_tiles * p.fc1.n_tiles > p.fc2.m_tiles * p.fc2.n_tiles)
+                        ? p.fc1.m_tiles * p.fc1.n_tiles
+                        : p.fc2.m_tiles * p.fc2.n_tiles;
+  const size_t cnt = part ? align256((size_t)tiles * 4) : 0;
+  p.xk = 0;
+  p.h = xk_bytes;
+  p.partial = xk_bytes + h_bytes;
+  p.counters = p.partial + part;
+  p.total = p.counters + cnt;
+  return p;
 }
 
-int gemm_bn(int n) { return n % 256 == 0 && n >= 1024 ? 256 : (n % 128 == 0 ? 128 : 64); }
+size_t rcmlp_ws_bytes(const Geo& g, int K, int C, int hidden) {
+  return mlp_plan(g, K, C, hidden).total;
+}
+
+int sm_count() {
+  static int cached[128] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return kPlanSMs;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      n = kPlanSMs;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
 
 }  // namespace
 }  // namespace ss
@@ -322,7 +363,9 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, c
   if (rc) return rc;
   if (!x || !w1 || !w2 || !keep || C < 1 || hidden < 1) return SS_EINVAL;
   if (C % 64 != 0 || hidden % 64 != 0) return SS_EUNSUPPORTED;
-  if (!aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16)) return SS_EINVAL;
+  if (!aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(b1, 16) ||
+      !aligned(b2, 16))
+    return SS_EINVAL;
   const int K = keep_count(cfg->density, g.T);
   const int64_t M = (int64_t)g.B * K;
   if (M * (hidden > C ? hidden : C) >= ((int64_t)1 << 31) || (M + 127) / 128 > 65535)
@@ -331,24 +374,31 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, c
   if (!ws || !aligned(ws, 256) || ws_bytes < need) return SS_EWORKSPACE;
   int* status = status_word();
   if (!status) return SS_ECUDA;
-  uint16_t* xk = static_cast<uint16_t*>(ws);
-  uint16_t* hbuf =
-      reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + align256((size_t)M * C * 2));
+  const MlpPlan plan = mlp_plan(g, K, C, hidden);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint16_t* xk = reinterpret_cast<uint16_t*>(wsb + plan.xk);
+  uint16_t* hbuf = reinterpret_cast<uint16_t*>(wsb + plan.h);
+  float* partial = reinterpret_cast<float*>(wsb + plan.partial);
+  int* counters = reinterpret_cast<int*>(wsb + plan.counters);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int sms = sm_count();
 
   rc = cuda_err(traced("gather_rows", st, [&] {
     return launch_gather_rows(x, keep, xk, g.B, g.T, K, C, st);
   }));
   if (rc) return rc;
 
-  const int bn1 = gemm_bn(hidden), bn2 = gemm_bn(C);
   CUtensorMap ta1, tb1, ta2, tb2;
   if (!encode_bf16(&ta1, 2, xk, C, M, 1, (uint64_t)C * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_bf16(&tb1, 2, w1, C, hidden, 1, (uint64_t)C * 2, 64, bn1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16(&tb1, 2, w1, C, hidden, 1, (uint64_t)C * 2, 64, plan.fc1.bn,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_bf16(&ta2, 2, hbuf, hidden, M, 1, (uint64_t)hidden * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_bf16(&tb2, 2, w2, hidden, C, 1, (uint64_t)hidden * 2, 64, bn2,
+      !encode_bf16(&tb2, 2, w2, hidden, C, 1, (uint64_t)hidden * 2, 64, plan.fc2.bn,
                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return SS_ECUDA;
+  if (plan.counters != plan.total &&
+      cudaMemsetAsync(counters, 0, plan.total - plan.counters, st) != cudaSuccess)
     return SS_ECUDA;
 
   GemmEpilogue e1 = {};
@@ -356,7 +406,8 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, c
   e1.bias = b1;
   e1.out = hbuf;
   rc = cuda_err(traced("rcmlp_fc1", st, [&] {
-    return launch_gemm(&ta1, &tb1, (int)M, hidden, C, bn1, e1, status, st);
+    return launch_gemm(&ta1, &tb1, plan.fc1, (int)M, hidden, C, e1, partial, counters, sms, status,
+                       st);
   }));
   if (rc) return rc;
   GemmEpilogue e2 = {};
@@ -367,7 +418,8 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, c
   e2.K_per_image = K;
   e2.T = g.T;
   return cuda_err(traced("rcmlp_fc2", st, [&] {
-    return launch_gemm(&ta2, &tb2, (int)M, C, hidden, bn2, e2, status, st);
+    return launch_gemm(&ta2, &tb2, plan.fc2, (int)M, C, hidden, e2, partial, counters, sms, status,
+                       st);
   }));
 }
 

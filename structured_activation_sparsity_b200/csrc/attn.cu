@@ -26,75 +26,90 @@ namespace ss {
 // ---------------------------------------------------------------------------------------------
 // Gather: Xp[(u*heads + h), q, :] = X[u, perm[u, p(q)], h, :]
 // ---------------------------------------------------------------------------------------------
+// One CTA per (unit, 8 consecutive block-major positions), a warp per position: the warp resolves
+// its source token, then copies the token's heads*dh row (contiguous in the source) as 16-byte
+// chunks into the per-head rows of the gathered buffers. CPR = 16-byte chunks per head.
+template <int CPR>
 __global__ void __launch_bounds__(256) k_gather_qkv(const uint16_t* __restrict__ q,
                                                     const uint16_t* __restrict__ k,
                                                     const uint16_t* __restrict__ v,
                                                     const int32_t* __restrict__ perm,
                                                     uint16_t* __restrict__ qp,
                                                     uint16_t* __restrict__ kp,
-                                                    uint16_t* __restrict__ vp, int U, int N,
-                                                    int heads, int dh, int b, int L) {
-  const uint16_t* src = blockIdx.y == 0 ? q : (blockIdx.y == 1 ? k : v);
-  uint16_t* dst = blockIdx.y == 0 ? qp : (blockIdx.y == 1 ? kp : vp);
-  const int cpr = dh / 8;            // 16-byte chunks per head row
-  const int per_tok = heads * cpr;   // 16-byte chunks per token (all heads)
-  const int total = U * N * per_tok;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
-    const int c = i % per_tok;
-    const int uq = i / per_tok;
-    const int qpos = uq % N;
-    const int u = uq / N;
-    const int h = c / cpr, cc = c - (c / cpr) * cpr;
-    const int p = blockmajor_to_canonical(qpos, b, L);
-    const int t = min(max(__ldg(perm + (size_t)u * N + p), 0), N - 1);   // never leave the unit
-    const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)(u * N + t) * heads * dh) + c;
-    uint4* d = reinterpret_cast<uint4*>(dst + ((size_t)(u * heads + h) * N + qpos) * dh) + cc;
-    *d = __ldg(s);
+                                                    uint16_t* __restrict__ vp, int N, int heads,
+                                                    int b, int L) {
+  const int u = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qpos = blockIdx.x * 8 + warp;
+  if (qpos >= N) return;
+  const int p = blockmajor_to_canonical(qpos, b, L);
+  const int tok = min(max(__ldg(perm + (size_t)u * N + p), 0), N - 1);   // stay in the unit
+  const int per_tok = heads * CPR;
+  const size_t plane = (size_t)N * CPR;       // 16-byte chunks per (unit, head) matrix
+  const size_t src_row = ((size_t)u * N + tok) * per_tok;
+  const size_t dst_row = (size_t)u * heads * plane + (size_t)qpos * CPR;
+#pragma unroll
+  for (int t = 0; t < 3; ++t) {
+    const uint4* src = reinterpret_cast<const uint4*>(t == 0 ? q : (t == 1 ? k : v)) + src_row;
+    uint4* dst = reinterpret_cast<uint4*>(t == 0 ? qp : (t == 1 ? kp : vp)) + dst_row;
+    for (int c = lane; c < per_tok; c += 32) {
+      const int h = c / CPR, cc = c - h * CPR;     // CPR is a compile-time constant
+      dst[h * plane + cc] = __ldg(src + c);
+    }
   }
 }
 
 cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                               const int32_t* perm, uint16_t* qp, uint16_t* kp, uint16_t* vp,
                               int U, int N, int heads, int dh, int b, cudaStream_t st) {
-  const int total = U * N * heads * (dh / 8);
-  int blocks = (total + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  k_gather_qkv<<<dim3(blocks, 3), 256, 0, st>>>(q, k, v, perm, qp, kp, vp, U, N, heads, dh, b,
-                                                N / kStripes);
+  dim3 grid((N + 7) / 8, U);
+  if (dh == 64)
+    k_gather_qkv<8><<<grid, 256, 0, st>>>(q, k, v, perm, qp, kp, vp, N, heads, b, N / kStripes);
+  else if (dh == 80)
+    k_gather_qkv<10><<<grid, 256, 0, st>>>(q, k, v, perm, qp, kp, vp, N, heads, b, N / kStripes);
+  else
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------------------------
 // Attention kernel
 // ---------------------------------------------------------------------------------------------
-constexpr int kBM = 128;          // query rows per CTA
-constexpr int kBN = 128;          // keys per tile
-constexpr int kStages = 3;        // K/V ring depth
-constexpr int kAttnThreads = 320; // 10 warps
+constexpr int kBM = 128;              // query rows per CTA
+constexpr int kBN = 128;              // keys per tile
+constexpr int kAttnThreads = 384;     // 12 warps = 3 warpgroups
 constexpr float kLazyRescale = 8.f;   // log2 headroom before O and l are rescaled
+// Register split (launch: 384 threads x 168): producer warpgroup 56, softmax warpgroups 224.
+constexpr uint32_t kRegsProducer = 56, kRegsSoftmax = 224;
+static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= 384 * 168, "register split too large");
 
 template <int DH>
 struct AttnSmem {
   static constexpr int kTail = DH - 64;                // 0 or 16 columns past the 128B atom
   static constexpr int kMain = kBM * 128;              // 128 rows x 128 B
   static constexpr int kTailBytes = kTail ? kBM * kTail * 2 : 0;
+  static constexpr int kTileBytes = ((kMain + kTailBytes + 1023) / 1024) * 1024;
+  static constexpr int kStages = DH == 64 ? 6 : 5;     // depth of each of the K and V rings
   static constexpr int kQ = 0;
-  static constexpr int kQTail = kQ + kMain;
-  static constexpr int kK = ((kQTail + kTailBytes + 1023) / 1024) * 1024;
-  static constexpr int kStageBytes = ((kMain + kTailBytes + 1023) / 1024) * 1024;
-  static constexpr int kV = kK + kStages * kStageBytes;
-  static constexpr int kP = kV + kStages * kStageBytes;  // two P buffers, one per softmax group
-  static constexpr int kPBytes = kBM * kBN * 2;        // two 128B-swizzled atoms of 64 keys
-  static constexpr int kML = kP + 2 * kPBytes;         // float m[2][128], l[2][128]
+  static constexpr int kK = kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kML = kV + kStages * kTileBytes;  // float m[2][128], l[2][128]
   static constexpr int kBar = kML + 4 * kBM * 4;
-  static constexpr int kBytes = kBar + 256;
+  static constexpr int kBytes = kBar + 512;
   static constexpr int kAlloc = kBytes + 1024;         // slack to align the base to 1024
 };
 
+// The key tiles of one query tile, visited from a CTA-dependent starting point: CTAs that share
+// key tiles (every query tile keeps the global block) then read different tiles at a time instead
+// of all hitting the same L2 lines. The softmax is order-independent up to rounding.
 struct KeyTiles {
-  int lo0, hi0, lo1, hi1;
+  int lo0, hi0, lo1, hi1, rot;
   __device__ int count() const { return (hi0 - lo0) + (hi1 - lo1); }
-  __device__ int tile(int n) const { return n < hi0 - lo0 ? lo0 + n : lo1 + (n - (hi0 - lo0)); }
+  __device__ int tile(int n) const {
+    const int c = count();
+    n = n + rot < c ? n + rot : n + rot - c;
+    return n < hi0 - lo0 ? lo0 + n : lo1 + (n - (hi0 - lo0));
+  }
 };
 
 // Key tiles a query tile [q0, q_last] needs: the global rows [0, g*4b) and the band rows
@@ -113,6 +128,7 @@ __device__ __forceinline__ KeyTiles key_tiles(int q0, int q_last, const AttnPara
     t.hi0 = max(t.hi0, t.hi1);
     t.lo1 = t.hi1 = t.hi0;
   }
+  t.rot = (int)((blockIdx.x * 5u + blockIdx.y * 3u) % (unsigned)max(1, t.count()));
   return t;
 }
 
@@ -132,11 +148,13 @@ __device__ __forceinline__ bool tile_full(int q0, int q_last, int c0, const Attn
 // group turns its S tile into probabilities, the tensor core runs the other group's P*V and the
 // next Q*K^T. Each group keeps its own running max m, sum l and accumulator O (in TMEM); at the
 // end the two partial results of every row are merged.
-//   warp 0      TMA producer (Q once, then K/V tiles into a 3-stage ring)
-//   warp 1      TMEM allocator and tcgen05.mma issuer
-//   warps 2-5   softmax group 0 (one thread per query row = TMEM lane)
-//   warps 6-9   softmax group 1
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256, 256+dh), O1 [384, 384+dh).
+//   warp 0        TMA producer (Q once; K and V tiles into two separate rings)
+//   warp 1        TMEM allocator and tcgen05.mma issuer
+//   warps 2-3     idle (they complete the producer warpgroup for the register split)
+//   warps 4-7     softmax group 0 (one thread per query row = TMEM lane)
+//   warps 8-11    softmax group 1
+// TMEM columns: S0 [0,128) with P0 over its first 64, S1 [128,256) with P1 likewise,
+// O0 [256, 256+dh), O1 [384, 384+dh). P is bf16, two per column: the A operand of P*V.
 template <int DH>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -144,6 +162,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
            const __grid_constant__ CUtensorMap tk_tail, const __grid_constant__ CUtensorMap tv_tail,
            const AttnParams P, int* status) {
   using S = AttnSmem<DH>;
+  constexpr int NS = S::kStages;
   constexpr bool kHasTail = S::kTail > 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -152,10 +171,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   float* s_l = s_m + 2 * kBM;                              // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;                 // [kStages]
-  uint64_t* v_full = k_full + kStages;         // [kStages]
-  uint64_t* kv_empty = v_full + kStages;       // [kStages]
-  uint64_t* s_full = kv_empty + kStages;       // [2]
+  uint64_t* k_full = bars + 1;                 // [NS]
+  uint64_t* k_empty = k_full + NS;             // [NS]
+  uint64_t* v_full = k_empty + NS;             // [NS]
+  uint64_t* v_empty = v_full + NS;             // [NS]
+  uint64_t* s_full = v_empty + NS;             // [2]
   uint64_t* p_full = s_full + 2;               // [2]
   uint64_t* o_done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
@@ -170,10 +190,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(k_full + i, 1);
+      mbar_init(k_empty + i, 1);
       mbar_init(v_full + i, 1);
-      mbar_init(kv_empty + i, 1);
+      mbar_init(v_empty + i, 1);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(s_full + w, 1);
@@ -189,44 +210,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------ TMA producer ------------------------------
-    if (lane == 0) {
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsProducer>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------ TMA producer ------------------------------
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
       mbar_expect_tx(q_full, S::kMain + S::kTailBytes);
       tma_load_3d(smem + S::kQ, &tq, q_full, 0, q0, uh);
-      if (kHasTail) tma_load_3d(smem + S::kQTail, &tq_tail, q_full, 64, q0, uh);
+      if (kHasTail) tma_load_3d(smem + S::kQ + S::kMain, &tq_tail, q_full, 64, q0, uh);
       for (int n = 0; n < ntiles; ++n) {
-        const int st = n % kStages;
-        if (n >= kStages && !mbar_wait(kv_empty + st, ((n / kStages) - 1) & 1, abort, status))
-          break;
+        const int st = n % NS;
+        const uint32_t ph = ((n / NS) - 1) & 1;
         const int c0 = tiles.tile(n) * kBN;
-        uint8_t* kb = smem + S::kK + st * S::kStageBytes;
-        uint8_t* vb = smem + S::kV + st * S::kStageBytes;
+        if (n >= NS && !mbar_wait(k_empty + st, ph, abort, status)) break;
+        uint8_t* kb = smem + S::kK + st * S::kTileBytes;
         mbar_expect_tx(k_full + st, S::kMain + S::kTailBytes);
         tma_load_3d(kb, &tk, k_full + st, 0, c0, uh);
         if (kHasTail) tma_load_3d(kb + S::kMain, &tk_tail, k_full + st, 64, c0, uh);
+        if (n >= NS && !mbar_wait(v_empty + st, ph, abort, status)) break;
+        uint8_t* vb = smem + S::kV + st * S::kTileBytes;
         mbar_expect_tx(v_full + st, S::kMain + S::kTailBytes);
         tma_load_3d(vb, &tv, v_full + st, 0, c0, uh);
         if (kHasTail) tma_load_3d(vb + S::kMain, &tv_tail, v_full + st, 64, c0, uh);
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------ MMA issuer --------------------------------
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------ MMA issuer --------------------------------
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, 64, false, true);
       constexpr uint32_t idesc_pv_tail = idesc_bf16_f32(kBM, 16, false, true);
       const uint32_t q_addr = smem_u32(smem + S::kQ);
       bool ok = mbar_wait(q_full, 0, abort, status);
-      // S_w = Q K_n^T for tile n (w = n % 2).
+      // S_w = Q K_n^T for tile n (w = n % 2); K's stage is released when it completes.
       auto issue_qk = [&](int n) -> bool {
-        const int st = n % kStages;
-        if (!mbar_wait(k_full + st, (n / kStages) & 1, abort, status)) return false;
+        const int st = n % NS;
+        if (!mbar_wait(k_full + st, (n / NS) & 1, abort, status)) return false;
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + S::kK + st * S::kStageBytes);
+        const uint32_t k_addr = smem_u32(smem + S::kK + st * S::kTileBytes);
         const uint32_t d = tmem + (n & 1) * kBN;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -236,30 +257,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           umma_bf16_ss(d, smem_desc(q_addr + S::kMain, 16, 256, kSwizzle32B),
                        smem_desc(k_addr + S::kMain, 16, 256, kSwizzle32B), idesc_qk, 1);
         umma_commit(s_full + (n & 1));
+        umma_commit(k_empty + st);
         return true;
       };
-      // O_w (+)= P_w V_n once group w has written P_w for tile n.
+      // O_w (+)= P_w V_n, P_w read from TMEM, once group w has written it for tile n.
       auto issue_pv = [&](int n) -> bool {
-        const int st = n % kStages, w = n & 1;
+        const int st = n % NS, w = n & 1;
         if (!mbar_wait(p_full + w, (n >> 1) & 1, abort, status)) return false;
-        if (!mbar_wait(v_full + st, (n / kStages) & 1, abort, status)) return false;
+        if (!mbar_wait(v_full + st, (n / NS) & 1, abort, status)) return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kStageBytes);
-        const uint32_t p_addr = smem_u32(smem + S::kP + w * S::kPBytes);
+        const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kTileBytes);
+        const uint32_t a = tmem + w * kBN;              // P_w: 128 lanes x 64 columns
         const uint32_t d = tmem + 256 + w * 128;
         const uint32_t acc = n >= 2;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t a = smem_desc(p_addr + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024,
-                                       kSwizzle128B);
-          umma_bf16_ss(d, a, smem_desc(v_addr + kk * 2048, kBN * 128, 1024, kSwizzle128B),
+          umma_bf16_ts(d, a + kk * 8, smem_desc(v_addr + kk * 2048, kBN * 128, 1024, kSwizzle128B),
                        idesc_pv, acc | (kk > 0));
           if (kHasTail)
-            umma_bf16_ss(d + 64, a,
+            umma_bf16_ts(d + 64, a + kk * 8,
                          smem_desc(v_addr + S::kMain + kk * 512, kBN * 32, 256, kSwizzle32B),
                          idesc_pv_tail, acc | (kk > 0));
         }
-        umma_commit(kv_empty + st);
+        umma_commit(v_empty + st);
         return true;
       };
       if (ok) tc_fence_after();
@@ -267,13 +287,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ok && ntiles > 1) ok = issue_qk(1);
       for (int n = 0; ok && n < ntiles; ++n) {
         ok = issue_pv(n);
+        // S_w of tile n+2 overwrites P_w of tile n: issued after that P*V, and tcgen05.mma
+        // operations of one thread execute in order.
         if (ok && n + 2 < ntiles) ok = issue_qk(n + 2);
       }
       if (ok) umma_commit(o_done);
     }
   } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------ softmax groups ----------------------------
-    const int grp = (warp - 2) >> 2;                    // 0 or 1
+    const int grp = (warp - 4) >> 2;                    // 0 or 1
     const int row = 32 * (warp & 3) + lane;             // TMEM lane == query row
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
     const uint32_t t_s = tmem + grp * kBN + lane_off;
@@ -283,7 +306,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int a_q = min(qrow, P.N - 1) / b4;
     const int s_q = band_start(a_q, P.W, P.nb);
     const int band_lo = s_q * b4, band_hi = (s_q + P.W) * b4, glob_hi = P.g * b4;
-    const uint32_t p_base = smem_u32(smem + S::kP + grp * S::kPBytes);
     const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
     float m_ref = -INFINITY, l_run = 0.f;
     bool ok = true;
@@ -337,25 +359,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
       const uint64_t nref2 = f2_pack(-ref, -ref);
       uint64_t sum2a = 0, sum2b = 0;   // two packed partial sums (bit pattern 0 = +0.0f pair)
+      // P row as bf16 pairs (column i holds keys 2i, 2i+1), written over the first 64 columns of
+      // S_w in two halves of 32 columns (the whole S row is already in registers).
 #pragma unroll
-      for (int at = 0; at < 2; ++at) {
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pw[32];
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = at * 64 + cc * 8 + 2 * e;
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), scale2, nref2), x0, x1);
-            const float p0 = ex2_mufu(x0), p1 = ex2_mufu(x1);
-            if (e & 1)
-              sum2b = f2_add(sum2b, f2_pack(p0, p1));
-            else
-              sum2a = f2_add(sum2a, f2_pack(p0, p1));
-            w[e] = pack_bf16(p0, p1);
-          }
-          st_shared_v4(p_base + at * (kBM * 128) + sw128_offset(row, cc), w[0], w[1], w[2], w[3]);
+        for (int i2 = 0; i2 < 32; ++i2) {
+          const int i = 64 * half + 2 * i2;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), scale2, nref2), x0, x1);
+          const float p0 = ex2_mufu(x0), p1 = ex2_mufu(x1);
+          if (i2 & 1)
+            sum2b = f2_add(sum2b, f2_pack(p0, p1));
+          else
+            sum2a = f2_add(sum2a, f2_pack(p0, p1));
+          pw[i2] = pack_bf16(p0, p1);
         }
+        tmem_st32(t_s + 32 * half, pw);
       }
       float sa0, sa1;
       f2_unpack(f2_add(sum2a, sum2b), sa0, sa1);
@@ -372,7 +393,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_st32(t_o + c * 32, o);
         }
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full + grp);
     }

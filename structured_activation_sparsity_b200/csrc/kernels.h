@@ -49,8 +49,17 @@ struct GemmEpilogue {
   const int32_t* keep;      // kind 1: [B*K]
   int K_per_image, T;       // kind 1
 };
-// C[M, N] = A[M, Kd] * B[N, Kd]^T on tcgen05 with the given epilogue.
-cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, int M, int N, int Kd,
-                        int BN, const GemmEpilogue& ep, int* status, cudaStream_t st);
+// Tile width and k-split of C[M, N] = A[M, Kd] * B[N, Kd]^T for `sms` persistent CTAs.
+struct GemmPlan {
+  int bn, splits, m_tiles, n_tiles, units;
+};
+GemmPlan gemm_plan(int M, int N, int Kd, int sms);
+// fp32 partial-tile bytes the plan needs (0 without a k-split); plus one int counter per tile.
+size_t gemm_partial_bytes(const GemmPlan& p);
+// C = A B^T on tcgen05 with the given epilogue. partial / counters: workspace for k-splits
+// (counters zero on entry).
+cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, const GemmPlan& p, int M,
+                        int N, int Kd, const GemmEpilogue& ep, float* partial, int* counters,
+                        int sms, int* status, cudaStream_t st);
 
 }  // namespace ss

@@ -41,49 +41,122 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* keep, uint16_t*
   return cudaGetLastError();
 }
 
-constexpr int kGemmThreads = 192;
+// Persistent warp-specialised GEMM. Work unit = (m-tile, n-tile, k-split); CTA c takes units
+// c, c + grid, c + 2*grid, ... The accumulator is double-buffered in TMEM, so the epilogue of one
+// unit overlaps the mainloop of the next.
+//   warp 0      TMA producer (A and B k-blocks into a multi-stage ring, across units)
+//   warp 1      TMEM allocator and tcgen05.mma issuer
+//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4).. and one half of the tile's columns
+// A k-split unit writes its fp32 partial tile to its own slot; the last unit of a tile to finish
+// (an atomic counter per tile) sums the slots in split order and applies the epilogue, so the
+// result does not depend on which split finished last.
+constexpr int kGemmThreads = 320;
+constexpr int kEpiThreads = 256;
 
 template <int BN>
 struct GemmCfg {
-  static constexpr int kStages = BN == 256 ? 3 : 4;
+  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
   static constexpr int kABytes = 128 * 128;       // 128 rows x 64 bf16
   static constexpr int kBBytes = BN * 128;        // BN rows x 64 bf16
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBar = kStages * kStageBytes;
-  static constexpr int kAlloc = kBar + 256 + 1024;
-  static constexpr int kTmemCols = BN < 32 ? 32 : BN;
+  static constexpr int kAlloc = kBar + 512 + 1024;
+  static constexpr int kTmemCols = 2 * BN;        // two accumulators
+  static constexpr int kHalf = BN / 2;            // columns per epilogue warp
 };
 
 __device__ __forceinline__ float bf16_to_f(uint16_t v) { return __uint_as_float(uint32_t(v) << 16); }
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 __device__ __forceinline__ float gelu_erf(float z) {
   return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
 }
 
+struct GemmShape {
+  int M, N, Kd;
+  int m_tiles, n_tiles, splits, kb_total;
+  float* partial;          // [tiles][splits][BN][128] fp32, column-major tiles (splits > 1)
+  int* counters;           // [tiles], zero on entry (splits > 1)
+};
+
+// Applies the epilogue to 32 consecutive columns [n, n+32) of row m (all m < M).
+__device__ __forceinline__ void epilogue32(const GemmEpilogue& ep, const GemmShape& g, int m,
+                                           int n, float (&v)[32]) {
+  if (ep.bias) {
+    const uint4* bp = reinterpret_cast<const uint4*>(ep.bias + n);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 bw = __ldg(bp + q);
+      const uint32_t w[4] = {bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[q * 8 + 2 * e] += bf16_lo(w[e]);
+        v[q * 8 + 2 * e + 1] += bf16_hi(w[e]);
+      }
+    }
+  }
+  uint4* d;
+  if (ep.kind == 0) {
+    d = reinterpret_cast<uint4*>(ep.out + (size_t)m * g.N + n);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+  } else {
+    const int b = m / ep.K_per_image;
+    const int t = min(max(__ldg(ep.keep + m), 0), ep.T - 1);   // never leave the image
+    d = reinterpret_cast<uint4*>(ep.x + ((size_t)b * ep.T + t) * g.N + n);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 xv = d[q];
+      const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[q * 8 + 2 * e] += bf16_lo(w[e]);
+        v[q * 8 + 2 * e + 1] += bf16_hi(w[e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16(v[q * 8 + 0], v[q * 8 + 1]);
+    w.y = pack_bf16(v[q * 8 + 2], v[q * 8 + 3]);
+    w.z = pack_bf16(v[q * 8 + 4], v[q * 8 + 5]);
+    w.w = pack_bf16(v[q * 8 + 6], v[q * 8 + 7]);
+    d[q] = w;
+  }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    k_gemm(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, int M,
-           int N, int Kd, const GemmEpilogue ep, int* status) {
+    k_gemm(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+           const GemmShape g, const GemmEpilogue ep, int* status) {
   using G = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::kBar);
   uint64_t* empty = full + G::kStages;
-  uint64_t* acc_full = empty + G::kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* acc_full = empty + G::kStages;   // [2]
+  uint64_t* acc_empty = acc_full + 2;        // [2]
+  uint64_t* epi_bar = acc_empty + 2;         // epilogue-warps rendezvous (bounded, unlike bar.sync)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_bar + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * BN;
-  const int kblocks = Kd / 64;
+  const int units = g.m_tiles * g.n_tiles * g.splits;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < G::kStages; ++i) {
       mbar_init(full + i, 1);
       mbar_init(empty + i, 1);
     }
-    mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full + b, 1);
+      mbar_init(acc_empty + b, kEpiThreads);
+    }
+    mbar_init(epi_bar, kEpiThreads);
     *abort = 0;
     fence_barrier_init();
   }
@@ -93,92 +166,147 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  auto decode = [&](int u, int& m, int& n, int& s, int& kb0, int& kb1) {
+    m = u % g.m_tiles;
+    const int r = u / g.m_tiles;
+    n = r % g.n_tiles;
+    s = r / g.n_tiles;
+    kb0 = (int)((long long)s * g.kb_total / g.splits);
+    kb1 = (int)((long long)(s + 1) * g.kb_total / g.splits);
+  };
+
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&ta);
       tma_prefetch_desc(&tb);
-      for (int kb = 0; kb < kblocks; ++kb) {
-        const int st = kb % G::kStages;
-        if (kb >= G::kStages &&
-            !mbar_wait(empty + st, ((kb / G::kStages) - 1) & 1, abort, status))
-          break;
-        uint8_t* sa = smem + st * G::kStageBytes;
-        mbar_expect_tx(full + st, G::kStageBytes);
-        tma_load_2d(sa, &ta, full + st, kb * 64, m0);
-        tma_load_2d(sa + G::kABytes, &tb, full + st, kb * 64, n0);
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
+        int m, n, s, kb0, kb1;
+        decode(u, m, n, s, kb0, kb1);
+        const int nkb = kb1 - kb0, rot = u % nkb;
+        for (int j = 0; j < nkb; ++j, ++it) {
+          const int kb = kb0 + (j + rot) % nkb;   // rotated start: CTAs spread over L2 slices
+          const int st = it % G::kStages;
+          if (it >= G::kStages &&
+              !(ok = mbar_wait(empty + st, ((it / G::kStages) - 1) & 1, abort, status)))
+            break;
+          uint8_t* sa = smem + st * G::kStageBytes;
+          mbar_expect_tx(full + st, G::kStageBytes);
+          tma_load_2d(sa, &ta, full + st, kb * 64, m * 128);
+          tma_load_2d(sa + G::kABytes, &tb, full + st, kb * 64, n * BN);
+        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
+      int it = 0, i = 0;
       bool ok = true;
-      for (int kb = 0; kb < kblocks; ++kb) {
-        const int st = kb % G::kStages;
-        if (!(ok = mbar_wait(full + st, (kb / G::kStages) & 1, abort, status))) break;
+      for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++i) {
+        int m, n, s, kb0, kb1;
+        decode(u, m, n, s, kb0, kb1);
+        const int buf = i & 1;
+        if (i >= 2 && !(ok = mbar_wait(acc_empty + buf, ((i >> 1) - 1) & 1, abort, status))) break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + st * G::kStageBytes);
-        const uint32_t b_addr = a_addr + G::kABytes;
+        const uint32_t d = tmem + buf * BN;
+        for (int j = 0; j < kb1 - kb0; ++j, ++it) {
+          const int st = it % G::kStages;
+          if (!(ok = mbar_wait(full + st, (it / G::kStages) & 1, abort, status))) break;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + st * G::kStageBytes);
+          const uint32_t b_addr = a_addr + G::kABytes;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_bf16_ss(tmem, smem_desc(a_addr + kk * 32, 16, 1024, kSwizzle128B),
-                       smem_desc(b_addr + kk * 32, 16, 1024, kSwizzle128B), idesc,
-                       (kb | kk) != 0);
-        umma_commit(empty + st);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ss(d, smem_desc(a_addr + kk * 32, 16, 1024, kSwizzle128B),
+                         smem_desc(b_addr + kk * 32, 16, 1024, kSwizzle128B), idesc,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(empty + st);
+        }
+        if (ok) umma_commit(acc_full + buf);
       }
-      if (ok) umma_commit(acc_full);
     }
   } else {
-    const int row = 32 * (warp & 3) + lane;
+    // ------------------------------ epilogue warps ----------------------------
+    const int ew = warp - 2;                              // 0..7
+    const int row = 32 * (warp & 3) + lane;               // TMEM lane
+    const int col0 = (ew >> 2) * G::kHalf;                // this warp's half of the columns
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
-    const int m = m0 + row;
-    const bool ok = mbar_wait(acc_full, 0, abort, status);
-    tc_fence_after();
-    if (ok) {
-      uint16_t* dst_row = nullptr;
-      if (ep.kind == 0) {
-        dst_row = ep.out + (size_t)m * N;
-      } else if (m < M) {
-        const int b = m / ep.K_per_image;
-        const int t = min(max(__ldg(ep.keep + m), 0), ep.T - 1);
-        dst_row = ep.x + ((size_t)b * ep.T + t) * N;
-      }
+    uint32_t epi_phase = 0;
+    // All epilogue threads meet here; a wait that gives up ends every caller's unit loop.
+    auto epi_sync = [&]() -> bool {
+      mbar_arrive(epi_bar);
+      const bool r = mbar_wait(epi_bar, epi_phase, abort, status);
+      epi_phase ^= 1;
+      return r;
+    };
+    int i = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
+      int m_t, n_t, s, kb0, kb1;
+      decode(u, m_t, n_t, s, kb0, kb1);
+      const int buf = i & 1;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full + buf, (i >> 1) & 1, abort, status));
+      if (!ok) break;
+      tc_fence_after();
+      const int m = m_t * 128 + row;
+      const int tile = n_t * g.m_tiles + m_t;
+      const uint32_t t_acc = tmem + buf * BN + lane_off + col0;
+      if (g.splits == 1) {
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_off + c * 32, r);
-                if (m >= M) continue;
-        const int n = n0 + c * 32;
-        float v[32];
+        for (int c = 0; c < G::kHalf / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_acc + c * 32, r);
+          if (c == G::kHalf / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(acc_empty + buf);   // accumulator fully read: MMA may reuse it
+          }
+          if (m < g.M) {
+            float v[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          v[i] = __uint_as_float(r[i]);
-          if (ep.bias) v[i] += bf16_to_f(__ldg(ep.bias + n + i));
-        }
-        uint4* d = reinterpret_cast<uint4*>(dst_row + n);
-        if (ep.kind == 0) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 xv = d[q];
-            const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              v[q * 8 + 2 * e] += __uint_as_float(w[e] << 16);
-              v[q * 8 + 2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
-            }
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+            epilogue32(ep, g, m, n_t * BN + col0 + c * 32, v);
           }
         }
+      } else {
+        // Write this split's partial tile (column-major, so a warp's 32 rows of one column are
+        // one 128-byte line), then let the last split of the tile finish it.
+        float* slot = g.partial + ((size_t)tile * g.splits + s) * 128 * BN + (size_t)col0 * 128 + row;
+#pragma unroll 1
+        for (int c = 0; c < G::kHalf / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_acc + c * 32, r);
+          if (c == G::kHalf / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(acc_empty + buf);
+          }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 w;
-          w.x = pack_bf16(v[q * 8 + 0], v[q * 8 + 1]);
-          w.y = pack_bf16(v[q * 8 + 2], v[q * 8 + 3]);
-          w.z = pack_bf16(v[q * 8 + 4], v[q * 8 + 5]);
-          w.w = pack_bf16(v[q * 8 + 6], v[q * 8 + 7]);
-          d[q] = w;
+          for (int e = 0; e < 32; ++e) slot[(size_t)(c * 32 + e) * 128] = __uint_as_float(r[e]);
         }
+        __threadfence();
+        if (!epi_sync()) break;
+        if (threadIdx.x == 64) *s_last = atomicAdd(g.counters + tile, 1) == g.splits - 1;
+        if (!epi_sync()) break;
+        if (*s_last) {
+          __threadfence();
+          if (m < g.M) {
+            const float* base =
+                g.partial + (size_t)tile * g.splits * 128 * BN + (size_t)col0 * 128 + row;
+#pragma unroll 1
+            for (int c = 0; c < G::kHalf / 32; ++c) {
+              float v[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = 0.f;
+              for (int sp = 0; sp < g.splits; ++sp) {   // fixed split order: deterministic sum
+                const float* src = base + (size_t)sp * 128 * BN + (size_t)c * 32 * 128;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] += __ldcg(src + (size_t)e * 128);
+              }
+              epilogue32(ep, g, m, n_t * BN + col0 + c * 32, v);
+            }
+          }
+          if (threadIdx.x == 64) g.counters[tile] = 0;
+        }
+        if (!epi_sync()) break;   // s_last is reused by the next unit
       }
     }
   }
@@ -190,24 +318,75 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+GemmPlan gemm_plan(int M, int N, int Kd, int sms) {
+  GemmPlan p;
+  const int m_tiles = (M + 127) / 128;
+  const int kb = Kd / 64;
+  // Pick the tile width and k-split with the smallest makespan: rounds of units over the CTAs,
+  // times k-blocks per unit, times the MMA time of one k-block (~ the tile width; N below 128 is
+  // bound by shared-memory bandwidth). A split costs a partial-tile round trip (~2 k-blocks per
+  // split) and is only considered for long K (>= 24 k-blocks).
+  long long best = -1;
+  p.bn = 64;
+  p.splits = 1;
+  for (int bn : {256, 128, 64}) {
+    if (N % bn) continue;
+    const int n_tiles = N / bn;
+    for (int s = 1; s <= 8; ++s) {
+      if (s > 1 && (kb < 24 || kb / s < 4)) break;
+      const long long units = (long long)m_tiles * n_tiles * s;
+      const long long rounds = (units + sms - 1) / sms;
+      const long long kb_unit = (kb + s - 1) / s;
+      const long long step = bn < 128 ? 128 : bn;
+      const long long cost = rounds * kb_unit * step + (s > 1 ? (long long)s * 2 * step : 0);
+      if (best < 0 || cost < best) {
+        best = cost;
+        p.bn = bn;
+        p.splits = s;
+      }
+    }
+  }
+  p.m_tiles = m_tiles;
+  p.n_tiles = N / p.bn;
+  p.units = m_tiles * p.n_tiles * p.splits;
+  return p;
+}
+
+size_t gemm_partial_bytes(const GemmPlan& p) {
+  if (p.splits == 1) return 0;
+  return (size_t)p.m_tiles * p.n_tiles * p.splits * 128 * p.bn * 4;
+}
+
 template <int BN>
-static cudaError_t launch_gemm_bn(const CUtensorMap* ta, const CUtensorMap* tb, int M, int N,
-                                  int Kd, const GemmEpilogue& ep, int* status, cudaStream_t st) {
+static cudaError_t launch_gemm_bn(const CUtensorMap* ta, const CUtensorMap* tb, const GemmPlan& p,
+                                  int M, int N, int Kd, const GemmEpilogue& ep, float* partial,
+                                  int* counters, int sms, int* status, cudaStream_t st) {
   using G = GemmCfg<BN>;
   cudaError_t e =
       cudaFuncSetAttribute(k_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kAlloc);
   if (e != cudaSuccess) return e;
-  dim3 grid((M + 127) / 128, N / BN);
-  k_gemm<BN><<<grid, kGemmThreads, G::kAlloc, st>>>(*ta, *tb, M, N, Kd, ep, status);
+  GemmShape g;
+  g.M = M;
+  g.N = N;
+  g.Kd = Kd;
+  g.m_tiles = p.m_tiles;
+  g.n_tiles = p.n_tiles;
+  g.splits = p.splits;
+  g.kb_total = Kd / 64;
+  g.partial = partial;
+  g.counters = counters;
+  const int grid = p.units < sms ? p.units : sms;
+  k_gemm<BN><<<grid, kGemmThreads, G::kAlloc, st>>>(*ta, *tb, g, ep, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, int M, int N, int Kd, int BN,
-                        const GemmEpilogue& ep, int* status, cudaStream_t st) {
-  switch (BN) {
-    case 64: return launch_gemm_bn<64>(ta, tb, M, N, Kd, ep, status, st);
-    case 128: return launch_gemm_bn<128>(ta, tb, M, N, Kd, ep, status, st);
-    case 256: return launch_gemm_bn<256>(ta, tb, M, N, Kd, ep, status, st);
+cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, const GemmPlan& p, int M,
+                        int N, int Kd, const GemmEpilogue& ep, float* partial, int* counters,
+                        int sms, int* status, cudaStream_t st) {
+  switch (p.bn) {
+    case 64: return launch_gemm_bn<64>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
+    case 128: return launch_gemm_bn<128>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
+    case 256: return launch_gemm_bn<256>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
   }
   return cudaErrorInvalidValue;
 }

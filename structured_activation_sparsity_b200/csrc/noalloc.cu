@@ -19,7 +19,7 @@
 namespace ss {
 namespace {
 
-constexpr size_t kRcmlpScratchBytes = size_t(16) << 20;   // 16 MiB
+constexpr size_t kRcmlpScratchBytes = size_t(32) << 20;   // 32 MiB
 static __device__ __align__(256) uint8_t g_rcmlp_scratch[kRcmlpScratchBytes];
 
 std::mutex g_scratch_mu;

@@ -69,11 +69,28 @@ __global__ void __launch_bounds__(256) k_stripe_rank(const double* __restrict__ 
   const unsigned long long kt = s_key[tt];
   const int chunk = (N + 7) / 8;
   const int lo = warp * chunk, hi = min(N, lo + chunk);
-  int cnt = 0;
-  for (int o = lo; o < hi; ++o) {
-    unsigned long long ko = s_key[o];
-    cnt += (ko > kt) | ((ko == kt) & (o < tt));
+  // Tokens before tt count when their key is >= kt (ties broken by the lower index), tokens
+  // after it only when strictly greater: two loops, no per-element index compare. Four
+  // independent counters keep the compare chain short.
+  const int mid = max(lo, min(hi, tt));
+  int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+  int o = lo;
+  for (; o + 4 <= mid; o += 4) {
+    c0 += s_key[o] >= kt;
+    c1 += s_key[o + 1] >= kt;
+    c2 += s_key[o + 2] >= kt;
+    c3 += s_key[o + 3] >= kt;
   }
+  for (; o < mid; ++o) c0 += s_key[o] >= kt;
+  o = mid;
+  for (; o + 4 <= hi; o += 4) {
+    c0 += s_key[o] > kt;
+    c1 += s_key[o + 1] > kt;
+    c2 += s_key[o + 2] > kt;
+    c3 += s_key[o + 3] > kt;
+  }
+  for (; o < hi; ++o) c0 += s_key[o] > kt;
+  const int cnt = (c0 + c1) + (c2 + c3);
   s_cnt[warp][lane] = cnt;
   __syncthreads();
   if (warp == 0 && t < N) {

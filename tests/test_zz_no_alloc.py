@@ -1,6 +1,6 @@
 """sparsesam_rcmlp_noalloc: the RC-MLP for callers that cannot allocate device memory (code under
 another runtime's stream capture, hosts that own all device memory, loops that must avoid
-cudaMalloc's device-wide synchronisation). It keeps its scratch in a fixed 16 MiB array inside the
+cudaMalloc's device-wide synchronisation). It keeps its scratch in a fixed 32 MiB array inside the
 library; its results must equal those of sparsesam_rcmlp with a caller-provided workspace.
 
 This file is collected last so that a failure here cannot stop the rest of a -x run."""
@@ -30,11 +30,11 @@ def _inputs(cfg, C, Hd, seed):
 
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_point_twice():
-    # The SAM ViT-B global block's MLP (768 -> 3072 -> 768 on 1639 kept tokens): 12.6 MB of scratch.
+    # The SAM ViT-B global block's MLP (768 -> 3072 -> 768 on 1639 kept tokens): 28 MB of scratch.
     cfg = L.make_cfg(1, 64, 64, "global", 14, 12, 64, 0.4)
     C, Hd = 768, 3072
     wsb = L.sparsesam_rcmlp_workspace(cfg, C, Hd)
-    assert wsb <= 16 << 20
+    assert wsb <= 32 << 20
     ws = torch.empty((wsb,), dtype=torch.uint8, device="cuda")
     for seed in (11, 12):                                  # two calls in a row on the shared array
         x, w1, b1, w2, b2, keep = (t.to("cuda") for t in _inputs(cfg, C, Hd, seed))
@@ -50,9 +50,9 @@ def test_noalloc_matches_workspace_entry_point_twice():
 
 
 def test_noalloc_rejects_shapes_beyond_its_array():
-    # batch 4 of the same block needs 4 x 12.6 MB: rejected on the host before any CUDA call.
+    # batch 4 of the same block needs about 4 x 28 MB: rejected on the host before any CUDA call.
     cfg = L.make_cfg(4, 64, 64, "global", 14, 12, 64, 0.4)
-    assert L.sparsesam_rcmlp_workspace(cfg, 768, 3072) > 16 << 20
+    assert L.sparsesam_rcmlp_workspace(cfg, 768, 3072) > 32 << 20
     with pytest.raises(L.SparseSAMError) as e:
         L.sparsesam_rcmlp_noalloc(cfg, 1 << 20, 768, 3072, 1 << 20, None, 1 << 20, None, 1 << 20)
     assert e.value.code == L.SS_EWORKSPACE
