@@ -18,6 +18,8 @@
 //              P written to shared memory as bf16 (128B-swizzled, K-major A operand),
 //              O accumulated in registers; epilogue scatters rows to out[perm[p]].
 // TMEM columns: [0,128) S (fp32), [128, 128+dh) P*V of the current tile (fp32).
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -79,6 +81,7 @@ constexpr int kBM = 128;              // query rows per CTA
 constexpr int kBN = 128;              // keys per tile
 constexpr int kAttnThreads = 384;     // 12 warps = 3 warpgroups
 constexpr float kLazyRescale = 8.f;   // log2 headroom before O and l are rescaled
+constexpr int kPolyPairs = 7;         // of every 16 exp pairs on full tiles, those on the FMA pipe
 // Register split (launch: 384 threads x 168): producer warpgroup 56, softmax warpgroups 224.
 constexpr uint32_t kRegsProducer = 56, kRegsSoftmax = 224;
 static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= 384 * 168, "register split too large");
@@ -132,15 +135,35 @@ __device__ __forceinline__ KeyTiles key_tiles(int q0, int q_last, const AttnPara
   return t;
 }
 
-// True if every (query row, key) pair of the tile is kept (no element mask needed).
-__device__ __forceinline__ bool tile_full(int q0, int q_last, int c0, const AttnParams& P) {
-  const int c_last = c0 + kBN - 1;
-  if (c_last >= P.N) return false;
-  const int b4 = P.b * kStripes;
-  for (int a = q0 / b4; a <= q_last / b4; ++a)
-    for (int ka = c0 / b4; ka <= c_last / b4; ++ka)
-      if (!block_kept(a, ka, P.W, P.nb, P.g)) return false;
-  return true;
+// Every (query row, key) pair of a key tile is kept when offset blocks are whole multiples of the
+// 128-row tile (4b % 128 == 0, e.g. b = 64): a query tile then lies in one offset block, and each
+// key tile of its list lies in one kept offset block. Otherwise (b = 16, 7, ...) tiles straddle
+// blocks and take the element mask; so does the ragged last key tile.
+__device__ __forceinline__ bool tile_full(int c0, const AttnParams& P) {
+  return (P.b * kStripes) % kBN == 0 && c0 + kBN <= P.N;
+}
+
+// 2^x on the FMA pipe for x in [-125, 8] (Cody-Waite style reduction 2^x = 2^n 2^f, n = round(x),
+// f in [-1/2, 1/2]; 2^f by the cubic that interpolates it at the four Chebyshev nodes of the
+// interval, coefficients from csrc/exp2_poly.py, relative error < 1e-4). Operates on a pair.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+  constexpr float kMagic = 12582912.f;   // 1.5 * 2^23: adding it rounds to an integer in the low bits
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  const uint64_t x2 = f2_pack(x0, x1);
+  const uint64_t t2 = f2_add(x2, f2_pack(kMagic, kMagic));
+  const uint64_t n2 = f2_add(t2, f2_pack(-kMagic, -kMagic));
+  const uint64_t fr = f2_fma(n2, f2_pack(-1.f, -1.f), x2);
+  uint64_t q = f2_fma(f2_pack(0.05583828315138817f, 0.05583828315138817f), fr,
+                      f2_pack(0.2426394820213318f, 0.2426394820213318f));
+  q = f2_fma(q, fr, f2_pack(0.6931367516517639f, 0.6931367516517639f));
+  q = f2_fma(q, fr, f2_pack(0.9999245405197144f, 0.9999245405197144f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t2, t0, t1);
+  // add n to the exponent field: the low mantissa bits of t hold n (two's complement)
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 // One CTA = one (unit, head, 128-row query tile). The key tiles are split between two softmax
@@ -323,7 +346,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(r[i]);
       }
       const int c0 = tiles.tile(n) * kBN;
-      if (!tile_full(q0, q_last, c0, P)) {
+      const bool full = tile_full(c0, P);
+      if (!full) {
 #pragma unroll
         for (int i = 0; i < kBN; ++i) {
           const int c = c0 + i;
@@ -360,24 +384,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t nref2 = f2_pack(-ref, -ref);
       uint64_t sum2a = 0, sum2b = 0;   // two packed partial sums (bit pattern 0 = +0.0f pair)
       // P row as bf16 pairs (column i holds keys 2i, 2i+1), written over the first 64 columns of
-      // S_w in two halves of 32 columns (the whole S row is already in registers).
+      // S_w in two halves of 32 columns (the whole S row is already in registers). On full tiles
+      // kPolyPairs of every 16 pairs take 2^x on the FMA pipe (exp2_poly2), the rest on MUFU, so
+      // neither pipe alone bounds the tile; masked tiles stay on MUFU (ex2(-inf) = 0 exactly).
+      auto softmax_row = [&](auto poly_tag) {
+        constexpr bool kPoly = decltype(poly_tag)::value;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pw[32];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pw[32];
 #pragma unroll
-        for (int i2 = 0; i2 < 32; ++i2) {
-          const int i = 64 * half + 2 * i2;
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), scale2, nref2), x0, x1);
-          const float p0 = ex2_mufu(x0), p1 = ex2_mufu(x1);
-          if (i2 & 1)
-            sum2b = f2_add(sum2b, f2_pack(p0, p1));
-          else
-            sum2a = f2_add(sum2a, f2_pack(p0, p1));
-          pw[i2] = pack_bf16(p0, p1);
+          for (int i2 = 0; i2 < 32; ++i2) {
+            const int i = 64 * half + 2 * i2;
+            float x0, x1, p0, p1;
+            f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), scale2, nref2), x0, x1);
+            if (kPoly && (i2 & 15) < kPolyPairs) {
+              exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2_mufu(x0);
+              p1 = ex2_mufu(x1);
+            }
+            if (i2 & 1)
+              sum2b = f2_add(sum2b, f2_pack(p0, p1));
+            else
+              sum2a = f2_add(sum2a, f2_pack(p0, p1));
+            pw[i2] = pack_bf16(p0, p1);
+          }
+          tmem_st32(t_s + 32 * half, pw);
         }
-        tmem_st32(t_s + 32 * half, pw);
-      }
+      };
+      if (full)
+        softmax_row(std::integral_constant<bool, true>());
+      else
+        softmax_row(std::integral_constant<bool, false>());
       float sa0, sa1;
       f2_unpack(f2_add(sum2a, sum2b), sa0, sa1);
       l_run += sa0 + sa1;
