@@ -81,7 +81,7 @@ constexpr int kBM = 128;              // query rows per CTA
 constexpr int kBN = 128;              // keys per tile
 constexpr int kAttnThreads = 384;     // 12 warps = 3 warpgroups
 constexpr float kLazyRescale = 8.f;   // log2 headroom before O and l are rescaled
-constexpr int kPolyPairs = 7;         // of every 16 exp pairs on full tiles, those on the FMA pipe
+constexpr int kPolyPairs = 0;         // of every 16 exp pairs on full tiles, those on the FMA pipe
 // Register split (launch: 384 threads x 168): producer warpgroup 56, softmax warpgroups 224.
 constexpr uint32_t kRegsProducer = 56, kRegsSoftmax = 224;
 static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= 384 * 168, "register split too large");
