@@ -50,14 +50,31 @@ __global__ void __launch_bounds__(256) k_gather_qkv(const uint16_t* __restrict__
   const size_t plane = (size_t)N * CPR;       // 16-byte chunks per (unit, head) matrix
   const size_t src_row = ((size_t)u * N + tok) * per_tok;
   const size_t dst_row = (size_t)u * heads * plane + (size_t)qpos * CPR;
+  const uint4* src[3] = {reinterpret_cast<const uint4*>(q) + src_row,
+                         reinterpret_cast<const uint4*>(k) + src_row,
+                         reinterpret_cast<const uint4*>(v) + src_row};
+  uint4* dst[3] = {reinterpret_cast<uint4*>(qp) + dst_row, reinterpret_cast<uint4*>(kp) + dst_row,
+                   reinterpret_cast<uint4*>(vp) + dst_row};
+  // Up to 4 chunks per tensor per lane per pass: all 12 loads are in flight before any store.
+  for (int c0 = 0; c0 < per_tok; c0 += 128) {
+    uint4 buf[3][4];
 #pragma unroll
-  for (int t = 0; t < 3; ++t) {
-    const uint4* src = reinterpret_cast<const uint4*>(t == 0 ? q : (t == 1 ? k : v)) + src_row;
-    uint4* dst = reinterpret_cast<uint4*>(t == 0 ? qp : (t == 1 ? kp : vp)) + dst_row;
-    for (int c = lane; c < per_tok; c += 32) {
-      const int h = c / CPR, cc = c - h * CPR;     // CPR is a compile-time constant
-      dst[h * plane + cc] = __ldg(src + c);
-    }
+    for (int t = 0; t < 3; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = c0 + e * 32 + lane;
+        if (c < per_tok) buf[t][e] = __ldg(src[t] + c);
+      }
+#pragma unroll
+    for (int t = 0; t < 3; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = c0 + e * 32 + lane;
+        if (c < per_tok) {
+          const int h = c / CPR, cc = c - h * CPR;   // CPR is a compile-time constant
+          dst[t][h * plane + cc] = buf[t][e];
+        }
+      }
   }
 }
 
@@ -384,9 +401,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t nref2 = f2_pack(-ref, -ref);
       uint64_t sum2a = 0, sum2b = 0;   // two packed partial sums (bit pattern 0 = +0.0f pair)
       // P row as bf16 pairs (column i holds keys 2i, 2i+1), written over the first 64 columns of
-      // S_w in two halves of 32 columns (the whole S row is already in registers). On full tiles
-      // kPolyPairs of every 16 pairs take 2^x on the FMA pipe (exp2_poly2), the rest on MUFU, so
-      // neither pipe alone bounds the tile; masked tiles stay on MUFU (ex2(-inf) = 0 exactly).
+      // S_w in two halves of 32 columns (the whole S row is already in registers). 2^x runs on
+      // MUFU as packed f16 pairs (half the MUFU operations of f32; P is rounded to bf16 anyway);
+      // on full tiles kPolyPairs of every 16 pairs may instead take the FMA-pipe exp2_poly2.
+      // Masked keys give ex2(-inf) = 0 exactly.
       auto softmax_row = [&](auto poly_tag) {
         constexpr bool kPoly = decltype(poly_tag)::value;
 #pragma unroll
@@ -400,8 +418,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (kPoly && (i2 & 15) < kPolyPairs) {
               exp2_poly2(x0, x1, p0, p1);
             } else {
-              p0 = ex2_mufu(x0);
-              p1 = ex2_mufu(x1);
+              ex2_pair_f16(x0, x1, p0, p1);   // one MUFU op per pair
             }
             if (i2 & 1)
               sum2b = f2_add(sum2b, f2_pack(p0, p1));

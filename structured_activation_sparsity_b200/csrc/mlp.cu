@@ -17,27 +17,34 @@
 
 namespace ss {
 
+// One warp per kept row: resolve the row's token, then copy its C bf16 (C/8 16-byte chunks) with
+// all of a lane's loads in flight before its stores.
 __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t* __restrict__ x,
                                                      const int32_t* __restrict__ keep,
                                                      uint16_t* __restrict__ xk, int B, int T,
                                                      int K, int C) {
+  const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (m >= B * K) return;
+  const int b = m / K;
+  const int t = min(max(__ldg(keep + m), 0), T - 1);   // never leave the image
   const int cpr = C / 8;
-  const int total = B * K * cpr;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
-    const int m = i / cpr, c = i - (i / cpr) * cpr;
-    const int b = m / K;
-    const int t = min(max(__ldg(keep + m), 0), T - 1);   // never leave the image
-    reinterpret_cast<uint4*>(xk)[(size_t)m * cpr + c] =
-        __ldg(reinterpret_cast<const uint4*>(x + ((size_t)b * T + t) * C) + c);
+  const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)b * T + t) * C);
+  uint4* dst = reinterpret_cast<uint4*>(xk) + (size_t)m * cpr;
+  for (int c0 = 0; c0 < cpr; c0 += 256) {
+    uint4 buf[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (c0 + e * 32 + lane < cpr) buf[e] = __ldg(src + c0 + e * 32 + lane);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (c0 + e * 32 + lane < cpr) dst[c0 + e * 32 + lane] = buf[e];
   }
 }
 
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* keep, uint16_t* xk, int B, int T,
                                int K, int C, cudaStream_t st) {
-  const int total = B * K * (C / 8);
-  int blocks = (total + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  k_gather_rows<<<blocks, 256, 0, st>>>(x, keep, xk, B, T, K, C);
+  const int rows = B * K;
+  k_gather_rows<<<(rows + 7) / 8, 256, 0, st>>>(x, keep, xk, B, T, K, C);
   return cudaGetLastError();
 }
 

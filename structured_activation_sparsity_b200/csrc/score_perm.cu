@@ -60,7 +60,20 @@ __global__ void __launch_bounds__(256) k_stripe_rank(const double* __restrict__ 
   extern __shared__ unsigned long long s_key[];
   __shared__ int s_cnt[8][32];
   const int u = blockIdx.y;
-  for (int t = threadIdx.x; t < N; t += blockDim.x) s_key[t] = m.key(score, u, t);
+  // Fill the unit's keys: eight independent loads in flight per thread before any store.
+  for (int t0 = threadIdx.x; t0 < N; t0 += 8 * blockDim.x) {
+    unsigned long long k8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int t = t0 + e * blockDim.x;
+      k8[e] = t < N ? m.key(score, u, t) : 0ull;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int t = t0 + e * blockDim.x;
+      if (t < N) s_key[t] = k8[e];
+    }
+  }
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
