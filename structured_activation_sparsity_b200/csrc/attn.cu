@@ -402,9 +402,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint64_t sum2a = 0, sum2b = 0;   // two packed partial sums (bit pattern 0 = +0.0f pair)
       // P row as bf16 pairs (column i holds keys 2i, 2i+1), written over the first 64 columns of
       // S_w in two halves of 32 columns (the whole S row is already in registers). 2^x runs on
-      // MUFU as packed f16 pairs (half the MUFU operations of f32; P is rounded to bf16 anyway);
-      // on full tiles kPolyPairs of every 16 pairs may instead take the FMA-pipe exp2_poly2.
-      // Masked keys give ex2(-inf) = 0 exactly.
+      // MUFU in f32 (measured faster here than packed-f16 MUFU or the FMA-pipe exp2_poly2, which
+      // full tiles can route kPolyPairs of every 16 pairs to). Masked keys give ex2(-inf) = 0.
       auto softmax_row = [&](auto poly_tag) {
         constexpr bool kPoly = decltype(poly_tag)::value;
 #pragma unroll
@@ -418,7 +417,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (kPoly && (i2 & 15) < kPolyPairs) {
               exp2_poly2(x0, x1, p0, p1);
             } else {
-              ex2_pair_f16(x0, x1, p0, p1);   // one MUFU op per pair
+              p0 = ex2_mufu(x0);
+              p1 = ex2_mufu(x1);
             }
             if (i2 & 1)
               sum2b = f2_add(sum2b, f2_pack(p0, p1));
@@ -426,8 +426,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               sum2a = f2_add(sum2a, f2_pack(p0, p1));
             pw[i2] = pack_bf16(p0, p1);
           }
-          tmem_st32(t_s + 32 * half, pw);
+          tmem_st32_async(t_s + 32 * half, pw);
         }
+        tmem_st_wait();   // P complete in TMEM before the arrive below releases it to the MMA
       };
       if (full)
         softmax_row(std::integral_constant<bool, true>());
