@@ -17,7 +17,7 @@
 //   warps 2-5  softmax: one thread per query row (TMEM lane), online softmax in fp32,
 //              P written to shared memory as bf16 (128B-swizzled, K-major A operand),
 //              O accumulated in registers; epilogue scatters rows to out[perm[p]].
-// TMEM columns: [0,128) S (fp32), [128, 128+dh) P*V of the current tile (fp32).
+// TMEM holds both groups' S tiles, O accumulators and P tiles (AttnTmem).
 #include <type_traits>
 
 #include "common.cuh"
@@ -102,6 +102,14 @@ constexpr int kPolyPairs = 0;         // of every 16 exp pairs on full tiles, th
 // Register split (launch: 384 threads x 168): producer warpgroup 56, softmax warpgroups 224.
 constexpr uint32_t kRegsProducer = 56, kRegsSoftmax = 224;
 static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= 384 * 168, "register split too large");
+
+template <int DH>
+struct AttnTmem {
+  static constexpr bool kSeparateP = DH <= 64;
+  static constexpr uint32_t kS = 0, kSStride = 128;
+  static constexpr uint32_t kO = 256, kOStride = DH <= 64 ? 64 : 128;
+  static constexpr uint32_t kP = kSeparateP ? 384 : 0, kPStride = kSeparateP ? 64 : 128;
+};
 
 template <int DH>
 struct AttnSmem {
@@ -193,8 +201,10 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float&
 //   warps 2-3     idle (they complete the producer warpgroup for the register split)
 //   warps 4-7     softmax group 0 (one thread per query row = TMEM lane)
 //   warps 8-11    softmax group 1
-// TMEM columns: S0 [0,128) with P0 over its first 64, S1 [128,256) with P1 likewise,
-// O0 [256, 256+dh), O1 [384, 384+dh). P is bf16, two per column: the A operand of P*V.
+// TMEM columns (AttnTmem): S0 [0,128), S1 [128,256); dh 64: O0 [256,320), O1 [320,384),
+// P0 [384,448), P1 [448,512); dh 80: O0 [256,336), O1 [384,464) and P_w over the first 64
+// columns of S_w. P is bf16, two per column: the A operand of P*V. Keeping P apart from S (when
+// it fits) lets Q*K^T of tile n+2 start while P*V of tile n still reads P.
 template <int DH>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -288,7 +298,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(k_full + st, (n / NS) & 1, abort, status)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + S::kK + st * S::kTileBytes);
-        const uint32_t d = tmem + (n & 1) * kBN;
+        const uint32_t d = tmem + AttnTmem<DH>::kS + (n & 1) * AttnTmem<DH>::kSStride;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_bf16_ss(d, smem_desc(q_addr + kk * 32, 16, 1024, kSwizzle128B),
@@ -307,8 +317,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(v_full + st, (n / NS) & 1, abort, status)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kTileBytes);
-        const uint32_t a = tmem + w * kBN;              // P_w: 128 lanes x 64 columns
-        const uint32_t d = tmem + 256 + w * 128;
+        const uint32_t a = tmem + AttnTmem<DH>::kP + w * AttnTmem<DH>::kPStride;   // P_w
+        const uint32_t d = tmem + AttnTmem<DH>::kO + w * AttnTmem<DH>::kOStride;
         const uint32_t acc = n >= 2;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
@@ -339,8 +349,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int grp = (warp - 4) >> 2;                    // 0 or 1
     const int row = 32 * (warp & 3) + lane;             // TMEM lane == query row
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
-    const uint32_t t_s = tmem + grp * kBN + lane_off;
-    const uint32_t t_o = tmem + 256 + grp * 128 + lane_off;
+    const uint32_t t_s = tmem + AttnTmem<DH>::kS + grp * AttnTmem<DH>::kSStride + lane_off;
+    const uint32_t t_p = tmem + AttnTmem<DH>::kP + grp * AttnTmem<DH>::kPStride + lane_off;
+    const uint32_t t_o = tmem + AttnTmem<DH>::kO + grp * AttnTmem<DH>::kOStride + lane_off;
     const int qrow = q0 + row;
     const int b4 = P.b * kStripes;
     const int a_q = min(qrow, P.N - 1) / b4;
@@ -400,8 +411,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
       const uint64_t nref2 = f2_pack(-ref, -ref);
       uint64_t sum2a = 0, sum2b = 0;   // two packed partial sums (bit pattern 0 = +0.0f pair)
-      // P row as bf16 pairs (column i holds keys 2i, 2i+1), written over the first 64 columns of
-      // S_w in two halves of 32 columns (the whole S row is already in registers). 2^x runs on
+      // P row as bf16 pairs (column i holds keys 2i, 2i+1), written to P_w (its own columns, or
+      // over S_w, whose row is already in registers) in two halves of 32 columns. 2^x runs on
       // MUFU in f32 (measured faster here than packed-f16 MUFU or the FMA-pipe exp2_poly2, which
       // full tiles can route kPolyPairs of every 16 pairs to). Masked keys give ex2(-inf) = 0.
       auto softmax_row = [&](auto poly_tag) {
@@ -426,7 +437,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               sum2a = f2_add(sum2a, f2_pack(p0, p1));
             pw[i2] = pack_bf16(p0, p1);
           }
-          tmem_st32_async(t_s + 32 * half, pw);
+          tmem_st32_async(t_p + 32 * half, pw);
         }
         tmem_st_wait();   // P complete in TMEM before the arrive below releases it to the MMA
       };
@@ -476,7 +487,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int t = min(max(__ldg(P.perm + (size_t)u * P.N + p), 0), P.N - 1);
         dst = P.out + ((size_t)(u * P.N + t) * P.heads + h) * DH;
       }
-      const uint32_t o0 = tmem + 256 + lane_off, o1 = tmem + 384 + lane_off;
+      const uint32_t o0 = tmem + AttnTmem<DH>::kO + lane_off;
+      const uint32_t o1 = o0 + AttnTmem<DH>::kOStride;
       constexpr int kChunks = DH / 8;            // 8 or 10 chunks of 8 columns
       for (int c = grp; c < kChunks; c += 2) {    // the two groups split the columns
         uint32_t x0[8], x1[8];
