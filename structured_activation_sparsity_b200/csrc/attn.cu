@@ -225,9 +225,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* k_empty = k_full + NS;             // [NS]
   uint64_t* v_full = k_empty + NS;             // [NS]
   uint64_t* v_empty = v_full + NS;             // [NS]
-  uint64_t* s_full = v_empty + NS;             // [2]
-  uint64_t* p_full = s_full + 2;               // [2]
-  uint64_t* o_done = p_full + 2;
+  uint64_t* s_full = v_empty + NS;             // [2] S_w computed
+  uint64_t* s_free = s_full + 2;               // [2] S_w read into registers by its group
+  uint64_t* p_full = s_free + 2;               // [2] P_w written (and O_w rescaled if needed)
+  uint64_t* p_free = p_full + 2;               // [2] P*V into O_w done: P_w and O_w reusable
+  uint64_t* o_done = p_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -248,7 +250,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(s_full + w, 1);
+      mbar_init(s_free + w, 128);
       mbar_init(p_full + w, 128);
+      mbar_init(p_free + w, 1);
     }
     mbar_init(o_done, 1);
     *abort = 0;
@@ -330,16 +334,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                          idesc_pv_tail, acc | (kk > 0));
         }
         umma_commit(v_empty + st);
+        umma_commit(p_free + w);
         return true;
       };
       if (ok) tc_fence_after();
       if (ok && ntiles > 0) ok = issue_qk(0);
       if (ok && ntiles > 1) ok = issue_qk(1);
       for (int n = 0; ok && n < ntiles; ++n) {
-        ok = issue_pv(n);
-        // S_w of tile n+2 overwrites P_w of tile n: issued after that P*V, and tcgen05.mma
-        // operations of one thread execute in order.
-        if (ok && n + 2 < ntiles) ok = issue_qk(n + 2);
+        if constexpr (AttnTmem<DH>::kSeparateP) {
+          // S_w is free once its group has loaded it into registers: Q*K^T of tile n+2 runs
+          // while that group still computes P of tile n, so each group finds its next S ready.
+          if (n + 2 < ntiles) {
+            ok = mbar_wait(s_free + (n & 1), (n >> 1) & 1, abort, status);
+            if (ok) ok = issue_qk(n + 2);
+          }
+          if (ok) ok = issue_pv(n);
+        } else {
+          ok = issue_pv(n);
+          // P_w lies over S_w: S of tile n+2 may only be written after this P*V (tcgen05.mma
+          // operations of one thread execute in order).
+          if (ok && n + 2 < ntiles) ok = issue_qk(n + 2);
+        }
       }
       if (ok) umma_commit(o_done);
     }
@@ -372,6 +387,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld128(t_s, r);
 #pragma unroll
         for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(r[i]);
+      }
+      if constexpr (AttnTmem<DH>::kSeparateP) {
+        tc_fence_before();
+        mbar_arrive(s_free + grp);   // S_w may now be overwritten by Q*K^T of tile n+2
       }
       const int c0 = tiles.tile(n) * kBN;
       const bool full = tile_full(c0, P);
@@ -415,6 +434,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // over S_w, whose row is already in registers) in two halves of 32 columns. 2^x runs on
       // MUFU in f32 (measured faster here than packed-f16 MUFU or the FMA-pipe exp2_poly2, which
       // full tiles can route kPolyPairs of every 16 pairs to). Masked keys give ex2(-inf) = 0.
+      // The group's previous P*V must be done before P_w is rewritten and O_w rescaled (with P
+      // over S it already is: this S was computed after that P*V).
+      if constexpr (AttnTmem<DH>::kSeparateP) {
+        if (j > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(p_free + grp, (j - 1) & 1, abort, status));
+          if (!ok) break;
+          tc_fence_after();
+        }
+      }
       auto softmax_row = [&](auto poly_tag) {
         constexpr bool kPoly = decltype(poly_tag)::value;
 #pragma unroll
