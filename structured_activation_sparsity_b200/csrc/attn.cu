@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               sum2b = f2_add(sum2b, f2_pack(p0, p1));
             else
               sum2a = f2_add(sum2a, f2_pack(p0, p1));
-            pw[i2] = pack_bf16(p0, p1);
+            pw[i2] = pack_bf16_pos(p0, p1);   // p >= 0: integer-pipe rounding
           }
           tmem_st32_async(t_p + 32 * half, pw);
         }

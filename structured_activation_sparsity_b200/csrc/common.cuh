@@ -326,6 +326,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Two non-negative finite floats to a bf16 pair (lo in the low half), rounded half-up, on the
+// integer pipes: an add that carries the rounding into bit 16, then one byte permute taking both
+// high halves. Keeps the conversion off the XU pipe, which the exponentials already saturate.
+__device__ __forceinline__ uint32_t pack_bf16_pos(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
