@@ -196,9 +196,10 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float&
 // group turns its S tile into probabilities, the tensor core runs the other group's P*V and the
 // next Q*K^T. Each group keeps its own running max m, sum l and accumulator O (in TMEM); at the
 // end the two partial results of every row are merged.
-//   warp 0        TMA producer (Q once; K and V tiles into two separate rings)
-//   warp 1        TMEM allocator and tcgen05.mma issuer
-//   warps 2-3     idle (they complete the producer warpgroup for the register split)
+//   warp 0        TMA producer (Q once; K and V tiles into a ring of stages)
+//   warp 1        TMEM allocator and Q*K^T issuer
+//   warp 2        P*V issuer
+//   warp 3        idle (completes the producer warpgroup for the register split)
 //   warps 4-7     softmax group 0 (one thread per query row = TMEM lane)
 //   warps 8-11    softmax group 1
 // TMEM columns (AttnTmem): S0 [0,128), S1 [128,256); dh 64: O0 [256,320), O1 [320,384),
@@ -221,15 +222,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   float* s_l = s_m + 2 * kBM;                              // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;                 // [NS]
-  uint64_t* k_empty = k_full + NS;             // [NS]
-  uint64_t* v_full = k_empty + NS;             // [NS]
-  uint64_t* v_empty = v_full + NS;             // [NS]
-  uint64_t* s_full = v_empty + NS;             // [2] S_w computed
+  uint64_t* kv_full = bars + 1;                // [NS] K and V of a stage landed
+  uint64_t* kv_empty = kv_full + NS;           // [NS] P*V of the stage's tile done (K, V free)
+  uint64_t* s_full = kv_empty + NS;            // [2] S_w computed
   uint64_t* s_free = s_full + 2;               // [2] S_w read into registers by its group
   uint64_t* p_full = s_free + 2;               // [2] P_w written (and O_w rescaled if needed)
-  uint64_t* p_free = p_full + 2;               // [2] P*V into O_w done: P_w and O_w reusable
-  uint64_t* o_done = p_free + 2;
+  uint64_t* o_done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -243,16 +241,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < NS; ++i) {
-      mbar_init(k_full + i, 1);
-      mbar_init(k_empty + i, 1);
-      mbar_init(v_full + i, 1);
-      mbar_init(v_empty + i, 1);
+      mbar_init(kv_full + i, 1);
+      mbar_init(kv_empty + i, 1);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(s_full + w, 1);
       mbar_init(s_free + w, 128);
       mbar_init(p_full + w, 128);
-      mbar_init(p_free + w, 1);
     }
     mbar_init(o_done, 1);
     *abort = 0;
@@ -264,6 +259,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // An mbarrier wait whose result gates the next instruction costs ~150 cycles even when the
+  // phase has already completed, so the two MMA streams get their own issuing threads: one for
+  // Q*K^T, one for P*V. Their data dependencies all go through the barriers above.
   if (warp < 4) {
     setmaxnreg_dec<kRegsProducer>();
     if (warp == 0 && lane == 0) {
@@ -276,33 +274,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (kHasTail) tma_load_3d(smem + S::kQ + S::kMain, &tq_tail, q_full, 64, q0, uh);
       for (int n = 0; n < ntiles; ++n) {
         const int st = n % NS;
-        const uint32_t ph = ((n / NS) - 1) & 1;
         const int c0 = tiles.tile(n) * kBN;
-        if (n >= NS && !mbar_wait(k_empty + st, ph, abort, status)) break;
+        if (n >= NS && !mbar_wait(kv_empty + st, ((n / NS) - 1) & 1, abort, status)) break;
         uint8_t* kb = smem + S::kK + st * S::kTileBytes;
-        mbar_expect_tx(k_full + st, S::kMain + S::kTailBytes);
-        tma_load_3d(kb, &tk, k_full + st, 0, c0, uh);
-        if (kHasTail) tma_load_3d(kb + S::kMain, &tk_tail, k_full + st, 64, c0, uh);
-        if (n >= NS && !mbar_wait(v_empty + st, ph, abort, status)) break;
         uint8_t* vb = smem + S::kV + st * S::kTileBytes;
-        mbar_expect_tx(v_full + st, S::kMain + S::kTailBytes);
-        tma_load_3d(vb, &tv, v_full + st, 0, c0, uh);
-        if (kHasTail) tma_load_3d(vb + S::kMain, &tv_tail, v_full + st, 64, c0, uh);
+        mbar_expect_tx(kv_full + st, 2 * (S::kMain + S::kTailBytes));
+        tma_load_3d(kb, &tk, kv_full + st, 0, c0, uh);
+        if (kHasTail) tma_load_3d(kb + S::kMain, &tk_tail, kv_full + st, 64, c0, uh);
+        tma_load_3d(vb, &tv, kv_full + st, 0, c0, uh);
+        if (kHasTail) tma_load_3d(vb + S::kMain, &tv_tail, kv_full + st, 64, c0, uh);
       }
     } else if (warp == 1 && lane == 0) {
-      // ------------------------------ MMA issuer --------------------------------
+      // ------------------------------ Q*K^T issuer ------------------------------
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, 64, false, true);
-      constexpr uint32_t idesc_pv_tail = idesc_bf16_f32(kBM, 16, false, true);
       const uint32_t q_addr = smem_u32(smem + S::kQ);
       bool ok = mbar_wait(q_full, 0, abort, status);
-      // S_w = Q K_n^T for tile n (w = n % 2); K's stage is released when it completes.
-      auto issue_qk = [&](int n) -> bool {
-        const int st = n % NS;
-        if (!mbar_wait(k_full + st, (n / NS) & 1, abort, status)) return false;
+      for (int n = 0; ok && n < ntiles; ++n) {
+        const int st = n % NS, w = n & 1;
+        if (n >= 2) {
+          // S_w is reusable once tile n-2's S is in its group's registers (P apart from S), or
+          // once tile n-2's P*V is done (P over S).
+          if constexpr (AttnTmem<DH>::kSeparateP)
+            ok = mbar_wait(s_free + w, ((n - 2) >> 1) & 1, abort, status);
+          else
+            ok = mbar_wait(kv_empty + (n - 2) % NS, ((n - 2) / NS) & 1, abort, status);
+          if (!ok) break;
+        }
+        if (!(ok = mbar_wait(kv_full + st, (n / NS) & 1, abort, status))) break;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + S::kK + st * S::kTileBytes);
-        const uint32_t d = tmem + AttnTmem<DH>::kS + (n & 1) * AttnTmem<DH>::kSStride;
+        const uint32_t d = tmem + AttnTmem<DH>::kS + w * AttnTmem<DH>::kSStride;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_bf16_ss(d, smem_desc(q_addr + kk * 32, 16, 1024, kSwizzle128B),
@@ -310,15 +311,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (kHasTail)
           umma_bf16_ss(d, smem_desc(q_addr + S::kMain, 16, 256, kSwizzle32B),
                        smem_desc(k_addr + S::kMain, 16, 256, kSwizzle32B), idesc_qk, 1);
-        umma_commit(s_full + (n & 1));
-        umma_commit(k_empty + st);
-        return true;
-      };
-      // O_w (+)= P_w V_n, P_w read from TMEM, once group w has written it for tile n.
-      auto issue_pv = [&](int n) -> bool {
+        umma_commit(s_full + w);
+      }
+    } else if (warp == 2 && lane == 0) {
+      // ------------------------------ P*V issuer --------------------------------
+      // P_w of tile n exists only after S of tile n, which followed that stage's K/V landing
+      // (observed by the Q*K^T issuer), so V is ready whenever P is.
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, 64, false, true);
+      constexpr uint32_t idesc_pv_tail = idesc_bf16_f32(kBM, 16, false, true);
+      bool ok = true;
+      for (int n = 0; ok && n < ntiles; ++n) {
         const int st = n % NS, w = n & 1;
-        if (!mbar_wait(p_full + w, (n >> 1) & 1, abort, status)) return false;
-        if (!mbar_wait(v_full + st, (n / NS) & 1, abort, status)) return false;
+        if (!(ok = mbar_wait(p_full + w, (n >> 1) & 1, abort, status))) break;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kTileBytes);
         const uint32_t a = tmem + AttnTmem<DH>::kP + w * AttnTmem<DH>::kPStride;   // P_w
@@ -333,28 +337,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                          smem_desc(v_addr + S::kMain + kk * 512, kBN * 32, 256, kSwizzle32B),
                          idesc_pv_tail, acc | (kk > 0));
         }
-        umma_commit(v_empty + st);
-        umma_commit(p_free + w);
-        return true;
-      };
-      if (ok) tc_fence_after();
-      if (ok && ntiles > 0) ok = issue_qk(0);
-      if (ok && ntiles > 1) ok = issue_qk(1);
-      for (int n = 0; ok && n < ntiles; ++n) {
-        if constexpr (AttnTmem<DH>::kSeparateP) {
-          // S_w is free once its group has loaded it into registers: Q*K^T of tile n+2 runs
-          // while that group still computes P of tile n, so each group finds its next S ready.
-          if (n + 2 < ntiles) {
-            ok = mbar_wait(s_free + (n & 1), (n >> 1) & 1, abort, status);
-            if (ok) ok = issue_qk(n + 2);
-          }
-          if (ok) ok = issue_pv(n);
-        } else {
-          ok = issue_pv(n);
-          // P_w lies over S_w: S of tile n+2 may only be written after this P*V (tcgen05.mma
-          // operations of one thread execute in order).
-          if (ok && n + 2 < ntiles) ok = issue_qk(n + 2);
-        }
+        umma_commit(kv_empty + st);   // Q*K^T of this tile finished before its P existed
       }
       if (ok) umma_commit(o_done);
     }
@@ -437,8 +420,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // The group's previous P*V must be done before P_w is rewritten and O_w rescaled (with P
       // over S it already is: this S was computed after that P*V).
       if constexpr (AttnTmem<DH>::kSeparateP) {
-        if (j > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(p_free + grp, (j - 1) & 1, abort, status));
+        if (n >= 2) {   // P*V of tile n-2 (this group's previous tile) released its stage
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(kv_empty + (n - 2) % NS, ((n - 2) / NS) & 1, abort, status));
           if (!ok) break;
           tc_fence_after();
         }
