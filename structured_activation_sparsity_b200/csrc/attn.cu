@@ -371,9 +371,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(r[i]);
       }
+      // Has P*V of this group's previous tile (n-2) released P_w and O_w? Tested now, used after
+      // the row max, so the test's latency is hidden behind the max.
+      bool prev_pv_done = true;
       if constexpr (AttnTmem<DH>::kSeparateP) {
         tc_fence_before();
         mbar_arrive(s_free + grp);   // S_w may now be overwritten by Q*K^T of tile n+2
+        if (n >= 2) prev_pv_done = mbar_test(kv_empty + (n - 2) % NS, ((n - 2) / NS) & 1);
       }
       const int c0 = tiles.tile(n) * kBN;
       const bool full = tile_full(c0, P);
@@ -421,9 +425,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // over S it already is: this S was computed after that P*V).
       if constexpr (AttnTmem<DH>::kSeparateP) {
         if (n >= 2) {   // P*V of tile n-2 (this group's previous tile) released its stage
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(kv_empty + (n - 2) % NS, ((n - 2) / NS) & 1, abort, status));
-          if (!ok) break;
+          if (!__all_sync(0xffffffffu, prev_pv_done)) {
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(kv_empty + (n - 2) % NS, ((n - 2) / NS) & 1, abort, status));
+            if (!ok) break;
+          }
           tc_fence_after();
         }
       }
