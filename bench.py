@@ -244,12 +244,18 @@ def time_steps(sets, steps, stream, dist=None):
 
 
 def max_over_ranks(x, dist, dev):
+    """The slowest rank's time: the job is done when every replica is."""
     if dist is None:
         return x
     import torch
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, units_per_step: int, steps: int, seconds: float) -> float:
+    """Weak scaling: every rank runs its own replica, so the job processes world x the units."""
+    return world * units_per_step * steps / seconds
 
 
 def run_ours(args, wl, rank, world, local_rank, dist):
@@ -286,7 +292,7 @@ def run_ours(args, wl, rank, world, local_rank, dist):
     clocks.stop()
     t = max_over_ranks(t, dist, dev)
     ms_per_step = t / args.steps * 1e3
-    value = world * tokens_per_step * args.steps / t
+    value = job_throughput(world, tokens_per_step, args.steps, t)
 
     # ---- per-kernel durations: the same K steps again with launch tracing on ---------------------
     L.sparsesam_trace_start(8 * args.steps + 16)
@@ -306,7 +312,7 @@ def run_ours(args, wl, rank, world, local_rank, dist):
         for i in range(args.warmup):
             dense_sets[i % n_sets].step(stream)
     td = max_over_ranks(time_steps(dense_sets, args.steps, stream, dist), dist, dev)
-    dense_value = world * tokens_per_step * args.steps / td
+    dense_value = job_throughput(world, tokens_per_step, args.steps, td)
     dpat = dense_sets[0].pattern
     dense_flops = (workloads.attn_flops(wl.units, wl.unit_tokens, wl.heads, wl.head_dim, dpat.rho)
                    + workloads.mlp_flops(wl.batch * dpat.keep, wl.dim, wl.hidden))
@@ -340,7 +346,7 @@ def run_ours(args, wl, rank, world, local_rank, dist):
     ev1.record(stream)
     torch.cuda.synchronize()
     te = max_over_ranks(ev0.elapsed_time(ev1) / 1e3, dist, dev)
-    e2e_value = world * tokens_per_step * args.steps / te
+    e2e_value = job_throughput(world, tokens_per_step, args.steps, te)
 
     if L.sparsesam_device_status(stream) != L.SS_OK:
         raise RuntimeError("a device wait timed out during timing")
