@@ -60,16 +60,19 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* keep, uint16_t*
 constexpr int kGemmThreads = 320;
 constexpr int kEpiThreads = 256;
 
-template <int BN>
+// KSUB 64-wide K sub-blocks per pipeline stage: each full/empty handshake (an mbarrier wait costs
+// ~150 cycles of latency on the thread that gates on it) then covers KSUB x 4 MMAs.
+template <int BN, int KSUB>
 struct GemmCfg {
-  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
-  static constexpr int kABytes = 128 * 128;       // 128 rows x 64 bf16
-  static constexpr int kBBytes = BN * 128;        // BN rows x 64 bf16
-  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kABytes = 128 * 128;       // 128 rows x 64 bf16 per sub-block
+  static constexpr int kBBytes = BN * 128;        // BN rows x 64 bf16 per sub-block
+  static constexpr int kStageBytes = KSUB * (kABytes + kBBytes);
+  static constexpr int kStages = (192 * 1024) / kStageBytes;
   static constexpr int kBar = kStages * kStageBytes;
   static constexpr int kAlloc = kBar + 512 + 1024;
   static constexpr int kTmemCols = 2 * BN;        // two accumulators
   static constexpr int kHalf = BN / 2;            // columns per epilogue warp
+  static_assert(kStages >= 2, "at least two stages");
 };
 
 __device__ __forceinline__ float bf16_to_f(uint16_t v) { return __uint_as_float(uint32_t(v) << 16); }
@@ -134,11 +137,11 @@ __device__ __forceinline__ void epilogue32(const GemmEpilogue& ep, const GemmSha
   }
 }
 
-template <int BN>
+template <int BN, int KSUB>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
            const GemmShape g, const GemmEpilogue ep, int* status) {
-  using G = GemmCfg<BN>;
+  using G = GemmCfg<BN, KSUB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -191,17 +194,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
         int m, n, s, kb0, kb1;
         decode(u, m, n, s, kb0, kb1);
-        const int nkb = kb1 - kb0, rot = u % nkb;
-        for (int j = 0; j < nkb; ++j, ++it) {
-          const int kb = kb0 + (j + rot) % nkb;   // rotated start: CTAs spread over L2 slices
+        const int nst = (kb1 - kb0) / KSUB, rot = u % nst;
+        for (int j = 0; j < nst; ++j, ++it) {
+          const int kb = kb0 + ((j + rot) % nst) * KSUB;   // rotated start: spread over L2 slices
           const int st = it % G::kStages;
           if (it >= G::kStages &&
               !(ok = mbar_wait(empty + st, ((it / G::kStages) - 1) & 1, abort, status)))
             break;
           uint8_t* sa = smem + st * G::kStageBytes;
+          uint8_t* sb = sa + KSUB * G::kABytes;
           mbar_expect_tx(full + st, G::kStageBytes);
-          tma_load_2d(sa, &ta, full + st, kb * 64, m * 128);
-          tma_load_2d(sa + G::kABytes, &tb, full + st, kb * 64, n * BN);
+#pragma unroll
+          for (int q = 0; q < KSUB; ++q) {
+            tma_load_2d(sa + q * G::kABytes, &ta, full + st, (kb + q) * 64, m * 128);
+            tma_load_2d(sb + q * G::kBBytes, &tb, full + st, (kb + q) * 64, n * BN);
+          }
         }
       }
     }
@@ -217,17 +224,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (i >= 2 && !(ok = mbar_wait(acc_empty + buf, ((i >> 1) - 1) & 1, abort, status))) break;
         tc_fence_after();
         const uint32_t d = tmem + buf * BN;
-        for (int j = 0; j < kb1 - kb0; ++j, ++it) {
+        const int nst = (kb1 - kb0) / KSUB;
+        bool ready = mbar_test(full + it % G::kStages, (it / G::kStages) & 1);
+        for (int j = 0; j < nst; ++j, ++it) {
           const int st = it % G::kStages;
-          if (!(ok = mbar_wait(full + st, (it / G::kStages) & 1, abort, status))) break;
+          if (!__builtin_expect(ready, 1) &&
+              !(ok = mbar_wait(full + st, (it / G::kStages) & 1, abort, status)))
+            break;
+          // test the next stage now: its latency hides behind this stage's MMA issue
+          if (j + 1 < nst) ready = mbar_test(full + (it + 1) % G::kStages, ((it + 1) / G::kStages) & 1);
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + st * G::kStageBytes);
-          const uint32_t b_addr = a_addr + G::kABytes;
+          const uint32_t b_addr = a_addr + KSUB * G::kABytes;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_ss(d, smem_desc(a_addr + kk * 32, 16, 1024, kSwizzle128B),
-                         smem_desc(b_addr + kk * 32, 16, 1024, kSwizzle128B), idesc,
-                         (j > 0 || kk > 0) ? 1u : 0u);
+          for (int q = 0; q < KSUB; ++q)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_ss(d, smem_desc(a_addr + q * G::kABytes + kk * 32, 16, 1024, kSwizzle128B),
+                           smem_desc(b_addr + q * G::kBBytes + kk * 32, 16, 1024, kSwizzle128B),
+                           idesc, (j > 0 || q > 0 || kk > 0) ? 1u : 0u);
           umma_commit(empty + st);
         }
         if (ok) umma_commit(acc_full + buf);
@@ -364,13 +379,13 @@ size_t gemm_partial_bytes(const GemmPlan& p) {
   return (size_t)p.m_tiles * p.n_tiles * p.splits * 128 * p.bn * 4;
 }
 
-template <int BN>
+template <int BN, int KSUB>
 static cudaError_t launch_gemm_bn(const CUtensorMap* ta, const CUtensorMap* tb, const GemmPlan& p,
                                   int M, int N, int Kd, const GemmEpilogue& ep, float* partial,
                                   int* counters, int sms, int* status, cudaStream_t st) {
-  using G = GemmCfg<BN>;
-  cudaError_t e =
-      cudaFuncSetAttribute(k_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kAlloc);
+  using G = GemmCfg<BN, KSUB>;
+  cudaError_t e = cudaFuncSetAttribute(k_gemm<BN, KSUB>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, G::kAlloc);
   if (e != cudaSuccess) return e;
   GemmShape g;
   g.M = M;
@@ -383,17 +398,26 @@ static cudaError_t launch_gemm_bn(const CUtensorMap* ta, const CUtensorMap* tb, 
   g.partial = partial;
   g.counters = counters;
   const int grid = p.units < sms ? p.units : sms;
-  k_gemm<BN><<<grid, kGemmThreads, G::kAlloc, st>>>(*ta, *tb, g, ep, status);
+  k_gemm<BN, KSUB><<<grid, kGemmThreads, G::kAlloc, st>>>(*ta, *tb, g, ep, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, const GemmPlan& p, int M,
                         int N, int Kd, const GemmEpilogue& ep, float* partial, int* counters,
                         int sms, int* status, cudaStream_t st) {
+  // Two sub-blocks per stage when every unit's k-range splits evenly (BN 256 keeps one: its
+  // 96 KB double stage would leave only two stages).
+  const int kb = Kd / 64;
+  const bool two = p.bn != 256 && kb % p.splits == 0 && (kb / p.splits) % 2 == 0;
   switch (p.bn) {
-    case 64: return launch_gemm_bn<64>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
-    case 128: return launch_gemm_bn<128>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
-    case 256: return launch_gemm_bn<256>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
+    case 64:
+      return two ? launch_gemm_bn<64, 2>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st)
+                 : launch_gemm_bn<64, 1>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
+    case 128:
+      return two ? launch_gemm_bn<128, 2>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st)
+                 : launch_gemm_bn<128, 1>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
+    case 256:
+      return launch_gemm_bn<256, 1>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
   }
   return cudaErrorInvalidValue;
 }
