@@ -36,9 +36,11 @@ METRIC = "Stripe-Sort attn + RC-MLP tokens/s per block; effective TFLOP/s vs bf1
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one attention launch, from the ncu capture
-# summarised in profiles/ (None until captured for the current kernel).
-ATTN_TRAFFIC_BYTES = {}
+# dram__bytes_read.sum + dram__bytes_write.sum of one attention launch on the ViT-B global block,
+# from the ncu --set full capture summarised in profiles/attn_vitb_global.md (cold caches; the
+# 6.3 MB output stays in L2 within the launch, so the write term is 0). Set to None whenever the
+# attention kernel changes until it is captured again.
+ATTN_TRAFFIC_BYTES = {"vitb_global": 18945536}
 
 
 def peaks():
