@@ -344,6 +344,7 @@ int sparsesam_attn(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k, cons
   ap.W = p.W;
   ap.g = p.g;
   ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dh));
+  ap.sms = sm_count();
   return cuda_err(traced("attn", st, [&] {
     return launch_attn(&tm[0], &tm[1], &tm[2], &tm[3], &tm[4], &tm[5], ap, dh, status, st);
   }));

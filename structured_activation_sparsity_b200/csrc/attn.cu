@@ -11,13 +11,12 @@
 // offset blocks [0, g) and [s(a), s(a)+W), i.e. at most two contiguous runs of 128-row key tiles.
 // The kernel derives that tile list from (b, nb, W, g) itself: no block list is read.
 //
-// One CTA = one (unit, head, 128-row query tile). Warp roles:
-//   warp 0     TMA producer (Q once, then K/V tiles into a 2-stage ring)
-//   warp 1     TMEM allocator and tcgen05.mma issuer (S = Q K^T, then O_tile = P V)
-//   warps 2-5  softmax: one thread per query row (TMEM lane), online softmax in fp32,
-//              P written to shared memory as bf16 (128B-swizzled, K-major A operand),
-//              O accumulated in registers; epilogue scatters rows to out[perm[p]].
-// TMEM holds both groups' S tiles, O accumulators and P tiles (AttnTmem).
+// Persistent: one CTA per SM walks the (unit, head, 128-row query tile) items. Per item a TMA
+// producer streams Q and the item's key tiles (K and V) into shared memory, two single-thread
+// issuers run S = Q K^T and O += P V on the tensor core with S, P and O in TMEM, and two softmax
+// warpgroups (one thread per query row) take alternate key tiles with an online softmax in fp32;
+// the epilogue merges the two groups' partial rows and scatters them to out[perm[p]].
+#include <algorithm>
 #include <type_traits>
 
 #include "common.cuh"
@@ -117,17 +116,18 @@ struct AttnSmem {
   static constexpr int kMain = kBM * 128;              // 128 rows x 128 B
   static constexpr int kTailBytes = kTail ? kBM * kTail * 2 : 0;
   static constexpr int kTileBytes = ((kMain + kTailBytes + 1023) / 1024) * 1024;
-  static constexpr int kStages = DH == 64 ? 6 : 5;     // depth of each of the K and V rings
-  static constexpr int kQ = 0;
-  static constexpr int kK = kTileBytes;
+  static constexpr int kStages = DH == 64 ? 5 : 4;     // depth of the K/V ring
+  static constexpr int kQ = 0;                         // two Q buffers (consecutive items)
+  static constexpr int kK = 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kML = kV + kStages * kTileBytes;  // float m[2][128], l[2][128]
   static constexpr int kBar = kML + 4 * kBM * 4;
   static constexpr int kBytes = kBar + 512;
   static constexpr int kAlloc = kBytes + 1024;         // slack to align the base to 1024
+  static_assert(kAlloc <= 227 * 1024, "attention shared memory above the per-CTA limit");
 };
 
-// The key tiles of one query tile, visited from a CTA-dependent starting point: CTAs that share
+// The key tiles of one query tile, visited from an item-dependent starting point: CTAs that share
 // key tiles (every query tile keeps the global block) then read different tiles at a time instead
 // of all hitting the same L2 lines. The softmax is order-independent up to rounding.
 struct KeyTiles {
@@ -142,7 +142,8 @@ struct KeyTiles {
 
 // Key tiles a query tile [q0, q_last] needs: the global rows [0, g*4b) and the band rows
 // [s(a_lo)*4b, (s(a_hi)+W)*4b), both clipped to N, as two (possibly merged) runs of tiles.
-__device__ __forceinline__ KeyTiles key_tiles(int q0, int q_last, const AttnParams& P) {
+__device__ __forceinline__ KeyTiles key_tiles(int q0, int q_last, int qt, int uh,
+                                              const AttnParams& P) {
   const int b4 = P.b * kStripes;
   const int a_lo = q0 / b4, a_hi = q_last / b4;
   const int s_lo = band_start(a_lo, P.W, P.nb), s_hi = band_start(a_hi, P.W, P.nb);
@@ -156,7 +157,7 @@ __device__ __forceinline__ KeyTiles key_tiles(int q0, int q_last, const AttnPara
     t.hi0 = max(t.hi0, t.hi1);
     t.lo1 = t.hi1 = t.hi0;
   }
-  t.rot = (int)((blockIdx.x * 5u + blockIdx.y * 3u) % (unsigned)max(1, t.count()));
+  t.rot = (int)((qt * 5u + uh * 3u) % (unsigned)max(1, t.count()));
   return t;
 }
 
@@ -191,12 +192,30 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float&
   p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
-// One CTA = one (unit, head, 128-row query tile). The key tiles are split between two softmax
-// warpgroups (tile n goes to group n % 2), so the MMA warp alternates between them: while one
-// group turns its S tile into probabilities, the tensor core runs the other group's P*V and the
-// next Q*K^T. Each group keeps its own running max m, sum l and accumulator O (in TMEM); at the
-// end the two partial results of every row are merged.
-//   warp 0        TMA producer (Q once; K and V tiles into a ring of stages)
+// Work item = (unit * heads + head, 128-row query tile), numbered head-major so that the CTAs
+// running at the same time share the K/V of a few heads in L2.
+struct Item {
+  int uh, q0, q_last;
+  KeyTiles tiles;
+};
+__device__ __forceinline__ Item item_of(int it, int nq, const AttnParams& P) {
+  Item I;
+  I.uh = it / nq;
+  const int qt = it - I.uh * nq;
+  I.q0 = qt * kBM;
+  I.q_last = min(I.q0 + kBM, P.N) - 1;
+  I.tiles = key_tiles(I.q0, I.q_last, qt, I.uh, P);
+  return I;
+}
+
+// Persistent: one CTA per SM walks the items it, it + gridDim.x, ... . The key tiles of an item
+// are split between two softmax warpgroups (tile n goes to group n % 2), so the MMA pipe
+// alternates between them: while one group turns its S tile into probabilities, the tensor core
+// runs the other group's P*V and the next Q*K^T. Each group keeps its own running max m, sum l
+// and accumulator O (in TMEM); at the end of an item the two partial results of every row are
+// merged and scattered. Q is double-buffered, so the next item's Q*K^T starts while this item's
+// last tiles and its epilogue are still running.
+//   warp 0        TMA producer (Q per item; K and V tiles into a ring of stages)
 //   warp 1        TMEM allocator and Q*K^T issuer
 //   warp 2        P*V issuer
 //   warp 3        idle (completes the producer warpgroup for the register split)
@@ -206,6 +225,7 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float&
 // P0 [384,448), P1 [448,512); dh 80: O0 [256,336), O1 [384,464) and P_w over the first 64
 // columns of S_w. P is bf16, two per column: the A operand of P*V. Keeping P apart from S (when
 // it fits) lets Q*K^T of tile n+2 start while P*V of tile n still reads P.
+// Barrier phases count uses across items: every role walks the same items and tiles in order.
 template <int DH>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -213,6 +233,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
            const __grid_constant__ CUtensorMap tk_tail, const __grid_constant__ CUtensorMap tv_tail,
            const AttnParams P, int* status) {
   using S = AttnSmem<DH>;
+  using T = AttnTmem<DH>;
   constexpr int NS = S::kStages;
   constexpr bool kHasTail = S::kTail > 0;
   extern __shared__ uint8_t smem_raw[];
@@ -221,33 +242,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   float* s_m = reinterpret_cast<float*>(smem + S::kML);   // [2][128]
   float* s_l = s_m + 2 * kBM;                              // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
-  uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;                // [NS] K and V of a stage landed
+  uint64_t* q_full = bars + 0;                 // [2] Q buffer landed
+  uint64_t* q_empty = q_full + 2;              // [2] Q*K^T of the buffer's item done
+  uint64_t* kv_full = q_empty + 2;             // [NS] K and V of a stage landed
   uint64_t* kv_empty = kv_full + NS;           // [NS] P*V of the stage's tile done (K, V free)
   uint64_t* s_full = kv_empty + NS;            // [2] S_w computed
   uint64_t* s_free = s_full + 2;               // [2] S_w read into registers by its group
   uint64_t* p_full = s_free + 2;               // [2] P_w written (and O_w rescaled if needed)
-  uint64_t* o_done = p_full + 2;
+  uint64_t* o_done = p_full + 2;               // an item's last P*V done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int uh = blockIdx.y;
-  const int q0 = blockIdx.x * kBM;
-  const int q_last = min(q0 + kBM, P.N) - 1;
-  const KeyTiles tiles = key_tiles(q0, q_last, P);
-  const int ntiles = tiles.count();
+  const int nq = (P.N + kBM - 1) / kBM;
+  const int n_items = nq * P.U * P.heads;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full + i, 1);
+      mbar_init(q_empty + i, 1);
+      mbar_init(s_full + i, 1);
+      mbar_init(s_free + i, 128);
+      mbar_init(p_full + i, 128);
+    }
     for (int i = 0; i < NS; ++i) {
       mbar_init(kv_full + i, 1);
       mbar_init(kv_empty + i, 1);
-    }
-    for (int w = 0; w < 2; ++w) {
-      mbar_init(s_full + w, 1);
-      mbar_init(s_free + w, 128);
-      mbar_init(p_full + w, 128);
     }
     mbar_init(o_done, 1);
     *abort = 0;
@@ -269,49 +289,72 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
-      mbar_expect_tx(q_full, S::kMain + S::kTailBytes);
-      tma_load_3d(smem + S::kQ, &tq, q_full, 0, q0, uh);
-      if (kHasTail) tma_load_3d(smem + S::kQ + S::kMain, &tq_tail, q_full, 64, q0, uh);
-      for (int n = 0; n < ntiles; ++n) {
-        const int st = n % NS;
-        const int c0 = tiles.tile(n) * kBN;
-        if (n >= NS && !mbar_wait(kv_empty + st, ((n / NS) - 1) & 1, abort, status)) break;
-        uint8_t* kb = smem + S::kK + st * S::kTileBytes;
-        uint8_t* vb = smem + S::kV + st * S::kTileBytes;
-        mbar_expect_tx(kv_full + st, 2 * (S::kMain + S::kTailBytes));
-        tma_load_3d(kb, &tk, kv_full + st, 0, c0, uh);
-        if (kHasTail) tma_load_3d(kb + S::kMain, &tk_tail, kv_full + st, 64, c0, uh);
-        tma_load_3d(vb, &tv, kv_full + st, 0, c0, uh);
-        if (kHasTail) tma_load_3d(vb + S::kMain, &tv_tail, kv_full + st, 64, c0, uh);
+      bool ok = true;
+      int gn = 0;   // tiles loaded so far (all items)
+      for (int it = blockIdx.x, li = 0; ok && it < n_items; it += gridDim.x, ++li) {
+        const Item I = item_of(it, nq, P);
+        const int qb = li & 1;
+        if (li >= 2 && !(ok = mbar_wait(q_empty + qb, ((li >> 1) - 1) & 1, abort, status))) break;
+        uint8_t* qbuf = smem + S::kQ + qb * S::kTileBytes;
+        mbar_expect_tx(q_full + qb, S::kMain + S::kTailBytes);
+        tma_load_3d(qbuf, &tq, q_full + qb, 0, I.q0, I.uh);
+        if (kHasTail) tma_load_3d(qbuf + S::kMain, &tq_tail, q_full + qb, 64, I.q0, I.uh);
+        const int nt = I.tiles.count();
+        for (int n = 0; n < nt; ++n, ++gn) {
+          const int st = gn % NS;
+          const int c0 = I.tiles.tile(n) * kBN;
+          if (gn >= NS && !(ok = mbar_wait(kv_empty + st, ((gn / NS) - 1) & 1, abort, status)))
+            break;
+          uint8_t* kb = smem + S::kK + st * S::kTileBytes;
+          uint8_t* vb = smem + S::kV + st * S::kTileBytes;
+          mbar_expect_tx(kv_full + st, 2 * (S::kMain + S::kTailBytes));
+          tma_load_3d(kb, &tk, kv_full + st, 0, c0, I.uh);
+          if (kHasTail) tma_load_3d(kb + S::kMain, &tk_tail, kv_full + st, 64, c0, I.uh);
+          tma_load_3d(vb, &tv, kv_full + st, 0, c0, I.uh);
+          if (kHasTail) tma_load_3d(vb + S::kMain, &tv_tail, kv_full + st, 64, c0, I.uh);
+        }
       }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------ Q*K^T issuer ------------------------------
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
-      const uint32_t q_addr = smem_u32(smem + S::kQ);
-      bool ok = mbar_wait(q_full, 0, abort, status);
-      for (int n = 0; ok && n < ntiles; ++n) {
-        const int st = n % NS, w = n & 1;
-        if (n >= 2) {
-          // S_w is reusable once tile n-2's S is in its group's registers (P apart from S), or
-          // once tile n-2's P*V is done (P over S).
-          if constexpr (AttnTmem<DH>::kSeparateP)
-            ok = mbar_wait(s_free + w, ((n - 2) >> 1) & 1, abort, status);
-          else
-            ok = mbar_wait(kv_empty + (n - 2) % NS, ((n - 2) / NS) & 1, abort, status);
-          if (!ok) break;
-        }
-        if (!(ok = mbar_wait(kv_full + st, (n / NS) & 1, abort, status))) break;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + S::kK + st * S::kTileBytes);
-        const uint32_t d = tmem + AttnTmem<DH>::kS + w * AttnTmem<DH>::kSStride;
+      bool ok = true;
+      int gn = 0;
+      int uses[2] = {0, 0};     // tiles computed into S_w so far
+      int last[2] = {0, 0};     // global index of the tile that last used S_w
+      for (int it = blockIdx.x, li = 0; ok && it < n_items; it += gridDim.x, ++li) {
+        const Item I = item_of(it, nq, P);
+        const int qb = li & 1;
+        if (!(ok = mbar_wait(q_full + qb, (li >> 1) & 1, abort, status))) break;
+        const uint32_t q_addr = smem_u32(smem + S::kQ + qb * S::kTileBytes);
+        const int nt = I.tiles.count();
+        for (int n = 0; n < nt; ++n, ++gn) {
+          const int st = gn % NS, w = n & 1;
+          if (uses[w] > 0) {
+            // S_w is reusable once its previous tile's S is in its group's registers (P apart
+            // from S), or once that tile's P*V is done (P over S).
+            if constexpr (T::kSeparateP)
+              ok = mbar_wait(s_free + w, (uses[w] - 1) & 1, abort, status);
+            else
+              ok = mbar_wait(kv_empty + last[w] % NS, (last[w] / NS) & 1, abort, status);
+            if (!ok) break;
+          }
+          if (!(ok = mbar_wait(kv_full + st, (gn / NS) & 1, abort, status))) break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(smem + S::kK + st * S::kTileBytes);
+          const uint32_t d = tmem + T::kS + w * T::kSStride;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_bf16_ss(d, smem_desc(q_addr + kk * 32, 16, 1024, kSwizzle128B),
-                       smem_desc(k_addr + kk * 32, 16, 1024, kSwizzle128B), idesc_qk, kk > 0);
-        if (kHasTail)
-          umma_bf16_ss(d, smem_desc(q_addr + S::kMain, 16, 256, kSwizzle32B),
-                       smem_desc(k_addr + S::kMain, 16, 256, kSwizzle32B), idesc_qk, 1);
-        umma_commit(s_full + w);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ss(d, smem_desc(q_addr + kk * 32, 16, 1024, kSwizzle128B),
+                         smem_desc(k_addr + kk * 32, 16, 1024, kSwizzle128B), idesc_qk, kk > 0);
+          if (kHasTail)
+            umma_bf16_ss(d, smem_desc(q_addr + S::kMain, 16, 256, kSwizzle32B),
+                         smem_desc(k_addr + S::kMain, 16, 256, kSwizzle32B), idesc_qk, 1);
+          umma_commit(s_full + w);
+          ++uses[w];
+          last[w] = gn;
+        }
+        if (!ok) break;
+        umma_commit(q_empty + qb);   // the Q buffer is free once this item's Q*K^T are done
       }
     } else if (warp == 2 && lane == 0) {
       // ------------------------------ P*V issuer --------------------------------
@@ -320,26 +363,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, 64, false, true);
       constexpr uint32_t idesc_pv_tail = idesc_bf16_f32(kBM, 16, false, true);
       bool ok = true;
-      for (int n = 0; ok && n < ntiles; ++n) {
-        const int st = n % NS, w = n & 1;
-        if (!(ok = mbar_wait(p_full + w, (n >> 1) & 1, abort, status))) break;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kTileBytes);
-        const uint32_t a = tmem + AttnTmem<DH>::kP + w * AttnTmem<DH>::kPStride;   // P_w
-        const uint32_t d = tmem + AttnTmem<DH>::kO + w * AttnTmem<DH>::kOStride;
-        const uint32_t acc = n >= 2;
+      int gn = 0;
+      int uses[2] = {0, 0};   // P_w handed over so far (p_full phases)
+      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+        const int nt = item_of(it, nq, P).tiles.count();
+        for (int n = 0; n < nt; ++n, ++gn) {
+          const int st = gn % NS, w = n & 1;
+          if (!(ok = mbar_wait(p_full + w, uses[w] & 1, abort, status))) break;
+          ++uses[w];
+          tc_fence_after();
+          const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kTileBytes);
+          const uint32_t a = tmem + T::kP + w * T::kPStride;   // P_w
+          const uint32_t d = tmem + T::kO + w * T::kOStride;
+          // The first tile of each group overwrites O_w: its group released the previous item's
+          // O (read in the epilogue) before handing over this P.
+          const uint32_t acc = n >= 2;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          umma_bf16_ts(d, a + kk * 8, smem_desc(v_addr + kk * 2048, kBN * 128, 1024, kSwizzle128B),
-                       idesc_pv, acc | (kk > 0));
-          if (kHasTail)
-            umma_bf16_ts(d + 64, a + kk * 8,
-                         smem_desc(v_addr + S::kMain + kk * 512, kBN * 32, 256, kSwizzle32B),
-                         idesc_pv_tail, acc | (kk > 0));
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            umma_bf16_ts(d, a + kk * 8, smem_desc(v_addr + kk * 2048, kBN * 128, 1024, kSwizzle128B),
+                         idesc_pv, acc | (kk > 0));
+            if (kHasTail)
+              umma_bf16_ts(d + 64, a + kk * 8,
+                           smem_desc(v_addr + S::kMain + kk * 512, kBN * 32, 256, kSwizzle32B),
+                           idesc_pv_tail, acc | (kk > 0));
+          }
+          umma_commit(kv_empty + st);   // Q*K^T of this tile finished before its P existed
         }
-        umma_commit(kv_empty + st);   // Q*K^T of this tile finished before its P existed
+        if (!ok) break;
+        umma_commit(o_done);   // phase = the item's parity in this CTA's sequence
       }
-      if (ok) umma_commit(o_done);
     }
   } else {
     setmaxnreg_inc<kRegsSoftmax>();
@@ -347,183 +399,209 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int grp = (warp - 4) >> 2;                    // 0 or 1
     const int row = 32 * (warp & 3) + lane;             // TMEM lane == query row
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
-    const uint32_t t_s = tmem + AttnTmem<DH>::kS + grp * AttnTmem<DH>::kSStride + lane_off;
-    const uint32_t t_p = tmem + AttnTmem<DH>::kP + grp * AttnTmem<DH>::kPStride + lane_off;
-    const uint32_t t_o = tmem + AttnTmem<DH>::kO + grp * AttnTmem<DH>::kOStride + lane_off;
-    const int qrow = q0 + row;
+    const uint32_t t_s = tmem + T::kS + grp * T::kSStride + lane_off;
+    const uint32_t t_p = tmem + T::kP + grp * T::kPStride + lane_off;
+    const uint32_t t_o = tmem + T::kO + grp * T::kOStride + lane_off;
     const int b4 = P.b * kStripes;
-    const int a_q = min(qrow, P.N - 1) / b4;
-    const int s_q = band_start(a_q, P.W, P.nb);
-    const int band_lo = s_q * b4, band_hi = (s_q + P.W) * b4, glob_hi = P.g * b4;
     const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
-    float m_ref = -INFINITY, l_run = 0.f;
     bool ok = true;
-    int j = 0;
-    for (int n = grp; n < ntiles; n += 2, ++j) {
-      // Warp-collective wait: either every lane goes on to the .sync.aligned TMEM ops or none.
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full + grp, j & 1, abort, status));
-      if (!ok) break;
-      tc_fence_after();
-      float sv[kBN];
-      {
-        uint32_t r[128];
-        tmem_ld128(t_s, r);
-#pragma unroll
-        for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(r[i]);
-      }
-      // Has P*V of this group's previous tile (n-2) released P_w and O_w? Tested now, used after
-      // the row max, so the test's latency is hidden behind the max.
-      bool prev_pv_done = true;
-      if constexpr (AttnTmem<DH>::kSeparateP) {
-        tc_fence_before();
-        mbar_arrive(s_free + grp);   // S_w may now be overwritten by Q*K^T of tile n+2
-        if (n >= 2) prev_pv_done = mbar_test(kv_empty + (n - 2) % NS, ((n - 2) / NS) & 1);
-      }
-      const int c0 = tiles.tile(n) * kBN;
-      const bool full = tile_full(c0, P);
-      if (!full) {
-#pragma unroll
-        for (int i = 0; i < kBN; ++i) {
-          const int c = c0 + i;
-          const bool kept = c < P.N && (c < glob_hi || (c >= band_lo && c < band_hi));
-          if (!kept) sv[i] = -INFINITY;
-        }
-      }
-      // Row max: eight independent chains of 3-input max over elements k, k+8, k+16, ...
-      float mx[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = fmax3(sv[k], sv[k + 8], sv[k + 16]);
-#pragma unroll
-      for (int t = 3; t + 1 < 16; t += 2)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv[k + 8 * t], sv[k + 8 * t + 8]);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], sv[k + 8 * 15]);
-      const float x_max =
-          fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])), fmaxf(mx[6], mx[7])) *
-          P.scale_log2;
-      // Lazy rescale: the reference max moves only when the row max passes it by 2^8, so O in
-      // TMEM is rescaled on few tiles. The decision is warp-wide (TMEM ops are warp-collective);
-      // the rescale itself runs after P is written, when the S registers are free.
-      const bool grow = x_max > m_ref + kLazyRescale;
-      const bool rescale = __any_sync(0xffffffffu, grow);
-      float alpha = 1.f;
-      if (rescale) {
-        const float m_new = grow ? x_max : m_ref;
-        alpha = (m_ref == -INFINITY) ? 0.f : ex2_mufu(m_ref - m_new);
-        l_run *= alpha;
-        m_ref = m_new;
-      }
-      const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
-      const uint64_t nref2 = f2_pack(-ref, -ref);
-      uint64_t sum2a = 0, sum2b = 0;   // two packed partial sums (bit pattern 0 = +0.0f pair)
-      // P row as bf16 pairs (column i holds keys 2i, 2i+1), written to P_w (its own columns, or
-      // over S_w, whose row is already in registers) in two halves of 32 columns. 2^x runs on
-      // MUFU in f32 (measured faster here than packed-f16 MUFU or the FMA-pipe exp2_poly2, which
-      // full tiles can route kPolyPairs of every 16 pairs to). Masked keys give ex2(-inf) = 0.
-      // The group's previous P*V must be done before P_w is rewritten and O_w rescaled (with P
-      // over S it already is: this S was computed after that P*V).
-      if constexpr (AttnTmem<DH>::kSeparateP) {
-        if (n >= 2) {   // P*V of tile n-2 (this group's previous tile) released its stage
-          if (!__all_sync(0xffffffffu, prev_pv_done)) {
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(kv_empty + (n - 2) % NS, ((n - 2) / NS) & 1, abort, status));
-            if (!ok) break;
-          }
-          tc_fence_after();
-        }
-      }
-      auto softmax_row = [&](auto poly_tag) {
-        constexpr bool kPoly = decltype(poly_tag)::value;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pw[32];
-#pragma unroll
-          for (int i2 = 0; i2 < 32; ++i2) {
-            const int i = 64 * half + 2 * i2;
-            float x0, x1, p0, p1;
-            f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), scale2, nref2), x0, x1);
-            if (kPoly && (i2 & 15) < kPolyPairs) {
-              exp2_poly2(x0, x1, p0, p1);
-            } else {
-              p0 = ex2_mufu(x0);
-              p1 = ex2_mufu(x1);
-            }
-            if (i2 & 1)
-              sum2b = f2_add(sum2b, f2_pack(p0, p1));
-            else
-              sum2a = f2_add(sum2a, f2_pack(p0, p1));
-            pw[i2] = pack_bf16_pos(p0, p1);   // p >= 0: integer-pipe rounding
-          }
-          tmem_st32_async(t_p + 32 * half, pw);
-        }
-        tmem_st_wait();   // P complete in TMEM before the arrive below releases it to the MMA
-      };
-      if (full)
-        softmax_row(std::integral_constant<bool, true>());
-      else
-        softmax_row(std::integral_constant<bool, false>());
-      float sa0, sa1;
-      f2_unpack(f2_add(sum2a, sum2b), sa0, sa1);
-      l_run += sa0 + sa1;
-      if (rescale && j > 0) {
-        // O_w holds the group's earlier tiles: their P*V completed before this S was committed,
-        // and this tile's P*V is issued only after the arrive below.
-#pragma unroll 1
-        for (int c = 0; c < (DH + 31) / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_o + c * 32, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(t_o + c * 32, o);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(p_full + grp);
-    }
-    // ---- merge the two groups' partial rows and scatter them to out[u, perm[p], h, :] ----
-    s_m[grp * kBM + row] = m_ref;
-    s_l[grp * kBM + row] = l_run;
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, 0, abort, status));
-    tc_fence_after();
-    named_barrier(1, 256);
-    if (ok) {
-      const float m0 = s_m[row], m1 = s_m[kBM + row];
-      const float l0 = s_l[row], l1 = s_l[kBM + row];
-      const float mm = fmaxf(m0, m1);
-      const float a0 = (m0 == -INFINITY) ? 0.f : ex2_mufu(m0 - mm);
-      const float a1 = (m1 == -INFINITY) ? 0.f : ex2_mufu(m1 - mm);
-      const float L = l0 * a0 + l1 * a1;
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-      const float f0 = a0 * inv, f1 = a1 * inv;
-      const bool has0 = ntiles > 0, has1 = ntiles > 1;   // a group with no tile has no O
+    int gn0 = 0;    // global index of the item's first tile
+    int uses = 0;   // tiles of this group so far (s_full phases)
+    for (int it = blockIdx.x, li = 0; it < n_items; it += gridDim.x, ++li) {
+      const Item I = item_of(it, nq, P);
+      const int nt = I.tiles.count();
+      const int qrow = I.q0 + row;
+      // Destination row, resolved now so that the perm load is long done by the epilogue.
       const bool store = qrow < P.N;
       uint16_t* dst = nullptr;
       if (store) {
-        const int u = uh / P.heads, h = uh - (uh / P.heads) * P.heads;
+        const int u = I.uh / P.heads, h = I.uh - u * P.heads;
         const int p = blockmajor_to_canonical(qrow, P.b, P.L);
         const int t = min(max(__ldg(P.perm + (size_t)u * P.N + p), 0), P.N - 1);
         dst = P.out + ((size_t)(u * P.N + t) * P.heads + h) * DH;
       }
-      const uint32_t o0 = tmem + AttnTmem<DH>::kO + lane_off;
-      const uint32_t o1 = o0 + AttnTmem<DH>::kOStride;
-      constexpr int kChunks = DH / 8;            // 8 or 10 chunks of 8 columns
-      for (int c = grp; c < kChunks; c += 2) {    // the two groups split the columns
-        uint32_t x0[8], x1[8];
-        tmem_ld8(o0 + c * 8, x0);                 // every lane loads (warp-collective) ...
-        tmem_ld8(o1 + c * 8, x1);
-        float v[8];
+      const int a_q = min(qrow, P.N - 1) / b4;
+      const int s_q = band_start(a_q, P.W, P.nb);
+      const int band_lo = s_q * b4, band_hi = (s_q + P.W) * b4, glob_hi = P.g * b4;
+      float m_ref = -INFINITY, l_run = 0.f;
+      int j = 0;
+      for (int n = grp; ok && n < nt; n += 2, ++j) {
+        // Warp-collective wait: either every lane goes on to the .sync.aligned TMEM ops or none.
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full + grp, uses & 1, abort, status));
+        ++uses;
+        if (!ok) break;
+        tc_fence_after();
+        float sv[kBN];
+        {
+          uint32_t r[128];
+          tmem_ld128(t_s, r);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          v[i] = (has0 ? __uint_as_float(x0[i]) * f0 : 0.f) +
-                 (has1 ? __uint_as_float(x1[i]) * f1 : 0.f);
-        uint4 wv;
-        wv.x = pack_bf16(v[0], v[1]);
-        wv.y = pack_bf16(v[2], v[3]);
-        wv.z = pack_bf16(v[4], v[5]);
-        wv.w = pack_bf16(v[6], v[7]);
-        if (store) reinterpret_cast<uint4*>(dst)[c] = wv;   // ... only rows < N store
+          for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(r[i]);
+        }
+        // Has P*V of this group's previous tile (n-2) released P_w and O_w? Tested now, used
+        // after the row max, so the test's latency is hidden behind the max. (The previous
+        // item's P*V are all done: the epilogue waited for them.)
+        const int gprev = gn0 + n - 2;
+        bool prev_pv_done = true;
+        if constexpr (T::kSeparateP) {
+          tc_fence_before();
+          mbar_arrive(s_free + grp);   // S_w may now be overwritten by the next Q*K^T into it
+          if (n >= 2) prev_pv_done = mbar_test(kv_empty + gprev % NS, (gprev / NS) & 1);
+        }
+        const int c0 = I.tiles.tile(n) * kBN;
+        const bool full = tile_full(c0, P);
+        if (!full) {
+#pragma unroll
+          for (int i = 0; i < kBN; ++i) {
+            const int c = c0 + i;
+            const bool kept = c < P.N && (c < glob_hi || (c >= band_lo && c < band_hi));
+            if (!kept) sv[i] = -INFINITY;
+          }
+        }
+        // Row max: eight independent chains of 3-input max over elements k, k+8, k+16, ...
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmax3(sv[k], sv[k + 8], sv[k + 16]);
+#pragma unroll
+        for (int t = 3; t + 1 < 16; t += 2)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv[k + 8 * t], sv[k + 8 * t + 8]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], sv[k + 8 * 15]);
+        const float x_max = fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])),
+                                  fmaxf(mx[6], mx[7])) *
+                            P.scale_log2;
+        // Lazy rescale: the reference max moves only when the row max passes it by 2^8, so O in
+        // TMEM is rescaled on few tiles. The decision is warp-wide (TMEM ops are warp-collective);
+        // the rescale itself runs after P is written, when the S registers are free.
+        const bool grow = x_max > m_ref + kLazyRescale;
+        const bool rescale = __any_sync(0xffffffffu, grow);
+        float alpha = 1.f;
+        if (rescale) {
+          const float m_new = grow ? x_max : m_ref;
+          alpha = (m_ref == -INFINITY) ? 0.f : ex2_mufu(m_ref - m_new);
+          l_run *= alpha;
+          m_ref = m_new;
+        }
+        const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const uint64_t nref2 = f2_pack(-ref, -ref);
+        uint64_t sum2a = 0, sum2b = 0;   // two packed partial sums (bit pattern 0 = +0.0f pair)
+        // The group's previous P*V must be done before P_w is rewritten and O_w rescaled (with P
+        // over S it already is: this S was computed after that P*V).
+        if constexpr (T::kSeparateP) {
+          if (n >= 2) {
+            if (!__all_sync(0xffffffffu, prev_pv_done)) {
+              ok = __all_sync(0xffffffffu,
+                              mbar_wait(kv_empty + gprev % NS, (gprev / NS) & 1, abort, status));
+              if (!ok) break;
+            }
+            tc_fence_after();
+          }
+        }
+        // P row as bf16 pairs (column i holds keys 2i, 2i+1), written to P_w (its own columns, or
+        // over S_w, whose row is already in registers) in two halves of 32 columns. 2^x runs on
+        // MUFU in f32 (measured faster here than packed-f16 MUFU or the FMA-pipe exp2_poly2, which
+        // full tiles can route kPolyPairs of every 16 pairs to). Masked keys give ex2(-inf) = 0.
+        auto softmax_row = [&](auto poly_tag) {
+          constexpr bool kPoly = decltype(poly_tag)::value;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t pw[32];
+#pragma unroll
+            for (int i2 = 0; i2 < 32; ++i2) {
+              const int i = 64 * half + 2 * i2;
+              float x0, x1, p0, p1;
+              f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), scale2, nref2), x0, x1);
+              if (kPoly && (i2 & 15) < kPolyPairs) {
+                exp2_poly2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2_mufu(x0);
+                p1 = ex2_mufu(x1);
+              }
+              if (i2 & 1)
+                sum2b = f2_add(sum2b, f2_pack(p0, p1));
+              else
+                sum2a = f2_add(sum2a, f2_pack(p0, p1));
+              pw[i2] = pack_bf16_pos(p0, p1);   // p >= 0: integer-pipe rounding
+            }
+            tmem_st32_async(t_p + 32 * half, pw);
+          }
+          tmem_st_wait();   // P complete in TMEM before the arrive below releases it to the MMA
+        };
+        if (full)
+          softmax_row(std::integral_constant<bool, true>());
+        else
+          softmax_row(std::integral_constant<bool, false>());
+        float sa0, sa1;
+        f2_unpack(f2_add(sum2a, sum2b), sa0, sa1);
+        l_run += sa0 + sa1;
+        if (rescale && j > 0) {
+          // O_w holds the group's earlier tiles: their P*V completed before this S was committed,
+          // and this tile's P*V is issued only after the arrive below.
+#pragma unroll 1
+          for (int c = 0; c < (DH + 31) / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_o + c * 32, o);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(p_full + grp);
       }
+      // ---- merge both groups' partial rows and scatter them to out[u, perm[p], h, :] ----
+      // Every softmax thread passes both named barriers once per item, also after a failed wait.
+      s_m[grp * kBM + row] = m_ref;
+      s_l[grp * kBM + row] = l_run;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, li & 1, abort, status));
+      tc_fence_after();
+      named_barrier(1, 256);
+      constexpr int kCols = DH / 2;   // this group's output columns [grp*kCols, (grp+1)*kCols)
+      uint32_t x0[32], x1[32], y0[8], y1[8];   // columns 0-31 and (dh 80) 32-39 of O0, O1
+      float m0 = 0.f, m1 = 0.f, l0 = 0.f, l1 = 0.f;
+      if (ok) {
+        m0 = s_m[row];
+        m1 = s_m[kBM + row];
+        l0 = s_l[row];
+        l1 = s_l[kBM + row];
+        const uint32_t o0 = tmem + T::kO + lane_off + grp * kCols;
+        const uint32_t o1 = o0 + T::kOStride;
+        tmem_ld32_pair(o0, o1, x0, x1);
+        if constexpr (kCols > 32) tmem_ld8_pair(o0 + 32, o1 + 32, y0, y1);
+      }
+      // Both groups have read O0 and O1 (and m, l) before either hands the next item's first P
+      // to the P*V issuer, whose first MMA into O_w overwrites it.
+      tc_fence_before();
+      named_barrier(1, 256);
+      if (ok && store) {
+        const float mm = fmaxf(m0, m1);
+        const float a0 = (m0 == -INFINITY) ? 0.f : ex2_mufu(m0 - mm);
+        const float a1 = (m1 == -INFINITY) ? 0.f : ex2_mufu(m1 - mm);
+        const float L = l0 * a0 + l1 * a1;
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const float f0 = a0 * inv, f1 = a1 * inv;
+        // A group with no tile in this item has a stale O: select, do not multiply by zero.
+        const bool has0 = nt > 0, has1 = nt > 1;
+        uint4* out4 = reinterpret_cast<uint4*>(dst + grp * kCols);
+#pragma unroll
+        for (int c = 0; c < kCols / 8; ++c) {
+          float v[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t u0 = c < 4 ? x0[8 * c + i] : y0[i];
+            const uint32_t u1 = c < 4 ? x1[8 * c + i] : y1[i];
+            v[i] = (has0 ? __uint_as_float(u0) * f0 : 0.f) + (has1 ? __uint_as_float(u1) * f1 : 0.f);
+          }
+          uint4 wv;
+          wv.x = pack_bf16(v[0], v[1]);
+          wv.y = pack_bf16(v[2], v[3]);
+          wv.z = pack_bf16(v[4], v[5]);
+          wv.w = pack_bf16(v[6], v[7]);
+          out4[c] = wv;
+        }
+      }
+      gn0 += nt;
     }
   }
   tc_fence_before();
@@ -543,7 +621,8 @@ static cudaError_t launch_attn_dh(const CUtensorMap* tq, const CUtensorMap* tk,
   cudaError_t e = cudaFuncSetAttribute(k_attn<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        S::kAlloc);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.N + kBM - 1) / kBM, p.U * p.heads);
+  const int items = ((p.N + kBM - 1) / kBM) * p.U * p.heads;
+  dim3 grid(std::max(1, std::min(items, p.sms)));
   k_attn<DH><<<grid, kAttnThreads, S::kAlloc, st>>>(*tq, *tk, *tv, *tq_tail, *tk_tail, *tv_tail, p,
                                                     status);
   return cudaGetLastError();

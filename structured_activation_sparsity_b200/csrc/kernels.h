@@ -29,6 +29,7 @@ struct AttnParams {
   uint16_t* out;         // [U, N, heads, dh]
   int U, N, heads, L, b, nb, W, g;
   float scale_log2;      // log2(e) / sqrt(dh)
+  int sms;               // persistent CTAs to launch (one per SM)
 };
 // Block-sparse attention over the gathered sequences (tensor maps over [U*heads, N, dh]).
 cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
