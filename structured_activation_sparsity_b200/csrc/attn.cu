@@ -121,7 +121,12 @@ struct AttnSmem {
   static constexpr int kK = 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kML = kV + kStages * kTileBytes;  // float m[2][128], l[2][128]
-  static constexpr int kBar = kML + 4 * kBM * 4;
+  // Output staging: 128 rows of DH bf16, padded by 16 bytes so that the 32 rows a warp writes
+  // at once spread over all banks; then the rows' destination tokens.
+  static constexpr int kStageStride = DH * 2 + 16;
+  static constexpr int kStage = kML + 4 * kBM * 4;
+  static constexpr int kDst = kStage + kBM * kStageStride;
+  static constexpr int kBar = kDst + kBM * 4;
   static constexpr int kBytes = kBar + 512;
   static constexpr int kAlloc = kBytes + 1024;         // slack to align the base to 1024
   static_assert(kAlloc <= 227 * 1024, "attention shared memory above the per-CTA limit");
@@ -167,6 +172,14 @@ __device__ __forceinline__ KeyTiles key_tiles(int q0, int q_last, int qt, int uh
 // blocks and take the element mask; so does the ragged last key tile.
 __device__ __forceinline__ bool tile_full(int c0, const AttnParams& P) {
   return (P.b * kStripes) % kBN == 0 && c0 + kBN <= P.N;
+}
+
+// Bits of the columns [lo, hi) that fall in [base, base + 32), as a 32-bit mask.
+__device__ __forceinline__ uint32_t run_bits(int lo, int hi, int base) {
+  const int l = min(max(lo - base, 0), 32), h = min(max(hi - base, 0), 32);
+  const uint32_t mh = h >= 32 ? 0xffffffffu : (1u << h) - 1u;
+  const uint32_t ml = l >= 32 ? 0xffffffffu : (1u << l) - 1u;
+  return h > l ? (mh & ~ml) : 0u;
 }
 
 // 2^x on the FMA pipe for x in [-125, 8] (Cody-Waite style reduction 2^x = 2^n 2^f, n = round(x),
@@ -241,6 +254,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                              ~uintptr_t(1023));
   float* s_m = reinterpret_cast<float*>(smem + S::kML);   // [2][128]
   float* s_l = s_m + 2 * kBM;                              // [2][128]
+  int* s_dst = reinterpret_cast<int*>(smem + S::kDst);     // [128] destination token or -1
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint64_t* q_full = bars + 0;                 // [2] Q buffer landed
   uint64_t* q_empty = q_full + 2;              // [2] Q*K^T of the buffer's item done
@@ -405,21 +419,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int b4 = P.b * kStripes;
     const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
     bool ok = true;
-    int gn0 = 0;    // global index of the item's first tile
-    int uses = 0;   // tiles of this group so far (s_full phases)
+    int gn0 = 0;           // global index of the item's first tile
+    int uses = 0;          // tiles of this group so far (s_full phases)
+    bool s_ready = false;  // the next s_full phase was already seen complete (non-blocking test)
     for (int it = blockIdx.x, li = 0; it < n_items; it += gridDim.x, ++li) {
       const Item I = item_of(it, nq, P);
       const int nt = I.tiles.count();
       const int qrow = I.q0 + row;
-      // Destination row, resolved now so that the perm load is long done by the epilogue.
+      // Destination token of the row: loaded now, used in the epilogue (the load's latency
+      // overlaps the item's tiles).
       const bool store = qrow < P.N;
-      uint16_t* dst = nullptr;
-      if (store) {
-        const int u = I.uh / P.heads, h = I.uh - u * P.heads;
-        const int p = blockmajor_to_canonical(qrow, P.b, P.L);
-        const int t = min(max(__ldg(P.perm + (size_t)u * P.N + p), 0), P.N - 1);
-        dst = P.out + ((size_t)(u * P.N + t) * P.heads + h) * DH;
-      }
+      const int u_i = I.uh / P.heads, h_i = I.uh - u_i * P.heads;
+      const int perm_t =
+          store ? __ldg(P.perm + (size_t)u_i * P.N + blockmajor_to_canonical(qrow, P.b, P.L)) : 0;
       const int a_q = min(qrow, P.N - 1) / b4;
       const int s_q = band_start(a_q, P.W, P.nb);
       const int band_lo = s_q * b4, band_hi = (s_q + P.W) * b4, glob_hi = P.g * b4;
@@ -427,7 +439,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int j = 0;
       for (int n = grp; ok && n < nt; n += 2, ++j) {
         // Warp-collective wait: either every lane goes on to the .sync.aligned TMEM ops or none.
-        ok = __all_sync(0xffffffffu, mbar_wait(s_full + grp, uses & 1, abort, status));
+        if (!__all_sync(0xffffffffu, s_ready))
+          ok = __all_sync(0xffffffffu, mbar_wait(s_full + grp, uses & 1, abort, status));
         ++uses;
         if (!ok) break;
         tc_fence_after();
@@ -451,12 +464,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int c0 = I.tiles.tile(n) * kBN;
         const bool full = tile_full(c0, P);
         if (!full) {
+          // The row's kept keys in this tile are two runs, [0, e0) and [s1, e1) relative to c0:
+          // turned into four 32-bit column masks, so the per-key test has no branch.
+          const int e0 = min(glob_hi, P.N) - c0, s1 = band_lo - c0, e1 = min(band_hi, P.N) - c0;
+          uint32_t km[4];
 #pragma unroll
-          for (int i = 0; i < kBN; ++i) {
-            const int c = c0 + i;
-            const bool kept = c < P.N && (c < glob_hi || (c >= band_lo && c < band_hi));
-            if (!kept) sv[i] = -INFINITY;
-          }
+          for (int k = 0; k < 4; ++k) km[k] = run_bits(0, e0, 32 * k) | run_bits(s1, e1, 32 * k);
+#pragma unroll
+          for (int i = 0; i < kBN; ++i)
+            sv[i] = (km[i >> 5] >> (i & 31)) & 1u ? sv[i] : -INFINITY;
         }
         // Row max: eight independent chains of 3-input max over elements k, k+8, k+16, ...
         float mx[8];
@@ -526,12 +542,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             tmem_st32_async(t_p + 32 * half, pw);
           }
+          // Is S of this group's next tile already there? Tested here, where the result is not
+          // needed at once, instead of by a blocking wait at the top of the next iteration.
           tmem_st_wait();   // P complete in TMEM before the arrive below releases it to the MMA
         };
         if (full)
           softmax_row(std::integral_constant<bool, true>());
         else
           softmax_row(std::integral_constant<bool, false>());
+        // Is S of this group's next tile already there? Tested here, where the result is not
+        // needed at once, instead of by a blocking wait at the top of the next iteration.
+        s_ready = mbar_test(s_full + grp, uses & 1);
         float sa0, sa1;
         f2_unpack(f2_add(sum2a, sum2b), sa0, sa1);
         l_run += sa0 + sa1;
@@ -574,7 +595,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // to the P*V issuer, whose first MMA into O_w overwrites it.
       tc_fence_before();
       named_barrier(1, 256);
-      if (ok && store) {
+      // Normalised half-row -> shared staging; then the 256 threads copy whole rows out, so
+      // that each warp store covers four contiguous 128-byte rows (dh 64) instead of 32 rows.
+      const uint32_t stage_row = smem_u32(smem + S::kStage) + row * S::kStageStride;
+      if (ok) {
         const float mm = fmaxf(m0, m1);
         const float a0 = (m0 == -INFINITY) ? 0.f : ex2_mufu(m0 - mm);
         const float a1 = (m1 == -INFINITY) ? 0.f : ex2_mufu(m1 - mm);
@@ -583,7 +607,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float f0 = a0 * inv, f1 = a1 * inv;
         // A group with no tile in this item has a stale O: select, do not multiply by zero.
         const bool has0 = nt > 0, has1 = nt > 1;
-        uint4* out4 = reinterpret_cast<uint4*>(dst + grp * kCols);
 #pragma unroll
         for (int c = 0; c < kCols / 8; ++c) {
           float v[8];
@@ -593,12 +616,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const uint32_t u1 = c < 4 ? x1[8 * c + i] : y1[i];
             v[i] = (has0 ? __uint_as_float(u0) * f0 : 0.f) + (has1 ? __uint_as_float(u1) * f1 : 0.f);
           }
-          uint4 wv;
-          wv.x = pack_bf16(v[0], v[1]);
-          wv.y = pack_bf16(v[2], v[3]);
-          wv.z = pack_bf16(v[4], v[5]);
-          wv.w = pack_bf16(v[6], v[7]);
-          out4[c] = wv;
+          st_shared_v4(stage_row + grp * kCols * 2 + c * 16, pack_bf16(v[0], v[1]),
+                       pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+        }
+        if (grp == 0) s_dst[row] = store ? min(max(perm_t, 0), P.N - 1) : -1;
+      }
+      named_barrier(1, 256);
+      if (ok) {
+        constexpr int kCpr = DH / 8;                  // 16-byte chunks per row
+        const int tid = threadIdx.x - 128;            // 0..255
+        const uint32_t stage = smem_u32(smem + S::kStage);
+        uint8_t* out_uh = reinterpret_cast<uint8_t*>(P.out) +
+                          ((size_t)u_i * P.N * P.heads + h_i) * DH * 2;
+#pragma unroll
+        for (int k = 0; k < kBM * kCpr / 256; ++k) {
+          const int q = tid + 256 * k;
+          const int r = q / kCpr, c = q - r * kCpr;
+          const int t = s_dst[r];
+          if (t >= 0) {
+            const uint4 v = ld_shared_v4(stage + r * S::kStageStride + c * 16);
+            *reinterpret_cast<uint4*>(out_uh + (size_t)t * P.heads * DH * 2 + c * 16) = v;
+          }
         }
       }
       gn0 += nt;
