@@ -248,6 +248,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   using S = AttnSmem<DH>;
   using T = AttnTmem<DH>;
   constexpr int NS = S::kStages;
+  constexpr bool kSplitHandoff = T::kSeparateP;   // P handed to P*V in two halves
   constexpr bool kHasTail = S::kTail > 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -262,8 +263,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* kv_empty = kv_full + NS;           // [NS] P*V of the stage's tile done (K, V free)
   uint64_t* s_full = kv_empty + NS;            // [2] S_w computed
   uint64_t* s_free = s_full + 2;               // [2] S_w read into registers by its group
-  uint64_t* p_full = s_free + 2;               // [2] P_w written (and O_w rescaled if needed)
-  uint64_t* o_done = p_full + 2;               // an item's last P*V done
+  uint64_t* p_full = s_free + 2;               // [2][2] half h of P_w written (O_w rescaled first)
+  uint64_t* o_done = p_full + 4;               // an item's last P*V done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -277,7 +278,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(q_empty + i, 1);
       mbar_init(s_full + i, 1);
       mbar_init(s_free + i, 128);
-      mbar_init(p_full + i, 128);
+      mbar_init(p_full + 2 * i, 128);
+      mbar_init(p_full + 2 * i + 1, 128);
     }
     for (int i = 0; i < NS; ++i) {
       mbar_init(kv_full + i, 1);
@@ -383,17 +385,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int nt = item_of(it, nq, P).tiles.count();
         for (int n = 0; n < nt; ++n, ++gn) {
           const int st = gn % NS, w = n & 1;
-          if (!(ok = mbar_wait(p_full + w, uses[w] & 1, abort, status))) break;
-          ++uses[w];
-          tc_fence_after();
           const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kTileBytes);
           const uint32_t a = tmem + T::kP + w * T::kPStride;   // P_w
           const uint32_t d = tmem + T::kO + w * T::kOStride;
           // The first tile of each group overwrites O_w: its group released the previous item's
           // O (read in the epilogue) before handing over this P.
           const uint32_t acc = n >= 2;
+          // P arrives in two halves (keys 0-63, 64-127): the first half's MMAs run while the
+          // softmax still computes the second.
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
+            if (kk % (kBN / 32) == 0) {
+              if (!(ok = mbar_wait(p_full + 2 * w + kk / (kBN / 32), uses[w] & 1, abort, status)))
+                break;
+              tc_fence_after();
+            }
             umma_bf16_ts(d, a + kk * 8, smem_desc(v_addr + kk * 2048, kBN * 128, 1024, kSwizzle128B),
                          idesc_pv, acc | (kk > 0));
             if (kHasTail)
@@ -401,6 +407,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                            smem_desc(v_addr + S::kMain + kk * 512, kBN * 32, 256, kSwizzle32B),
                            idesc_pv_tail, acc | (kk > 0));
           }
+          if (!ok) break;
+          ++uses[w];
           umma_commit(kv_empty + st);   // Q*K^T of this tile finished before its P existed
         }
         if (!ok) break;
@@ -541,10 +549,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               pw[i2] = pack_bf16_pos(p0, p1);   // p >= 0: integer-pipe rounding
             }
             tmem_st32_async(t_p + 32 * half, pw);
+            if constexpr (kSplitHandoff) {
+              // Each half is handed over as soon as it is written.
+              if (half == 0 && rescale && j > 0) {
+                // O_w holds the group's earlier tiles (their P*V completed: waited above); it is
+                // rescaled before this tile's first P*V accumulates into it.
+#pragma unroll 1
+                for (int c = 0; c < (DH + 31) / 32; ++c) {
+                  uint32_t o[32];
+                  tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+                  for (int i = 0; i < 32; ++i)
+                    o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                  tmem_st32_async(t_o + c * 32, o);
+                }
+              }
+              tmem_st_wait();   // P (and O) complete in TMEM before the arrive releases it
+              tc_fence_before();
+              mbar_arrive(p_full + 2 * grp + half);
+            }
           }
-          // Is S of this group's next tile already there? Tested here, where the result is not
-          // needed at once, instead of by a blocking wait at the top of the next iteration.
-          tmem_st_wait();   // P complete in TMEM before the arrive below releases it to the MMA
         };
         if (full)
           softmax_row(std::integral_constant<bool, true>());
@@ -556,20 +580,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float sa0, sa1;
         f2_unpack(f2_add(sum2a, sum2b), sa0, sa1);
         l_run += sa0 + sa1;
-        if (rescale && j > 0) {
-          // O_w holds the group's earlier tiles: their P*V completed before this S was committed,
-          // and this tile's P*V is issued only after the arrive below.
+        if constexpr (!kSplitHandoff) {
+          // Both halves go together (the split costs the dh 80 variant registers it does not
+          // have): P written, then O_w rescaled if needed (its earlier P*V completed before this
+          // S was committed), then the hand-over.
+          tmem_st_wait();
+          if (rescale && j > 0) {
 #pragma unroll 1
-          for (int c = 0; c < (DH + 31) / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_o + c * 32, o);
+            for (int c = 0; c < (DH + 31) / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(t_o + c * 32, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(t_o + c * 32, o);
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(t_o + c * 32, o);
+            }
           }
+          tc_fence_before();
+          mbar_arrive(p_full + 2 * grp);
+          mbar_arrive(p_full + 2 * grp + 1);
         }
-        tc_fence_before();
-        mbar_arrive(p_full + grp);
       }
       // ---- merge both groups' partial rows and scatter them to out[u, perm[p], h, :] ----
       // Every softmax thread passes both named barriers once per item, also after a failed wait.
