@@ -384,8 +384,11 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, c
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int sms = sm_count();
 
+  // The gather also zeroes the GEMMs' k-split counters (a memset here would stand between two
+  // kernels and end their launch overlap).
+  const int n_counters = (int)((plan.total - plan.counters) / sizeof(int));
   rc = cuda_err(traced("gather_rows", st, [&] {
-    return launch_gather_rows(x, keep, xk, g.B, g.T, K, C, st);
+    return launch_gather_rows(x, keep, xk, g.B, g.T, K, C, counters, n_counters, st);
   }));
   if (rc) return rc;
 
@@ -397,9 +400,6 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, c
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_bf16(&tb2, 2, w2, hidden, C, 1, (uint64_t)hidden * 2, 64, plan.fc2.bn,
                    CU_TENSOR_MAP_SWIZZLE_128B))
-    return SS_ECUDA;
-  if (plan.counters != plan.total &&
-      cudaMemsetAsync(counters, 0, plan.total - plan.counters, st) != cudaSuccess)
     return SS_ECUDA;
 
   GemmEpilogue e1 = {};

@@ -39,6 +39,8 @@ __global__ void __launch_bounds__(256) k_gather_qkv(const uint16_t* __restrict__
                                                     uint16_t* __restrict__ kp,
                                                     uint16_t* __restrict__ vp, int N, int heads,
                                                     int b, int L) {
+  griddep_wait();
+  griddep_launch();
   const int u = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qpos = blockIdx.x * 8 + warp;
@@ -82,12 +84,12 @@ cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16
                               int U, int N, int heads, int dh, int b, cudaStream_t st) {
   dim3 grid((N + 7) / 8, U);
   if (dh == 64)
-    k_gather_qkv<8><<<grid, 256, 0, st>>>(q, k, v, perm, qp, kp, vp, N, heads, b, N / kStripes);
-  else if (dh == 80)
-    k_gather_qkv<10><<<grid, 256, 0, st>>>(q, k, v, perm, qp, kp, vp, N, heads, b, N / kStripes);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+    return launch_pdl(k_gather_qkv<8>, grid, dim3(256), 0, st, q, k, v, perm, qp, kp, vp, N, heads,
+                      b, N / kStripes);
+  if (dh == 80)
+    return launch_pdl(k_gather_qkv<10>, grid, dim3(256), 0, st, q, k, v, perm, qp, kp, vp, N, heads,
+                      b, N / kStripes);
+  return cudaErrorInvalidValue;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -294,6 +296,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();   // Q, K, V and perm come from the work before this launch
+  griddep_launch();
 
   // An mbarrier wait whose result gates the next instruction costs ~150 cycles even when the
   // phase has already completed, so the two MMA streams get their own issuing threads: one for
@@ -690,9 +694,8 @@ static cudaError_t launch_attn_dh(const CUtensorMap* tq, const CUtensorMap* tk,
   if (e != cudaSuccess) return e;
   const int items = ((p.N + kBM - 1) / kBM) * p.U * p.heads;
   dim3 grid(std::max(1, std::min(items, p.sms)));
-  k_attn<DH><<<grid, kAttnThreads, S::kAlloc, st>>>(*tq, *tk, *tv, *tq_tail, *tk_tail, *tv_tail, p,
-                                                    status);
-  return cudaGetLastError();
+  return launch_pdl(k_attn<DH>, grid, dim3(kAttnThreads), S::kAlloc, st, *tq, *tk, *tv, *tq_tail,
+                    *tk_tail, *tv_tail, p, status);
 }
 
 cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,

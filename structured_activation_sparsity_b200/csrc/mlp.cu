@@ -18,11 +18,17 @@
 namespace ss {
 
 // One warp per kept row: resolve the row's token, then copy its C bf16 (C/8 16-byte chunks) with
-// all of a lane's loads in flight before its stores.
+// all of a lane's loads in flight before its stores. CTA 0 also zeroes the GEMMs' k-split
+// counters (`zero`, `nzero` ints), which the two GEMM launches that follow expect at zero.
 __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t* __restrict__ x,
                                                      const int32_t* __restrict__ keep,
                                                      uint16_t* __restrict__ xk, int B, int T,
-                                                     int K, int C) {
+                                                     int K, int C, int* __restrict__ zero,
+                                                     int nzero) {
+  griddep_wait();
+  griddep_launch();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
   const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (m >= B * K) return;
   const int b = m / K;
@@ -42,10 +48,10 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t* __restrict_
 }
 
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* keep, uint16_t* xk, int B, int T,
-                               int K, int C, cudaStream_t st) {
+                               int K, int C, int* zero, int nzero, cudaStream_t st) {
   const int rows = B * K;
-  k_gather_rows<<<(rows + 7) / 8, 256, 0, st>>>(x, keep, xk, B, T, K, C);
-  return cudaGetLastError();
+  return launch_pdl(k_gather_rows, dim3((rows + 7) / 8), dim3(256), 0, st, x, keep, xk, B, T, K, C,
+                    zero, nzero);
 }
 
 // Persistent warp-specialised GEMM. Work unit = (m-tile, n-tile, k-split); CTA c takes units
@@ -175,6 +181,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();   // A, B and the epilogue's x come from the work before this launch
+  griddep_launch();
 
   auto decode = [&](int u, int& m, int& n, int& s, int& kb0, int& kb1) {
     m = u % g.m_tiles;
@@ -398,8 +406,8 @@ static cudaError_t launch_gemm_bn(const CUtensorMap* ta, const CUtensorMap* tb, 
   g.partial = partial;
   g.counters = counters;
   const int grid = p.units < sms ? p.units : sms;
-  k_gemm<BN, KSUB><<<grid, kGemmThreads, G::kAlloc, st>>>(*ta, *tb, g, ep, status);
-  return cudaGetLastError();
+  return launch_pdl(k_gemm<BN, KSUB>, dim3(grid), dim3(kGemmThreads), G::kAlloc, st, *ta, *tb, g, ep,
+                    status);
 }
 
 cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, const GemmPlan& p, int M,

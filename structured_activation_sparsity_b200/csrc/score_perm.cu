@@ -9,6 +9,7 @@
 // independent compares spread over the whole GPU (32 target tokens per CTA, 8 warps splitting the
 // other tokens), no synchronisation beyond one CTA-level reduction, and the result is the stable
 // order by construction. Each rank is scattered straight into perm, inv and the keep list.
+#include "common.cuh"
 #include "kernels.h"
 
 namespace ss {
@@ -16,6 +17,8 @@ namespace ss {
 __global__ void __launch_bounds__(256) k_sobel_score(const float* __restrict__ lum,
                                                      double* __restrict__ score, int B, int H,
                                                      int W) {
+  griddep_wait();
+  griddep_launch();
   int idx = blockIdx.x * blockDim.x + threadIdx.x;
   int per = H * W;
   if (idx >= B * per) return;
@@ -59,6 +62,8 @@ __global__ void __launch_bounds__(256) k_stripe_rank(const double* __restrict__ 
                                                      int32_t* __restrict__ keep) {
   extern __shared__ unsigned long long s_key[];
   __shared__ int s_cnt[8][32];
+  griddep_wait();
+  griddep_launch();
   const int u = blockIdx.y;
   // Fill the unit's keys: eight independent loads in flight per thread before any store.
   for (int t0 = threadIdx.x; t0 < N; t0 += 8 * blockDim.x) {
@@ -121,8 +126,7 @@ __global__ void __launch_bounds__(256) k_stripe_rank(const double* __restrict__ 
 cudaError_t launch_sobel_score(const float* lum, double* score, int B, int H, int W,
                                cudaStream_t st) {
   int n = B * H * W;
-  k_sobel_score<<<(n + 255) / 256, 256, 0, st>>>(lum, score, B, H, W);
-  return cudaGetLastError();
+  return launch_pdl(k_sobel_score, dim3((n + 255) / 256), dim3(256), 0, st, lum, score, B, H, W);
 }
 
 cudaError_t launch_stripe_rank(const double* score, int window_mode, int B, int Hg, int Wg, int ws,
@@ -142,8 +146,7 @@ cudaError_t launch_stripe_rank(const double* score, int window_mode, int B, int 
     if (e != cudaSuccess) return e;
   }
   dim3 grid((N + 31) / 32, units);
-  k_stripe_rank<<<grid, 256, smem, st>>>(score, m, N, K, perm, inv, keep);
-  return cudaGetLastError();
+  return launch_pdl(k_stripe_rank, grid, dim3(256), smem, st, score, m, N, K, perm, inv, keep);
 }
 
 }  // namespace ss
