@@ -55,13 +55,17 @@ struct UnitMap {
   }
 };
 
-// grid (ceil(N/32), units), block 256, dynamic smem N * 8 bytes.
-__global__ void __launch_bounds__(256) k_stripe_rank(const double* __restrict__ score, UnitMap m,
-                                                     int N, int K, int32_t* __restrict__ perm,
-                                                     int32_t* __restrict__ inv,
-                                                     int32_t* __restrict__ keep) {
-  extern __shared__ unsigned long long s_key[];
-  __shared__ int s_cnt[8][32];
+// grid (ceil(N/32), units), block 32 * WARPS, dynamic smem N * 8 bytes (16-byte aligned).
+// Each CTA ranks 32 target tokens; its WARPS warps split the unit's keys and count, for all 32
+// targets at once, the keys that come before each target.
+template <int WARPS>
+__global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __restrict__ score,
+                                                            UnitMap m, int N, int K,
+                                                            int32_t* __restrict__ perm,
+                                                            int32_t* __restrict__ inv,
+                                                            int32_t* __restrict__ keep) {
+  extern __shared__ __align__(16) unsigned long long s_key[];
+  __shared__ int s_cnt[WARPS][32];
   griddep_wait();
   griddep_launch();
   const int u = blockIdx.y;
@@ -85,27 +89,31 @@ __global__ void __launch_bounds__(256) k_stripe_rank(const double* __restrict__ 
   const int t = blockIdx.x * 32 + lane;
   const int tt = t < N ? t : N - 1;
   const unsigned long long kt = s_key[tt];
-  const int chunk = (N + 7) / 8;
-  const int lo = warp * chunk, hi = min(N, lo + chunk);
+  const int chunk = (((N + WARPS - 1) / WARPS) + 1) & ~1;   // even: pairs stay 16-byte aligned
+  const int lo = min(N, warp * chunk), hi = min(N, lo + chunk);
+  const ulonglong2* s_pair = reinterpret_cast<const ulonglong2*>(s_key);
   // Tokens before tt count when their key is >= kt (ties broken by the lower index), tokens
-  // after it only when strictly greater: two loops, no per-element index compare. Four
-  // independent counters keep the compare chain short.
+  // after it only when strictly greater: two runs, no per-element index compare. Keys are read
+  // in pairs (one 16-byte shared load, the same address across the warp: a broadcast); four
+  // independent counters keep the compare chains short.
   const int mid = max(lo, min(hi, tt));
   int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
   int o = lo;
   for (; o + 4 <= mid; o += 4) {
-    c0 += s_key[o] >= kt;
-    c1 += s_key[o + 1] >= kt;
-    c2 += s_key[o + 2] >= kt;
-    c3 += s_key[o + 3] >= kt;
+    const ulonglong2 p = s_pair[o >> 1], q = s_pair[(o >> 1) + 1];
+    c0 += p.x >= kt;
+    c1 += p.y >= kt;
+    c2 += q.x >= kt;
+    c3 += q.y >= kt;
   }
   for (; o < mid; ++o) c0 += s_key[o] >= kt;
-  o = mid;
+  if ((o & 1) && o < hi) c1 += s_key[o++] > kt;   // back to an even index
   for (; o + 4 <= hi; o += 4) {
-    c0 += s_key[o] > kt;
-    c1 += s_key[o + 1] > kt;
-    c2 += s_key[o + 2] > kt;
-    c3 += s_key[o + 3] > kt;
+    const ulonglong2 p = s_pair[o >> 1], q = s_pair[(o >> 1) + 1];
+    c0 += p.x > kt;
+    c1 += p.y > kt;
+    c2 += q.x > kt;
+    c3 += q.y > kt;
   }
   for (; o < hi; ++o) c0 += s_key[o] > kt;
   const int cnt = (c0 + c1) + (c2 + c3);
@@ -114,7 +122,7 @@ __global__ void __launch_bounds__(256) k_stripe_rank(const double* __restrict__ 
   if (warp == 0 && t < N) {
     int r = 0;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) r += s_cnt[w][lane];
+    for (int w = 0; w < WARPS; ++w) r += s_cnt[w][lane];
     const int L = N / kStripes;
     const int pos = (r % kStripes) * L + r / kStripes;   // stripe transpose
     if (perm) perm[(size_t)u * N + pos] = t;
@@ -140,13 +148,18 @@ cudaError_t launch_stripe_rank(const double* score, int window_mode, int B, int 
   m.wpr = window_mode ? (Wg + ws - 1) / ws : 1;
   m.nwin = window_mode ? m.wpr * ((Hg + ws - 1) / ws) : 1;
   size_t smem = (size_t)N * sizeof(unsigned long long);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k_stripe_rank, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-  }
   dim3 grid((N + 31) / 32, units);
-  return launch_pdl(k_stripe_rank, grid, dim3(256), smem, st, score, m, N, K, perm, inv, keep);
+  // Long units split their keys over 32 warps per CTA (a shorter count per warp), short ones
+  // over 8 (more CTAs per SM).
+  auto go = [&](auto kernel, int warps) -> cudaError_t {
+    if (smem > 48 * 1024) {
+      cudaError_t e =
+          cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(kernel, grid, dim3(32 * warps), smem, st, score, m, N, K, perm, inv, keep);
+  };
+  return N >= 2048 ? go(k_stripe_rank<32>, 32) : go(k_stripe_rank<8>, 8);
 }
 
 }  // namespace ss
