@@ -76,7 +76,8 @@ struct GemmCfg {
   static constexpr int kStages = (192 * 1024) / kStageBytes;
   static constexpr int kBar = kStages * kStageBytes;
   static constexpr int kAlloc = kBar + 512 + 1024;
-  static constexpr int kTmemCols = 2 * BN;        // two accumulators
+  // two accumulators; TMEM is allocated in powers of two columns
+  static constexpr int kTmemCols = 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
   static constexpr int kHalf = BN / 2;            // columns per epilogue warp
   static_assert(kStages >= 2, "at least two stages");
 };
@@ -85,8 +86,20 @@ __device__ __forceinline__ float bf16_to_f(uint16_t v) { return __uint_as_float(
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// GELU(z) = z/2 (1 + erf(z / sqrt 2)), with erf from Abramowitz & Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26 (|error| <= 1.5e-7, far below the bf16 rounding of the
+// result): for x >= 0, erfc(x) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) e^(-x^2), t = 1/(1 + p x).
+// Then GELU(z) = z/2 erfc(|z|/sqrt 2) for z < 0 and z/2 (2 - erfc(|z|/sqrt 2)) for z >= 0, which
+// keeps the relative accuracy of the small negative tail. Two MUFU ops (reciprocal, 2^x) and a
+// handful of FMAs, so the fc1 epilogue does not crowd out the MMA-issuing thread.
 __device__ __forceinline__ float gelu_erf(float z) {
-  return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+  const float x = fabsf(z) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, x, 1.0f));
+  const float poly =
+      t * fmaf(fmaf(fmaf(fmaf(1.061405429f, t, -1.453152027f), t, 1.421413741f), t, -0.284496736f),
+               t, 0.254829592f);
+  const float erfc_x = poly * ex2_mufu(-(x * x) * 1.4426950408889634f);
+  return 0.5f * z * (z >= 0.f ? 2.0f - erfc_x : erfc_x);
 }
 
 struct GemmShape {
@@ -352,14 +365,16 @@ GemmPlan gemm_plan(int M, int N, int Kd, int sms) {
   GemmPlan p;
   const int m_tiles = (M + 127) / 128;
   const int kb = Kd / 64;
-  // Pick the tile width and k-split with the smallest makespan: rounds of units over the CTAs,
-  // times k-blocks per unit, times the MMA time of one k-block (~ the tile width; N below 128 is
-  // bound by shared-memory bandwidth). A split costs a partial-tile round trip (~2 k-blocks per
-  // split) and is only considered for long K (>= 24 k-blocks).
+  // Pick the tile width and k-split with the smallest makespan, counted in operand bytes that
+  // the busiest CTA moves from L2 into shared memory (the measured bound of these GEMMs: one
+  // 64-wide k-block of a 128 x BN tile reads 128 + BN rows of 128 B). Rounds of (tile, split)
+  // units over the CTAs, times k-blocks per unit, times (128 + BN); a k-split adds the unit's fp32
+  // partial tile written (4 BN rows' worth) and, for the unit that finishes the tile, all `s`
+  // partials read back. Splits only for long K (>= 24 k-blocks).
   long long best = -1;
   p.bn = 64;
   p.splits = 1;
-  for (int bn : {256, 128, 64}) {
+  for (int bn : {256, 192, 128, 64}) {
     if (N % bn) continue;
     const int n_tiles = N / bn;
     for (int s = 1; s <= 8; ++s) {
@@ -367,8 +382,8 @@ GemmPlan gemm_plan(int M, int N, int Kd, int sms) {
       const long long units = (long long)m_tiles * n_tiles * s;
       const long long rounds = (units + sms - 1) / sms;
       const long long kb_unit = (kb + s - 1) / s;
-      const long long step = bn < 128 ? 128 : bn;
-      const long long cost = rounds * kb_unit * step + (s > 1 ? (long long)s * 2 * step : 0);
+      const long long partial = s > 1 ? (rounds + s) * 4LL * bn : 0;
+      const long long cost = rounds * kb_unit * (128 + bn) + partial;
       if (best < 0 || cost < best) {
         best = cost;
         p.bn = bn;
@@ -413,10 +428,10 @@ static cudaError_t launch_gemm_bn(const CUtensorMap* ta, const CUtensorMap* tb, 
 cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, const GemmPlan& p, int M,
                         int N, int Kd, const GemmEpilogue& ep, float* partial, int* counters,
                         int sms, int* status, cudaStream_t st) {
-  // Two sub-blocks per stage when every unit's k-range splits evenly (BN 256 keeps one: its
-  // 96 KB double stage would leave only two stages).
+  // Two sub-blocks per stage when every unit's k-range splits evenly (BN 192 and 256 keep one:
+  // their 80 and 96 KB double stages would leave only two stages).
   const int kb = Kd / 64;
-  const bool two = p.bn != 256 && kb % p.splits == 0 && (kb / p.splits) % 2 == 0;
+  const bool two = p.bn <= 128 && kb % p.splits == 0 && (kb / p.splits) % 2 == 0;
   switch (p.bn) {
     case 64:
       return two ? launch_gemm_bn<64, 2>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st)
@@ -424,6 +439,8 @@ cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, const Gemm
     case 128:
       return two ? launch_gemm_bn<128, 2>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st)
                  : launch_gemm_bn<128, 1>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
+    case 192:
+      return launch_gemm_bn<192, 1>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
     case 256:
       return launch_gemm_bn<256, 1>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st);
   }
