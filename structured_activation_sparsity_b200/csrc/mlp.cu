@@ -109,15 +109,38 @@ struct GemmShape {
   int* counters;           // [tiles], zero on entry (splits > 1)
 };
 
-// Applies the epilogue to 32 consecutive columns [n, n+32) of row m (all m < M).
-__device__ __forceinline__ void epilogue32(const GemmEpilogue& ep, const GemmShape& g, int m,
-                                           int n, float (&v)[32]) {
+// The epilogue of one output row m (< M) in chunks of 32 columns. The row's destination (and, for
+// kind 1, the keep lookup behind it) is resolved once per unit; a chunk's bias and residual words
+// are loaded before its accumulator values are needed, so their latency overlaps those reads.
+__device__ __forceinline__ uint16_t* epi_row(const GemmEpilogue& ep, const GemmShape& g, int m) {
+  if (ep.kind == 0) return ep.out + (size_t)m * g.N;
+  const int b = m / ep.K_per_image;
+  const int t = min(max(__ldg(ep.keep + m), 0), ep.T - 1);   // never leave the image
+  return ep.x + ((size_t)b * ep.T + t) * g.N;
+}
+struct Epi32In {
+  uint4 b[4], x[4];   // bias and (kind 1) residual bf16 words of 32 columns
+};
+__device__ __forceinline__ void epi_load(const GemmEpilogue& ep, const uint16_t* row, int n,
+                                         Epi32In& in) {
   if (ep.bias) {
     const uint4* bp = reinterpret_cast<const uint4*>(ep.bias + n);
 #pragma unroll
+    for (int q = 0; q < 4; ++q) in.b[q] = __ldg(bp + q);
+  }
+  if (ep.kind == 1) {
+    const uint4* xp = reinterpret_cast<const uint4*>(row + n);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) in.x[q] = xp[q];
+  }
+}
+// Kind 0: row[n..n+32) = bf16(GELU(v + bias)). Kind 1: row[n..n+32) = bf16(x + v + bias).
+__device__ __forceinline__ void epi_store(const GemmEpilogue& ep, uint16_t* row, int n,
+                                          const Epi32In& in, float (&v)[32]) {
+  if (ep.bias) {
+#pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const uint4 bw = __ldg(bp + q);
-      const uint32_t w[4] = {bw.x, bw.y, bw.z, bw.w};
+      const uint32_t w[4] = {in.b[q].x, in.b[q].y, in.b[q].z, in.b[q].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         v[q * 8 + 2 * e] += bf16_lo(w[e]);
@@ -125,19 +148,13 @@ __device__ __forceinline__ void epilogue32(const GemmEpilogue& ep, const GemmSha
       }
     }
   }
-  uint4* d;
   if (ep.kind == 0) {
-    d = reinterpret_cast<uint4*>(ep.out + (size_t)m * g.N + n);
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
   } else {
-    const int b = m / ep.K_per_image;
-    const int t = min(max(__ldg(ep.keep + m), 0), ep.T - 1);   // never leave the image
-    d = reinterpret_cast<uint4*>(ep.x + ((size_t)b * ep.T + t) * g.N + n);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const uint4 xv = d[q];
-      const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+      const uint32_t w[4] = {in.x[q].x, in.x[q].y, in.x[q].z, in.x[q].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         v[q * 8 + 2 * e] += bf16_lo(w[e]);
@@ -145,6 +162,7 @@ __device__ __forceinline__ void epilogue32(const GemmEpilogue& ep, const GemmSha
       }
     }
   }
+  uint4* d = reinterpret_cast<uint4*>(row + n);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint4 w;
@@ -294,20 +312,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int m = m_t * 128 + row;
       const int tile = n_t * g.m_tiles + m_t;
       const uint32_t t_acc = tmem + buf * BN + lane_off + col0;
+      uint16_t* drow = m < g.M ? epi_row(ep, g, m) : nullptr;
       if (g.splits == 1) {
 #pragma unroll 1
         for (int c = 0; c < G::kHalf / 32; ++c) {
+          const int n = n_t * BN + col0 + c * 32;
+          Epi32In in;
+          if (drow) epi_load(ep, drow, n, in);
           uint32_t r[32];
           tmem_ld32(t_acc + c * 32, r);
           if (c == G::kHalf / 32 - 1) {
             tc_fence_before();
             mbar_arrive(acc_empty + buf);   // accumulator fully read: MMA may reuse it
           }
-          if (m < g.M) {
+          if (drow) {
             float v[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
-            epilogue32(ep, g, m, n_t * BN + col0 + c * 32, v);
+            epi_store(ep, drow, n, in, v);
           }
         }
       } else {
@@ -331,20 +353,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!epi_sync()) break;
         if (*s_last) {
           __threadfence();
-          if (m < g.M) {
+          if (drow) {
             const float* base =
                 g.partial + (size_t)tile * g.splits * 128 * BN + (size_t)col0 * 128 + row;
 #pragma unroll 1
             for (int c = 0; c < G::kHalf / 32; ++c) {
+              const int n = n_t * BN + col0 + c * 32;
+              Epi32In in;
+              epi_load(ep, drow, n, in);
+              // Split 0's values and split 1's are loaded before either is added (64 loads in
+              // flight); further splits follow in the same fixed order: a deterministic sum.
+              const float* src = base + (size_t)c * 32 * 128;
               float v[32];
 #pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] = 0.f;
-              for (int sp = 0; sp < g.splits; ++sp) {   // fixed split order: deterministic sum
-                const float* src = base + (size_t)sp * 128 * BN + (size_t)c * 32 * 128;
+              for (int e = 0; e < 32; ++e) v[e] = __ldcg(src + (size_t)e * 128);
+              for (int sp = 1; sp < g.splits; ++sp) {
+                const float* s2 = src + (size_t)sp * 128 * BN;
+                float w[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] += __ldcg(src + (size_t)e * 128);
+                for (int e = 0; e < 32; ++e) w[e] = __ldcg(s2 + (size_t)e * 128);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] += w[e];
               }
-              epilogue32(ep, g, m, n_t * BN + col0 + c * 32, v);
+              epi_store(ep, drow, n, in, v);
             }
           }
           if (threadIdx.x == 64) g.counters[tile] = 0;
