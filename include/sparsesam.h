@@ -7,6 +7,7 @@
  *
  *   sparsesam_score  S1  Sobel gradient score per token
  *   sparsesam_perm   S2  stable sort by score + stripe transpose -> permutation; top-K keep list
+ *   sparsesam_score_perm  S1 + S2 in one pass (the same results, one launch fewer)
  *   sparsesam_attn   S3  static block-sparse attention over the permuted sequence
  *   sparsesam_rcmlp  S4  fc1-GELU-fc2 on the kept tokens, added to the residual in place
  *
@@ -114,6 +115,14 @@ int sparsesam_score(const ss_cfg* cfg, const float* lum, double* score, void* st
  * window). Any of perm/inv/keep may be NULL to skip it (not all three). Scores must not be NaN. */
 int sparsesam_perm(const ss_cfg* cfg, const double* score, int32_t* perm, int32_t* inv,
                    int32_t* keep, void* stream);
+
+/* S1 and S2 in one pass: the same results as sparsesam_score(cfg, lum, score) followed by
+ * sparsesam_perm(cfg, score, perm, inv, keep), bit for bit, with one launch fewer (global mode:
+ * one launch in all; window mode with keep: two). Each ranking CTA computes its unit's Sobel
+ * scores itself and writes its own tokens' scores to score. lum, score (device) as for
+ * sparsesam_score, both non-NULL; perm, inv, keep as for sparsesam_perm. */
+int sparsesam_score_perm(const ss_cfg* cfg, const float* lum, double* score, int32_t* perm,
+                         int32_t* inv, int32_t* keep, void* stream);
 
 /* Bytes of device workspace sparsesam_attn needs for cfg (0 on an invalid cfg). */
 size_t sparsesam_attn_workspace(const ss_cfg* cfg);

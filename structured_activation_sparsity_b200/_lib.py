@@ -53,6 +53,7 @@ def _load():
         "sparsesam_blocklist": (ctypes.c_int, [cfgp, P, P, I32]),
         "sparsesam_score": (ctypes.c_int, [cfgp, P, P, VP]),
         "sparsesam_perm": (ctypes.c_int, [cfgp, P, P, P, P, VP]),
+        "sparsesam_score_perm": (ctypes.c_int, [cfgp, P, P, P, P, P, VP]),
         "sparsesam_attn_workspace": (SZ, [cfgp]),
         "sparsesam_attn": (ctypes.c_int, [cfgp, P, P, P, P, P, P, SZ, VP]),
         "sparsesam_rcmlp_workspace": (SZ, [cfgp, I32, I32]),
@@ -140,6 +141,12 @@ def sparsesam_perm(cfg, score, perm, inv, keep, stream=None):
     return _check("sparsesam_perm",
                   lib.sparsesam_perm(ctypes.byref(cfg), _ptr(score), _ptr(perm), _ptr(inv),
                                      _ptr(keep), _stream(stream)))
+
+
+def sparsesam_score_perm(cfg, lum, score, perm, inv, keep, stream=None):
+    return _check("sparsesam_score_perm",
+                  lib.sparsesam_score_perm(ctypes.byref(cfg), _ptr(lum), _ptr(score), _ptr(perm),
+                                           _ptr(inv), _ptr(keep), _stream(stream)))
 
 
 def sparsesam_attn_workspace(cfg) -> int:

@@ -251,12 +251,14 @@ int sparsesam_score(const ss_cfg* cfg, const float* lum, double* score, void* st
   }));
 }
 
-int sparsesam_perm(const ss_cfg* cfg, const double* score, int32_t* perm, int32_t* inv,
-                   int32_t* keep, void* stream) {
+// S2 from given scores (score non-null, lum null) or S1 + S2 in one pass (lum non-null; the scores
+// are computed from lum and written to score when it is non-null).
+static int rank_path(const ss_cfg* cfg, const float* lum, const double* score, double* score_out,
+                     int32_t* perm, int32_t* inv, int32_t* keep, void* stream) {
   Geo g;
   int rc = geometry(cfg, &g);
   if (rc) return rc;
-  if (!score || (!perm && !inv && !keep)) return SS_EINVAL;
+  if (!perm && !inv && !keep) return SS_EINVAL;
   ss_pattern p;
   if ((perm || inv) && (rc = pattern_of(cfg, g, &p))) return rc;
   if (g.N > kMaxRankTokens || g.T > kMaxRankTokens) return SS_EUNSUPPORTED;
@@ -264,24 +266,40 @@ int sparsesam_perm(const ss_cfg* cfg, const double* score, int32_t* perm, int32_
   const int K = keep_count(cfg->density, g.T);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!g.window_mode) {
-    return cuda_err(traced("stripe_rank", st, [&] {
-      return launch_stripe_rank(score, 0, g.B, g.Hg, g.Wg, 0, g.B, g.T, K, perm, inv, keep, st);
+    return cuda_err(traced(lum ? "score_rank" : "stripe_rank", st, [&] {
+      return launch_stripe_rank(score, lum, score_out, 0, g.B, g.Hg, g.Wg, 0, g.B, g.T, K, perm,
+                                inv, keep, st);
     }));
   }
   if (perm || inv) {
-    rc = cuda_err(traced("stripe_rank_window", st, [&] {
-      return launch_stripe_rank(score, 1, g.B, g.Hg, g.Wg, g.ws, g.U, g.N, 0, perm, inv, nullptr,
-                                st);
+    rc = cuda_err(traced(lum ? "score_rank_window" : "stripe_rank_window", st, [&] {
+      return launch_stripe_rank(score, lum, score_out, 1, g.B, g.Hg, g.Wg, g.ws, g.U, g.N, 0, perm,
+                                inv, nullptr, st);
     }));
     if (rc) return rc;
   }
   if (keep) {
+    // The per-image keep ranking reads the scores: those the window pass just wrote, or the
+    // caller's.
+    const double* sc = lum ? score_out : score;
     rc = cuda_err(traced("keep_rank", st, [&] {
-      return launch_stripe_rank(score, 0, g.B, g.Hg, g.Wg, 0, g.B, g.T, K, nullptr, nullptr, keep,
-                                st);
+      return launch_stripe_rank(sc, nullptr, nullptr, 0, g.B, g.Hg, g.Wg, 0, g.B, g.T, K, nullptr,
+                                nullptr, keep, st);
     }));
   }
   return rc;
+}
+
+int sparsesam_perm(const ss_cfg* cfg, const double* score, int32_t* perm, int32_t* inv,
+                   int32_t* keep, void* stream) {
+  if (!score) return SS_EINVAL;
+  return rank_path(cfg, nullptr, score, nullptr, perm, inv, keep, stream);
+}
+
+int sparsesam_score_perm(const ss_cfg* cfg, const float* lum, double* score, int32_t* perm,
+                         int32_t* inv, int32_t* keep, void* stream) {
+  if (!lum || !score) return SS_EINVAL;
+  return rank_path(cfg, lum, nullptr, score, perm, inv, keep, stream);
 }
 
 size_t sparsesam_attn_workspace(const ss_cfg* cfg) {

@@ -15,9 +15,12 @@ constexpr int kMaxRankTokens = 16384;   // tokens per unit the rank kernel holds
 cudaError_t launch_sobel_score(const float* lum, double* score, int B, int H, int W,
                                cudaStream_t st);
 
-cudaError_t launch_stripe_rank(const double* score, int window_mode, int B, int Hg, int Wg, int ws,
-                               int units, int N, int K, int32_t* perm, int32_t* inv,
-                               int32_t* keep, cudaStream_t st);
+// Ranks the unit's tokens by score. With lum non-null the scores are computed from lum (S1 fused
+// in) instead of read from `score`, and written to score_out (when non-null).
+cudaError_t launch_stripe_rank(const double* score, const float* lum, double* score_out,
+                               int window_mode, int B, int Hg, int Wg, int ws, int units, int N,
+                               int K, int32_t* perm, int32_t* inv, int32_t* keep,
+                               cudaStream_t st);
 
 // Gathers q, k, v [U, N, heads, dh] into the block-major permuted layout [U*heads, N, dh].
 cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16_t* v,

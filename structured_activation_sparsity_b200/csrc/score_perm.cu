@@ -14,6 +14,23 @@
 
 namespace ss {
 
+// Squared Sobel gradient magnitude of pixel (y, x) of an H x W image, replicate border. Each step
+// is one fp64 round-to-nearest operation, in a fixed order, never fused, so every caller gets the
+// same bits.
+__device__ __forceinline__ double sobel_at(const float* __restrict__ img, int H, int W, int y,
+                                           int x) {
+  int ym = y > 0 ? y - 1 : 0, yp = y < H - 1 ? y + 1 : H - 1;
+  int xm = x > 0 ? x - 1 : 0, xp = x < W - 1 ? x + 1 : W - 1;
+  double l_mm = img[ym * W + xm], l_m0 = img[ym * W + x], l_mp = img[ym * W + xp];
+  double l_0m = img[y * W + xm], l_0p = img[y * W + xp];
+  double l_pm = img[yp * W + xm], l_p0 = img[yp * W + x], l_pp = img[yp * W + xp];
+  double gx = __dadd_rn(__dadd_rn(__dsub_rn(l_mp, l_mm), __dmul_rn(2.0, __dsub_rn(l_0p, l_0m))),
+                        __dsub_rn(l_pp, l_pm));
+  double gy = __dadd_rn(__dadd_rn(__dsub_rn(l_pm, l_mm), __dmul_rn(2.0, __dsub_rn(l_p0, l_m0))),
+                        __dsub_rn(l_pp, l_mp));
+  return __dadd_rn(__dmul_rn(gx, gx), __dmul_rn(gy, gy));
+}
+
 __global__ void __launch_bounds__(256) k_sobel_score(const float* __restrict__ lum,
                                                      double* __restrict__ score, int B, int H,
                                                      int W) {
@@ -25,41 +42,52 @@ __global__ void __launch_bounds__(256) k_sobel_score(const float* __restrict__ l
   int b = idx / per;
   int r = idx - b * per;
   int y = r / W, x = r - (r / W) * W;
-  int ym = y > 0 ? y - 1 : 0, yp = y < H - 1 ? y + 1 : H - 1;
-  int xm = x > 0 ? x - 1 : 0, xp = x < W - 1 ? x + 1 : W - 1;
-  const float* img = lum + (size_t)b * per;
-  double l_mm = img[ym * W + xm], l_m0 = img[ym * W + x], l_mp = img[ym * W + xp];
-  double l_0m = img[y * W + xm], l_0p = img[y * W + xp];
-  double l_pm = img[yp * W + xm], l_p0 = img[yp * W + x], l_pp = img[yp * W + xp];
-  // Each step is one fp64 round-to-nearest operation, in a fixed order, never fused.
-  double gx = __dadd_rn(__dadd_rn(__dsub_rn(l_mp, l_mm), __dmul_rn(2.0, __dsub_rn(l_0p, l_0m))),
-                        __dsub_rn(l_pp, l_pm));
-  double gy = __dadd_rn(__dadd_rn(__dsub_rn(l_pm, l_mm), __dmul_rn(2.0, __dsub_rn(l_p0, l_m0))),
-                        __dsub_rn(l_pp, l_mp));
-  score[idx] = __dadd_rn(__dmul_rn(gx, gx), __dmul_rn(gy, gy));
+  score[idx] = sobel_at(lum + (size_t)b * per, H, W, y, x);
 }
 
 // Unit-local token t -> its score key (bits of a non-negative double, which order like the value).
 struct UnitMap {
   int window_mode;   // 0: unit = image, t = raster index; 1: unit = window, t = window raster
   int Hg, Wg, ws, wpr, nwin;
-  __device__ __forceinline__ unsigned long long key(const double* score, int u, int t) const {
+  // Image b and pixel (y, x) of unit-local token t; false for a window's pad token.
+  __device__ __forceinline__ bool locate(int u, int t, int& b, int& y, int& x) const {
     if (!window_mode) {
-      return (unsigned long long)__double_as_longlong(score[(size_t)u * Hg * Wg + t]);
+      b = u;
+      y = t / Wg;
+      x = t - y * Wg;
+      return true;
     }
-    int b = u / nwin, w = u - (u / nwin) * nwin;
-    int wy = w / wpr, wx = w - (w / wpr) * wpr;
-    int y = wy * ws + t / ws, x = wx * ws + t % ws;
-    if (y >= Hg || x >= Wg) return 0ull;   // pad token: +0.0
-    return (unsigned long long)__double_as_longlong(score[(size_t)b * Hg * Wg + y * Wg + x]);
+    b = u / nwin;
+    const int w = u - b * nwin;
+    const int wy = w / wpr, wx = w - (w / wpr) * wpr;
+    y = wy * ws + t / ws;
+    x = wx * ws + t % ws;
+    return y < Hg && x < Wg;
+  }
+  __device__ __forceinline__ unsigned long long key(const double* score, int u, int t) const {
+    int b, y, x;
+    if (!locate(u, t, b, y, x)) return 0ull;   // pad token: +0.0
+    return (unsigned long long)__double_as_longlong(score[((size_t)b * Hg + y) * Wg + x]);
+  }
+  // The same key computed from the luminance (S1 fused into S2).
+  __device__ __forceinline__ unsigned long long key_lum(const float* lum, int u, int t) const {
+    int b, y, x;
+    if (!locate(u, t, b, y, x)) return 0ull;
+    return (unsigned long long)__double_as_longlong(
+        sobel_at(lum + (size_t)b * Hg * Wg, Hg, Wg, y, x));
   }
 };
 
 // grid (ceil(N/32), units), block 32 * WARPS, dynamic smem N * 8 bytes (16-byte aligned).
 // Each CTA ranks 32 target tokens; its WARPS warps split the unit's keys and count, for all 32
 // targets at once, the keys that come before each target.
-template <int WARPS>
+// FROM_LUM: the keys are the Sobel scores computed here from `lum` (S1 fused into S2); each CTA
+// also stores the scores of its 32 target tokens into `score_out`, so every real token's score is
+// written once.
+template <int WARPS, bool FROM_LUM>
 __global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __restrict__ score,
+                                                            const float* __restrict__ lum,
+                                                            double* __restrict__ score_out,
                                                             UnitMap m, int N, int K,
                                                             int32_t* __restrict__ perm,
                                                             int32_t* __restrict__ inv,
@@ -75,7 +103,7 @@ __global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __rest
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int t = t0 + e * blockDim.x;
-      k8[e] = t < N ? m.key(score, u, t) : 0ull;
+      k8[e] = t >= N ? 0ull : FROM_LUM ? m.key_lum(lum, u, t) : m.key(score, u, t);
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -128,6 +156,10 @@ __global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __rest
     if (perm) perm[(size_t)u * N + pos] = t;
     if (inv) inv[(size_t)u * N + t] = pos;
     if (keep && r < K) keep[(size_t)u * K + r] = t;
+    if (FROM_LUM && score_out) {
+      int b, y, x;
+      if (m.locate(u, t, b, y, x)) score_out[((size_t)b * m.Hg + y) * m.Wg + x] = __longlong_as_double((long long)kt);
+    }
   }
 }
 
@@ -137,9 +169,10 @@ cudaError_t launch_sobel_score(const float* lum, double* score, int B, int H, in
   return launch_pdl(k_sobel_score, dim3((n + 255) / 256), dim3(256), 0, st, lum, score, B, H, W);
 }
 
-cudaError_t launch_stripe_rank(const double* score, int window_mode, int B, int Hg, int Wg, int ws,
-                               int units, int N, int K, int32_t* perm, int32_t* inv,
-                               int32_t* keep, cudaStream_t st) {
+cudaError_t launch_stripe_rank(const double* score, const float* lum, double* score_out,
+                               int window_mode, int B, int Hg, int Wg, int ws, int units, int N,
+                               int K, int32_t* perm, int32_t* inv, int32_t* keep,
+                               cudaStream_t st) {
   UnitMap m;
   m.window_mode = window_mode;
   m.Hg = Hg;
@@ -157,9 +190,12 @@ cudaError_t launch_stripe_rank(const double* score, int window_mode, int B, int 
           cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
-    return launch_pdl(kernel, grid, dim3(32 * warps), smem, st, score, m, N, K, perm, inv, keep);
+    return launch_pdl(kernel, grid, dim3(32 * warps), smem, st, score, lum, score_out, m, N, K,
+                      perm, inv, keep);
   };
-  return N >= 2048 ? go(k_stripe_rank<32>, 32) : go(k_stripe_rank<8>, 8);
+  if (lum)
+    return N >= 2048 ? go(k_stripe_rank<32, true>, 32) : go(k_stripe_rank<8, true>, 8);
+  return N >= 2048 ? go(k_stripe_rank<32, false>, 32) : go(k_stripe_rank<8, false>, 8);
 }
 
 }  // namespace ss

@@ -59,6 +59,11 @@ class HotPath:
     def perm_step(self, stream=None):
         L.sparsesam_perm(self.cfg, self.score, self.perm, self.inv, self.keep, stream)
 
+    def score_perm_step(self, stream=None):
+        """S1 and S2 in one pass (the same score, perm, inv and keep as score_step + perm_step)."""
+        L.sparsesam_score_perm(self.cfg, self.lum, self.score, self.perm, self.inv, self.keep,
+                               stream)
+
     def attn_step(self, stream=None):
         L.sparsesam_attn(self.cfg, self.q, self.k, self.v, self.perm, self.out, self.ws_attn,
                          self.ws_attn_bytes, stream)
@@ -68,8 +73,8 @@ class HotPath:
                           self.w2, self.b2, self.keep, self.ws_mlp, self.ws_mlp_bytes, stream)
 
     def step(self, stream=None):
-        """S1..S4 of one block, asynchronously on `stream` (a torch.cuda.Stream or None)."""
-        self.score_step(stream)
-        self.perm_step(stream)
+        """S1..S4 of one block, asynchronously on `stream` (a torch.cuda.Stream or None); S1 and S2
+        run as one fused pass."""
+        self.score_perm_step(stream)
         self.attn_step(stream)
         self.mlp_step(stream)

@@ -98,6 +98,9 @@ def test_validation_codes():
     # null pointers
     assert lib.sparsesam_score(by(good), None, FAKE, None) == L.SS_EINVAL
     assert lib.sparsesam_perm(by(good), FAKE, None, None, None, None) == L.SS_EINVAL
+    assert lib.sparsesam_score_perm(by(good), None, FAKE, FAKE, None, None, None) == L.SS_EINVAL
+    assert lib.sparsesam_score_perm(by(good), FAKE, None, FAKE, None, None, None) == L.SS_EINVAL
+    assert lib.sparsesam_score_perm(by(good), FAKE, FAKE, None, None, None, None) == L.SS_EINVAL
     assert lib.sparsesam_attn(by(good), None, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == L.SS_EINVAL
     # unsupported head_dim
     bad_dh = L.make_cfg(1, 16, 16, "global", 14, 1, 96, 0.4)

@@ -41,30 +41,36 @@ SCORE_CASES = [
 ]
 
 
-def _score_perm(cfg, lum_np):
+def _score_perm(cfg, lum_np, fused=False):
+    """S1 then S2 (two calls), or both through the fused call; the outputs start as NaN / -1."""
     B, H, W = lum_np.shape
     geo = _geo(cfg)
     lum = torch.from_numpy(lum_np).to(DEV)
-    score = torch.empty((B, H * W), dtype=torch.float64, device=DEV)
-    L.sparsesam_score(cfg, lum, score)
-    perm = torch.empty((geo.units, geo.unit_tokens), dtype=torch.int32, device=DEV)
-    inv = torch.empty_like(perm)
+    score = torch.full((B, H * W), float("nan"), dtype=torch.float64, device=DEV)
+    perm = torch.full((geo.units, geo.unit_tokens), -1, dtype=torch.int32, device=DEV)
+    inv = torch.full_like(perm, -1)
     K = O.keep_count(cfg.density, H * W)
-    keep = torch.empty((B, K), dtype=torch.int32, device=DEV)
-    L.sparsesam_perm(cfg, score, perm, inv, keep)
+    keep = torch.full((B, K), -1, dtype=torch.int32, device=DEV)
+    if fused:
+        L.sparsesam_score_perm(cfg, lum, score, perm, inv, keep)
+    else:
+        L.sparsesam_score(cfg, lum, score)
+        L.sparsesam_perm(cfg, score, perm, inv, keep)
     torch.cuda.synchronize()
     return score.cpu().numpy(), perm.cpu().numpy(), inv.cpu().numpy(), keep.cpu().numpy()
 
 
 def _check_score_perm(cfg, lum_np):
-    score, perm, inv, keep = _score_perm(cfg, lum_np)
     geo = _geo(cfg)
     o_score = O.sobel_score(lum_np)
-    assert np.array_equal(score.view(np.int64), o_score.view(np.int64))
     o_perm, o_inv = O.stripe_sort(o_score, geo)
-    assert np.array_equal(perm, o_perm)
-    assert np.array_equal(inv, o_inv)
-    assert np.array_equal(keep, O.keep_list(o_score, cfg.density))
+    o_keep = O.keep_list(o_score, cfg.density)
+    for fused in (False, True):   # both paths, bit-exact against the oracle
+        score, perm, inv, keep = _score_perm(cfg, lum_np, fused)
+        assert np.array_equal(score.view(np.int64), o_score.view(np.int64)), fused
+        assert np.array_equal(perm, o_perm), fused
+        assert np.array_equal(inv, o_inv), fused
+        assert np.array_equal(keep, o_keep), fused
     _status_ok()
 
 
@@ -216,11 +222,13 @@ def test_hotpath_tiny_end_to_end():
     n0 = L.sparsesam_launch_count()
     hp.step()
     torch.cuda.synchronize()
-    assert L.sparsesam_launch_count() - n0 == 7
+    assert L.sparsesam_launch_count() - n0 == 6   # S1+S2 fused, gather, attn, gather, fc1, fc2
     geo = O.Geometry(1, 16, 16, "global", 14)
     score, perm, inv, keep, out, y = O.hot_path(
         lum, *(synth.bf16_to_f64(t) for t in (q, k, v, xb, w1b, b1b, w2b, b2b)), geo, wl.density)
+    assert np.array_equal(hp.score.cpu().numpy().view(np.int64), score.view(np.int64))
     assert np.array_equal(hp.perm.cpu().numpy(), perm)
+    assert np.array_equal(hp.inv.cpu().numpy(), inv)
     assert np.array_equal(hp.keep.cpu().numpy(), keep)
     _assert_close(synth.bf16_to_f64(hp.out), out, "hotpath attn")
     _assert_close(synth.bf16_to_f64(hp.x), y, "hotpath rcmlp")
@@ -236,6 +244,5 @@ def test_trace_records_each_launch():
     hp.step()
     recs = L.sparsesam_trace_stop()
     names = [n for n, _ in recs]
-    assert names == ["sobel_score", "stripe_rank", "gather_qkv", "attn", "gather_rows",
-                     "rcmlp_fc1", "rcmlp_fc2"]
+    assert names == ["score_rank", "gather_qkv", "attn", "gather_rows", "rcmlp_fc1", "rcmlp_fc2"]
     assert all(ms > 0 for _, ms in recs)
