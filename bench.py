@@ -11,6 +11,12 @@ One process per GPU (torchrun for N > 1). The path has no exchange step: each ra
 independent replica of the workload (weak scaling) and the job's throughput is all ranks' tokens
 over the slowest rank's device time. Rank 0 prints one JSON line.
 
+`value` times the steps with inputs resident on the device (rotating over input sets larger than
+L2). `e2e` times the same steps through the same calls with every step's inputs copied in from
+pinned host memory and its results (out, x) read back, pipelined the way a serving loop runs:
+the copy-in of one step, the compute of the previous one and the read-back of the one before
+overlap on three streams over two device buffer sets.
+
 --impl reference times the float64 CPU oracle (the only reference this method has) on the host
 cores, on a bounded sample of the same workload, and prints the same line with "impl": "reference".
 """
@@ -321,31 +327,48 @@ def run_ours(args, wl, rank, world, local_rank, dist):
     del dense_sets
 
     # ---- end to end: pinned host inputs in, results out, through the same C-ABI calls ------------
-    hp = sets[0]
-    host_in = [t_.detach().to("cpu").pin_memory() for t_ in hp.input_tensors()]
-    host_out = [torch.empty(hp.out.shape, dtype=hp.out.dtype).pin_memory(),
-                torch.empty(hp.x.shape, dtype=hp.x.dtype).pin_memory()]
+    # Pipelined over two device buffer sets and three streams, as a serving loop runs: step i's
+    # inputs are copied in (one stream) while step i-1 computes (the compute stream) and step
+    # i-2's results are read back (a third stream). Every step copies all of its inputs in and all
+    # of its results (out, x) back.
+    e2e_sets = sets[:2]
+    host_in = [t_.detach().to("cpu").pin_memory() for t_ in e2e_sets[0].input_tensors()]
+    host_out = [[torch.empty(h.out.shape, dtype=h.out.dtype).pin_memory(),
+                 torch.empty(h.x.shape, dtype=h.x.dtype).pin_memory()] for h in e2e_sets]
     h2d = sum(x.numel() * x.element_size() for x in host_in)
-    d2h = sum(x.numel() * x.element_size() for x in host_out)
+    d2h = sum(x.numel() * x.element_size() for x in host_out[0])
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in e2e_sets]
+    ev_c = [torch.cuda.Event() for _ in e2e_sets]
+    ev_out = [torch.cuda.Event() for _ in e2e_sets]
 
-    def e2e_step():
-        with torch.cuda.stream(stream):
-            for dst, src in zip(hp.input_tensors(), host_in):
+    def e2e_step(i):
+        b = i % len(e2e_sets)
+        h = e2e_sets[b]
+        s_in.wait_event(ev_out[b])   # set b's previous results have been read back
+        with torch.cuda.stream(s_in):
+            for dst, src in zip(h.input_tensors(), host_in):
                 dst.copy_(src, non_blocking=True)
-            hp.step(stream)
-            host_out[0].copy_(hp.out, non_blocking=True)
-            host_out[1].copy_(hp.x, non_blocking=True)
+            ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        h.step(stream)
+        ev_c[b].record(stream)
+        s_out.wait_event(ev_c[b])
+        with torch.cuda.stream(s_out):
+            host_out[b][0].copy_(h.out, non_blocking=True)
+            host_out[b][1].copy_(h.x, non_blocking=True)
+            ev_out[b].record(s_out)
 
-    for _ in range(max(3, args.warmup // 4)):
-        e2e_step()
+    for i in range(max(3, args.warmup // 4)):
+        e2e_step(i)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    ev1.record(stream)
+    ev0.record(s_in)
+    for i in range(args.steps):
+        e2e_step(i)
+    ev1.record(s_out)   # after the last read-back, which follows every other step's work
     torch.cuda.synchronize()
     te = max_over_ranks(ev0.elapsed_time(ev1) / 1e3, dist, dev)
     e2e_value = job_throughput(world, tokens_per_step, args.steps, te)
