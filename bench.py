@@ -231,7 +231,7 @@ def make_sets(wl, n_sets, dev, density=None):
 
 def set_bytes(hp):
     ts = [hp.lum, hp.score, hp.perm, hp.inv, hp.keep, hp.q, hp.k, hp.v, hp.out, hp.x, hp.w1,
-          hp.w2, hp.ws_attn, hp.ws_mlp]
+          hp.w2, hp.ws_block]
     return sum(t.numel() * t.element_size() for t in ts if t is not None)
 
 

@@ -8,6 +8,7 @@
  *   sparsesam_score  S1  Sobel gradient score per token
  *   sparsesam_perm   S2  stable sort by score + stripe transpose -> permutation; top-K keep list
  *   sparsesam_score_perm  S1 + S2 in one pass (the same results, one launch fewer)
+ *   sparsesam_block       S1..S4 in one call with one workspace
  *   sparsesam_attn   S3  static block-sparse attention over the permuted sequence
  *   sparsesam_rcmlp  S4  fc1-GELU-fc2 on the kept tokens, added to the residual in place
  *
@@ -154,6 +155,21 @@ size_t sparsesam_rcmlp_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden);
 int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden,
                     const uint16_t* w1, const uint16_t* b1, const uint16_t* w2, const uint16_t* b2,
                     const int32_t* keep, void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace sparsesam_block needs (0 on an invalid cfg). */
+size_t sparsesam_block_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden);
+
+/* S1..S4 of one encoder block in one call: sparsesam_score_perm(cfg, lum, score, perm, inv, keep),
+ * then sparsesam_attn(cfg, q, k, v, perm, out), then sparsesam_rcmlp(cfg, x, C, hidden, w1, b1,
+ * w2, b2, keep), with one workspace: the same launches and results, bit for bit. Arguments and
+ * their layouts, alignment and error codes as in those calls (lum, score, perm, keep, out
+ * non-NULL; inv may be NULL). ws (device, 256-byte aligned) >= sparsesam_block_workspace(cfg, C,
+ * hidden) bytes; its contents on entry do not matter. */
+int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, const uint16_t* k,
+                    const uint16_t* v, uint16_t* x, int32_t C, int32_t hidden, const uint16_t* w1,
+                    const uint16_t* b1, const uint16_t* w2, const uint16_t* b2, double* score,
+                    int32_t* perm, int32_t* inv, int32_t* keep, uint16_t* out, void* ws,
+                    size_t ws_bytes, void* stream);
 
 /* S4 without a caller-provided workspace. The SparseSAM pages have no counterpart to this call;
  * it exists for callers that cannot allocate device memory where they run the block: code inside

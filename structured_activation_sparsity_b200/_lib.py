@@ -54,6 +54,9 @@ def _load():
         "sparsesam_score": (ctypes.c_int, [cfgp, P, P, VP]),
         "sparsesam_perm": (ctypes.c_int, [cfgp, P, P, P, P, VP]),
         "sparsesam_score_perm": (ctypes.c_int, [cfgp, P, P, P, P, P, VP]),
+        "sparsesam_block_workspace": (SZ, [cfgp, I32, I32]),
+        "sparsesam_block": (ctypes.c_int, [cfgp, P, P, P, P, P, I32, I32, P, P, P, P, P, P, P, P,
+                                           P, P, SZ, VP]),
         "sparsesam_attn_workspace": (SZ, [cfgp]),
         "sparsesam_attn": (ctypes.c_int, [cfgp, P, P, P, P, P, P, SZ, VP]),
         "sparsesam_rcmlp_workspace": (SZ, [cfgp, I32, I32]),
@@ -147,6 +150,19 @@ def sparsesam_score_perm(cfg, lum, score, perm, inv, keep, stream=None):
     return _check("sparsesam_score_perm",
                   lib.sparsesam_score_perm(ctypes.byref(cfg), _ptr(lum), _ptr(score), _ptr(perm),
                                            _ptr(inv), _ptr(keep), _stream(stream)))
+
+
+def sparsesam_block_workspace(cfg, C, hidden) -> int:
+    return int(lib.sparsesam_block_workspace(ctypes.byref(cfg), C, hidden))
+
+
+def sparsesam_block(cfg, lum, q, k, v, x, C, hidden, w1, b1, w2, b2, score, perm, inv, keep, out,
+                    ws, ws_bytes, stream=None):
+    return _check("sparsesam_block",
+                  lib.sparsesam_block(ctypes.byref(cfg), _ptr(lum), _ptr(q), _ptr(k), _ptr(v),
+                                      _ptr(x), C, hidden, _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2),
+                                      _ptr(score), _ptr(perm), _ptr(inv), _ptr(keep), _ptr(out),
+                                      _ptr(ws), ws_bytes, _stream(stream)))
 
 
 def sparsesam_attn_workspace(cfg) -> int:

@@ -308,40 +308,32 @@ size_t sparsesam_attn_workspace(const ss_cfg* cfg) {
   return attn_ws_bytes(g, cfg->heads, cfg->head_dim);
 }
 
-int sparsesam_attn(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                   const int32_t* perm, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
-  Geo g;
-  int rc = geometry(cfg, &g);
-  if (rc) return rc;
+// Argument checks of the attention step (also for the whole-block path); fills the pattern.
+static int attn_check(const ss_cfg* cfg, const Geo& g, const uint16_t* q, const uint16_t* k,
+                      const uint16_t* v, const int32_t* perm, const uint16_t* out, ss_pattern* p) {
   if (cfg->heads < 1 || cfg->head_dim < 1) return SS_EINVAL;
   if (!q || !k || !v || !perm || !out) return SS_EINVAL;
   if (cfg->head_dim != 64 && cfg->head_dim != 80) return SS_EUNSUPPORTED;
-  ss_pattern p;
-  if ((rc = pattern_of(cfg, g, &p))) return rc;
+  int rc = pattern_of(cfg, g, p);
+  if (rc) return rc;
   const int heads = cfg->heads, dh = cfg->head_dim;
   if ((int64_t)g.U * heads > 65535) return SS_EUNSUPPORTED;
   if ((int64_t)g.U * g.N * heads * (dh / 8) >= (int64_t)1 << 31) return SS_EUNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
     return SS_EINVAL;
-  const size_t need = attn_ws_bytes(g, heads, dh);
-  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SS_EWORKSPACE;
-  int* status = status_word();
-  if (!status) return SS_ECUDA;
+  return SS_OK;
+}
 
-  const size_t one = need / 3;
-  uint16_t* qp = static_cast<uint16_t*>(ws);
-  uint16_t* kp = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + one);
-  uint16_t* vp = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + 2 * one);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-
-  rc = cuda_err(traced("gather_qkv", st, [&] {
-    return launch_gather_qkv(q, k, v, perm, qp, kp, vp, g.U, g.N, heads, dh, p.b, st);
-  }));
-  if (rc) return rc;
-
+// The attention over the gathered Q, K, V in ws (laid out as attn_ws_bytes describes).
+static int attn_launch(const ss_cfg* cfg, const Geo& g, const ss_pattern& p, uint8_t* ws,
+                       const int32_t* perm, uint16_t* out, int* status, cudaStream_t st) {
+  const int heads = cfg->heads, dh = cfg->head_dim;
+  const size_t one = attn_ws_bytes(g, heads, dh) / 3;
+  const uint16_t* bufs[3] = {reinterpret_cast<uint16_t*>(ws),
+                             reinterpret_cast<uint16_t*>(ws + one),
+                             reinterpret_cast<uint16_t*>(ws + 2 * one)};
   CUtensorMap tm[6];
   const uint64_t mats = (uint64_t)g.U * heads;
-  const uint16_t* bufs[3] = {qp, kp, vp};
   for (int i = 0; i < 3; ++i) {
     if (!encode_bf16(&tm[i], 3, bufs[i], dh, g.N, mats, (uint64_t)dh * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B))
@@ -368,18 +360,41 @@ int sparsesam_attn(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k, cons
   }));
 }
 
+int sparsesam_attn(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const int32_t* perm, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  ss_pattern p;
+  if ((rc = attn_check(cfg, g, q, k, v, perm, out, &p))) return rc;
+  const int heads = cfg->heads, dh = cfg->head_dim;
+  const size_t need = attn_ws_bytes(g, heads, dh);
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SS_EWORKSPACE;
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const size_t one = need / 3;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = cuda_err(traced("gather_qkv", st, [&] {
+    return launch_gather_qkv(q, k, v, perm, reinterpret_cast<uint16_t*>(wsb),
+                             reinterpret_cast<uint16_t*>(wsb + one),
+                             reinterpret_cast<uint16_t*>(wsb + 2 * one), g.U, g.N, heads, dh, p.b,
+                             st);
+  }));
+  if (rc) return rc;
+  return attn_launch(cfg, g, p, wsb, perm, out, status, st);
+}
+
 size_t sparsesam_rcmlp_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden) {
   Geo g;
   if (geometry(cfg, &g) || C < 1 || hidden < 1) return 0;
   return rcmlp_ws_bytes(g, keep_count(cfg->density, g.T), C, hidden);
 }
 
-int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, const uint16_t* w1,
-                    const uint16_t* b1, const uint16_t* w2, const uint16_t* b2,
-                    const int32_t* keep, void* ws, size_t ws_bytes, void* stream) {
-  Geo g;
-  int rc = geometry(cfg, &g);
-  if (rc) return rc;
+// Argument checks of the RC-MLP step (also for the whole-block path).
+static int rcmlp_check(const ss_cfg* cfg, const Geo& g, const uint16_t* x, int32_t C,
+                       int32_t hidden, const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
+                       const uint16_t* b2, const int32_t* keep) {
   if (!x || !w1 || !w2 || !keep || C < 1 || hidden < 1) return SS_EINVAL;
   if (C % 64 != 0 || hidden % 64 != 0) return SS_EUNSUPPORTED;
   if (!aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(b1, 16) ||
@@ -389,27 +404,21 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, c
   const int64_t M = (int64_t)g.B * K;
   if (M * (hidden > C ? hidden : C) >= ((int64_t)1 << 31) || (M + 127) / 128 > 65535)
     return SS_EUNSUPPORTED;
-  const size_t need = rcmlp_ws_bytes(g, K, C, hidden);
-  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SS_EWORKSPACE;
-  int* status = status_word();
-  if (!status) return SS_ECUDA;
+  return SS_OK;
+}
+
+// fc1 and fc2 over the gathered rows in ws (laid out as mlp_plan describes).
+static int rcmlp_launch(const Geo& g, int K, uint16_t* x, int32_t C, int32_t hidden,
+                        const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
+                        const uint16_t* b2, const int32_t* keep, uint8_t* wsb, int* status,
+                        cudaStream_t st) {
   const MlpPlan plan = mlp_plan(g, K, C, hidden);
-  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const int64_t M = (int64_t)g.B * K;
   uint16_t* xk = reinterpret_cast<uint16_t*>(wsb + plan.xk);
   uint16_t* hbuf = reinterpret_cast<uint16_t*>(wsb + plan.h);
   float* partial = reinterpret_cast<float*>(wsb + plan.partial);
   int* counters = reinterpret_cast<int*>(wsb + plan.counters);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int sms = sm_count();
-
-  // The gather also zeroes the GEMMs' k-split counters (a memset here would stand between two
-  // kernels and end their launch overlap).
-  const int n_counters = (int)((plan.total - plan.counters) / sizeof(int));
-  rc = cuda_err(traced("gather_rows", st, [&] {
-    return launch_gather_rows(x, keep, xk, g.B, g.T, K, C, counters, n_counters, st);
-  }));
-  if (rc) return rc;
-
   CUtensorMap ta1, tb1, ta2, tb2;
   if (!encode_bf16(&ta1, 2, xk, C, M, 1, (uint64_t)C * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_bf16(&tb1, 2, w1, C, hidden, 1, (uint64_t)C * 2, 64, plan.fc1.bn,
@@ -419,12 +428,11 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, c
       !encode_bf16(&tb2, 2, w2, hidden, C, 1, (uint64_t)hidden * 2, 64, plan.fc2.bn,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return SS_ECUDA;
-
   GemmEpilogue e1 = {};
   e1.kind = 0;
   e1.bias = b1;
   e1.out = hbuf;
-  rc = cuda_err(traced("rcmlp_fc1", st, [&] {
+  int rc = cuda_err(traced("rcmlp_fc1", st, [&] {
     return launch_gemm(&ta1, &tb1, plan.fc1, (int)M, hidden, C, e1, partial, counters, sms, status,
                        st);
   }));
@@ -440,6 +448,86 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, c
     return launch_gemm(&ta2, &tb2, plan.fc2, (int)M, C, hidden, e2, partial, counters, sms, status,
                        st);
   }));
+}
+
+int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, const uint16_t* w1,
+                    const uint16_t* b1, const uint16_t* w2, const uint16_t* b2,
+                    const int32_t* keep, void* ws, size_t ws_bytes, void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  if ((rc = rcmlp_check(cfg, g, x, C, hidden, w1, b1, w2, b2, keep))) return rc;
+  const int K = keep_count(cfg->density, g.T);
+  const size_t need = rcmlp_ws_bytes(g, K, C, hidden);
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SS_EWORKSPACE;
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+  const MlpPlan plan = mlp_plan(g, K, C, hidden);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The gather also zeroes the GEMMs' k-split counters (a memset here would stand between two
+  // kernels and end their launch overlap).
+  const int n_counters = (int)((plan.total - plan.counters) / sizeof(int));
+  rc = cuda_err(traced("gather_rows", st, [&] {
+    return launch_gather_rows(x, keep, reinterpret_cast<uint16_t*>(wsb + plan.xk), g.B, g.T, K, C,
+                              reinterpret_cast<int*>(wsb + plan.counters), n_counters, st);
+  }));
+  if (rc) return rc;
+  return rcmlp_launch(g, K, x, C, hidden, w1, b1, w2, b2, keep, wsb, status, st);
+}
+
+size_t sparsesam_block_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden) {
+  Geo g;
+  if (geometry(cfg, &g) || cfg->heads < 1 || cfg->head_dim < 1 || C < 1 || hidden < 1) return 0;
+  return align256(attn_ws_bytes(g, cfg->heads, cfg->head_dim)) +
+         rcmlp_ws_bytes(g, keep_count(cfg->density, g.T), C, hidden);
+}
+
+int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, const uint16_t* k,
+                    const uint16_t* v, uint16_t* x, int32_t C, int32_t hidden, const uint16_t* w1,
+                    const uint16_t* b1, const uint16_t* w2, const uint16_t* b2, double* score,
+                    int32_t* perm, int32_t* inv, int32_t* keep, uint16_t* out, void* ws,
+                    size_t ws_bytes, void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  if (!lum || !score) return SS_EINVAL;
+  ss_pattern p;
+  if ((rc = attn_check(cfg, g, q, k, v, perm, out, &p))) return rc;
+  if ((rc = rcmlp_check(cfg, g, x, C, hidden, w1, b1, w2, b2, keep))) return rc;
+  if (g.N > kMaxRankTokens || g.T > kMaxRankTokens) return SS_EUNSUPPORTED;
+  const int heads = cfg->heads, dh = cfg->head_dim;
+  const int K = keep_count(cfg->density, g.T);
+  const size_t attn_part = align256(attn_ws_bytes(g, heads, dh));
+  if (!ws || !aligned(ws, 256) || ws_bytes < attn_part + rcmlp_ws_bytes(g, K, C, hidden))
+    return SS_EWORKSPACE;
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+  uint8_t* wsa = static_cast<uint8_t*>(ws);
+  uint8_t* wsm = wsa + attn_part;
+  const size_t one = attn_ws_bytes(g, heads, dh) / 3;
+  const MlpPlan plan = mlp_plan(g, K, C, hidden);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // S1 + S2 in one pass, the attention's gather and the attention, the MLP's gather (which also
+  // zeroes the GEMMs' k-split counters) and fc1, fc2: the launches of the per-step calls. (Fusing
+  // the two gathers into the ranking launch was measured slower: its 128 ranking CTAs copy the
+  // rows less efficiently than the gathers spread over every SM.)
+  if ((rc = rank_path(cfg, lum, nullptr, score, perm, inv, keep, stream))) return rc;
+  rc = cuda_err(traced("gather_qkv", st, [&] {
+    return launch_gather_qkv(q, k, v, perm, reinterpret_cast<uint16_t*>(wsa),
+                             reinterpret_cast<uint16_t*>(wsa + one),
+                             reinterpret_cast<uint16_t*>(wsa + 2 * one), g.U, g.N, heads, dh, p.b,
+                             st);
+  }));
+  if (rc) return rc;
+  if ((rc = attn_launch(cfg, g, p, wsa, perm, out, status, st))) return rc;
+  const int n_counters = (int)((plan.total - plan.counters) / sizeof(int));
+  rc = cuda_err(traced("gather_rows", st, [&] {
+    return launch_gather_rows(x, keep, reinterpret_cast<uint16_t*>(wsm + plan.xk), g.B, g.T, K, C,
+                              reinterpret_cast<int*>(wsm + plan.counters), n_counters, st);
+  }));
+  if (rc) return rc;
+  return rcmlp_launch(g, K, x, C, hidden, w1, b1, w2, b2, keep, wsm, status, st);
 }
 
 int sparsesam_device_status(int32_t* out, void* stream) {

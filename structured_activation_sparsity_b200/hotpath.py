@@ -36,10 +36,15 @@ class HotPath:
         self.w2 = torch.empty((C, Hd), dtype=torch.bfloat16, **e)
         self.b1 = torch.zeros((Hd,), dtype=torch.bfloat16, **e) if bias else None
         self.b2 = torch.zeros((C,), dtype=torch.bfloat16, **e) if bias else None
+        # One workspace for the whole-block call; the per-step calls use its two parts (the
+        # attention's first, 256-byte aligned, then the MLP's).
         self.ws_attn_bytes = L.sparsesam_attn_workspace(self.cfg)
         self.ws_mlp_bytes = L.sparsesam_rcmlp_workspace(self.cfg, C, Hd)
-        self.ws_attn = torch.empty((self.ws_attn_bytes,), dtype=torch.uint8, **e)
-        self.ws_mlp = torch.empty((self.ws_mlp_bytes,), dtype=torch.uint8, **e)
+        self.ws_block_bytes = L.sparsesam_block_workspace(self.cfg, C, Hd)
+        self.ws_block = torch.empty((self.ws_block_bytes,), dtype=torch.uint8, **e)
+        attn_part = -(-self.ws_attn_bytes // 256) * 256
+        self.ws_attn = self.ws_block[:attn_part]
+        self.ws_mlp = self.ws_block[attn_part:]
 
     # -- inputs --------------------------------------------------------------------------------
     def load(self, lum, q, k, v, x, w1, b1, w2, b2):
@@ -73,8 +78,14 @@ class HotPath:
                           self.w2, self.b2, self.keep, self.ws_mlp, self.ws_mlp_bytes, stream)
 
     def step(self, stream=None):
-        """S1..S4 of one block, asynchronously on `stream` (a torch.cuda.Stream or None); S1 and S2
-        run as one fused pass."""
+        """S1..S4 of one block, asynchronously on `stream` (a torch.cuda.Stream or None), in the
+        whole-block call (S1 and S2 as one fused pass)."""
+        L.sparsesam_block(self.cfg, self.lum, self.q, self.k, self.v, self.x, self.wl.dim,
+                          self.wl.hidden, self.w1, self.b1, self.w2, self.b2, self.score, self.perm,
+                          self.inv, self.keep, self.out, self.ws_block, self.ws_block_bytes, stream)
+
+    def step_by_calls(self, stream=None):
+        """The same step through the per-step calls (S1+S2 fused, then S3, then S4)."""
         self.score_perm_step(stream)
         self.attn_step(stream)
         self.mlp_step(stream)

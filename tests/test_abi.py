@@ -101,6 +101,16 @@ def test_validation_codes():
     assert lib.sparsesam_score_perm(by(good), None, FAKE, FAKE, None, None, None) == L.SS_EINVAL
     assert lib.sparsesam_score_perm(by(good), FAKE, None, FAKE, None, None, None) == L.SS_EINVAL
     assert lib.sparsesam_score_perm(by(good), FAKE, FAKE, None, None, None, None) == L.SS_EINVAL
+    assert lib.sparsesam_block_workspace(None, 64, 256) == 0
+    assert lib.sparsesam_block_workspace(by(good), 0, 256) == 0
+    assert lib.sparsesam_block_workspace(by(good), 64, 256) >= (
+        lib.sparsesam_attn_workspace(by(good)) + lib.sparsesam_rcmlp_workspace(by(good), 64, 256))
+    blk = [FAKE] * 5 + [64, 256] + [FAKE] * 4 + [FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, None]
+    assert lib.sparsesam_block(by(good), *blk) == L.SS_EWORKSPACE   # 1 byte of workspace
+    for i in (0, 1, 11, 12, 14, 15):   # lum, q, score, perm, keep, out
+        bad = list(blk)
+        bad[i] = None
+        assert lib.sparsesam_block(by(good), *bad) == L.SS_EINVAL, i
     assert lib.sparsesam_attn(by(good), None, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == L.SS_EINVAL
     # unsupported head_dim
     bad_dh = L.make_cfg(1, 16, 16, "global", 14, 1, 96, 0.4)

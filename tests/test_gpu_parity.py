@@ -246,3 +246,26 @@ def test_trace_records_each_launch():
     names = [n for n, _ in recs]
     assert names == ["score_rank", "gather_qkv", "attn", "gather_rows", "rcmlp_fc1", "rcmlp_fc2"]
     assert all(ms > 0 for _, ms in recs)
+
+
+# ------------------------------------------------------------------------------------------------
+# The whole-block call against the per-step calls: the same kernels on the same data, so every
+# output is bit-identical.
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["tiny", "vitb_global", "vitb_window", "vith_global"])
+def test_block_call_equals_step_calls(name):
+    wl = workloads.get(name)
+    a, b = HotPath(wl), HotPath(wl)
+    lum = torch.from_numpy(synth.luminance(wl))
+    q, k, v = (synth.to_bf16(t) for t in synth.qkv(wl))
+    mlp = [synth.to_bf16(t) for t in synth.mlp_params(wl, bias_scale=0.1)]
+    a.load(lum, q, k, v, *mlp)
+    b.load(lum, q, k, v, *mlp)
+    a.step()
+    b.step_by_calls()
+    torch.cuda.synchronize()
+    for ta, tb in ((a.score, b.score), (a.perm, b.perm), (a.inv, b.inv), (a.keep, b.keep),
+                   (a.out, b.out), (a.x, b.x)):
+        assert torch.equal(ta.view(torch.int8) if ta.dtype != torch.int32 else ta,
+                           tb.view(torch.int8) if tb.dtype != torch.int32 else tb), name
+    _status_ok()
