@@ -229,6 +229,22 @@ def make_sets(wl, n_sets, dev, density=None):
     return sets, (lum, q, k, v, mlp)
 
 
+def kernel_bytes(wl, pat):
+    """Algorithmic DRAM bytes per launch of the bandwidth-bound kernels of one step."""
+    T = wl.batch * wl.grid_h * wl.grid_w              # real tokens
+    units_tokens = wl.units * wl.unit_tokens          # tokens incl. window pads
+    K = wl.batch * pat.keep
+    row = wl.heads * wl.head_dim * 2                  # one token's bf16 Q (or K, V) row
+    return {
+        # lum in, score out, perm and inv out, keep out
+        "score_rank": T * 4 + T * 8 + units_tokens * 8 + K * 4,
+        "sobel_score": T * 4 + T * 8,
+        "stripe_rank": T * 8 + units_tokens * 8 + K * 4,
+        "gather_qkv": 2 * 3 * units_tokens * row,     # Q, K, V read once and written once
+        "gather_rows": 2 * K * wl.dim * 2,            # kept rows of x read and written
+    }
+
+
 def set_bytes(hp):
     ts = [hp.lum, hp.score, hp.perm, hp.inv, hp.keep, hp.q, hp.k, hp.v, hp.out, hp.x, hp.w1,
           hp.w2, hp.ws_block]
@@ -310,6 +326,14 @@ def run_ours(args, wl, rank, world, local_rank, dist):
     for name, ms in recs:
         per_kernel.setdefault(name, []).append(ms)
     kernels = {n: {"launches": len(v), "avg_us": 1e3 * sum(v) / len(v)} for n, v in per_kernel.items()}
+    # Algorithmic bytes of the bandwidth-bound launches (reads + writes each must make at least
+    # once) and their rate against the measured HBM copy peak. The per-launch times come from the
+    # traced pass (CUDA events around each launch), so they include the launch's own latency.
+    moved = kernel_bytes(wl, pat)
+    for n, nbytes in moved.items():
+        if n in kernels:
+            gbs = nbytes / (kernels[n]["avg_us"] * 1e-6) / 1e9
+            kernels[n].update({"bytes": nbytes, "gbs": gbs, "frac_hbm": gbs / hbm_peak})
     attn_us = kernels["attn"]["avg_us"]
     achieved = attn_flops / (attn_us * 1e-6) / 1e12
     traffic = ATTN_TRAFFIC_BYTES.get(wl.name)
@@ -433,6 +457,64 @@ def run_kernel_loop(args, wl, local_rank):
                       "note": "inputs stay resident in L2 across calls"}), flush=True)
 
 
+def run_stack(args, local_rank):
+    """The ViT-L encoder stack (24 blocks: global at 5, 11, 17, 23, the rest 14x14 windowed;
+    8 images of 64x64 tokens, 16 heads x 64, MLP 1024->4096) at each density of the sweep, as the
+    sum of its blocks' steps: S1+S2 once per image for each of the two geometries (the permutation
+    depends on the image only), then S3 and S4 for every block. One JSON line per density."""
+    import torch
+
+    from structured_activation_sparsity_b200 import _lib as L
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    wg, ww = workloads.get("vitl_global"), workloads.get("vitl_window")
+    n_global, n_window = 4, 20
+    bf16_peak = peaks()[0]
+    for d in (1.0, 0.5, 0.4, 0.3):
+        hg = make_sets(wg, 1, dev, density=d)[0][0]
+        hw = make_sets(ww, 1, dev, density=d)[0][0]
+
+        def stack_step():
+            hg.score_perm_step(stream)
+            hw.score_perm_step(stream)
+            for i in range(n_global + n_window):
+                h = hg if i % 6 == 5 else hw   # blocks 5, 11, 17, 23 are global
+                h.attn_step(stream)
+                h.mlp_step(stream)
+
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                stack_step()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                stack_step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        t = ev0.elapsed_time(ev1) / 1e3 / args.steps
+        if L.sparsesam_device_status(stream) != L.SS_OK:
+            raise RuntimeError("a device wait timed out during timing")
+        flops = 0.0
+        for h, w, n in ((hg, wg, n_global), (hw, ww, n_window)):
+            pat = h.pattern
+            flops += n * (workloads.attn_flops(w.units, w.unit_tokens, w.heads, w.head_dim, pat.rho)
+                          + workloads.mlp_flops(w.batch * pat.keep, w.dim, w.hidden))
+        tokens = wg.batch * wg.grid_h * wg.grid_w
+        print(json.dumps({"stack": "vitl_24_blocks", "density": d, "ms_per_stack": t * 1e3,
+                          "tokens_per_s": tokens / t, "effective_tflops": flops / t / 1e12,
+                          "frac_bf16_peak": flops / t / 1e12 / bf16_peak,
+                          "global_rho": hg.pattern.rho, "window_rho": hw.pattern.rho,
+                          "steps": args.steps, "warmup": args.warmup,
+                          "note": "sum of block steps; the full block (LN, projections) is not in "
+                                  "the hot path"}), flush=True)
+        del hg, hw
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -442,6 +524,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--kernel-loop", default=None, choices=["score", "perm", "attn", "rcmlp"],
                     help="run only this library call in a loop (profiling aid; no bench line)")
+    ap.add_argument("--stack", action="store_true",
+                    help="time the ViT-L 24-block stack at densities 1.0/0.5/0.4/0.3 (no bench line)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = workloads.get(args.workload)
@@ -454,6 +538,9 @@ def main():
         return
     if args.kernel_loop:
         run_kernel_loop(args, wl, local_rank)
+        return
+    if args.stack:
+        run_stack(args, local_rank)
         return
     dist = None
     if world > 1:
