@@ -99,6 +99,8 @@ constexpr int kBM = 128;              // query rows per CTA
 constexpr int kBN = 128;              // keys per tile
 constexpr int kAttnThreads = 384;     // 12 warps = 3 warpgroups
 constexpr float kLazyRescale = 8.f;   // log2 headroom before O and l are rescaled
+constexpr int kPairTiles = 4;         // items of at most this many key tiles: k_attn_pairs
+constexpr bool kPairInterleave = true;   // k_attn_pairs ring order A_0, B_0, A_1, B_1, ...
 constexpr int kPolyPairs = 0;         // of every 16 exp pairs on full tiles, those on the FMA pipe
 // Register split (launch: 384 threads x 168): producer warpgroup 56, softmax warpgroups 224.
 constexpr uint32_t kRegsProducer = 56, kRegsSoftmax = 224;
@@ -139,7 +141,7 @@ struct AttnSmem {
 // of all hitting the same L2 lines. The softmax is order-independent up to rounding.
 struct KeyTiles {
   int lo0, hi0, lo1, hi1, rot;
-  __device__ int count() const { return (hi0 - lo0) + (hi1 - lo1); }
+  __host__ __device__ int count() const { return (hi0 - lo0) + (hi1 - lo1); }
   __device__ int tile(int n) const {
     const int c = count();
     n = n + rot < c ? n + rot : n + rot - c;
@@ -149,8 +151,8 @@ struct KeyTiles {
 
 // Key tiles a query tile [q0, q_last] needs: the global rows [0, g*4b) and the band rows
 // [s(a_lo)*4b, (s(a_hi)+W)*4b), both clipped to N, as two (possibly merged) runs of tiles.
-__device__ __forceinline__ KeyTiles key_tiles(int q0, int q_last, int qt, int uh,
-                                              const AttnParams& P) {
+__host__ __device__ __forceinline__ KeyTiles key_tiles(int q0, int q_last, int qt, int uh,
+                                                       const AttnParams& P) {
   const int b4 = P.b * kStripes;
   const int a_lo = q0 / b4, a_hi = q_last / b4;
   const int s_lo = band_start(a_lo, P.W, P.nb), s_hi = band_start(a_hi, P.W, P.nb);
@@ -683,6 +685,419 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Short items (windowed blocks: about two key tiles per item): whole items per softmax group.
+// ---------------------------------------------------------------------------------------------
+// With two key tiles per item, splitting an item's tiles between the two groups (k_attn) leaves
+// each group one tile per item, then a wait for both P*V and a merged epilogue behind two
+// CTA-wide barriers: the exposed latencies dominate. Here the CTA takes its items in pairs (A =
+// its item 2p, B = its item 2p+1); group 0 runs A and group 1 runs B, each a whole item with its
+// own Q buffer, S, P and O, each normalising and scattering its own rows (no merge). The pair's
+// key tiles go through one K/V ring in the order A_0, B_0, A_1, B_1, ... (kInterleave) or
+// A_0, A_1, ..., B_0, B_1, ... . Head dim 64 (the windowed configurations).
+struct AttnPairSmem {
+  static constexpr int kTileBytes = kBM * 128;                  // 128 rows x 64 bf16
+  static constexpr int kStages = 4;                             // depth of the K/V ring
+  static constexpr int kQ = 0;                                  // Q of A, Q of B
+  static constexpr int kK = 2 * kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kStageStride = 64 * 2 + 16;              // padded output staging rows
+  static constexpr int kStage = kV + kStages * kTileBytes;      // [2 groups][128 rows]
+  static constexpr int kDst = kStage + 2 * kBM * kStageStride;  // [2 groups][128] tokens
+  static constexpr int kBar = kDst + 2 * kBM * 4;
+  static constexpr int kBytes = kBar + 512;
+  static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 227 * 1024, "attention shared memory above the per-CTA limit");
+};
+
+// Position of tile n of the pair's item g in the pair's ring order.
+template <bool kInterleave>
+__device__ __forceinline__ int pair_tile_index(int g, int n, int ntA, int ntB) {
+  if (kInterleave) return min(n, ntA) + min(n, ntB) + (g == 1 && n < ntA ? 1 : 0);
+  return g == 0 ? n : ntA + n;
+}
+
+template <bool kInterleave>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    k_attn_pairs(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                 const __grid_constant__ CUtensorMap tv, const AttnParams P, int* status) {
+  using S = AttnPairSmem;
+  using T = AttnTmem<64>;
+  constexpr int NS = S::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  int* s_dst = reinterpret_cast<int*>(smem + S::kDst);     // [2][128] destination token or -1
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint64_t* q_full = bars + 0;                 // [2] Q of group g's item landed
+  uint64_t* q_empty = q_full + 2;              // [2] Q*K^T of group g's item done
+  uint64_t* kv_full = q_empty + 2;             // [NS]
+  uint64_t* kv_empty = kv_full + NS;           // [NS] P*V of the stage's tile done
+  uint64_t* s_full = kv_empty + NS;            // [2] S_g computed
+  uint64_t* s_free = s_full + 2;               // [2] S_g read into registers
+  uint64_t* p_full = s_free + 2;               // [2][2] half h of P_g written
+  uint64_t* o_done = p_full + 4;               // [2] last P*V of group g's item done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 2);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nq = (P.N + kBM - 1) / kBM;
+  const int n_items = nq * P.U * P.heads;
+  const int G = gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full + i, 1);
+      mbar_init(q_empty + i, 1);
+      mbar_init(s_full + i, 1);
+      mbar_init(s_free + i, 128);
+      mbar_init(p_full + 2 * i, 128);
+      mbar_init(p_full + 2 * i + 1, 128);
+      mbar_init(o_done + i, 1);
+    }
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(kv_full + i, 1);
+      mbar_init(kv_empty + i, 1);
+    }
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_wait();   // Q, K, V and perm come from the work before this launch
+  griddep_launch();
+
+  // Every role walks the pairs p = 0, 1, ... with item A = blockIdx.x + 2pG and B = A + G; every
+  // item has at least one key tile (its own band).
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsProducer>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------ TMA producer ------------------------------
+      tma_prefetch_desc(&tq);
+      tma_prefetch_desc(&tk);
+      tma_prefetch_desc(&tv);
+      bool ok = true;
+      int gn0 = 0;   // ring index of the pair's first tile
+      for (int p = 0, itA = blockIdx.x; ok && itA < n_items; ++p, itA += 2 * G) {
+        const bool hasB = itA + G < n_items;
+        const Item A = item_of(itA, nq, P);
+        Item B = A;
+        if (hasB) B = item_of(itA + G, nq, P);
+        const int ntA = A.tiles.count(), ntB = hasB ? B.tiles.count() : 0;
+        if (p >= 1 && !(ok = mbar_wait(q_empty + 0, (p - 1) & 1, abort, status))) break;
+        mbar_expect_tx(q_full + 0, S::kTileBytes);
+        tma_load_3d(smem + S::kQ, &tq, q_full + 0, 0, A.q0, A.uh);
+        if (hasB) {
+          if (p >= 1 && !(ok = mbar_wait(q_empty + 1, (p - 1) & 1, abort, status))) break;
+          mbar_expect_tx(q_full + 1, S::kTileBytes);
+          tma_load_3d(smem + S::kQ + S::kTileBytes, &tq, q_full + 1, 0, B.q0, B.uh);
+        }
+        for (int j = 0; ok && j < ntA + ntB; ++j) {
+          // tile j of the ring order -> (item, tile)
+          int g, n;
+          if (kInterleave) {
+            const int both = 2 * min(ntA, ntB);
+            if (j < both) {
+              g = j & 1;
+              n = j >> 1;
+            } else {
+              g = ntA > ntB ? 0 : 1;
+              n = (j - both) + min(ntA, ntB);
+            }
+          } else {
+            g = j < ntA ? 0 : 1;
+            n = j < ntA ? j : j - ntA;
+          }
+          const int gn = gn0 + j, st = gn % NS;
+          if (gn >= NS && !(ok = mbar_wait(kv_empty + st, ((gn / NS) - 1) & 1, abort, status)))
+            break;
+          const int c0 = (g ? B.tiles.tile(n) : A.tiles.tile(n)) * kBN;
+          const int uh = g ? B.uh : A.uh;
+          mbar_expect_tx(kv_full + st, 2 * S::kTileBytes);
+          tma_load_3d(smem + S::kK + st * S::kTileBytes, &tk, kv_full + st, 0, c0, uh);
+          tma_load_3d(smem + S::kV + st * S::kTileBytes, &tv, kv_full + st, 0, c0, uh);
+        }
+        gn0 += ntA + ntB;
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------ Q*K^T issuer ------------------------------
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
+      bool ok = true;
+      int gn0 = 0;
+      int uses[2] = {0, 0};   // tiles computed into S_g so far
+      for (int p = 0, itA = blockIdx.x; ok && itA < n_items; ++p, itA += 2 * G) {
+        const bool hasB = itA + G < n_items;
+        const int ntA = item_of(itA, nq, P).tiles.count();
+        const int ntB = hasB ? item_of(itA + G, nq, P).tiles.count() : 0;
+        bool q_in0 = false, q_in1 = false;
+        for (int j = 0; ok && j < ntA + ntB; ++j) {
+          int g, n;
+          if (kInterleave) {
+            const int both = 2 * min(ntA, ntB);
+            g = j < both ? (j & 1) : (ntA > ntB ? 0 : 1);
+            n = j < both ? (j >> 1) : (j - both) + min(ntA, ntB);
+          } else {
+            g = j < ntA ? 0 : 1;
+            n = j < ntA ? j : j - ntA;
+          }
+          bool& q_in = g ? q_in1 : q_in0;
+          if (!q_in) {
+            if (!(ok = mbar_wait(q_full + g, p & 1, abort, status))) break;
+            q_in = true;
+          }
+          const int gn = gn0 + j, st = gn % NS;
+          const int ug = g ? uses[1] : uses[0];
+          // S_g is reusable once its previous tile's S is in its group's registers.
+          if (ug > 0 && !(ok = mbar_wait(s_free + g, (ug - 1) & 1, abort, status))) break;
+          if (!(ok = mbar_wait(kv_full + st, (gn / NS) & 1, abort, status))) break;
+          tc_fence_after();
+          const uint32_t q_addr = smem_u32(smem + S::kQ + g * S::kTileBytes);
+          const uint32_t k_addr = smem_u32(smem + S::kK + st * S::kTileBytes);
+          const uint32_t d = tmem + T::kS + g * T::kSStride;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ss(d, smem_desc(q_addr + kk * 32, 16, 1024, kSwizzle128B),
+                         smem_desc(k_addr + kk * 32, 16, 1024, kSwizzle128B), idesc_qk, kk > 0);
+          umma_commit(s_full + g);
+          if (g) ++uses[1]; else ++uses[0];
+          if (n == (g ? ntB : ntA) - 1) umma_commit(q_empty + g);   // the item's Q is free
+        }
+        gn0 += ntA + ntB;
+      }
+    } else if (warp == 2 && lane == 0) {
+      // ------------------------------ P*V issuer --------------------------------
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, 64, false, true);
+      bool ok = true;
+      int gn0 = 0;
+      int uses[2] = {0, 0};   // P_g handed over so far (p_full phases)
+      for (int p = 0, itA = blockIdx.x; ok && itA < n_items; ++p, itA += 2 * G) {
+        const bool hasB = itA + G < n_items;
+        const int ntA = item_of(itA, nq, P).tiles.count();
+        const int ntB = hasB ? item_of(itA + G, nq, P).tiles.count() : 0;
+        for (int j = 0; ok && j < ntA + ntB; ++j) {
+          int g, n;
+          if (kInterleave) {
+            const int both = 2 * min(ntA, ntB);
+            g = j < both ? (j & 1) : (ntA > ntB ? 0 : 1);
+            n = j < both ? (j >> 1) : (j - both) + min(ntA, ntB);
+          } else {
+            g = j < ntA ? 0 : 1;
+            n = j < ntA ? j : j - ntA;
+          }
+          const int gn = gn0 + j, st = gn % NS;
+          const int ug = g ? uses[1] : uses[0];
+          const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kTileBytes);
+          const uint32_t a = tmem + T::kP + g * T::kPStride;
+          const uint32_t d = tmem + T::kO + g * T::kOStride;
+          // An item's first tile overwrites O_g: its group read the previous item's O in the
+          // epilogue before handing over this P.
+          const uint32_t acc = n > 0;
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            if (kk % (kBN / 32) == 0) {
+              if (!(ok = mbar_wait(p_full + 2 * g + kk / (kBN / 32), ug & 1, abort, status)))
+                break;
+              tc_fence_after();
+            }
+            umma_bf16_ts(d, a + kk * 8, smem_desc(v_addr + kk * 2048, kBN * 128, 1024, kSwizzle128B),
+                         idesc_pv, acc | (kk > 0));
+          }
+          if (!ok) break;
+          if (g) ++uses[1]; else ++uses[0];
+          umma_commit(kv_empty + st);
+          if (n == (g ? ntB : ntA) - 1) umma_commit(o_done + g);   // the item's O is complete
+        }
+        gn0 += ntA + ntB;
+      }
+    }
+  } else {
+    setmaxnreg_inc<kRegsSoftmax>();
+    // ------------------------------ softmax groups ----------------------------
+    const int grp = (warp - 4) >> 2;                    // 0: the pairs' A items, 1: their B items
+    const int row = 32 * (warp & 3) + lane;             // TMEM lane == query row
+    const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
+    const uint32_t t_s = tmem + T::kS + grp * T::kSStride + lane_off;
+    const uint32_t t_p = tmem + T::kP + grp * T::kPStride + lane_off;
+    const uint32_t t_o = tmem + T::kO + grp * T::kOStride + lane_off;
+    const uint32_t bar = 2 + grp;                       // the group's named barrier
+    const uint32_t stage_row = smem_u32(smem + S::kStage) + (grp * kBM + row) * S::kStageStride;
+    int* dst_tok = s_dst + grp * kBM;
+    const int b4 = P.b * kStripes;
+    const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
+    bool ok = true;
+    int gn0 = 0;           // ring index of the pair's first tile
+    int uses = 0;          // tiles of this group so far (s_full phases)
+    bool s_ready = false;  // the next s_full phase was already seen complete
+    for (int p = 0, itA = blockIdx.x; itA < n_items; ++p, itA += 2 * G) {
+      const int itB = itA + G;
+      const bool hasB = itB < n_items;
+      if (grp == 1 && !hasB) break;                    // the CTA's last pair has no B
+      const Item I = item_of(grp ? itB : itA, nq, P);
+      const int nt = I.tiles.count();
+      const int nt_other = grp ? item_of(itA, nq, P).tiles.count()
+                               : (hasB ? item_of(itB, nq, P).tiles.count() : 0);
+      const int ntA = grp ? nt_other : nt, ntB = grp ? nt : nt_other;
+      const int qrow = I.q0 + row;
+      const bool store = qrow < P.N;
+      const int u_i = I.uh / P.heads, h_i = I.uh - u_i * P.heads;
+      const int perm_t =
+          store ? __ldg(P.perm + (size_t)u_i * P.N + blockmajor_to_canonical(qrow, P.b, P.L)) : 0;
+      const int a_q = min(qrow, P.N - 1) / b4;
+      const int s_q = band_start(a_q, P.W, P.nb);
+      const int band_lo = s_q * b4, band_hi = (s_q + P.W) * b4, glob_hi = P.g * b4;
+      float m_ref = -INFINITY, l_run = 0.f;
+      for (int n = 0; ok && n < nt; ++n) {
+        if (!__all_sync(0xffffffffu, s_ready))
+          ok = __all_sync(0xffffffffu, mbar_wait(s_full + grp, uses & 1, abort, status));
+        ++uses;
+        if (!ok) break;
+        tc_fence_after();
+        float sv[kBN];
+        {
+          uint32_t r[128];
+          tmem_ld128(t_s, r);
+#pragma unroll
+          for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(r[i]);
+        }
+        // P*V of the item's previous tile must be done before P_g is rewritten (the previous
+        // item's are: the epilogue waited for them). Tested now, waited for after the row max.
+        const int gprev = n >= 1 ? gn0 + pair_tile_index<kInterleave>(grp, n - 1, ntA, ntB) : 0;
+        tc_fence_before();
+        mbar_arrive(s_free + grp);   // S_g may now be overwritten by the next Q*K^T into it
+        const bool prev_pv_done = n == 0 || mbar_test(kv_empty + gprev % NS, (gprev / NS) & 1);
+        const int c0 = I.tiles.tile(n) * kBN;
+        if (!tile_full(c0, P)) {
+          const int e0 = min(glob_hi, P.N) - c0, s1 = band_lo - c0, e1 = min(band_hi, P.N) - c0;
+          uint32_t km[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) km[k] = run_bits(0, e0, 32 * k) | run_bits(s1, e1, 32 * k);
+#pragma unroll
+          for (int i = 0; i < kBN; ++i)
+            sv[i] = (km[i >> 5] >> (i & 31)) & 1u ? sv[i] : -INFINITY;
+        }
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmax3(sv[k], sv[k + 8], sv[k + 16]);
+#pragma unroll
+        for (int t = 3; t + 1 < 16; t += 2)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv[k + 8 * t], sv[k + 8 * t + 8]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], sv[k + 8 * 15]);
+        const float x_max = fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])),
+                                  fmaxf(mx[6], mx[7])) *
+                            P.scale_log2;
+        // Lazy rescale of the reference max, as in k_attn.
+        const bool grow = x_max > m_ref + kLazyRescale;
+        const bool rescale = __any_sync(0xffffffffu, grow);
+        float alpha = 1.f;
+        if (rescale) {
+          const float m_new = grow ? x_max : m_ref;
+          alpha = (m_ref == -INFINITY) ? 0.f : ex2_mufu(m_ref - m_new);
+          l_run *= alpha;
+          m_ref = m_new;
+        }
+        const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const uint64_t nref2 = f2_pack(-ref, -ref);
+        uint64_t sum2a = 0, sum2b = 0;
+        if (n >= 1) {
+          if (!__all_sync(0xffffffffu, prev_pv_done)) {
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(kv_empty + gprev % NS, (gprev / NS) & 1, abort, status));
+            if (!ok) break;
+          }
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pw[32];
+#pragma unroll
+          for (int i2 = 0; i2 < 32; ++i2) {
+            const int i = 64 * half + 2 * i2;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), scale2, nref2), x0, x1);
+            const float p0 = ex2_mufu(x0), p1 = ex2_mufu(x1);
+            if (i2 & 1)
+              sum2b = f2_add(sum2b, f2_pack(p0, p1));
+            else
+              sum2a = f2_add(sum2a, f2_pack(p0, p1));
+            pw[i2] = pack_bf16_pos(p0, p1);
+          }
+          tmem_st32_async(t_p + 32 * half, pw);
+          if (half == 0 && rescale && n > 0) {
+            // O_g holds the item's earlier tiles (their P*V completed: waited above).
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+              uint32_t o[32];
+              tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32_async(t_o + c * 32, o);
+            }
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(p_full + 2 * grp + half);
+        }
+        s_ready = mbar_test(s_full + grp, uses & 1);
+        float sa0, sa1;
+        f2_unpack(f2_add(sum2a, sum2b), sa0, sa1);
+        l_run += sa0 + sa1;
+      }
+      // ---- the group's item: normalise its rows and scatter them to out[u, perm[p], h, :] ----
+      // The group's threads all pass both named barriers once per item, also after a failed
+      // wait.
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done + grp, p & 1, abort, status));
+      tc_fence_after();
+      named_barrier(bar, 128);   // the group's previous copy-out is done with the staging rows
+      if (ok) {
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        uint32_t x0[32], x1[32];
+        tmem_ld32_pair(t_o, t_o + 32, x0, x1);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t* u = c < 4 ? x0 + 8 * c : x1 + 8 * (c - 4);
+          st_shared_v4(stage_row + c * 16,
+                       pack_bf16(__uint_as_float(u[0]) * inv, __uint_as_float(u[1]) * inv),
+                       pack_bf16(__uint_as_float(u[2]) * inv, __uint_as_float(u[3]) * inv),
+                       pack_bf16(__uint_as_float(u[4]) * inv, __uint_as_float(u[5]) * inv),
+                       pack_bf16(__uint_as_float(u[6]) * inv, __uint_as_float(u[7]) * inv));
+        }
+        dst_tok[row] = store ? min(max(perm_t, 0), P.N - 1) : -1;
+      }
+      tc_fence_before();   // O_g is read before the next item's first P goes to P*V
+      named_barrier(bar, 128);
+      if (ok) {
+        constexpr int kCpr = 8;                          // 16-byte chunks per 64-column row
+        const int tid = threadIdx.x - 128 * (1 + grp);   // 0..127 within the group
+        const uint32_t stage = smem_u32(smem + S::kStage) + grp * kBM * S::kStageStride;
+        uint8_t* out_uh =
+            reinterpret_cast<uint8_t*>(P.out) + ((size_t)u_i * P.N * P.heads + h_i) * 64 * 2;
+#pragma unroll 4
+        for (int k = 0; k < kBM * kCpr / 128; ++k) {
+          const int q = tid + 128 * k;
+          const int r = q / kCpr, c = q - r * kCpr;
+          const int t = dst_tok[r];
+          if (t >= 0) {
+            const uint4 v = ld_shared_v4(stage + r * S::kStageStride + c * 16);
+            *reinterpret_cast<uint4*>(out_uh + (size_t)t * P.heads * 64 * 2 + c * 16) = v;
+          }
+        }
+      }
+      gn0 += ntA + ntB;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 template <int DH>
 static cudaError_t launch_attn_dh(const CUtensorMap* tq, const CUtensorMap* tk,
                                   const CUtensorMap* tv, const CUtensorMap* tq_tail,
@@ -698,11 +1113,34 @@ static cudaError_t launch_attn_dh(const CUtensorMap* tq, const CUtensorMap* tk,
                     *tk_tail, *tv_tail, p, status);
 }
 
+static cudaError_t launch_attn_pairs(const CUtensorMap* tq, const CUtensorMap* tk,
+                                     const CUtensorMap* tv, const AttnParams& p, int* status,
+                                     cudaStream_t st) {
+  using S = AttnPairSmem;
+  auto kernel = k_attn_pairs<kPairInterleave>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc);
+  if (e != cudaSuccess) return e;
+  const int items = ((p.N + kBM - 1) / kBM) * p.U * p.heads;
+  dim3 grid(std::max(1, std::min((items + 1) / 2, p.sms)));
+  return launch_pdl(kernel, grid, dim3(kAttnThreads), S::kAlloc, st, *tq, *tk, *tv, p, status);
+}
+
 cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                         const CUtensorMap* tq_tail, const CUtensorMap* tk_tail,
                         const CUtensorMap* tv_tail, const AttnParams& p, int dh, int* status,
                         cudaStream_t st) {
-  if (dh == 64) return launch_attn_dh<64>(tq, tk, tv, tq, tk, tv, p, status, st);
+  if (dh == 64) {
+    // Short items (at most kPairTiles key tiles per query tile, as in windowed blocks) go to the
+    // whole-item-per-group kernel.
+    const int nq = (p.N + kBM - 1) / kBM;
+    int nt_max = 0;
+    for (int qt = 0; qt < nq; ++qt)
+      nt_max = std::max(nt_max,
+                        key_tiles(qt * kBM, std::min(qt * kBM + kBM, p.N) - 1, qt, 0, p).count());
+    if (nt_max <= kPairTiles) return launch_attn_pairs(tq, tk, tv, p, status, st);
+    return launch_attn_dh<64>(tq, tk, tv, tq, tk, tv, p, status, st);
+  }
   if (dh == 80) return launch_attn_dh<80>(tq, tk, tv, tq_tail, tk_tail, tv_tail, p, status, st);
   return cudaErrorInvalidValue;
 }

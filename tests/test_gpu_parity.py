@@ -133,6 +133,7 @@ def _attn_case(cfg, seed, scale=1.0, heads_check=None, units_check=None):
     (1, 16, 16, "global", 2, 80, 0.4),     # head_dim 80
     (1, 28, 28, "window", 2, 64, 0.3),     # 4 windows of 196 tokens: ragged tail tile
     (1, 20, 20, "window", 1, 80, 0.5),     # windows with pads, dh 80
+    (4, 56, 56, "window", 4, 64, 0.4),     # 512 short items: CTAs run two or more item pairs
     (1, 4, 4, "global", 1, 64, 0.6),       # N=16, b=1
     (1, 6, 6, "global", 3, 64, 0.5),       # N=36, b=1, nb=9
     (1, 48, 48, "global", 2, 64, 0.4),     # N=2304, b=64 (L=576 -> b=64, nb=9)
