@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
-  __syncthreads();
+  cta_sync_converged();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   griddep_wait();   // Q, K, V and perm come from the work before this launch
@@ -678,7 +678,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync_converged();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -764,7 +764,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
-  __syncthreads();
+  cta_sync_converged();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   griddep_wait();   // Q, K, V and perm come from the work before this launch
@@ -1091,7 +1091,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync_converged();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

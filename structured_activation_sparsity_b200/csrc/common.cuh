@@ -59,6 +59,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// CTA-wide barrier for kernels whose warps split into roles: each warp first reconverges (its
+// lanes may come from different paths, e.g. lane 0 from a long producer loop and lanes 1-31
+// straight from the role dispatch), then the whole CTA meets. Without the warp reconvergence,
+// measured on B200, a lane returning late from a role loop passed the final __syncthreads while
+// the epilogue warps were still working: the barrier did not order their TMEM reads before the
+// dealloc that follows it.
+__device__ __forceinline__ void cta_sync_converged() {
+  __syncwarp();
+  __syncthreads();
+}
 // Non-blocking test of a phase (no suspend). Its ~150-cycle latency overlaps whatever work sits
 // between it and the first use of the result.
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {

@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   if (warp == 1) tmem_alloc(tmem_slot, G::kTmemCols);
   tc_fence_before();
-  __syncthreads();
+  cta_sync_converged();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   griddep_wait();   // A, B and the epilogue's x come from the work before this launch
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync_converged();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, G::kTmemCols);

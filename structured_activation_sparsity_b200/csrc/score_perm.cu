@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __rest
       if (t < N) s_key[t] = k8[e];
     }
   }
-  __syncthreads();
+  cta_sync_converged();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 32 + lane;
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __rest
   for (; o < hi; ++o) c0 += s_key[o] > kt;
   const int cnt = (c0 + c1) + (c2 + c3);
   s_cnt[warp][lane] = cnt;
-  __syncthreads();
+  cta_sync_converged();
   if (warp == 0 && t < N) {
     int r = 0;
 #pragma unroll
