@@ -183,7 +183,7 @@ MlpPlan mlp_plan(const Geo& g, int K, int C, int hidden) {
   const int tiles = (p.fc1.m_tiles * p.fc1.n_tiles > p.fc2.m_tiles * p.fc2.n_tiles)
                         ? p.fc1.m_tiles * p.fc1.n_tiles
                         : p.fc2.m_tiles * p.fc2.n_tiles;
-  const size_t cnt = part ? align256((size_t)tiles * 4) : 0;
+  const size_t cnt = part ? align256((size_t)tiles * 2 * 4) : 0;   // two counters per tile
   p.xk = 0;
   p.h = xk_bytes;
   p.partial = xk_bytes + h_bytes;

@@ -99,6 +99,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Waits until the global counter reaches `target` (acquire: what the writers stored before their
+// release is visible afterwards). Bounded like mbar_wait.
+__device__ __forceinline__ bool wait_counter_geq(const int* counter, int target,
+                                                 volatile int* abort, int* status) {
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+    if (v >= target) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_timeout(status);
+      *abort = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
+// Adds to a global counter with release semantics (this thread's earlier writes, and those it
+// has observed, become visible to an acquire that sees the new value).
+__device__ __forceinline__ int add_release(int* counter, int v) {
+  int old;
+  asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(counter), "r"(v)
+               : "memory");
+  return old;
+}
+
 // ---------------------------------------------------------------------------------------------
 // TMA tile loads (no multicast)
 // ---------------------------------------------------------------------------------------------
@@ -299,6 +328,16 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float rcp_mufu(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

@@ -59,12 +59,17 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* keep, uint16_t*
 // unit overlaps the mainloop of the next.
 //   warp 0      TMA producer (A and B k-blocks into a multi-stage ring, across units)
 //   warp 1      TMEM allocator and tcgen05.mma issuer
-//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4).. and one half of the tile's columns
+//   warps 2-3   idle (complete the first warpgroup for the register split)
+//   warps 4-11  epilogue: warp w reads TMEM lanes 32*(w%4).. and one half of the tile's columns
 // A k-split unit writes its fp32 partial tile to its own slot; the last unit of a tile to finish
 // (an atomic counter per tile) sums the slots in split order and applies the epilogue, so the
 // result does not depend on which split finished last.
-constexpr int kGemmThreads = 320;
+constexpr int kGemmThreads = 384;
 constexpr int kEpiThreads = 256;
+// Register split (launch: 384 threads x 168): producer warpgroup 56, epilogue warpgroups 224.
+constexpr uint32_t kGemmRegsProducer = 56, kGemmRegsEpilogue = 224;
+static_assert(128 * kGemmRegsProducer + 256 * kGemmRegsEpilogue <= 384 * 168,
+              "GEMM register split too large");
 
 // KSUB 64-wide K sub-blocks per pipeline stage: each full/empty handshake (an mbarrier wait costs
 // ~150 cycles of latency on the thread that gates on it) then covers KSUB x 4 MMAs.
@@ -90,23 +95,36 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // Mathematical Functions, formula 7.1.26 (|error| <= 1.5e-7, far below the bf16 rounding of the
 // result): for x >= 0, erfc(x) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) e^(-x^2), t = 1/(1 + p x).
 // Then GELU(z) = z/2 erfc(|z|/sqrt 2) for z < 0 and z/2 (2 - erfc(|z|/sqrt 2)) for z >= 0, which
-// keeps the relative accuracy of the small negative tail. Two MUFU ops (reciprocal, 2^x) and a
-// handful of FMAs, so the fc1 epilogue does not crowd out the MMA-issuing thread.
-__device__ __forceinline__ float gelu_erf(float z) {
-  const float x = fabsf(z) * 0.70710678118654752f;
-  const float t = __fdividef(1.0f, fmaf(0.3275911f, x, 1.0f));
-  const float poly =
-      t * fmaf(fmaf(fmaf(fmaf(1.061405429f, t, -1.453152027f), t, 1.421413741f), t, -0.284496736f),
-               t, 0.254829592f);
-  const float erfc_x = poly * ex2_mufu(-(x * x) * 1.4426950408889634f);
-  return 0.5f * z * (z >= 0.f ? 2.0f - erfc_x : erfc_x);
+// keeps the relative accuracy of the small negative tail. Two MUFU ops (reciprocal, 2^x) per value;
+// the rest runs on a pair of values at once in packed fp32x2 arithmetic (the same roundings as
+// scalar operations), halving the FMA-pipe instructions of the fc1 epilogue.
+__device__ __forceinline__ void gelu_erf2(float& z0, float& z1) {
+  const uint64_t x = f2_mul(f2_pack(fabsf(z0), fabsf(z1)),
+                            f2_pack(0.70710678118654752f, 0.70710678118654752f));
+  float d0, d1;
+  f2_unpack(f2_fma(f2_pack(0.3275911f, 0.3275911f), x, f2_pack(1.0f, 1.0f)), d0, d1);
+  const uint64_t t = f2_pack(rcp_mufu(d0), rcp_mufu(d1));
+  uint64_t q = f2_fma(f2_pack(1.061405429f, 1.061405429f), t, f2_pack(-1.453152027f, -1.453152027f));
+  q = f2_fma(q, t, f2_pack(1.421413741f, 1.421413741f));
+  q = f2_fma(q, t, f2_pack(-0.284496736f, -0.284496736f));
+  q = f2_fma(q, t, f2_pack(0.254829592f, 0.254829592f));
+  float a0, a1;   // -x^2 log2(e)
+  f2_unpack(f2_mul(f2_mul(x, x), f2_pack(-1.4426950408889634f, -1.4426950408889634f)), a0, a1);
+  const uint64_t erfc = f2_mul(f2_mul(t, q), f2_pack(ex2_mufu(a0), ex2_mufu(a1)));
+  float e0, e1, m0, m1;   // erfc and 2 - erfc
+  f2_unpack(erfc, e0, e1);
+  f2_unpack(f2_fma(erfc, f2_pack(-1.0f, -1.0f), f2_pack(2.0f, 2.0f)), m0, m1);
+  const uint64_t w = f2_pack(z0 >= 0.f ? m0 : e0, z1 >= 0.f ? m1 : e1);
+  f2_unpack(f2_mul(f2_mul(f2_pack(z0, z1), f2_pack(0.5f, 0.5f)), w), z0, z1);
 }
 
 struct GemmShape {
   int M, N, Kd;
   int m_tiles, n_tiles, splits, kb_total;
-  float* partial;          // [tiles][splits][BN][128] fp32, column-major tiles (splits > 1)
-  int* counters;           // [tiles], zero on entry (splits > 1)
+  int paired;              // two k-splits, every unit resident at once: each finishes half
+  float* partial;          // splits > 1: [tiles][splits][BN][128] fp32, column-major tiles;
+                           // paired: [tiles][2 halves][BN/2][128]
+  int* counters;           // [tiles][2], zero on entry (splits > 1)
 };
 
 // The epilogue of one output row m (< M) in chunks of 32 columns. The row's destination (and, for
@@ -134,6 +152,10 @@ __device__ __forceinline__ void epi_load(const GemmEpilogue& ep, const uint16_t*
     for (int q = 0; q < 4; ++q) in.x[q] = xp[q];
   }
 }
+// v0, v1 += the two bf16 values of w (packed fp32x2 add).
+__device__ __forceinline__ void f2_add_bf16(float& v0, float& v1, uint32_t w) {
+  f2_unpack(f2_add(f2_pack(v0, v1), f2_pack(bf16_lo(w), bf16_hi(w))), v0, v1);
+}
 // Kind 0: row[n..n+32) = bf16(GELU(v + bias)). Kind 1: row[n..n+32) = bf16(x + v + bias).
 __device__ __forceinline__ void epi_store(const GemmEpilogue& ep, uint16_t* row, int n,
                                           const Epi32In& in, float (&v)[32]) {
@@ -142,24 +164,18 @@ __device__ __forceinline__ void epi_store(const GemmEpilogue& ep, uint16_t* row,
     for (int q = 0; q < 4; ++q) {
       const uint32_t w[4] = {in.b[q].x, in.b[q].y, in.b[q].z, in.b[q].w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[q * 8 + 2 * e] += bf16_lo(w[e]);
-        v[q * 8 + 2 * e + 1] += bf16_hi(w[e]);
-      }
+      for (int e = 0; e < 4; ++e) f2_add_bf16(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1], w[e]);
     }
   }
   if (ep.kind == 0) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+    for (int i = 0; i < 16; ++i) gelu_erf2(v[2 * i], v[2 * i + 1]);
   } else {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint32_t w[4] = {in.x[q].x, in.x[q].y, in.x[q].z, in.x[q].w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[q * 8 + 2 * e] += bf16_lo(w[e]);
-        v[q * 8 + 2 * e + 1] += bf16_hi(w[e]);
-      }
+      for (int e = 0; e < 4; ++e) f2_add_bf16(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1], w[e]);
     }
   }
   uint4* d = reinterpret_cast<uint4*>(row + n);
@@ -212,8 +228,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   cta_sync_converged();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  griddep_wait();   // A, B and the epilogue's x come from the work before this launch
-  griddep_launch();
+  // A and the epilogue's x come from the work before this launch; the producer waits for it
+  // itself, after requesting the B (weight) tiles that do not depend on it.
+  const bool producer = warp == 0 && lane == 0;
+  if (!producer) {
+    griddep_wait();
+    griddep_launch();
+  }
 
   auto decode = [&](int u, int& m, int& n, int& s, int& kb0, int& kb1) {
     m = u % g.m_tiles;
@@ -224,10 +245,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     kb1 = (int)((long long)(s + 1) * g.kb_total / g.splits);
   };
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp < 4) {
+    setmaxnreg_dec<kGemmRegsProducer>();
+    if (producer) {
       tma_prefetch_desc(&ta);
       tma_prefetch_desc(&tb);
+      // B tiles of the first unit's first stages, before the wait for the previous work.
+      int pre = 0;
+      if (blockIdx.x < units) {
+        int m, n, s, kb0, kb1;
+        decode(blockIdx.x, m, n, s, kb0, kb1);
+        const int nst = (kb1 - kb0) / KSUB, rot = blockIdx.x % nst;
+        pre = nst < G::kStages ? nst : G::kStages;
+        for (int j = 0; j < pre; ++j) {
+          const int kb = kb0 + ((j + rot) % nst) * KSUB;
+          uint8_t* sb = smem + j * G::kStageBytes + KSUB * G::kABytes;
+          mbar_expect_tx(full + j, G::kStageBytes);
+#pragma unroll
+          for (int q = 0; q < KSUB; ++q)
+            tma_load_2d(sb + q * G::kBBytes, &tb, full + j, (kb + q) * 64, n * BN);
+        }
+      }
+      griddep_wait();
+      griddep_launch();
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
@@ -242,17 +282,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           uint8_t* sa = smem + st * G::kStageBytes;
           uint8_t* sb = sa + KSUB * G::kABytes;
-          mbar_expect_tx(full + st, G::kStageBytes);
+          const bool b_done = it < pre;   // B of this stage requested before the wait
+          if (!b_done) mbar_expect_tx(full + st, G::kStageBytes);
 #pragma unroll
           for (int q = 0; q < KSUB; ++q) {
             tma_load_2d(sa + q * G::kABytes, &ta, full + st, (kb + q) * 64, m * 128);
-            tma_load_2d(sb + q * G::kBBytes, &tb, full + st, (kb + q) * 64, n * BN);
+            if (!b_done) tma_load_2d(sb + q * G::kBBytes, &tb, full + st, (kb + q) * 64, n * BN);
           }
         }
       }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
       int it = 0, i = 0;
       bool ok = true;
@@ -288,8 +327,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else {
+    setmaxnreg_inc<kGemmRegsEpilogue>();
     // ------------------------------ epilogue warps ----------------------------
-    const int ew = warp - 2;                              // 0..7
+    const int ew = warp - 4;                              // 0..7
     const int row = 32 * (warp & 3) + lane;               // TMEM lane
     const int col0 = (ew >> 2) * G::kHalf;                // this warp's half of the columns
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
@@ -332,6 +372,60 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             epi_store(ep, drow, n, in, v);
           }
         }
+      } else if (g.paired) {
+        // Two k-splits of the tile run at the same time in two CTAs; split s finishes column half
+        // s. This unit's warps of the other half hand their accumulator columns to the partner
+        // as an fp32 partial (column-major: a warp's 32 rows of one column are one 128-byte
+        // line) and count themselves on that half's counter; the warps of half s wait for the
+        // partner's four, then add its partial to their own columns (acc_s + partial_(1-s): for
+        // two terms the same sum as p0 + p1 in either order) and apply the epilogue.
+        const int half = ew >> 2;
+        float* part = g.partial + ((size_t)tile * 2 + half) * 128 * G::kHalf + row;
+        int* count = g.counters + tile * 2 + half;
+        if (half != s) {
+#pragma unroll 1
+          for (int c = 0; c < G::kHalf / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(t_acc + c * 32, r);
+            if (c == G::kHalf / 32 - 1) {
+              tc_fence_before();
+              mbar_arrive(acc_empty + buf);
+            }
+#pragma unroll
+            for (int e = 0; e < 32; ++e) part[(size_t)(c * 32 + e) * 128] = __uint_as_float(r[e]);
+          }
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) add_release(count, 1);   // the warp's 32 rows of the half are written
+        } else {
+          // Every lane acquires the counter itself before reading the partial.
+          if (!__all_sync(0xffffffffu, wait_counter_geq(count, 4, abort, status))) break;
+#pragma unroll 1
+          for (int c = 0; c < G::kHalf / 32; ++c) {
+            const int n = n_t * BN + col0 + c * 32;
+            Epi32In in;
+            float w[32];
+            if (drow) {
+              epi_load(ep, drow, n, in);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) w[e] = __ldcg(part + (size_t)(c * 32 + e) * 128);
+            }
+            uint32_t r[32];
+            tmem_ld32(t_acc + c * 32, r);
+            if (c == G::kHalf / 32 - 1) {
+              tc_fence_before();
+              mbar_arrive(acc_empty + buf);
+            }
+            if (drow) {
+              float v[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]) + w[e];
+              epi_store(ep, drow, n, in, v);
+            }
+          }
+          // The last of the four owner warps re-arms the counter (for a later GEMM sharing it).
+          if (lane == 0 && atomicAdd(count, 1) == 7) atomicExch(count, 0);
+        }
       } else {
         // Write this split's partial tile (column-major, so a warp's 32 rows of one column are
         // one 128-byte line), then let the last split of the tile finish it.
@@ -349,7 +443,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __threadfence();
         if (!epi_sync()) break;
-        if (threadIdx.x == 64) *s_last = atomicAdd(g.counters + tile, 1) == g.splits - 1;
+        if (threadIdx.x == 128) *s_last = atomicAdd(g.counters + tile, 1) == g.splits - 1;
         if (!epi_sync()) break;
         if (*s_last) {
           __threadfence();
@@ -378,7 +472,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               epi_store(ep, drow, n, in, v);
             }
           }
-          if (threadIdx.x == 64) g.counters[tile] = 0;
+          if (threadIdx.x == 128) g.counters[tile] = 0;
         }
         if (!epi_sync()) break;   // s_last is reused by the next unit
       }
@@ -452,6 +546,9 @@ static cudaError_t launch_gemm_bn(const CUtensorMap* ta, const CUtensorMap* tb, 
   g.partial = partial;
   g.counters = counters;
   const int grid = p.units < sms ? p.units : sms;
+  // Every unit has its own CTA (one per SM, all resident together), so the two splits of a tile
+  // can wait for each other.
+  g.paired = p.splits == 2 && p.units <= grid;
   return launch_pdl(k_gemm<BN, KSUB>, dim3(grid), dim3(kGemmThreads), G::kAlloc, st, *ta, *tb, g, ep,
                     status);
 }

@@ -1,4 +1,4 @@
-"""The fc1 epilogue's GELU (csrc/mlp.cu, gelu_erf): erf by Abramowitz & Stegun, Handbook of
+"""The fc1 epilogue's GELU (csrc/mlp.cu, gelu_erf2): erf by Abramowitz & Stegun, Handbook of
 Mathematical Functions, formula 7.1.26, emulated step by step in float32 with the constants read from
 the kernel source, against the exact erf GELU in float64."""
 import os
@@ -13,12 +13,17 @@ MLP = os.path.join(ROOT, "structured_activation_sparsity_b200", "csrc", "mlp.cu"
 
 def _kernel_constants():
     src = open(MLP).read()
-    body = src[src.index("float gelu_erf(float z)"):]
+    body = src[src.index("void gelu_erf2(float& z0, float& z1)"):]
     body = body[: body.index("\n}\n")]
     nums = [float(v) for v in re.findall(r"-?\d+\.\d+(?=f)", body)]
-    # the literals other than the exact 0.5, 1, 2, in source order: 1/sqrt2, p, a5, a4, a3, a2,
-    # a1, log2(e)
-    return [np.float32(v) for v in nums if v not in (0.5, 1.0, 2.0)]
+    # each constant is written twice (one per lane of a packed pair)
+    assert all(a == b for a, b in zip(nums[0::2], nums[1::2])) and len(nums) % 2 == 0
+    nums = nums[0::2]
+    # the literals other than the exact 0.5, +-1, 2, in source order: 1/sqrt2, p, a5, a4, a3, a2,
+    # a1, -log2(e) (the kernel multiplies x^2 by it)
+    c = [v for v in nums if v not in (0.5, 1.0, -1.0, 2.0)]
+    c[-1] = -c[-1]
+    return [np.float32(v) for v in c]
 
 
 def _emulate(z, c):

@@ -196,6 +196,8 @@ def _mlp_case(cfg, C, Hd, seed, bias=True, images_check=None):
     (2, 16, 16, 128, 512, 0.5, False),
     (1, 32, 32, 256, 1024, 0.3, True),
     (3, 20, 20, 192, 320, 1.0, True),      # dense, N not a multiple of 128 (BN 64)
+    (1, 32, 32, 128, 2048, 0.4, True),     # fc2 split four ways along K: the last split finishes
+    (1, 48, 48, 384, 1536, 0.5, True),     # fc2 split two ways, all units resident: paired finish
 ])
 def test_rcmlp_small(B, H, W, C, Hd, d, bias):
     cfg = L.make_cfg(B, H, W, "global", 14, 1, 64, d)
