@@ -54,10 +54,14 @@ struct GemmEpilogue {
   int K_per_image, T;       // kind 1
 };
 // Tile width and k-split of C[M, N] = A[M, Kd] * B[N, Kd]^T for `sms` persistent CTAs.
+// tail: without a k-split, the tiles of a last, partial round of units that are each split in two
+// along K (two CTAs, finished as a pair), so that round takes half a unit (0: none).
 struct GemmPlan {
-  int bn, splits, m_tiles, n_tiles, units;
+  int bn, splits, m_tiles, n_tiles, units, tail;
 };
 GemmPlan gemm_plan(int M, int N, int Kd, int sms);
+// Tiles of the tail for `tiles` whole tiles of kb k-blocks over `sms` CTAs (0: no tail).
+int gemm_tail(int tiles, int kb, int sms);
 // fp32 partial-tile bytes the plan needs (0 without a k-split); plus one int counter per tile.
 size_t gemm_partial_bytes(const GemmPlan& p);
 // C = A B^T on tcgen05 with the given epilogue. partial / counters: workspace for k-splits

@@ -122,8 +122,9 @@ struct GemmShape {
   int M, N, Kd;
   int m_tiles, n_tiles, splits, kb_total;
   int paired;              // two k-splits, every unit resident at once: each finishes half
+  int units, whole;        // units; those from `whole` on are tail halves (see GemmPlan::tail)
   float* partial;          // splits > 1: [tiles][splits][BN][128] fp32, column-major tiles;
-                           // paired: [tiles][2 halves][BN/2][128]
+                           // paired: [tiles][2 halves][BN/2][128]; tail: [tail tiles][2][BN/2][128]
   int* counters;           // [tiles][2], zero on entry (splits > 1)
 };
 
@@ -208,7 +209,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int units = g.m_tiles * g.n_tiles * g.splits;
+  const int units = g.units;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < G::kStages; ++i) {
@@ -236,13 +237,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     griddep_launch();
   }
 
-  auto decode = [&](int u, int& m, int& n, int& s, int& kb0, int& kb1) {
-    m = u % g.m_tiles;
-    const int r = u / g.m_tiles;
-    n = r % g.n_tiles;
-    s = r / g.n_tiles;
-    kb0 = (int)((long long)s * g.kb_total / g.splits);
-    kb1 = (int)((long long)(s + 1) * g.kb_total / g.splits);
+  // Unit u -> tile (m, n), k-split s and its k-block range; pair: finished with its partner
+  // split (paired protocol), slot: the pair's partial and counter slot.
+  auto decode = [&](int u, int& m, int& n, int& s, int& kb0, int& kb1, int& slot, bool& pair) {
+    if (u < g.whole) {
+      m = u % g.m_tiles;
+      const int r = u / g.m_tiles;
+      n = r % g.n_tiles;
+      s = r / g.n_tiles;
+      kb0 = (int)((long long)s * g.kb_total / g.splits);
+      kb1 = (int)((long long)(s + 1) * g.kb_total / g.splits);
+      slot = n * g.m_tiles + m;
+      pair = g.paired;
+    } else {
+      // tail: units whole + 2i and whole + 2i + 1 are the two k-halves of tile whole + i
+      const int v = u - g.whole, t = g.whole + (v >> 1);
+      m = t % g.m_tiles;
+      n = t / g.m_tiles;
+      s = v & 1;
+      kb0 = s ? g.kb_total / 2 : 0;
+      kb1 = s ? g.kb_total : g.kb_total / 2;
+      slot = v >> 1;
+      pair = true;
+    }
   };
 
   if (warp < 4) {
@@ -253,8 +270,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // B tiles of the first unit's first stages, before the wait for the previous work.
       int pre = 0;
       if (blockIdx.x < units) {
-        int m, n, s, kb0, kb1;
-        decode(blockIdx.x, m, n, s, kb0, kb1);
+        int m, n, s, kb0, kb1, slot;
+        bool pair;
+        decode(blockIdx.x, m, n, s, kb0, kb1, slot, pair);
         const int nst = (kb1 - kb0) / KSUB, rot = blockIdx.x % nst;
         pre = nst < G::kStages ? nst : G::kStages;
         for (int j = 0; j < pre; ++j) {
@@ -271,8 +289,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
-        int m, n, s, kb0, kb1;
-        decode(u, m, n, s, kb0, kb1);
+        int m, n, s, kb0, kb1, slot;
+        bool pair;
+        decode(u, m, n, s, kb0, kb1, slot, pair);
         const int nst = (kb1 - kb0) / KSUB, rot = u % nst;
         for (int j = 0; j < nst; ++j, ++it) {
           const int kb = kb0 + ((j + rot) % nst) * KSUB;   // rotated start: spread over L2 slices
@@ -296,8 +315,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int it = 0, i = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++i) {
-        int m, n, s, kb0, kb1;
-        decode(u, m, n, s, kb0, kb1);
+        int m, n, s, kb0, kb1, slot;
+        bool pair;
+        decode(u, m, n, s, kb0, kb1, slot, pair);
         const int buf = i & 1;
         if (i >= 2 && !(ok = mbar_wait(acc_empty + buf, ((i >> 1) - 1) & 1, abort, status))) break;
         tc_fence_after();
@@ -343,8 +363,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     };
     int i = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
-      int m_t, n_t, s, kb0, kb1;
-      decode(u, m_t, n_t, s, kb0, kb1);
+      int m_t, n_t, s, kb0, kb1, slot;
+      bool pair;
+      decode(u, m_t, n_t, s, kb0, kb1, slot, pair);
       const int buf = i & 1;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full + buf, (i >> 1) & 1, abort, status));
       if (!ok) break;
@@ -353,7 +374,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int tile = n_t * g.m_tiles + m_t;
       const uint32_t t_acc = tmem + buf * BN + lane_off + col0;
       uint16_t* drow = m < g.M ? epi_row(ep, g, m) : nullptr;
-      if (g.splits == 1) {
+      if (g.splits == 1 && !pair) {
 #pragma unroll 1
         for (int c = 0; c < G::kHalf / 32; ++c) {
           const int n = n_t * BN + col0 + c * 32;
@@ -372,7 +393,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             epi_store(ep, drow, n, in, v);
           }
         }
-      } else if (g.paired) {
+      } else if (pair) {
         // Two k-splits of the tile run at the same time in two CTAs; split s finishes column half
         // s. This unit's warps of the other half hand their accumulator columns to the partner
         // as an fp32 partial (column-major: a warp's 32 rows of one column are one 128-byte
@@ -380,8 +401,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // partner's four, then add its partial to their own columns (acc_s + partial_(1-s): for
         // two terms the same sum as p0 + p1 in either order) and apply the epilogue.
         const int half = ew >> 2;
-        float* part = g.partial + ((size_t)tile * 2 + half) * 128 * G::kHalf + row;
-        int* count = g.counters + tile * 2 + half;
+        float* part = g.partial + ((size_t)slot * 2 + half) * 128 * G::kHalf + row;
+        int* count = g.counters + slot * 2 + half;
         if (half != s) {
 #pragma unroll 1
           for (int c = 0; c < G::kHalf / 32; ++c) {
@@ -496,34 +517,52 @@ GemmPlan gemm_plan(int M, int N, int Kd, int sms) {
   // units over the CTAs, times k-blocks per unit, times (128 + BN); a k-split adds the unit's fp32
   // partial tile written (4 BN rows' worth) and, for the unit that finishes the tile, all `s`
   // partials read back. Splits only for long K (>= 24 k-blocks).
+  // Without a k-split, a last partial round of R <= sms/2 tiles runs as 2R k-halves (the tail),
+  // which costs half a unit plus the pair's partial exchange.
   long long best = -1;
   p.bn = 64;
   p.splits = 1;
+  p.tail = 0;
   for (int bn : {256, 192, 128, 64}) {
     if (N % bn) continue;
     const int n_tiles = N / bn;
     for (int s = 1; s <= 8; ++s) {
       if (s > 1 && (kb < 24 || kb / s < 4)) break;
       const long long units = (long long)m_tiles * n_tiles * s;
-      const long long rounds = (units + sms - 1) / sms;
+      long long rounds = (units + sms - 1) / sms;
       const long long kb_unit = (kb + s - 1) / s;
       const long long partial = s > 1 ? (rounds + s) * 4LL * bn : 0;
-      const long long cost = rounds * kb_unit * (128 + bn) + partial;
+      long long cost = rounds * kb_unit * (128 + bn) + partial;
+      int tail = 0;
+      if (s == 1) {
+        tail = gemm_tail(m_tiles * n_tiles, kb, sms);
+        if (tail) cost = (rounds - 1) * kb * (128 + bn) + (kb / 2) * (128 + bn) + 2 * 4LL * bn;
+      }
       if (best < 0 || cost < best) {
         best = cost;
         p.bn = bn;
         p.splits = s;
+        p.tail = tail;
       }
     }
   }
   p.m_tiles = m_tiles;
   p.n_tiles = N / p.bn;
-  p.units = m_tiles * p.n_tiles * p.splits;
+  p.units = m_tiles * p.n_tiles * p.splits + p.tail;
   return p;
 }
 
+// Only for long K: the halves save kb/2 k-blocks of mainloop, while the pair's partial exchange
+// and the unchanged epilogue of the last unit cost a fixed amount (measured on B200: a loss at 12
+// k-blocks, about even at 16 and 20, a clear gain at 80).
+constexpr int kTailMinKb = 24;
+int gemm_tail(int tiles, int kb, int sms) {
+  const int r = tiles % sms;
+  return tiles > sms && r > 0 && 2 * r <= sms && kb >= kTailMinKb && kb % 2 == 0 ? r : 0;
+}
+
 size_t gemm_partial_bytes(const GemmPlan& p) {
-  if (p.splits == 1) return 0;
+  if (p.splits == 1) return (size_t)p.tail * 128 * p.bn * 4;
   return (size_t)p.m_tiles * p.n_tiles * p.splits * 128 * p.bn * 4;
 }
 
@@ -545,10 +584,18 @@ static cudaError_t launch_gemm_bn(const CUtensorMap* ta, const CUtensorMap* tb, 
   g.kb_total = Kd / 64;
   g.partial = partial;
   g.counters = counters;
-  const int grid = p.units < sms ? p.units : sms;
+  // The tail as planned holds only for the SM count it was planned for (its partial workspace
+  // is sized by it); on another count the last round runs whole tiles.
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int tail =
+      p.splits == 1 && p.tail > 0 && gemm_tail(tiles, g.kb_total, sms) == p.tail ? p.tail : 0;
+  g.units = tiles * p.splits + tail;
+  g.whole = tiles * p.splits - tail;
+  const int grid = g.units < sms ? g.units : sms;
   // Every unit has its own CTA (one per SM, all resident together), so the two splits of a tile
-  // can wait for each other.
-  g.paired = p.splits == 2 && p.units <= grid;
+  // can wait for each other; the tail halves all run in the last round, every CTA's earlier units
+  // waiting on nothing.
+  g.paired = p.splits == 2 && g.units <= grid;
   return launch_pdl(k_gemm<BN, KSUB>, dim3(grid), dim3(kGemmThreads), G::kAlloc, st, *ta, *tb, g, ep,
                     status);
 }
@@ -559,7 +606,8 @@ cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, const Gemm
   // Two sub-blocks per stage when every unit's k-range splits evenly (BN 192 and 256 keep one:
   // their 80 and 96 KB double stages would leave only two stages).
   const int kb = Kd / 64;
-  const bool two = p.bn <= 128 && kb % p.splits == 0 && (kb / p.splits) % 2 == 0;
+  const bool two = p.bn <= 128 && kb % p.splits == 0 && (kb / p.splits) % 2 == 0 &&
+                   (p.tail == 0 || (kb / 2) % 2 == 0);
   switch (p.bn) {
     case 64:
       return two ? launch_gemm_bn<64, 2>(ta, tb, p, M, N, Kd, ep, partial, counters, sms, status, st)
