@@ -124,7 +124,9 @@ struct AttnSmem {
   static constexpr int kQ = 0;                         // two Q buffers (consecutive items)
   static constexpr int kK = 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kML = kV + kStages * kTileBytes;  // float m[2][128], l[2][128]
+  // group 0's float m[2 items][128], l[2 items][128]: one item's rows stay intact while the
+  // next item's are written
+  static constexpr int kML = kV + kStages * kTileBytes;
   // Output staging: 128 rows of DH bf16, padded by 16 bytes so that the 32 rows a warp writes
   // at once spread over all banks; then the rows' destination tokens.
   static constexpr int kStageStride = DH * 2 + 16;
@@ -254,10 +256,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   constexpr int NS = S::kStages;
   constexpr bool kSplitHandoff = T::kSeparateP;   // P handed to P*V in two halves
   constexpr bool kHasTail = S::kTail > 0;
+  // Epilogue: dh 80 lets group 1 merge and emit each item while group 0 moves on to the next
+  // (measured faster there: ViT-H 284 -> 273 us); dh 64 keeps both groups on the merge (the
+  // one-group form measured slower: ViT-B 52.8 -> 55.2 us).
+  constexpr bool kOneGroupEpi = DH == 80;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  float* s_m = reinterpret_cast<float*>(smem + S::kML);   // [2][128]
+  float* s_m = reinterpret_cast<float*>(smem + S::kML);   // [2][128] group 0's, by item parity
   float* s_l = s_m + 2 * kBM;                              // [2][128]
   int* s_dst = reinterpret_cast<int*>(smem + S::kDst);     // [128] destination token or -1
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
@@ -269,7 +275,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* s_free = s_full + 2;               // [2] S_w read into registers by its group
   uint64_t* p_full = s_free + 2;               // [2][2] half h of P_w written (O_w rescaled first)
   uint64_t* o_done = p_full + 4;               // an item's last P*V done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
+  // [2] by item parity: group 0's m, l of the item written. Two, so that group 0 (which moves on
+  // to the next item at once) cannot complete a second phase before group 1 has waited the first.
+  uint64_t* ml_ready = o_done + 1;
+  uint64_t* o_free = ml_ready + 2;             // O0, O1 of the item read (next item may reuse them)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -290,6 +300,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(kv_empty + i, 1);
     }
     mbar_init(o_done, 1);
+    if constexpr (kOneGroupEpi) {
+      mbar_init(ml_ready, 128);
+      mbar_init(ml_ready + 1, 128);
+      mbar_init(o_free, 128);
+    }
     *abort = 0;
     fence_barrier_init();
   }
@@ -387,15 +402,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool ok = true;
       int gn = 0;
       int uses[2] = {0, 0};   // P_w handed over so far (p_full phases)
-      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+      for (int it = blockIdx.x, li = 0; ok && it < n_items; it += gridDim.x, ++li) {
         const int nt = item_of(it, nq, P).tiles.count();
+        // The item's first P*V into O_w overwrites it: the previous item's epilogue must have
+        // read O0 and O1.
+        if (kOneGroupEpi && li > 0 && !(ok = mbar_wait(o_free, (li - 1) & 1, abort, status)))
+          break;
         for (int n = 0; n < nt; ++n, ++gn) {
           const int st = gn % NS, w = n & 1;
           const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kTileBytes);
           const uint32_t a = tmem + T::kP + w * T::kPStride;   // P_w
           const uint32_t d = tmem + T::kO + w * T::kOStride;
-          // The first tile of each group overwrites O_w: its group released the previous item's
-          // O (read in the epilogue) before handing over this P.
+          // The first tile of each group overwrites O_w: released by o_free above, or (two-group
+          // epilogue) by the group itself, which read the previous item's O before handing over
+          // this P.
           const uint32_t acc = n >= 2;
           // P arrives in two halves (keys 0-63, 64-127): the first half's MMAs run while the
           // softmax still computes the second.
@@ -436,6 +456,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int gn0 = 0;           // global index of the item's first tile
     int uses = 0;          // tiles of this group so far (s_full phases)
     bool s_ready = false;  // the next s_full phase was already seen complete (non-blocking test)
+    int g_last = -1;       // global index of this group's previous tile (any item), -1: none
     for (int it = blockIdx.x, li = 0; it < n_items; it += gridDim.x, ++li) {
       const Item I = item_of(it, nq, P);
       const int nt = I.tiles.count();
@@ -465,15 +486,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(r[i]);
         }
-        // Has P*V of this group's previous tile (n-2) released P_w and O_w? Tested now, used
-        // after the row max, so the test's latency is hidden behind the max. (The previous
-        // item's P*V are all done: the epilogue waited for them.)
-        const int gprev = gn0 + n - 2;
+        // Has P*V of this group's previous tile (in this item or the last) released P_w? Tested
+        // now, used after the row max, so the test's latency is hidden behind the max.
+        // (With the two-group epilogue both groups waited for the previous item's P*V, so only
+        // this item's earlier tiles count.)
+        int gprev = n >= 2 ? gn0 + n - 2 : -1;
+        if constexpr (kOneGroupEpi) {
+          gprev = g_last;
+          g_last = gn0 + n;
+        }
         bool prev_pv_done = true;
         if constexpr (T::kSeparateP) {
           tc_fence_before();
           mbar_arrive(s_free + grp);   // S_w may now be overwritten by the next Q*K^T into it
-          if (n >= 2) prev_pv_done = mbar_test(kv_empty + gprev % NS, (gprev / NS) & 1);
+          if (gprev >= 0) prev_pv_done = mbar_test(kv_empty + gprev % NS, (gprev / NS) & 1);
         }
         const int c0 = I.tiles.tile(n) * kBN;
         const bool full = tile_full(c0, P);
@@ -519,7 +545,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // The group's previous P*V must be done before P_w is rewritten and O_w rescaled (with P
         // over S it already is: this S was computed after that P*V).
         if constexpr (T::kSeparateP) {
-          if (n >= 2) {
+          if (gprev >= 0) {
             if (!__all_sync(0xffffffffu, prev_pv_done)) {
               ok = __all_sync(0xffffffffu,
                               mbar_wait(kv_empty + gprev % NS, (gprev / NS) & 1, abort, status));
@@ -606,71 +632,151 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mbar_arrive(p_full + 2 * grp + 1);
         }
       }
-      // ---- merge both groups' partial rows and scatter them to out[u, perm[p], h, :] ----
-      // Every softmax thread passes both named barriers once per item, also after a failed wait.
-      s_m[grp * kBM + row] = m_ref;
-      s_l[grp * kBM + row] = l_run;
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, li & 1, abort, status));
-      tc_fence_after();
-      named_barrier(1, 256);
-      constexpr int kCols = DH / 2;   // this group's output columns [grp*kCols, (grp+1)*kCols)
-      uint32_t x0[32], x1[32], y0[8], y1[8];   // columns 0-31 and (dh 80) 32-39 of O0, O1
-      float m0 = 0.f, m1 = 0.f, l0 = 0.f, l1 = 0.f;
-      if (ok) {
-        m0 = s_m[row];
-        m1 = s_m[kBM + row];
-        l0 = s_l[row];
-        l1 = s_l[kBM + row];
-        const uint32_t o0 = tmem + T::kO + lane_off + grp * kCols;
-        const uint32_t o1 = o0 + T::kOStride;
-        tmem_ld32_pair(o0, o1, x0, x1);
-        if constexpr (kCols > 32) tmem_ld8_pair(o0 + 32, o1 + 32, y0, y1);
-      }
-      // Both groups have read O0 and O1 (and m, l) before either hands the next item's first P
-      // to the P*V issuer, whose first MMA into O_w overwrites it.
-      tc_fence_before();
-      named_barrier(1, 256);
-      // Normalised half-row -> shared staging; then the 256 threads copy whole rows out, so
-      // that each warp store covers four contiguous 128-byte rows (dh 64) instead of 32 rows.
-      const uint32_t stage_row = smem_u32(smem + S::kStage) + row * S::kStageStride;
-      if (ok) {
-        const float mm = fmaxf(m0, m1);
-        const float a0 = (m0 == -INFINITY) ? 0.f : ex2_mufu(m0 - mm);
-        const float a1 = (m1 == -INFINITY) ? 0.f : ex2_mufu(m1 - mm);
-        const float L = l0 * a0 + l1 * a1;
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        const float f0 = a0 * inv, f1 = a1 * inv;
-        // A group with no tile in this item has a stale O: select, do not multiply by zero.
-        const bool has0 = nt > 0, has1 = nt > 1;
-#pragma unroll
-        for (int c = 0; c < kCols / 8; ++c) {
-          float v[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t u0 = c < 4 ? x0[8 * c + i] : y0[i];
-            const uint32_t u1 = c < 4 ? x1[8 * c + i] : y1[i];
-            v[i] = (has0 ? __uint_as_float(u0) * f0 : 0.f) + (has1 ? __uint_as_float(u1) * f1 : 0.f);
+      if constexpr (kOneGroupEpi) {
+        // ---- merge both groups' partial rows and scatter them to out[u, perm[p], h, :] ----
+        // Group 1 merges and emits the item; group 0 hands over its row max and sum and goes on to
+        // the next item at once (its first P*V there waits for o_free, i.e. for group 1 to have
+        // read O0 and O1). Every wait and barrier below is passed also after a failed wait.
+        const int mb = li & 1;   // this item's m, l buffer
+        if (grp == 0) {
+          s_m[mb * kBM + row] = m_ref;
+          s_l[mb * kBM + row] = l_run;
+          mbar_arrive(ml_ready + mb);
+        } else {
+          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ml_ready + mb, (li >> 1) & 1, abort, status));
+          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, li & 1, abort, status));
+          tc_fence_after();
+          const float m0 = s_m[mb * kBM + row], l0 = s_l[mb * kBM + row];
+          const float m1 = m_ref, l1 = l_run;
+          const float mm = fmaxf(m0, m1);
+          const float a0 = (m0 == -INFINITY) ? 0.f : ex2_mufu(m0 - mm);
+          const float a1 = (m1 == -INFINITY) ? 0.f : ex2_mufu(m1 - mm);
+          const float L = l0 * a0 + l1 * a1;
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          const float f0 = a0 * inv, f1 = a1 * inv;
+          const bool has0 = nt > 0, has1 = nt > 1;   // a group with no tile has a stale O
+          // The previous item's copy-out is finished before the staging rows are rewritten.
+          named_barrier(2, 128);
+          // Normalised row -> shared staging (rows padded by 16 bytes against bank conflicts); then
+          // the group copies whole rows out, so that each warp store covers contiguous rows.
+          const uint32_t stage_row = smem_u32(smem + S::kStage) + row * S::kStageStride;
+          if (ok) {
+            const uint32_t o0 = tmem + T::kO + lane_off;
+            const uint32_t o1 = o0 + T::kOStride;
+            auto emit8 = [&](const uint32_t* u0, const uint32_t* u1, int col) {
+              float v[8];
+  #pragma unroll
+              for (int i = 0; i < 8; ++i)
+                v[i] = (has0 ? __uint_as_float(u0[i]) * f0 : 0.f) +
+                       (has1 ? __uint_as_float(u1[i]) * f1 : 0.f);
+              st_shared_v4(stage_row + col * 2, pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                           pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+            };
+  #pragma unroll 1
+            for (int c = 0; c < DH / 32; ++c) {   // 32 columns of O0 and O1 at a time
+              uint32_t x0[32], x1[32];
+              tmem_ld32_pair(o0 + c * 32, o1 + c * 32, x0, x1);
+  #pragma unroll
+              for (int e = 0; e < 4; ++e) emit8(x0 + 8 * e, x1 + 8 * e, c * 32 + 8 * e);
+            }
+            if constexpr (DH % 32) {   // dh 80: columns 64..79
+  #pragma unroll
+              for (int c = (DH / 32) * 32; c < DH; c += 8) {
+                uint32_t x0[8], x1[8];
+                tmem_ld8_pair(o0 + c, o1 + c, x0, x1);
+                emit8(x0, x1, c);
+              }
+            }
+            s_dst[row] = store ? min(max(perm_t, 0), P.N - 1) : -1;
           }
-          st_shared_v4(stage_row + grp * kCols * 2 + c * 16, pack_bf16(v[0], v[1]),
-                       pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+          tc_fence_before();
+          mbar_arrive(o_free);   // O0, O1 read: the next item's first P*V may overwrite them
+          named_barrier(2, 128);
+          if (ok) {
+            constexpr int kCpr = DH / 8;                  // 16-byte chunks per row
+            const int tid = threadIdx.x - 256;            // 0..127: group 1
+            const uint32_t stage = smem_u32(smem + S::kStage);
+            uint8_t* out_uh = reinterpret_cast<uint8_t*>(P.out) +
+                              ((size_t)u_i * P.N * P.heads + h_i) * DH * 2;
+  #pragma unroll 2
+            for (int k = 0; k < kBM * kCpr / 128; ++k) {
+              const int q = tid + 128 * k;
+              const int r = q / kCpr, c = q - r * kCpr;
+              const int t = s_dst[r];
+              if (t >= 0) {
+                const uint4 v = ld_shared_v4(stage + r * S::kStageStride + c * 16);
+                *reinterpret_cast<uint4*>(out_uh + (size_t)t * P.heads * DH * 2 + c * 16) = v;
+              }
+            }
+          }
         }
-        if (grp == 0) s_dst[row] = store ? min(max(perm_t, 0), P.N - 1) : -1;
-      }
-      named_barrier(1, 256);
-      if (ok) {
-        constexpr int kCpr = DH / 8;                  // 16-byte chunks per row
-        const int tid = threadIdx.x - 128;            // 0..255
-        const uint32_t stage = smem_u32(smem + S::kStage);
-        uint8_t* out_uh = reinterpret_cast<uint8_t*>(P.out) +
-                          ((size_t)u_i * P.N * P.heads + h_i) * DH * 2;
-#pragma unroll
-        for (int k = 0; k < kBM * kCpr / 256; ++k) {
-          const int q = tid + 256 * k;
-          const int r = q / kCpr, c = q - r * kCpr;
-          const int t = s_dst[r];
-          if (t >= 0) {
-            const uint4 v = ld_shared_v4(stage + r * S::kStageStride + c * 16);
-            *reinterpret_cast<uint4*>(out_uh + (size_t)t * P.heads * DH * 2 + c * 16) = v;
+      } else {
+        // ---- merge both groups' partial rows and scatter them to out[u, perm[p], h, :] ----
+        // Every softmax thread passes both named barriers once per item, also after a failed wait.
+        s_m[grp * kBM + row] = m_ref;
+        s_l[grp * kBM + row] = l_run;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, li & 1, abort, status));
+        tc_fence_after();
+        named_barrier(1, 256);
+        constexpr int kCols = DH / 2;   // this group's output columns [grp*kCols, (grp+1)*kCols)
+        uint32_t x0[32], x1[32], y0[8], y1[8];   // columns 0-31 and (dh 80) 32-39 of O0, O1
+        float m0 = 0.f, m1 = 0.f, l0 = 0.f, l1 = 0.f;
+        if (ok) {
+          m0 = s_m[row];
+          m1 = s_m[kBM + row];
+          l0 = s_l[row];
+          l1 = s_l[kBM + row];
+          const uint32_t o0 = tmem + T::kO + lane_off + grp * kCols;
+          const uint32_t o1 = o0 + T::kOStride;
+          tmem_ld32_pair(o0, o1, x0, x1);
+          if constexpr (kCols > 32) tmem_ld8_pair(o0 + 32, o1 + 32, y0, y1);
+        }
+        // Both groups have read O0 and O1 (and m, l) before either hands the next item's first P
+        // to the P*V issuer, whose first MMA into O_w overwrites it.
+        tc_fence_before();
+        named_barrier(1, 256);
+        // Normalised half-row -> shared staging; then the 256 threads copy whole rows out, so
+        // that each warp store covers four contiguous 128-byte rows (dh 64) instead of 32 rows.
+        const uint32_t stage_row = smem_u32(smem + S::kStage) + row * S::kStageStride;
+        if (ok) {
+          const float mm = fmaxf(m0, m1);
+          const float a0 = (m0 == -INFINITY) ? 0.f : ex2_mufu(m0 - mm);
+          const float a1 = (m1 == -INFINITY) ? 0.f : ex2_mufu(m1 - mm);
+          const float L = l0 * a0 + l1 * a1;
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          const float f0 = a0 * inv, f1 = a1 * inv;
+          // A group with no tile in this item has a stale O: select, do not multiply by zero.
+          const bool has0 = nt > 0, has1 = nt > 1;
+  #pragma unroll
+          for (int c = 0; c < kCols / 8; ++c) {
+            float v[8];
+  #pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t u0 = c < 4 ? x0[8 * c + i] : y0[i];
+              const uint32_t u1 = c < 4 ? x1[8 * c + i] : y1[i];
+              v[i] = (has0 ? __uint_as_float(u0) * f0 : 0.f) + (has1 ? __uint_as_float(u1) * f1 : 0.f);
+            }
+            st_shared_v4(stage_row + grp * kCols * 2 + c * 16, pack_bf16(v[0], v[1]),
+                         pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+          }
+          if (grp == 0) s_dst[row] = store ? min(max(perm_t, 0), P.N - 1) : -1;
+        }
+        named_barrier(1, 256);
+        if (ok) {
+          constexpr int kCpr = DH / 8;                  // 16-byte chunks per row
+          const int tid = threadIdx.x - 128;            // 0..255
+          const uint32_t stage = smem_u32(smem + S::kStage);
+          uint8_t* out_uh = reinterpret_cast<uint8_t*>(P.out) +
+                            ((size_t)u_i * P.N * P.heads + h_i) * DH * 2;
+  #pragma unroll
+          for (int k = 0; k < kBM * kCpr / 256; ++k) {
+            const int q = tid + 256 * k;
+            const int r = q / kCpr, c = q - r * kCpr;
+            const int t = s_dst[r];
+            if (t >= 0) {
+              const uint4 v = ld_shared_v4(stage + r * S::kStageStride + c * 16);
+              *reinterpret_cast<uint4*>(out_uh + (size_t)t * P.heads * DH * 2 + c * 16) = v;
+            }
           }
         }
       }
