@@ -14,21 +14,24 @@
 
 namespace ss {
 
-// Squared Sobel gradient magnitude of pixel (y, x) of an H x W image, replicate border. Each step
-// is one fp64 round-to-nearest operation, in a fixed order, never fused, so every caller gets the
-// same bits.
-__device__ __forceinline__ double sobel_at(const float* __restrict__ img, int H, int W, int y,
-                                           int x) {
-  int ym = y > 0 ? y - 1 : 0, yp = y < H - 1 ? y + 1 : H - 1;
-  int xm = x > 0 ? x - 1 : 0, xp = x < W - 1 ? x + 1 : W - 1;
-  double l_mm = img[ym * W + xm], l_m0 = img[ym * W + x], l_mp = img[ym * W + xp];
-  double l_0m = img[y * W + xm], l_0p = img[y * W + xp];
-  double l_pm = img[yp * W + xm], l_p0 = img[yp * W + x], l_pp = img[yp * W + xp];
+// Squared Sobel gradient magnitude from the 3 x 3 neighbourhood (rows m, 0, p = y-1, y, y+1;
+// columns m, 0, p = x-1, x, x+1). Each step is one fp64 round-to-nearest operation, in a fixed
+// order, never fused, so every caller gets the same bits.
+__device__ __forceinline__ double sobel_of(double l_mm, double l_m0, double l_mp, double l_0m,
+                                           double l_0p, double l_pm, double l_p0, double l_pp) {
   double gx = __dadd_rn(__dadd_rn(__dsub_rn(l_mp, l_mm), __dmul_rn(2.0, __dsub_rn(l_0p, l_0m))),
                         __dsub_rn(l_pp, l_pm));
   double gy = __dadd_rn(__dadd_rn(__dsub_rn(l_pm, l_mm), __dmul_rn(2.0, __dsub_rn(l_p0, l_m0))),
                         __dsub_rn(l_pp, l_mp));
   return __dadd_rn(__dmul_rn(gx, gx), __dmul_rn(gy, gy));
+}
+// Of pixel (y, x) of an H x W image, replicate border.
+__device__ __forceinline__ double sobel_at(const float* __restrict__ img, int H, int W, int y,
+                                           int x) {
+  int ym = y > 0 ? y - 1 : 0, yp = y < H - 1 ? y + 1 : H - 1;
+  int xm = x > 0 ? x - 1 : 0, xp = x < W - 1 ? x + 1 : W - 1;
+  return sobel_of(img[ym * W + xm], img[ym * W + x], img[ym * W + xp], img[y * W + xm],
+                  img[y * W + xp], img[yp * W + xm], img[yp * W + x], img[yp * W + xp]);
 }
 
 __global__ void __launch_bounds__(256) k_sobel_score(const float* __restrict__ lum,
@@ -97,6 +100,34 @@ __global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __rest
   griddep_wait();
   griddep_launch();
   const int u = blockIdx.y;
+  if (FROM_LUM && !m.window_mode && (m.Wg & 3) == 0) {
+    // The whole image's keys, four horizontally adjacent pixels per thread from one 3 x 6
+    // neighbourhood (18 loads and conversions for four keys instead of 32).
+    const float* img = lum + (size_t)u * N;
+    const int W = m.Wg, H = m.Hg, qpr = W >> 2;
+    for (int q = threadIdx.x; q < N / 4; q += blockDim.x) {
+      const int y = q / qpr, x0 = (q - y * qpr) * 4;
+      const int rows[3] = {y > 0 ? y - 1 : 0, y, y < H - 1 ? y + 1 : H - 1};
+      double l[3][6];
+#pragma unroll
+      for (int r = 0; r < 3; ++r)
+#pragma unroll
+        for (int c = 0; c < 6; ++c) {
+          const int x = min(max(x0 - 1 + c, 0), W - 1);
+          l[r][c] = img[rows[r] * W + x];
+        }
+      ulonglong2 k2[2];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const double v = sobel_of(l[0][k], l[0][k + 1], l[0][k + 2], l[1][k], l[1][k + 2],
+                                  l[2][k], l[2][k + 1], l[2][k + 2]);
+        const unsigned long long bits = (unsigned long long)__double_as_longlong(v);
+        if (k & 1) k2[k >> 1].y = bits; else k2[k >> 1].x = bits;
+      }
+      reinterpret_cast<ulonglong2*>(s_key)[2 * q] = k2[0];       // y*W + x0 is a multiple of 4
+      reinterpret_cast<ulonglong2*>(s_key)[2 * q + 1] = k2[1];
+    }
+  } else
   // Fill the unit's keys: eight independent loads in flight per thread before any store.
   for (int t0 = threadIdx.x; t0 < N; t0 += 8 * blockDim.x) {
     unsigned long long k8[8];
