@@ -29,16 +29,18 @@ namespace ss {
 // ---------------------------------------------------------------------------------------------
 // One CTA per (unit, 8 consecutive block-major positions), a warp per position: the warp resolves
 // its source token, then copies the token's heads*dh row (contiguous in the source) as 16-byte
-// chunks into the per-head rows of the gathered buffers. CPR = 16-byte chunks per head.
-template <int CPR>
-__global__ void __launch_bounds__(256) k_gather_qkv(const uint16_t* __restrict__ q,
-                                                    const uint16_t* __restrict__ k,
-                                                    const uint16_t* __restrict__ v,
-                                                    const int32_t* __restrict__ perm,
-                                                    uint16_t* __restrict__ qp,
-                                                    uint16_t* __restrict__ kp,
-                                                    uint16_t* __restrict__ vp, int N, int heads,
-                                                    int b, int L) {
+// chunks into the per-head rows of the gathered buffers. CPR = 16-byte chunks per head; KPL =
+// chunks of one tensor per lane (heads*CPR <= 32*KPL), all 3*KPL loads of a lane in flight before
+// its stores. MINB: CTAs per SM the registers are sized for.
+template <int CPR, int KPL, int MINB>
+__global__ void __launch_bounds__(256, MINB) k_gather_qkv(const uint16_t* __restrict__ q,
+                                                       const uint16_t* __restrict__ k,
+                                                       const uint16_t* __restrict__ v,
+                                                       const int32_t* __restrict__ perm,
+                                                       uint16_t* __restrict__ qp,
+                                                       uint16_t* __restrict__ kp,
+                                                       uint16_t* __restrict__ vp, int N,
+                                                       int heads, int b, int L) {
   griddep_wait();
   griddep_launch();
   const int u = blockIdx.y;
@@ -56,40 +58,43 @@ __global__ void __launch_bounds__(256) k_gather_qkv(const uint16_t* __restrict__
                          reinterpret_cast<const uint4*>(v) + src_row};
   uint4* dst[3] = {reinterpret_cast<uint4*>(qp) + dst_row, reinterpret_cast<uint4*>(kp) + dst_row,
                    reinterpret_cast<uint4*>(vp) + dst_row};
-  // Up to 4 chunks per tensor per lane per pass: all 12 loads are in flight before any store.
-  for (int c0 = 0; c0 < per_tok; c0 += 128) {
-    uint4 buf[3][4];
+  uint4 buf[3][KPL];
 #pragma unroll
-    for (int t = 0; t < 3; ++t)
+  for (int t = 0; t < 3; ++t)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = c0 + e * 32 + lane;
-        if (c < per_tok) buf[t][e] = __ldg(src[t] + c);
+    for (int e = 0; e < KPL; ++e) {
+      const int c = e * 32 + lane;
+      if (c < per_tok) buf[t][e] = __ldg(src[t] + c);
+    }
+#pragma unroll
+  for (int t = 0; t < 3; ++t)
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+      const int c = e * 32 + lane;
+      if (c < per_tok) {
+        const int h = c / CPR, cc = c - h * CPR;   // CPR is a compile-time constant
+        dst[t][h * plane + cc] = buf[t][e];
       }
-#pragma unroll
-    for (int t = 0; t < 3; ++t)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = c0 + e * 32 + lane;
-        if (c < per_tok) {
-          const int h = c / CPR, cc = c - h * CPR;   // CPR is a compile-time constant
-          dst[t][h * plane + cc] = buf[t][e];
-        }
-      }
-  }
+    }
 }
 
 cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                               const int32_t* perm, uint16_t* qp, uint16_t* kp, uint16_t* vp,
                               int U, int N, int heads, int dh, int b, cudaStream_t st) {
   dim3 grid((N + 7) / 8, U);
-  if (dh == 64)
-    return launch_pdl(k_gather_qkv<8>, grid, dim3(256), 0, st, q, k, v, perm, qp, kp, vp, N, heads,
-                      b, N / kStripes);
-  if (dh == 80)
-    return launch_pdl(k_gather_qkv<10>, grid, dim3(256), 0, st, q, k, v, perm, qp, kp, vp, N, heads,
-                      b, N / kStripes);
-  return cudaErrorInvalidValue;
+  const int L = N / kStripes;
+  auto go = [&](auto kernel) {
+    return launch_pdl(kernel, grid, dim3(256), 0, st, q, k, v, perm, qp, kp, vp, N, heads, b, L);
+  };
+  const int per_tok = heads * (dh / 8);
+  if (dh != 64 && dh != 80) return cudaErrorInvalidValue;
+  if (per_tok > 32 * 8) return cudaErrorInvalidValue;   // heads * dh > 2048
+  const int kpl = (per_tok + 31) / 32;
+  // Measured on one B200 (block step): head dim 80 with five chunks per lane sized for three CTAs
+  // per SM, ViT-H 441.5 -> 435.2 us against the four-chunk form; at head dim 64 sizing for four
+  // CTAs per SM (one wave at ViT-B) measured slower (108.8 -> 110.2 us), so it keeps its shape.
+  if (dh == 64) return kpl <= 4 ? go(k_gather_qkv<8, 4, 1>) : go(k_gather_qkv<8, 8, 1>);
+  return kpl <= 5 ? go(k_gather_qkv<10, 5, 3>) : go(k_gather_qkv<10, 8, 2>);
 }
 
 // ---------------------------------------------------------------------------------------------
