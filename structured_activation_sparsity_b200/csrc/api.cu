@@ -521,10 +521,14 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
   }));
   if (rc) return rc;
   if ((rc = attn_launch(cfg, g, p, wsa, perm, out, status, st))) return rc;
+  // The row gather's inputs are final: keep came from the ranking launch, which the Q/K/V gather
+  // and the attention waited for before this launch can start, and x is not written before fc2.
+  // Its copy runs in the attention's tail; its dependency wait comes last (late_wait).
   const int n_counters = (int)((plan.total - plan.counters) / sizeof(int));
   rc = cuda_err(traced("gather_rows", st, [&] {
     return launch_gather_rows(x, keep, reinterpret_cast<uint16_t*>(wsm + plan.xk), g.B, g.T, K, C,
-                              reinterpret_cast<int*>(wsm + plan.counters), n_counters, st);
+                              reinterpret_cast<int*>(wsm + plan.counters), n_counters, st,
+                              /*late_wait=*/true);
   }));
   if (rc) return rc;
   return rcmlp_launch(g, K, x, C, hidden, w1, b1, w2, b2, keep, wsm, status, st);

@@ -40,9 +40,12 @@ cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUte
                         const CUtensorMap* tv_tail, const AttnParams& p, int dh, int* status,
                         cudaStream_t st);
 
-// Gathers the kept rows of x [B, T, C] into xk [B*K, C]; zeroes zero[0, nzero).
+// Gathers the kept rows of x [B, T, C] into xk [B*K, C]; zeroes zero[0, nzero). late_wait: keep
+// and x are known final at launch (see k_gather_rows), the copy need not wait for the previous
+// launch.
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* keep, uint16_t* xk, int B, int T,
-                               int K, int C, int* zero, int nzero, cudaStream_t st);
+                               int K, int C, int* zero, int nzero, cudaStream_t st,
+                               bool late_wait = false);
 
 struct GemmEpilogue {
   int kind;                 // 0: out = bf16(GELU(acc + bias)) into out[M, N]

@@ -20,38 +20,46 @@ namespace ss {
 // One warp per kept row: resolve the row's token, then copy its C bf16 (C/8 16-byte chunks) with
 // all of a lane's loads in flight before its stores. CTA 0 also zeroes the GEMMs' k-split
 // counters (`zero`, `nzero` ints), which the two GEMM launches that follow expect at zero.
+// late_wait: the caller guarantees that keep and x are already final when this launch starts
+// (earlier launches of the same call waited for the work that wrote them) and that nothing still
+// running reads xk or the counters. The copy then runs at once, in the previous launch's tail,
+// and every thread takes the dependency wait at its end, so this launch still completes after the
+// previous one for everything that follows.
 __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t* __restrict__ x,
                                                      const int32_t* __restrict__ keep,
                                                      uint16_t* __restrict__ xk, int B, int T,
                                                      int K, int C, int* __restrict__ zero,
-                                                     int nzero) {
-  griddep_wait();
+                                                     int nzero, int late_wait) {
+  if (!late_wait) griddep_wait();
   griddep_launch();
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
   const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (m >= B * K) return;
-  const int b = m / K;
-  const int t = min(max(__ldg(keep + m), 0), T - 1);   // never leave the image
-  const int cpr = C / 8;
-  const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)b * T + t) * C);
-  uint4* dst = reinterpret_cast<uint4*>(xk) + (size_t)m * cpr;
-  for (int c0 = 0; c0 < cpr; c0 += 256) {
-    uint4 buf[8];
+  if (m < B * K) {
+    const int b = m / K;
+    const int t = min(max(__ldg(keep + m), 0), T - 1);   // never leave the image
+    const int cpr = C / 8;
+    const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)b * T + t) * C);
+    uint4* dst = reinterpret_cast<uint4*>(xk) + (size_t)m * cpr;
+    for (int c0 = 0; c0 < cpr; c0 += 256) {
+      uint4 buf[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if (c0 + e * 32 + lane < cpr) buf[e] = __ldg(src + c0 + e * 32 + lane);
+      for (int e = 0; e < 8; ++e)
+        if (c0 + e * 32 + lane < cpr) buf[e] = __ldg(src + c0 + e * 32 + lane);
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if (c0 + e * 32 + lane < cpr) dst[c0 + e * 32 + lane] = buf[e];
+      for (int e = 0; e < 8; ++e)
+        if (c0 + e * 32 + lane < cpr) dst[c0 + e * 32 + lane] = buf[e];
+    }
   }
+  if (late_wait) griddep_wait();
 }
 
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* keep, uint16_t* xk, int B, int T,
-                               int K, int C, int* zero, int nzero, cudaStream_t st) {
+                               int K, int C, int* zero, int nzero, cudaStream_t st,
+                               bool late_wait) {
   const int rows = B * K;
   return launch_pdl(k_gather_rows, dim3((rows + 7) / 8), dim3(256), 0, st, x, keep, xk, B, T, K, C,
-                    zero, nzero);
+                    zero, nzero, late_wait ? 1 : 0);
 }
 
 // Persistent warp-specialised GEMM. Work unit = (m-tile, n-tile, k-split); CTA c takes units
