@@ -163,8 +163,9 @@ size_t sparsesam_block_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden);
  * then sparsesam_attn(cfg, q, k, v, perm, out), then sparsesam_rcmlp(cfg, x, C, hidden, w1, b1,
  * w2, b2, keep), with one workspace: the same launches and results, bit for bit. Arguments and
  * their layouts, alignment and error codes as in those calls (lum, score, perm, keep, out
- * non-NULL; inv may be NULL). ws (device, 256-byte aligned) >= sparsesam_block_workspace(cfg, C,
- * hidden) bytes; its contents on entry do not matter. */
+ * non-NULL; inv may be NULL); in addition out may not overlap x (SS_EINVAL), since S4's row gather
+ * is allowed to start before S3 has finished. ws (device, 256-byte aligned) >=
+ * sparsesam_block_workspace(cfg, C, hidden) bytes; its contents on entry do not matter. */
 int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, const uint16_t* k,
                     const uint16_t* v, uint16_t* x, int32_t C, int32_t hidden, const uint16_t* w1,
                     const uint16_t* b1, const uint16_t* w2, const uint16_t* b2, double* score,

@@ -501,6 +501,14 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
   const size_t attn_part = align256(attn_ws_bytes(g, heads, dh));
   if (!ws || !aligned(ws, 256) || ws_bytes < attn_part + rcmlp_ws_bytes(g, K, C, hidden))
     return SS_EWORKSPACE;
+  // out may not overlap x: S4's row gather starts before S3 has finished writing out.
+  {
+    const uintptr_t o0 = reinterpret_cast<uintptr_t>(out);
+    const uintptr_t o1 = o0 + (size_t)g.U * g.N * heads * dh * 2;
+    const uintptr_t x0 = reinterpret_cast<uintptr_t>(x);
+    const uintptr_t x1 = x0 + (size_t)g.B * g.T * C * 2;
+    if (o0 < x1 && x0 < o1) return SS_EINVAL;
+  }
   int* status = status_word();
   if (!status) return SS_ECUDA;
   uint8_t* wsa = static_cast<uint8_t*>(ws);

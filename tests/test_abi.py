@@ -111,6 +111,10 @@ def test_validation_codes():
         bad = list(blk)
         bad[i] = None
         assert lib.sparsesam_block(by(good), *bad) == L.SS_EINVAL, i
+    overlap = list(blk)
+    overlap[17] = 1 << 30   # enough workspace: the x / out overlap is what is refused
+    assert overlap[4] == overlap[15]   # x and out are the same fake buffer
+    assert lib.sparsesam_block(by(good), *overlap) == L.SS_EINVAL
     assert lib.sparsesam_attn(by(good), None, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == L.SS_EINVAL
     # unsupported head_dim
     bad_dh = L.make_cfg(1, 16, 16, "global", 14, 1, 96, 0.4)
