@@ -133,6 +133,16 @@ def test_validation_codes():
     K = O.keep_count(0.4, 256)
     assert need_m == math.ceil(K * 64 * 2 / 256) * 256 + math.ceil(K * 256 * 2 / 256) * 256
     assert lib.sparsesam_rcmlp(by(good), FAKE, 64, 256, FAKE, None, FAKE, None, FAKE, FAKE, need_m - 1, None) == L.SS_EWORKSPACE
+    # A long-K fc2 (ViT-H: K = 5120, 80 k-blocks; 4 images, 4916 kept rows) has a last partial
+    # round of tiles split in two along K: the workspace holds their fp32 halves and counters
+    # beyond xk and H.
+    vith = L.make_cfg(4, 64, 64, "global", 14, 16, 80, 0.3)
+    M = 4 * O.keep_count(0.3, 4096)
+    xk_h = math.ceil(M * 1280 * 2 / 256) * 256 + math.ceil(M * 5120 * 2 / 256) * 256
+    # 47 tail tiles of 128 x 256 fp32 (6.2 MB), where a two-way split of all 195 tiles would need
+    # 51 MB of partials
+    extra = L.sparsesam_rcmlp_workspace(vith, 1280, 5120) - xk_h
+    assert 47 * 128 * 256 * 4 <= extra < 8 << 20
     # blocklist capacity
     rp = (ctypes.c_int32 * 8)()
     ci = (ctypes.c_int32 * 2)()
