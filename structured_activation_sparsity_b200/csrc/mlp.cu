@@ -403,58 +403,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       } else if (pair) {
         // Two k-splits of the tile run at the same time in two CTAs; split s finishes column half
-        // s. This unit's warps of the other half hand their accumulator columns to the partner
-        // as an fp32 partial (column-major: a warp's 32 rows of one column are one 128-byte
-        // line) and count themselves on that half's counter; the warps of half s wait for the
-        // partner's four, then add its partial to their own columns (acc_s + partial_(1-s): for
-        // two terms the same sum as p0 + p1 in either order) and apply the epilogue.
-        const int half = ew >> 2;
-        float* part = g.partial + ((size_t)slot * 2 + half) * 128 * G::kHalf + row;
-        int* count = g.counters + slot * 2 + half;
-        if (half != s) {
+        // s. All eight epilogue warps take part in both jobs, 32-column chunk by chunk (warp group
+        // hg takes chunks hg, hg + 2, ...): first they hand the partner's half of their rows to the
+        // partner as an fp32 partial (column-major: a warp's 32 rows of one column are one
+        // 128-byte line) and count themselves on that half's counter; then each waits for the
+        // partner's eight warps and adds its partial to its own half's chunks (acc_s +
+        // partial_(1-s): for two terms the same sum as p0 + p1 in either order) and applies the
+        // epilogue.
+        constexpr int kChunks = G::kHalf / 32;
+        const int hg = ew >> 2, other = 1 - s;
+        const uint32_t t_row = tmem + buf * BN + lane_off;
+        float* part_out = g.partial + ((size_t)slot * 2 + other) * 128 * G::kHalf + row;
+        float* part_in = g.partial + ((size_t)slot * 2 + s) * 128 * G::kHalf + row;
+        int* count_out = g.counters + slot * 2 + other;
+        int* count_in = g.counters + slot * 2 + s;
 #pragma unroll 1
-          for (int c = 0; c < G::kHalf / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(t_acc + c * 32, r);
-            if (c == G::kHalf / 32 - 1) {
-              tc_fence_before();
-              mbar_arrive(acc_empty + buf);
-            }
+        for (int c = hg; c < kChunks; c += 2) {
+          uint32_t r[32];
+          tmem_ld32(t_row + other * G::kHalf + c * 32, r);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) part[(size_t)(c * 32 + e) * 128] = __uint_as_float(r[e]);
-          }
-          __threadfence();
-          __syncwarp();
-          if (lane == 0) add_release(count, 1);   // the warp's 32 rows of the half are written
-        } else {
-          // Every lane acquires the counter itself before reading the partial.
-          if (!__all_sync(0xffffffffu, wait_counter_geq(count, 4, abort, status))) break;
-#pragma unroll 1
-          for (int c = 0; c < G::kHalf / 32; ++c) {
-            const int n = n_t * BN + col0 + c * 32;
-            Epi32In in;
-            float w[32];
-            if (drow) {
-              epi_load(ep, drow, n, in);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) w[e] = __ldcg(part + (size_t)(c * 32 + e) * 128);
-            }
-            uint32_t r[32];
-            tmem_ld32(t_acc + c * 32, r);
-            if (c == G::kHalf / 32 - 1) {
-              tc_fence_before();
-              mbar_arrive(acc_empty + buf);
-            }
-            if (drow) {
-              float v[32];
-#pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]) + w[e];
-              epi_store(ep, drow, n, in, v);
-            }
-          }
-          // The last of the four owner warps re-arms the counter (for a later GEMM sharing it).
-          if (lane == 0 && atomicAdd(count, 1) == 7) atomicExch(count, 0);
+          for (int e = 0; e < 32; ++e)
+            part_out[(size_t)(c * 32 + e) * 128] = __uint_as_float(r[e]);
         }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) add_release(count_out, 1);   // this warp's share of the partner's half
+        // Every lane acquires the counter itself before reading the partial.
+        if (!__all_sync(0xffffffffu, wait_counter_geq(count_in, 8, abort, status))) break;
+#pragma unroll 1
+        for (int c = hg; c < kChunks; c += 2) {
+          const int n = n_t * BN + s * G::kHalf + c * 32;
+          Epi32In in;
+          float w[32];
+          if (drow) {
+            epi_load(ep, drow, n, in);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) w[e] = __ldcg(part_in + (size_t)(c * 32 + e) * 128);
+          }
+          uint32_t r[32];
+          tmem_ld32(t_row + s * G::kHalf + c * 32, r);
+          if (drow) {
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]) + w[e];
+            epi_store(ep, drow, n, in, v);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(acc_empty + buf);   // this warp's reads of the accumulator are done
+        // The last of the sixteen arrivals on this half's counter (the partner's eight writer
+        // arrivals, then this CTA's eight warps once finished) re-arms it for a later GEMM.
+        if (lane == 0 && atomicAdd(count_in, 1) == 15) atomicExch(count_in, 0);
       } else {
         // Write this split's partial tile (column-major, so a warp's 32 rows of one column are
         // one 128-byte line), then let the last split of the tile finish it.
