@@ -11,7 +11,8 @@
 //
 // GEMM: C[M, N] = A[M, Kd] B[N, Kd]^T, A and B K-major bf16 in 128B-swizzled 64-wide K blocks
 // loaded by TMA into a multi-stage ring; one thread issues 128 x BN x 16 MMAs into a TMEM fp32
-// accumulator; four epilogue warps read it back with tcgen05.ld (one row per thread).
+// accumulator; eight epilogue warps read it back with tcgen05.ld (one row per thread, two warps
+// per TMEM lane quadrant, each on half of the columns).
 #include "common.cuh"
 #include "kernels.h"
 
