@@ -198,6 +198,8 @@ def _mlp_case(cfg, C, Hd, seed, bias=True, images_check=None):
     (3, 20, 20, 192, 320, 1.0, True),      # dense, N not a multiple of 128 (BN 64)
     (1, 32, 32, 128, 2048, 0.4, True),     # fc2 split four ways along K: the last split finishes
     (1, 48, 48, 384, 1536, 0.5, True),     # fc2 split two ways, all units resident: paired finish
+    (1, 64, 64, 768, 3072, 0.625, True),   # paired finish with 256-wide tiles (120 units)
+    (2, 48, 48, 512, 2048, 0.5, True),     # paired finish with 128-wide tiles (144 units)
 ])
 def test_rcmlp_small(B, H, W, C, Hd, d, bias):
     cfg = L.make_cfg(B, H, W, "global", 14, 1, 64, d)
