@@ -3,7 +3,9 @@
 
 A step is one pass of the whole path -- Sobel score, stripe-sort permutation, Stripe-Sort sparse
 attention, Residual-Consistency MLP -- over one batch of the named synthetic workload (default:
-SAM ViT-B global block, 1 x 64x64 tokens, 12 heads x 64, density 0.4, MLP 768->3072->768).
+SAM ViT-H global block, 4 x 64x64 tokens, 16 heads x 80, density 0.3, MLP 1280->5120->1280, the
+largest single-block configuration). The SAM ViT-B global and windowed blocks are measured the same
+way and reported under "also".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -42,11 +44,10 @@ METRIC = "Stripe-Sort attn + RC-MLP tokens/s per block; effective TFLOP/s vs bf1
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one attention launch on the ViT-B global block,
-# from the ncu --set full capture of the attention kernel on this workload (cold caches; the
-# 6.3 MB output stays in L2 within the launch, so the write term is 0). Set to None whenever the
-# attention kernel changes until it is captured again.
-ATTN_TRAFFIC_BYTES = {"vitb_global": 18964480}
+# dram__bytes_read.sum + dram__bytes_write.sum of one attention launch per workload, from an ncu
+# capture of the current attention kernel on that workload (profiles/ names the capture). A
+# workload is absent (traffic null) until its capture is taken again after a kernel change.
+ATTN_TRAFFIC_BYTES = {}
 
 
 def peaks():
@@ -282,15 +283,30 @@ def job_throughput(world: int, units_per_step: int, steps: int, seconds: float) 
     return world * units_per_step * steps / seconds
 
 
-def run_ours(args, wl, rank, world, local_rank, dist):
+def time_attn_kernel(sets, launches, stream, warmup=3):
+    """Average duration of the attention kernel alone: CUDA events on the launching stream around
+    `launches` back-to-back launches over the rotating input sets (their workspaces hold the
+    permuted Q, K, V their last step left), so that consecutive launches overlap as inside a step
+    (programmatic dependent launch) and no per-launch event stands between them."""
+    import torch
+    for i in range(warmup):
+        sets[i % len(sets)].attn_kernel_step(stream)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for i in range(launches):
+        sets[i % len(sets)].attn_kernel_step(stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    return ev0.elapsed_time(ev1) * 1e3 / launches
+
+
+def measure(args, wl, dist, dev, stream, world):
+    """The timed steps of one workload and the per-kernel figures behind them."""
     import torch
     from structured_activation_sparsity_b200 import _lib as L
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    stream = torch.cuda.Stream(device=dev)
-    bf16_peak, bf16_sust, hbm_peak, peak_src = peaks()
-
+    bf16_peak, _, hbm_peak, peak_src = peaks()
     probe, _ = make_sets(wl, 1, dev)
     per_set = set_bytes(probe[0])
     n_sets = max(2, math.ceil(3 * L2_BYTES / per_set))
@@ -308,7 +324,7 @@ def run_ours(args, wl, rank, world, local_rank, dist):
         raise RuntimeError("a device wait timed out during warm-up")
 
     # ---- timed region: exactly K steps --------------------------------------------------------
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(dev.index or 0)
     clocks.start()
     n0 = L.sparsesam_launch_count()
     t = time_steps(sets, args.steps, stream, dist)
@@ -318,25 +334,52 @@ def run_ours(args, wl, rank, world, local_rank, dist):
     ms_per_step = t / args.steps * 1e3
     value = job_throughput(world, tokens_per_step, args.steps, t)
 
-    # ---- per-kernel durations: the same K steps again with launch tracing on ---------------------
+    # ---- per-kernel durations: the same K steps again with an event pair around every launch ----
+    # (the events keep each launch from overlapping its neighbours, so these include launch
+    # latency; the attention's own figure below has no event between launches)
     L.sparsesam_trace_start(8 * args.steps + 16)
     time_steps(sets, args.steps, stream, dist)
     recs = L.sparsesam_trace_stop()
     per_kernel = {}
     for name, ms in recs:
         per_kernel.setdefault(name, []).append(ms)
-    kernels = {n: {"launches": len(v), "avg_us": 1e3 * sum(v) / len(v)} for n, v in per_kernel.items()}
-    # Algorithmic bytes of the bandwidth-bound launches (reads + writes each must make at least
-    # once) and their rate against the measured HBM copy peak. The per-launch times come from the
-    # traced pass (CUDA events around each launch), so they include the launch's own latency.
+    kernels = {n: {"launches": len(v), "avg_us_traced": 1e3 * sum(v) / len(v)}
+               for n, v in per_kernel.items()}
     moved = kernel_bytes(wl, pat)
     for n, nbytes in moved.items():
         if n in kernels:
-            gbs = nbytes / (kernels[n]["avg_us"] * 1e-6) / 1e9
-            kernels[n].update({"bytes": nbytes, "gbs": gbs, "frac_hbm": gbs / hbm_peak})
-    attn_us = kernels["attn"]["avg_us"]
+            gbs = nbytes / (kernels[n]["avg_us_traced"] * 1e-6) / 1e9
+            kernels[n].update({"bytes": nbytes, "gbs_traced": gbs, "frac_hbm_traced": gbs / hbm_peak})
+
+    # ---- the attention kernel by itself (the roofline's kernel) --------------------------------
+    attn_us = time_attn_kernel(sets, max(50, args.steps), stream)
+    kernels.setdefault("attn", {})["avg_us"] = attn_us
     achieved = attn_flops / (attn_us * 1e-6) / 1e12
-    traffic = ATTN_TRAFFIC_BYTES.get(wl.name)
+    roofline = {"bound": "tensor", "kernel": "attn", "achieved": achieved, "peak": bf16_peak,
+                "unit": "TFLOP/s", "frac": achieved / bf16_peak,
+                "traffic": ATTN_TRAFFIC_BYTES.get(wl.name),
+                "peak_source": f"{peak_src} bf16 burst",
+                "algorithmic_flops_per_launch": attn_flops,
+                "timing": f"CUDA events around {max(50, args.steps)} back-to-back launches of the "
+                          f"attention kernel over {n_sets} rotating input sets"}
+    if L.sparsesam_device_status(stream) != L.SS_OK:
+        raise RuntimeError("a device wait timed out during timing")
+    return {"sets": sets, "n_sets": n_sets, "per_set": per_set, "pat": pat, "value": value,
+            "t": t, "ms_per_step": ms_per_step, "launches": launches, "clocks": clocks,
+            "kernels": kernels, "roofline": roofline, "attn_flops": attn_flops,
+            "mlp_flops": mlp_flops, "tokens_per_step": tokens_per_step}
+
+
+def run_ours(args, wl, rank, world, local_rank, dist):
+    import torch
+    from structured_activation_sparsity_b200 import _lib as L
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    m = measure(args, wl, dist, dev, stream, world)
+    sets, n_sets, pat = m["sets"], m["n_sets"], m["pat"]
+    t, value, tokens_per_step = m["t"], m["value"], m["tokens_per_step"]
 
     # ---- dense comparison: the same kernels at density 1.0 -----------------------------------------
     dense_sets = make_sets(wl, n_sets, dev, density=1.0)[0]
@@ -396,32 +439,45 @@ def run_ours(args, wl, rank, world, local_rank, dist):
     torch.cuda.synchronize()
     te = max_over_ranks(ev0.elapsed_time(ev1) / 1e3, dist, dev)
     e2e_value = job_throughput(world, tokens_per_step, args.steps, te)
-
     if L.sparsesam_device_status(stream) != L.SS_OK:
         raise RuntimeError("a device wait timed out during timing")
+    del sets, e2e_sets, m["sets"]
+    torch.cuda.empty_cache()
+
+    # ---- the other single-block workloads, measured the same way (extra keys of the line) -------
+    also = {}
+    for name in [n for n in args.also.split(",") if n and n != wl.name]:
+        w2 = workloads.get(name)
+        m2 = measure(args, w2, dist, dev, stream, world)
+        also[name] = {"value": m2["value"], "unit": UNIT, "ms_per_step": m2["ms_per_step"],
+                      "config": config_of(w2, args, {"realised_density": m2["pat"].rho}),
+                      "roofline": m2["roofline"], "clocks": m2["clocks"].summary(),
+                      "gpu_launches": int(m2["launches"]),
+                      "effective_tflops": (m2["attn_flops"] + m2["mlp_flops"]) * args.steps
+                      * world / m2["t"] / 1e12}
+        del m2
+        torch.cuda.empty_cache()
 
     if rank != 0:
         return
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_of(wl, args, {
-            "l2": f"{n_sets} rotating input sets of {per_set / 2**20:.0f} MiB (> 3x L2)",
+            "l2": f"{n_sets} rotating input sets of {m['per_set'] / 2**20:.0f} MiB (> 3x L2)",
             "realised_density": pat.rho, "mlp_tokens_per_image": pat.keep}),
-        "clocks": clocks.summary(),
+        "clocks": m["clocks"].summary(),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": int(launches),
-        "effective_tflops": (attn_flops + mlp_flops) * args.steps * world / t / 1e12,
-        "roofline": {"bound": "tensor", "kernel": "attn", "achieved": achieved,
-                     "peak": bf16_peak, "unit": "TFLOP/s", "frac": achieved / bf16_peak,
-                     "traffic": traffic, "peak_source": f"{peak_src} bf16 burst",
-                     "algorithmic_flops_per_launch": attn_flops},
-        "kernels": kernels,
+        "gpu_launches": int(m["launches"]),
+        "effective_tflops": (m["attn_flops"] + m["mlp_flops"]) * args.steps * world / t / 1e12,
+        "roofline": m["roofline"],
+        "kernels": m["kernels"],
         "dense": {"value": dense_value, "unit": UNIT, "ms_per_step": td / args.steps * 1e3,
                   "effective_tflops": dense_flops * args.steps * world / td / 1e12,
                   "sparse_speedup": value / dense_value},
+        "also": also,
     }
     if world == 1:
         step_s, desc, cores, _ = cpu_sample(wl)
@@ -441,8 +497,9 @@ def run_kernel_loop(args, wl, local_rank):
     with torch.cuda.stream(stream):
         hp.score_step(stream)
         hp.perm_step(stream)
+    hp.attn_step(stream)   # leaves the permuted Q, K, V in the workspace for attn_kernel
     fn = {"score": hp.score_step, "perm": hp.perm_step, "attn": hp.attn_step,
-          "rcmlp": hp.mlp_step}[args.kernel_loop]
+          "attn_kernel": hp.attn_kernel_step, "rcmlp": hp.mlp_step}[args.kernel_loop]
     for _ in range(args.warmup):
         fn(stream)
     torch.cuda.synchronize()
@@ -520,9 +577,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="vitb_global", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="vith_global", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--also", default="vitb_global,vitb_window",
+                    help="other workloads measured the same way, reported under 'also' "
+                         "(comma-separated; empty for none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--kernel-loop", default=None, choices=["score", "perm", "attn", "rcmlp"],
+    ap.add_argument("--kernel-loop", default=None,
+                    choices=["score", "perm", "attn", "attn_kernel", "rcmlp"],
                     help="run only this library call in a loop (profiling aid; no bench line)")
     ap.add_argument("--stack", action="store_true",
                     help="time the ViT-L 24-block stack at densities 1.0/0.5/0.4/0.3 (no bench line)")

@@ -22,7 +22,9 @@
  *   - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
  *   - A device-side wait that gives up (it never should) records SS_ETIMEOUT in a device status
  *     word, makes the kernel return early and leaves the context usable; sparsesam_device_status()
- *     reads and clears that word.
+ *     reads and clears that word. Every perm / keep index a kernel reads is range-checked: one
+ *     outside its unit (perm) or image (keep) records SS_EINDEX in the same word and the row it
+ *     would have addressed is skipped (no access outside the caller's tensors).
  *
  * Layouts (shared by the calls; U = attention units, N = tokens per unit)
  *   global mode: U = batch, N = grid_h*grid_w (raster order).
@@ -54,6 +56,8 @@ extern "C" {
 #define SS_EWORKSPACE   (-3)  /* workspace pointer null/misaligned or smaller than required     */
 #define SS_ECUDA        (-4)  /* a CUDA runtime/driver call failed (launch, tensor-map encode)   */
 #define SS_ETIMEOUT     (-5)  /* a device-side wait gave up (read via sparsesam_device_status)   */
+#define SS_EINDEX       (-6)  /* a perm or keep index outside its unit or image reached a kernel;
+                                 the access was skipped (read via sparsesam_device_status)       */
 
 #define SS_GLOBAL 0
 #define SS_WINDOW 1
@@ -113,7 +117,9 @@ int sparsesam_score(const ss_cfg* cfg, const float* lum, double* score, void* st
  * lower enumeration index first) giving ranked tokens t_0..t_{N-1}; then perm[j*L + k] = t_{4k+j}.
  * score (device) -> perm, inv (device) int32 [U, N]; keep (device) int32 [batch, K]: the first K
  * tokens of each image's own ranking over its real tokens (window mode: per image, not per
- * window). Any of perm/inv/keep may be NULL to skip it (not all three). Scores must not be NaN. */
+ * window). Any of perm/inv/keep may be NULL to skip it (not all three). Scores may be any
+ * non-NaN doubles (negative, zero of either sign, infinite): they rank by value, and -0.0 ties with
+ * +0.0. A NaN score gives an unspecified (but in-bounds) permutation. */
 int sparsesam_perm(const ss_cfg* cfg, const double* score, int32_t* perm, int32_t* inv,
                    int32_t* keep, void* stream);
 
@@ -138,8 +144,19 @@ size_t sparsesam_attn_workspace(const ss_cfg* cfg);
 int sparsesam_attn(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                    const int32_t* perm, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
 
-/* Bytes of device workspace sparsesam_rcmlp needs (0 on invalid arguments). */
-size_t sparsesam_rcmlp_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden);
+/* S3 without its gather: the attention kernel alone, over the permuted Q, K, V that an earlier
+ * sparsesam_attn (or sparsesam_block) call with the same cfg and perm left in ws. ws holds three
+ * bf16 arrays of sparsesam_attn_workspace(cfg)/3 bytes each (Q, then K, then V), each laid out as
+ * [U*heads][N][head_dim]: row q of matrix u*heads+h is the token perm[u][j*L + a*b + r] for the
+ * block-major position q = a*4b + j*b + r (offset block a of stripe j; L, b from the pattern).
+ * out, perm and the results as for sparsesam_attn. For re-running the attention on prepared
+ * operands (and timing the kernel by itself). */
+int sparsesam_attn_gathered(const ss_cfg* cfg, const void* ws, size_t ws_bytes,
+                            const int32_t* perm, uint16_t* out, void* stream);
+
+/* Bytes of device workspace sparsesam_rcmlp needs for K kept tokens per image (0 on invalid
+ * arguments). */
+size_t sparsesam_rcmlp_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden, int32_t K);
 
 /* S4 (same summary, "Residual-Consistency MLP": only the top-K keep-set runs through the MLP; the
  * residual set bypasses it unchanged). In place on x (device) bf16 [batch, grid_h*grid_w, C]:
@@ -148,13 +165,16 @@ size_t sparsesam_rcmlp_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden);
  * every other row is left bit-for-bit untouched. w1 bf16 [hidden, C], w2 bf16 [C, hidden]
  * (row-major, PyTorch nn.Linear weight layout); b1 [hidden], b2 [C] bf16 or NULL (zero); x, w1,
  * w2, b1 and b2 16-byte aligned. keep
- * (device) int32 [batch, K] with distinct rows per image (as sparsesam_perm writes it).
+ * (device) int32 [batch, K] with distinct rows per image: the keep list sparsesam_perm writes
+ * (K = the pattern's `keep`, from the density) or one from another criterion
+ * (sparsesam_keep_by_update, sparsesam_random_perm), 0 <= K <= grid_h*grid_w; K = 0 launches
+ * nothing.
  * C and hidden must be multiples of 64. bf16 operands, fp32 accumulation; the hidden activation
  * is rounded to bf16 between the two products. ws (device, 256-byte aligned) >=
  * sparsesam_rcmlp_workspace bytes. */
 int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden,
                     const uint16_t* w1, const uint16_t* b1, const uint16_t* w2, const uint16_t* b2,
-                    const int32_t* keep, void* ws, size_t ws_bytes, void* stream);
+                    const int32_t* keep, int32_t K, void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of device workspace sparsesam_block needs (0 on an invalid cfg). */
 size_t sparsesam_block_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden);
@@ -179,21 +199,37 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
  * implicit device-wide synchronisation. Same arguments, semantics and results as sparsesam_rcmlp,
  * minus ws/ws_bytes: the scratch lives in a 32 MiB array inside this library (a file-scope
  * __device__ array that every GPU loading the library holds until the process exits).
- *   - Returns SS_EWORKSPACE, before any CUDA call, when sparsesam_rcmlp_workspace(cfg, C, hidden)
- *     exceeds 32 MiB (e.g. the SAM ViT-B global block, 28 MB, fits; batch 4 does not).
+ *   - Arguments are checked as sparsesam_rcmlp checks them (same codes); then, before any CUDA
+ *     call, SS_EWORKSPACE when sparsesam_rcmlp_workspace(cfg, C, hidden, K) exceeds 32 MiB (e.g.
+ *     the SAM ViT-B global block, 28 MB, fits; batch 4 does not).
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
- *     that device current); make that first call before any stream capture.
+ *     that device current); make that first call before any stream capture. The address is kept
+ *     for the process; after a cudaDeviceReset of that device it is stale (so is the status
+ *     word's address that every call looks up the same way), and the library must not be used on
+ *     that device again.
  *   - All calls on a device share the one array and leave their contents in it; nothing needs
  *     clearing because each call writes every scratch byte before reading it. Calls whose GPU
  *     execution overlaps (different streams, no ordering between them) race on the array. */
 int sparsesam_rcmlp_noalloc(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden,
                             const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
-                            const uint16_t* b2, const int32_t* keep, void* stream);
+                            const uint16_t* b2, const int32_t* keep, int32_t K, void* stream);
 
-/* Reads (and clears) the device status word that bounded device waits write. Synchronises the
- * given stream. *status receives SS_OK or SS_ETIMEOUT. Returns SS_OK or SS_ECUDA. */
+/* Reads (and clears) the device status word that bounded device waits and index checks write.
+ * Synchronises the given stream. *status receives SS_OK, SS_ETIMEOUT or SS_EINDEX. Returns SS_OK or
+ * SS_ECUDA. */
 int sparsesam_device_status(int32_t* status, void* stream);
+
+/* Test support for the failure path of the bounded device waits (no counterpart on the pages).
+ * sparsesam_set_wait_limit_ns sets, on the current device, how long a device wait may take before
+ * it gives up (default 500 ms; 0 restores the default). sparsesam_wait_selftest launches one CTA
+ * that waits on an mbarrier no thread arrives on (`which` = 0) or on a global counter nothing
+ * increments (`which` = 1), through the same bounded waits the kernels use, so that the wait runs
+ * out and records SS_ETIMEOUT in the status word; with `which` = 2 or 3 the barrier is arrived on /
+ * the counter is set first, so the wait succeeds and records nothing. Nothing else is in flight in
+ * that CTA. Both return SS_OK, SS_EINVAL or SS_ECUDA. */
+int sparsesam_set_wait_limit_ns(uint64_t ns);
+int sparsesam_wait_selftest(int32_t which, void* stream);
 
 /* Kernel launches this library has issued since it was loaded (host counter). */
 uint64_t sparsesam_launch_count(void);

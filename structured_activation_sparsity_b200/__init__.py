@@ -11,9 +11,10 @@ works before the library exists; using any of them without the built library rai
 import importlib
 
 _LIB_NAMES = {
-    "SS_ECUDA", "SS_EINVAL", "SS_EUNSUPPORTED", "SS_EWORKSPACE", "SS_ETIMEOUT", "SS_GLOBAL",
+    "SS_ECUDA", "SS_EINVAL", "SS_EUNSUPPORTED", "SS_EWORKSPACE", "SS_ETIMEOUT", "SS_EINDEX",
+    "SS_GLOBAL", "sparsesam_set_wait_limit_ns", "sparsesam_wait_selftest",
     "SS_OK", "SS_WINDOW", "SparseSAMError", "SsCfg", "SsPattern", "cfg_for", "make_cfg",
-    "sparsesam_attn", "sparsesam_attn_workspace", "sparsesam_blocklist",
+    "sparsesam_attn", "sparsesam_attn_gathered", "sparsesam_attn_workspace", "sparsesam_blocklist",
     "sparsesam_device_status", "sparsesam_launch_count", "sparsesam_pattern", "sparsesam_perm",
     "sparsesam_rcmlp", "sparsesam_rcmlp_noalloc", "sparsesam_rcmlp_workspace", "sparsesam_score",
     "sparsesam_score_perm", "sparsesam_block", "sparsesam_block_workspace",

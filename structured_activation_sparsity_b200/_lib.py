@@ -18,6 +18,7 @@ SS_EUNSUPPORTED = -2
 SS_EWORKSPACE = -3
 SS_ECUDA = -4
 SS_ETIMEOUT = -5
+SS_EINDEX = -6
 SS_GLOBAL = 0
 SS_WINDOW = 1
 
@@ -59,9 +60,12 @@ def _load():
                                            P, P, SZ, VP]),
         "sparsesam_attn_workspace": (SZ, [cfgp]),
         "sparsesam_attn": (ctypes.c_int, [cfgp, P, P, P, P, P, P, SZ, VP]),
-        "sparsesam_rcmlp_workspace": (SZ, [cfgp, I32, I32]),
-        "sparsesam_rcmlp": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, P, SZ, VP]),
-        "sparsesam_rcmlp_noalloc": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, VP]),
+        "sparsesam_attn_gathered": (ctypes.c_int, [cfgp, P, SZ, P, P, VP]),
+        "sparsesam_rcmlp_workspace": (SZ, [cfgp, I32, I32, I32]),
+        "sparsesam_rcmlp": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, I32, P, SZ, VP]),
+        "sparsesam_rcmlp_noalloc": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, I32, VP]),
+        "sparsesam_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
+        "sparsesam_wait_selftest": (ctypes.c_int, [I32, VP]),
         "sparsesam_device_status": (ctypes.c_int, [ctypes.POINTER(I32), VP]),
         "sparsesam_launch_count": (ctypes.c_uint64, []),
         "sparsesam_trace_start": (ctypes.c_int, [I32]),
@@ -175,24 +179,43 @@ def sparsesam_attn(cfg, q, k, v, perm, out, ws, ws_bytes, stream=None):
                                      _ptr(out), _ptr(ws), int(ws_bytes), _stream(stream)))
 
 
-def sparsesam_rcmlp_workspace(cfg, C: int, hidden: int) -> int:
-    return int(lib.sparsesam_rcmlp_workspace(ctypes.byref(cfg), int(C), int(hidden)))
+def sparsesam_attn_gathered(cfg, ws, ws_bytes, perm, out, stream=None):
+    """The attention kernel alone over the permuted Q, K, V an earlier sparsesam_attn left in ws."""
+    return _check("sparsesam_attn_gathered",
+                  lib.sparsesam_attn_gathered(ctypes.byref(cfg), _ptr(ws), int(ws_bytes), _ptr(perm),
+                                              _ptr(out), _stream(stream)))
 
 
-def sparsesam_rcmlp(cfg, x, C, hidden, w1, b1, w2, b2, keep, ws, ws_bytes, stream=None):
+def sparsesam_rcmlp_workspace(cfg, C: int, hidden: int, K: int) -> int:
+    return int(lib.sparsesam_rcmlp_workspace(ctypes.byref(cfg), int(C), int(hidden), int(K)))
+
+
+def sparsesam_rcmlp(cfg, x, C, hidden, w1, b1, w2, b2, keep, K, ws, ws_bytes, stream=None):
     return _check("sparsesam_rcmlp",
                   lib.sparsesam_rcmlp(ctypes.byref(cfg), _ptr(x), int(C), int(hidden), _ptr(w1),
-                                      _ptr(b1), _ptr(w2), _ptr(b2), _ptr(keep), _ptr(ws),
+                                      _ptr(b1), _ptr(w2), _ptr(b2), _ptr(keep), int(K), _ptr(ws),
                                       int(ws_bytes), _stream(stream)))
 
 
-def sparsesam_rcmlp_noalloc(cfg, x, C, hidden, w1, b1, w2, b2, keep, stream=None):
+def sparsesam_rcmlp_noalloc(cfg, x, C, hidden, w1, b1, w2, b2, keep, K, stream=None):
     """sparsesam_rcmlp with its scratch in the library's fixed 32 MiB device array (no workspace
     argument, nothing allocated). For callers that cannot allocate device memory."""
     return _check("sparsesam_rcmlp_noalloc",
                   lib.sparsesam_rcmlp_noalloc(ctypes.byref(cfg), _ptr(x), int(C), int(hidden),
                                               _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(keep),
-                                              _stream(stream)))
+                                              int(K), _stream(stream)))
+
+
+def sparsesam_set_wait_limit_ns(ns: int):
+    """Test support: the device waits' time limit on the current device (0 = the default)."""
+    return _check("sparsesam_set_wait_limit_ns", lib.sparsesam_set_wait_limit_ns(int(ns)))
+
+
+def sparsesam_wait_selftest(which: int, stream=None):
+    """Test support: one bounded device wait that runs out (which 0: mbarrier, 1: counter) or is
+    satisfied (2, 3)."""
+    return _check("sparsesam_wait_selftest",
+                  lib.sparsesam_wait_selftest(int(which), _stream(stream)))
 
 
 def sparsesam_device_status(stream=None) -> int:

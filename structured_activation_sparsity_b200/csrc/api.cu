@@ -8,12 +8,41 @@
 #include <mutex>
 #include <vector>
 
+#include "common.cuh"
 #include "kernels.h"
 
 namespace ss {
 
 // Device status word written by bounded device waits that give up (see sparsesam_device_status).
 __device__ int g_status = 0;
+// A counter nothing increments unless the self-test asks for it (sparsesam_wait_selftest).
+__device__ int g_selftest_counter = 0;
+
+// One CTA of 32 threads; thread 0 runs one bounded wait that (which 0, 1) nobody satisfies or
+// (which 2, 3) is satisfied before it starts: an mbarrier phase (0, 2) or a global counter (1, 3).
+// No copy or MMA is in flight, so giving up leaves nothing behind.
+__global__ void k_wait_selftest(int which, int* counter, int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (which == 0 || which == 2) {
+      if (which == 2) mbar_arrive(&bar);
+      mbar_wait(&bar, 0, &abort_flag, status);
+    } else {
+      *counter = which == 3 ? 1 : 0;
+      __threadfence();
+      wait_counter_geq(counter, 1, &abort_flag, status);
+      *counter = 0;
+    }
+  }
+  __syncthreads();
+}
 
 namespace {
 
@@ -379,28 +408,45 @@ int sparsesam_attn(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k, cons
     return launch_gather_qkv(q, k, v, perm, reinterpret_cast<uint16_t*>(wsb),
                              reinterpret_cast<uint16_t*>(wsb + one),
                              reinterpret_cast<uint16_t*>(wsb + 2 * one), g.U, g.N, heads, dh, p.b,
-                             st);
+                             status, st);
   }));
   if (rc) return rc;
   return attn_launch(cfg, g, p, wsb, perm, out, status, st);
 }
 
-size_t sparsesam_rcmlp_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden) {
+int sparsesam_attn_gathered(const ss_cfg* cfg, const void* ws, size_t ws_bytes,
+                            const int32_t* perm, uint16_t* out, void* stream) {
   Geo g;
-  if (geometry(cfg, &g) || C < 1 || hidden < 1) return 0;
-  return rcmlp_ws_bytes(g, keep_count(cfg->density, g.T), C, hidden);
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  ss_pattern p;
+  // The checks of sparsesam_attn, with the workspace standing in for q, k and v.
+  if ((rc = attn_check(cfg, g, static_cast<const uint16_t*>(ws), static_cast<const uint16_t*>(ws),
+                       static_cast<const uint16_t*>(ws), perm, out, &p)))
+    return rc == SS_EINVAL && !ws ? SS_EWORKSPACE : rc;
+  const size_t need = attn_ws_bytes(g, cfg->heads, cfg->head_dim);
+  if (!aligned(ws, 256) || ws_bytes < need) return SS_EWORKSPACE;
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+  return attn_launch(cfg, g, p, static_cast<uint8_t*>(const_cast<void*>(ws)), perm, out, status,
+                     static_cast<cudaStream_t>(stream));
+}
+
+size_t sparsesam_rcmlp_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden, int32_t K) {
+  Geo g;
+  if (geometry(cfg, &g) || C < 1 || hidden < 1 || K < 0 || K > g.T) return 0;
+  return rcmlp_ws_bytes(g, K, C, hidden);
 }
 
 // Argument checks of the RC-MLP step (also for the whole-block path).
-static int rcmlp_check(const ss_cfg* cfg, const Geo& g, const uint16_t* x, int32_t C,
-                       int32_t hidden, const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
-                       const uint16_t* b2, const int32_t* keep) {
-  if (!x || !w1 || !w2 || !keep || C < 1 || hidden < 1) return SS_EINVAL;
+static int rcmlp_check(const Geo& g, const uint16_t* x, int32_t C, int32_t hidden,
+                       const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
+                       const uint16_t* b2, const int32_t* keep, int32_t K) {
+  if (!x || !w1 || !w2 || !keep || C < 1 || hidden < 1 || K < 0 || K > g.T) return SS_EINVAL;
   if (C % 64 != 0 || hidden % 64 != 0) return SS_EUNSUPPORTED;
   if (!aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(b1, 16) ||
       !aligned(b2, 16))
     return SS_EINVAL;
-  const int K = keep_count(cfg->density, g.T);
   const int64_t M = (int64_t)g.B * K;
   if (M * (hidden > C ? hidden : C) >= ((int64_t)1 << 31) || (M + 127) / 128 > 65535)
     return SS_EUNSUPPORTED;
@@ -452,12 +498,12 @@ static int rcmlp_launch(const Geo& g, int K, uint16_t* x, int32_t C, int32_t hid
 
 int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, const uint16_t* w1,
                     const uint16_t* b1, const uint16_t* w2, const uint16_t* b2,
-                    const int32_t* keep, void* ws, size_t ws_bytes, void* stream) {
+                    const int32_t* keep, int32_t K, void* ws, size_t ws_bytes, void* stream) {
   Geo g;
   int rc = geometry(cfg, &g);
   if (rc) return rc;
-  if ((rc = rcmlp_check(cfg, g, x, C, hidden, w1, b1, w2, b2, keep))) return rc;
-  const int K = keep_count(cfg->density, g.T);
+  if ((rc = rcmlp_check(g, x, C, hidden, w1, b1, w2, b2, keep, K))) return rc;
+  if (K == 0) return SS_OK;   // an empty keep-set: every row is residual, nothing to launch
   const size_t need = rcmlp_ws_bytes(g, K, C, hidden);
   if (!ws || !aligned(ws, 256) || ws_bytes < need) return SS_EWORKSPACE;
   int* status = status_word();
@@ -470,7 +516,8 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, c
   const int n_counters = (int)((plan.total - plan.counters) / sizeof(int));
   rc = cuda_err(traced("gather_rows", st, [&] {
     return launch_gather_rows(x, keep, reinterpret_cast<uint16_t*>(wsb + plan.xk), g.B, g.T, K, C,
-                              reinterpret_cast<int*>(wsb + plan.counters), n_counters, st);
+                              reinterpret_cast<int*>(wsb + plan.counters), n_counters, status,
+                              st);
   }));
   if (rc) return rc;
   return rcmlp_launch(g, K, x, C, hidden, w1, b1, w2, b2, keep, wsb, status, st);
@@ -494,10 +541,10 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
   if (!lum || !score) return SS_EINVAL;
   ss_pattern p;
   if ((rc = attn_check(cfg, g, q, k, v, perm, out, &p))) return rc;
-  if ((rc = rcmlp_check(cfg, g, x, C, hidden, w1, b1, w2, b2, keep))) return rc;
+  const int K = keep_count(cfg->density, g.T);
+  if ((rc = rcmlp_check(g, x, C, hidden, w1, b1, w2, b2, keep, K))) return rc;
   if (g.N > kMaxRankTokens || g.T > kMaxRankTokens) return SS_EUNSUPPORTED;
   const int heads = cfg->heads, dh = cfg->head_dim;
-  const int K = keep_count(cfg->density, g.T);
   const size_t attn_part = align256(attn_ws_bytes(g, heads, dh));
   if (!ws || !aligned(ws, 256) || ws_bytes < attn_part + rcmlp_ws_bytes(g, K, C, hidden))
     return SS_EWORKSPACE;
@@ -525,7 +572,7 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
     return launch_gather_qkv(q, k, v, perm, reinterpret_cast<uint16_t*>(wsa),
                              reinterpret_cast<uint16_t*>(wsa + one),
                              reinterpret_cast<uint16_t*>(wsa + 2 * one), g.U, g.N, heads, dh, p.b,
-                             st);
+                             status, st);
   }));
   if (rc) return rc;
   if ((rc = attn_launch(cfg, g, p, wsa, perm, out, status, st))) return rc;
@@ -535,7 +582,7 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
   const int n_counters = (int)((plan.total - plan.counters) / sizeof(int));
   rc = cuda_err(traced("gather_rows", st, [&] {
     return launch_gather_rows(x, keep, reinterpret_cast<uint16_t*>(wsm + plan.xk), g.B, g.T, K, C,
-                              reinterpret_cast<int*>(wsm + plan.counters), n_counters, st,
+                              reinterpret_cast<int*>(wsm + plan.counters), n_counters, status, st,
                               /*late_wait=*/true);
   }));
   if (rc) return rc;
@@ -557,6 +604,28 @@ int sparsesam_device_status(int32_t* out, void* stream) {
 }
 
 uint64_t sparsesam_launch_count(void) { return g_launches.load(); }
+
+int sparsesam_set_wait_limit_ns(uint64_t ns) {
+  const uint64_t v = ns ? ns : kWaitLimitNs;
+  if (set_wait_limit_here(v) != cudaSuccess || set_wait_limit_attn(v) != cudaSuccess ||
+      set_wait_limit_mlp(v) != cudaSuccess)
+    return SS_ECUDA;
+  return SS_OK;
+}
+
+int sparsesam_wait_selftest(int32_t which, void* stream) {
+  if (which < 0 || which > 3) return SS_EINVAL;
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+  int* counter = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&counter), g_selftest_counter) != cudaSuccess)
+    return SS_ECUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_err(traced("wait_selftest", st, [&] {
+    k_wait_selftest<<<1, 32, 0, st>>>(which, counter, status);
+    return cudaGetLastError();
+  }));
+}
 
 int sparsesam_trace_start(int32_t capacity) {
   if (capacity < 1) return SS_EINVAL;
@@ -601,8 +670,22 @@ const char* sparsesam_strerror(int code) {
     case SS_EWORKSPACE: return "workspace missing, misaligned or too small";
     case SS_ECUDA: return "CUDA call failed";
     case SS_ETIMEOUT: return "device wait timed out";
+    case SS_EINDEX: return "perm or keep index outside its unit or image (access skipped)";
   }
   return "unknown error";
 }
 
 }  // extern "C"
+
+// The argument checks of sparsesam_rcmlp, in its order, and its workspace size (for the entry point
+// without a workspace, which must answer as sparsesam_rcmlp does).
+int ss::rcmlp_validate(const ss_cfg* cfg, const uint16_t* x, int32_t C, int32_t hidden,
+                       const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
+                       const uint16_t* b2, const int32_t* keep, int32_t K, size_t* need) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  if ((rc = rcmlp_check(g, x, C, hidden, w1, b1, w2, b2, keep, K))) return rc;
+  *need = K == 0 ? 0 : rcmlp_ws_bytes(g, K, C, hidden);
+  return SS_OK;
+}

@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(256, MINB) k_gather_qkv(const uint16_t* __rest
                                                        uint16_t* __restrict__ qp,
                                                        uint16_t* __restrict__ kp,
                                                        uint16_t* __restrict__ vp, int N,
-                                                       int heads, int b, int L) {
+                                                       int heads, int b, int L, int* status) {
   griddep_wait();
   griddep_launch();
   const int u = blockIdx.y;
@@ -48,7 +48,11 @@ __global__ void __launch_bounds__(256, MINB) k_gather_qkv(const uint16_t* __rest
   const int qpos = blockIdx.x * 8 + warp;
   if (qpos >= N) return;
   const int p = blockmajor_to_canonical(qpos, b, L);
-  const int tok = min(max(__ldg(perm + (size_t)u * N + p), 0), N - 1);   // stay in the unit
+  const int tok = __ldg(perm + (size_t)u * N + p);
+  if ((unsigned)tok >= (unsigned)N) {   // not a token of this unit: skip the row, report it
+    if (lane == 0) record_bad_index(status);
+    return;
+  }
   const int per_tok = heads * CPR;
   const size_t plane = (size_t)N * CPR;       // 16-byte chunks per (unit, head) matrix
   const size_t src_row = ((size_t)u * N + tok) * per_tok;
@@ -80,11 +84,13 @@ __global__ void __launch_bounds__(256, MINB) k_gather_qkv(const uint16_t* __rest
 
 cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                               const int32_t* perm, uint16_t* qp, uint16_t* kp, uint16_t* vp,
-                              int U, int N, int heads, int dh, int b, cudaStream_t st) {
+                              int U, int N, int heads, int dh, int b, int* status,
+                              cudaStream_t st) {
   dim3 grid((N + 7) / 8, U);
   const int L = N / kStripes;
   auto go = [&](auto kernel) {
-    return launch_pdl(kernel, grid, dim3(256), 0, st, q, k, v, perm, qp, kp, vp, N, heads, b, L);
+    return launch_pdl(kernel, grid, dim3(256), 0, st, q, k, v, perm, qp, kp, vp, N, heads, b, L,
+                      status);
   };
   const int per_tok = heads * (dh / 8);
   if (dh != 64 && dh != 80) return cudaErrorInvalidValue;
@@ -214,6 +220,14 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float&
   // add n to the exponent field: the low mantissa bits of t hold n (two's complement)
   p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
   p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+// Destination token of an output row: perm's entry if it lies in the unit, else -1 (the row is
+// not stored) with SS_EINDEX recorded.
+__device__ __forceinline__ int dst_token(int perm_t, int N, int* status) {
+  if ((unsigned)perm_t < (unsigned)N) return perm_t;
+  record_bad_index(status);
+  return -1;
 }
 
 // Work item = (unit * heads + head, 128-row query tile), numbered head-major so that the CTAs
@@ -692,7 +706,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 emit8(x0, x1, c);
               }
             }
-            s_dst[row] = store ? min(max(perm_t, 0), P.N - 1) : -1;
+            s_dst[row] = store ? dst_token(perm_t, P.N, status) : -1;
           }
           tc_fence_before();
           mbar_arrive(o_free);   // O0, O1 read: the next item's first P*V may overwrite them
@@ -764,7 +778,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             st_shared_v4(stage_row + grp * kCols * 2 + c * 16, pack_bf16(v[0], v[1]),
                          pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
           }
-          if (grp == 0) s_dst[row] = store ? min(max(perm_t, 0), P.N - 1) : -1;
+          if (grp == 0) s_dst[row] = store ? dst_token(perm_t, P.N, status) : -1;
         }
         named_barrier(1, 256);
         if (ok) {
@@ -1177,7 +1191,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                        pack_bf16(__uint_as_float(u[4]) * inv, __uint_as_float(u[5]) * inv),
                        pack_bf16(__uint_as_float(u[6]) * inv, __uint_as_float(u[7]) * inv));
         }
-        dst_tok[row] = store ? min(max(perm_t, 0), P.N - 1) : -1;
+        dst_tok[row] = store ? dst_token(perm_t, P.N, status) : -1;
       }
       tc_fence_before();   // O_g is read before the next item's first P goes to P*V
       named_barrier(bar, 128);
@@ -1255,5 +1269,7 @@ cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUte
   if (dh == 80) return launch_attn_dh<80>(tq, tk, tv, tq_tail, tk_tail, tv_tail, p, status, st);
   return cudaErrorInvalidValue;
 }
+
+cudaError_t set_wait_limit_attn(uint64_t ns) { return set_wait_limit_here(ns); }
 
 }  // namespace ss

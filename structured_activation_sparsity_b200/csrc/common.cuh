@@ -16,6 +16,13 @@ namespace ss {
 // Time limit of a bounded mbarrier wait. Every wait in these kernels is on work of the same CTA
 // that takes microseconds, so a wait this long means the pipeline is stuck.
 constexpr uint64_t kWaitLimitNs = 500ull * 1000ull * 1000ull;
+// The limit the waits use: kWaitLimitNs unless changed for a test (sparsesam_set_wait_limit_ns).
+// Each compiled source file of the library is its own device module with its own copy, which
+// set_wait_limit_here() (called through each file's exported setter) writes on the current device.
+static __constant__ uint64_t c_wait_limit_ns = kWaitLimitNs;
+static inline cudaError_t set_wait_limit_here(uint64_t ns) {
+  return cudaMemcpyToSymbol(c_wait_limit_ns, &ns, sizeof(ns));
+}
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -30,6 +37,9 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // A bounded wait that gives up writes SS_ETIMEOUT to the library's device status word (first
 // writer wins); kernels receive that word's address as an argument.
 __device__ __forceinline__ void record_timeout(int* status) { atomicCAS(status, 0, SS_ETIMEOUT); }
+// An index read from a caller's perm / keep tensor that falls outside its unit or image: the
+// access is skipped and SS_EINDEX recorded (first writer wins).
+__device__ __forceinline__ void record_bad_index(int* status) { atomicCAS(status, 0, SS_EINDEX); }
 
 // ---------------------------------------------------------------------------------------------
 // mbarrier
@@ -83,7 +93,7 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Waits for the phase with the given parity to complete. Returns false (and records a timeout)
-// if it has not completed within kWaitLimitNs, or as soon as *abort is set by another warp.
+// if it has not completed within c_wait_limit_ns, or as soon as *abort is set by another warp.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                          int* status) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -91,7 +101,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > c_wait_limit_ns) {
       record_timeout(status);
       *abort = 1;
       return false;
@@ -109,7 +119,7 @@ __device__ __forceinline__ bool wait_counter_geq(const int* counter, int target,
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
     if (v >= target) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > c_wait_limit_ns) {
       record_timeout(status);
       *abort = 1;
       return false;

@@ -12,6 +12,15 @@ namespace ss {
 
 constexpr int kMaxRankTokens = 16384;   // tokens per unit the rank kernel holds in shared memory
 
+// The bounded-wait limit of each source file's kernels (see c_wait_limit_ns), current device.
+cudaError_t set_wait_limit_attn(uint64_t ns);
+cudaError_t set_wait_limit_mlp(uint64_t ns);
+
+// sparsesam_rcmlp's argument checks (same codes, same order) and its workspace bytes in *need.
+int rcmlp_validate(const ss_cfg* cfg, const uint16_t* x, int32_t C, int32_t hidden,
+                   const uint16_t* w1, const uint16_t* b1, const uint16_t* w2, const uint16_t* b2,
+                   const int32_t* keep, int32_t K, size_t* need);
+
 cudaError_t launch_sobel_score(const float* lum, double* score, int B, int H, int W,
                                cudaStream_t st);
 
@@ -25,7 +34,8 @@ cudaError_t launch_stripe_rank(const double* score, const float* lum, double* sc
 // Gathers q, k, v [U, N, heads, dh] into the block-major permuted layout [U*heads, N, dh].
 cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                               const int32_t* perm, uint16_t* qp, uint16_t* kp, uint16_t* vp,
-                              int U, int N, int heads, int dh, int b, cudaStream_t st);
+                              int U, int N, int heads, int dh, int b, int* status,
+                              cudaStream_t st);
 
 struct AttnParams {
   const int32_t* perm;   // [U, N]
@@ -44,7 +54,7 @@ cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUte
 // and x are known final at launch (see k_gather_rows), the copy need not wait for the previous
 // launch.
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* keep, uint16_t* xk, int B, int T,
-                               int K, int C, int* zero, int nzero, cudaStream_t st,
+                               int K, int C, int* zero, int nzero, int* status, cudaStream_t st,
                                bool late_wait = false);
 
 struct GemmEpilogue {

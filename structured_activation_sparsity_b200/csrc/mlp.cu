@@ -30,15 +30,16 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t* __restrict_
                                                      const int32_t* __restrict__ keep,
                                                      uint16_t* __restrict__ xk, int B, int T,
                                                      int K, int C, int* __restrict__ zero,
-                                                     int nzero, int late_wait) {
+                                                     int nzero, int late_wait, int* status) {
   if (!late_wait) griddep_wait();
   griddep_launch();
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
   const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (m < B * K) {
+  const int t = m < B * K ? __ldg(keep + m) : 0;
+  if (m < B * K && (unsigned)t >= (unsigned)T && lane == 0) record_bad_index(status);
+  if (m < B * K && (unsigned)t < (unsigned)T) {   // a keep entry outside the image is skipped
     const int b = m / K;
-    const int t = min(max(__ldg(keep + m), 0), T - 1);   // never leave the image
     const int cpr = C / 8;
     const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)b * T + t) * C);
     uint4* dst = reinterpret_cast<uint4*>(xk) + (size_t)m * cpr;
@@ -56,11 +57,11 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t* __restrict_
 }
 
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* keep, uint16_t* xk, int B, int T,
-                               int K, int C, int* zero, int nzero, cudaStream_t st,
+                               int K, int C, int* zero, int nzero, int* status, cudaStream_t st,
                                bool late_wait) {
   const int rows = B * K;
   return launch_pdl(k_gather_rows, dim3((rows + 7) / 8), dim3(256), 0, st, x, keep, xk, B, T, K, C,
-                    zero, nzero, late_wait ? 1 : 0);
+                    zero, nzero, late_wait ? 1 : 0, status);
 }
 
 // Persistent warp-specialised GEMM. Work unit = (m-tile, n-tile, k-split); CTA c takes units
@@ -140,10 +141,17 @@ struct GemmShape {
 // The epilogue of one output row m (< M) in chunks of 32 columns. The row's destination (and, for
 // kind 1, the keep lookup behind it) is resolved once per unit; a chunk's bias and residual words
 // are loaded before its accumulator values are needed, so their latency overlaps those reads.
-__device__ __forceinline__ uint16_t* epi_row(const GemmEpilogue& ep, const GemmShape& g, int m) {
+// Kind 1: a keep entry outside the image gives no row (nullptr: the row is skipped) and records
+// SS_EINDEX.
+__device__ __forceinline__ uint16_t* epi_row(const GemmEpilogue& ep, const GemmShape& g, int m,
+                                             int* status) {
   if (ep.kind == 0) return ep.out + (size_t)m * g.N;
   const int b = m / ep.K_per_image;
-  const int t = min(max(__ldg(ep.keep + m), 0), ep.T - 1);   // never leave the image
+  const int t = __ldg(ep.keep + m);
+  if ((unsigned)t >= (unsigned)ep.T) {
+    record_bad_index(status);
+    return nullptr;
+  }
   return ep.x + ((size_t)b * ep.T + t) * g.N;
 }
 struct Epi32In {
@@ -382,7 +390,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int m = m_t * 128 + row;
       const int tile = n_t * g.m_tiles + m_t;
       const uint32_t t_acc = tmem + buf * BN + lane_off + col0;
-      uint16_t* drow = m < g.M ? epi_row(ep, g, m) : nullptr;
+      uint16_t* drow = m < g.M ? epi_row(ep, g, m, status) : nullptr;
       if (g.splits == 1 && !pair) {
 #pragma unroll 1
         for (int c = 0; c < G::kHalf / 32; ++c) {
@@ -630,5 +638,7 @@ cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, const Gemm
   }
   return cudaErrorInvalidValue;
 }
+
+cudaError_t set_wait_limit_mlp(uint64_t ns) { return set_wait_limit_here(ns); }
 
 }  // namespace ss

@@ -11,7 +11,8 @@
 // The array is a file-scope __device__ variable: every GPU that loads this library holds its
 // kRcmlpScratchBytes until the process exits. Host code may not use its name as a device address;
 // the address is looked up once per device with cudaGetSymbolAddress (with that device current)
-// and passed to the kernels.
+// and passed to the kernels. That cached address (like the status word's) is not looked up again,
+// so it is stale after a cudaDeviceReset of the device.
 #include <mutex>
 
 #include "kernels.h"
@@ -44,11 +45,13 @@ int scratch_address(void** out) {
 
 extern "C" int sparsesam_rcmlp_noalloc(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden,
                                        const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
-                                       const uint16_t* b2, const int32_t* keep, void* stream) {
-  // Size check first, on the host: a shape whose scratch exceeds the fixed array is rejected
-  // before any CUDA call.
-  const size_t need = sparsesam_rcmlp_workspace(cfg, C, hidden);
-  if (need == 0) return SS_EINVAL;
+                                       const uint16_t* b2, const int32_t* keep, int32_t K,
+                                       void* stream) {
+  // The same argument checks as sparsesam_rcmlp, then the size check, all on the host: a shape
+  // whose scratch exceeds the fixed array is rejected before any CUDA call.
+  size_t need = 0;
+  int rc0 = ss::rcmlp_validate(cfg, x, C, hidden, w1, b1, w2, b2, keep, K, &need);
+  if (rc0) return rc0;
   if (need > ss::kRcmlpScratchBytes) return SS_EWORKSPACE;
   void* scratch = nullptr;
   int rc = ss::scratch_address(&scratch);
@@ -56,6 +59,6 @@ extern "C" int sparsesam_rcmlp_noalloc(const ss_cfg* cfg, uint16_t* x, int32_t C
   // Every scratch byte the MLP reads is written earlier in the same call (the gather fills the
   // kept rows, fc1 fills the hidden rows it covers, TMA zero-fills rows past the end), so nothing
   // left from a previous call has to be cleared.
-  return sparsesam_rcmlp(cfg, x, C, hidden, w1, b1, w2, b2, keep, scratch, ss::kRcmlpScratchBytes,
-                         stream);
+  return sparsesam_rcmlp(cfg, x, C, hidden, w1, b1, w2, b2, keep, K, scratch,
+                         ss::kRcmlpScratchBytes, stream);
 }

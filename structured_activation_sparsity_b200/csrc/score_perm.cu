@@ -48,7 +48,22 @@ __global__ void __launch_bounds__(256) k_sobel_score(const float* __restrict__ l
   score[idx] = sobel_at(lum + (size_t)b * per, H, W, y, x);
 }
 
-// Unit-local token t -> its score key (bits of a non-negative double, which order like the value).
+// Order-preserving 64-bit key of a double: for any non-NaN a, b, a < b exactly when
+// key(a) < key(b) as unsigned integers, and -0.0 and +0.0 share one key (they compare equal, so the
+// stable sort keeps their enumeration order). Negative values have their bits inverted (so a more
+// negative value gets a smaller key), non-negative values get the sign bit set (so they sit above
+// every negative one).
+__device__ __forceinline__ unsigned long long order_key(double v) {
+  unsigned long long u = (unsigned long long)__double_as_longlong(v);
+  if (u == 0x8000000000000000ull) u = 0ull;   // -0.0 -> +0.0
+  return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+// The double whose order_key is k (for -0.0, +0.0).
+__device__ __forceinline__ double key_value(unsigned long long k) {
+  return __longlong_as_double((long long)((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
+}
+
+// Unit-local token t -> its score's order key.
 struct UnitMap {
   int window_mode;   // 0: unit = image, t = raster index; 1: unit = window, t = window raster
   int Hg, Wg, ws, wpr, nwin;
@@ -69,15 +84,14 @@ struct UnitMap {
   }
   __device__ __forceinline__ unsigned long long key(const double* score, int u, int t) const {
     int b, y, x;
-    if (!locate(u, t, b, y, x)) return 0ull;   // pad token: +0.0
-    return (unsigned long long)__double_as_longlong(score[((size_t)b * Hg + y) * Wg + x]);
+    if (!locate(u, t, b, y, x)) return order_key(0.0);   // pad token: +0.0
+    return order_key(score[((size_t)b * Hg + y) * Wg + x]);
   }
   // The same key computed from the luminance (S1 fused into S2).
   __device__ __forceinline__ unsigned long long key_lum(const float* lum, int u, int t) const {
     int b, y, x;
-    if (!locate(u, t, b, y, x)) return 0ull;
-    return (unsigned long long)__double_as_longlong(
-        sobel_at(lum + (size_t)b * Hg * Wg, Hg, Wg, y, x));
+    if (!locate(u, t, b, y, x)) return order_key(0.0);
+    return order_key(sobel_at(lum + (size_t)b * Hg * Wg, Hg, Wg, y, x));
   }
 };
 
@@ -121,8 +135,8 @@ __global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __rest
       for (int k = 0; k < 4; ++k) {
         const double v = sobel_of(l[0][k], l[0][k + 1], l[0][k + 2], l[1][k], l[1][k + 2],
                                   l[2][k], l[2][k + 1], l[2][k + 2]);
-        const unsigned long long bits = (unsigned long long)__double_as_longlong(v);
-        if (k & 1) k2[k >> 1].y = bits; else k2[k >> 1].x = bits;
+        const unsigned long long key = order_key(v);
+        if (k & 1) k2[k >> 1].y = key; else k2[k >> 1].x = key;
       }
       reinterpret_cast<ulonglong2*>(s_key)[2 * q] = k2[0];       // y*W + x0 is a multiple of 4
       reinterpret_cast<ulonglong2*>(s_key)[2 * q + 1] = k2[1];
@@ -189,7 +203,7 @@ __global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __rest
     if (keep && r < K) keep[(size_t)u * K + r] = t;
     if (FROM_LUM && score_out) {
       int b, y, x;
-      if (m.locate(u, t, b, y, x)) score_out[((size_t)b * m.Hg + y) * m.Wg + x] = __longlong_as_double((long long)kt);
+      if (m.locate(u, t, b, y, x)) score_out[((size_t)b * m.Hg + y) * m.Wg + x] = key_value(kt);
     }
   }
 }

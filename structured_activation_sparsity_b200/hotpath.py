@@ -39,7 +39,7 @@ class HotPath:
         # One workspace for the whole-block call; the per-step calls use its two parts (the
         # attention's first, 256-byte aligned, then the MLP's).
         self.ws_attn_bytes = L.sparsesam_attn_workspace(self.cfg)
-        self.ws_mlp_bytes = L.sparsesam_rcmlp_workspace(self.cfg, C, Hd)
+        self.ws_mlp_bytes = L.sparsesam_rcmlp_workspace(self.cfg, C, Hd, self.K)
         self.ws_block_bytes = L.sparsesam_block_workspace(self.cfg, C, Hd)
         self.ws_block = torch.empty((self.ws_block_bytes,), dtype=torch.uint8, **e)
         attn_part = -(-self.ws_attn_bytes // 256) * 256
@@ -73,9 +73,16 @@ class HotPath:
         L.sparsesam_attn(self.cfg, self.q, self.k, self.v, self.perm, self.out, self.ws_attn,
                          self.ws_attn_bytes, stream)
 
+    def attn_kernel_step(self, stream=None):
+        """The attention kernel alone over the permuted Q, K, V the last attn_step / step left in
+        the workspace (for timing the kernel by itself)."""
+        L.sparsesam_attn_gathered(self.cfg, self.ws_attn, self.ws_attn_bytes, self.perm, self.out,
+                                  stream)
+
     def mlp_step(self, stream=None):
         L.sparsesam_rcmlp(self.cfg, self.x, self.wl.dim, self.wl.hidden, self.w1, self.b1,
-                          self.w2, self.b2, self.keep, self.ws_mlp, self.ws_mlp_bytes, stream)
+                          self.w2, self.b2, self.keep, self.K, self.ws_mlp, self.ws_mlp_bytes,
+                          stream)
 
     def step(self, stream=None):
         """S1..S4 of one block, asynchronously on `stream` (a torch.cuda.Stream or None), in the

@@ -39,7 +39,7 @@ def test_no_launches_without_gpu_work():
 
 def test_strerror():
     assert L.strerror(0) == "ok"
-    for c in (-1, -2, -3, -4, -5):
+    for c in (-1, -2, -3, -4, -5, -6):
         assert L.strerror(c) != "unknown error"
     assert L.strerror(-99) == "unknown error"
 
@@ -104,7 +104,8 @@ def test_validation_codes():
     assert lib.sparsesam_block_workspace(None, 64, 256) == 0
     assert lib.sparsesam_block_workspace(by(good), 0, 256) == 0
     assert lib.sparsesam_block_workspace(by(good), 64, 256) >= (
-        lib.sparsesam_attn_workspace(by(good)) + lib.sparsesam_rcmlp_workspace(by(good), 64, 256))
+        lib.sparsesam_attn_workspace(by(good))
+        + lib.sparsesam_rcmlp_workspace(by(good), 64, 256, O.keep_count(0.4, 256)))
     blk = [FAKE] * 5 + [64, 256] + [FAKE] * 4 + [FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, None]
     assert lib.sparsesam_block(by(good), *blk) == L.SS_EWORKSPACE   # 1 byte of workspace
     for i in (0, 1, 11, 12, 14, 15):   # lum, q, score, perm, keep, out
@@ -127,12 +128,19 @@ def test_validation_codes():
     assert lib.sparsesam_attn(by(good), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, None) == L.SS_EWORKSPACE
     assert lib.sparsesam_attn(by(good), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 16, need, None) == L.SS_EWORKSPACE
     assert lib.sparsesam_attn(by(good), FAKE, FAKE, FAKE, FAKE, FAKE, None, need, None) == L.SS_EWORKSPACE
-    # rcmlp: C not a multiple of 64, workspace
-    assert lib.sparsesam_rcmlp(by(good), FAKE, 48, 256, FAKE, None, FAKE, None, FAKE, FAKE, 1 << 30, None) == L.SS_EUNSUPPORTED
-    need_m = L.sparsesam_rcmlp_workspace(good, 64, 256)
+    # rcmlp: C not a multiple of 64, K outside [0, T], workspace
     K = O.keep_count(0.4, 256)
+    assert lib.sparsesam_rcmlp(by(good), FAKE, 48, 256, FAKE, None, FAKE, None, FAKE, K, FAKE, 1 << 30, None) == L.SS_EUNSUPPORTED
+    for badK in (-1, 257):
+        assert lib.sparsesam_rcmlp(by(good), FAKE, 64, 256, FAKE, None, FAKE, None, FAKE, badK, FAKE, 1 << 30, None) == L.SS_EINVAL
+        assert lib.sparsesam_rcmlp_workspace(by(good), 64, 256, badK) == 0
+    need_m = L.sparsesam_rcmlp_workspace(good, 64, 256, K)
     assert need_m == math.ceil(K * 64 * 2 / 256) * 256 + math.ceil(K * 256 * 2 / 256) * 256
-    assert lib.sparsesam_rcmlp(by(good), FAKE, 64, 256, FAKE, None, FAKE, None, FAKE, FAKE, need_m - 1, None) == L.SS_EWORKSPACE
+    assert lib.sparsesam_rcmlp(by(good), FAKE, 64, 256, FAKE, None, FAKE, None, FAKE, K, FAKE, need_m - 1, None) == L.SS_EWORKSPACE
+    # a caller K other than the density's (another keep criterion) sizes the workspace by that K
+    assert L.sparsesam_rcmlp_workspace(good, 64, 256, 200) > need_m
+    # K = 0: every row is residual; nothing is launched, even without a workspace
+    assert lib.sparsesam_rcmlp(by(good), FAKE, 64, 256, FAKE, None, FAKE, None, FAKE, 0, None, 0, None) == L.SS_OK
     # A long-K fc2 (ViT-H: K = 5120, 80 k-blocks; 4 images, 4916 kept rows) has a last partial
     # round of tiles split in two along K: the workspace holds their fp32 halves and counters
     # beyond xk and H.
@@ -141,7 +149,7 @@ def test_validation_codes():
     xk_h = math.ceil(M * 1280 * 2 / 256) * 256 + math.ceil(M * 5120 * 2 / 256) * 256
     # 47 tail tiles of 128 x 256 fp32 (6.2 MB), where a two-way split of all 195 tiles would need
     # 51 MB of partials
-    extra = L.sparsesam_rcmlp_workspace(vith, 1280, 5120) - xk_h
+    extra = L.sparsesam_rcmlp_workspace(vith, 1280, 5120, O.keep_count(0.3, 4096)) - xk_h
     assert 47 * 128 * 256 * 4 <= extra < 8 << 20
     # blocklist capacity
     rp = (ctypes.c_int32 * 8)()

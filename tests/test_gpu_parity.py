@@ -99,10 +99,58 @@ def test_perm_ties_flat_and_quantised():
     assert np.array_equal(perm[0], [4 * k + j for j in range(4) for k in range(64)])
 
 
+def _caller_scores(B, T, seed):
+    """Scores a caller may pass: negatives, mixed signs, both zeros, huge and tiny magnitudes,
+    infinities, subnormals and ties across signs (equal magnitudes of both signs)."""
+    g = np.random.default_rng(seed)
+    pool = np.array([0.0, -0.0, 1.0, -1.0, 1e308, -1e308, 1e-308, -1e-308, 5e-324, -5e-324,
+                     np.inf, -np.inf, 2.5, -2.5, 3.0e-5, -3.0e-5])
+    s = g.standard_normal((B, T)) * 10.0 ** g.integers(-30, 30, (B, T))
+    pick = g.random((B, T)) < 0.35
+    s[pick] = pool[g.integers(0, pool.size, int(pick.sum()))]
+    return s
+
+
+@pytest.mark.parametrize("B,H,W,mode,ws,d", [
+    (2, 16, 16, "global", 14, 0.4), (1, 64, 64, "global", 14, 0.3), (2, 30, 30, "window", 14, 0.5),
+    (1, 64, 64, "window", 14, 0.3),
+])
+def test_perm_caller_scores_any_sign(B, H, W, mode, ws, d):
+    """sparsesam_perm on scores it did not compute: it must rank by value, -0.0 tying with +0.0."""
+    cfg = L.make_cfg(B, H, W, mode, ws, 1, 64, d)
+    geo = _geo(cfg)
+    sc = _caller_scores(B, H * W, seed=B * 100 + H)
+    o_perm, o_inv = O.stripe_sort(sc, geo)
+    o_keep = O.keep_list(sc, cfg.density)
+    dsc = torch.from_numpy(sc).to(DEV)
+    perm = torch.full((geo.units, geo.unit_tokens), -1, dtype=torch.int32, device=DEV)
+    inv = torch.full_like(perm, -1)
+    keep = torch.full(o_keep.shape, -1, dtype=torch.int32, device=DEV)
+    L.sparsesam_perm(cfg, dsc, perm, inv, keep)
+    torch.cuda.synchronize()
+    assert np.array_equal(perm.cpu().numpy(), o_perm)
+    assert np.array_equal(inv.cpu().numpy(), o_inv)
+    assert np.array_equal(keep.cpu().numpy(), o_keep)
+    _status_ok()
+
+
+def test_perm_negative_zero_ties_positive_zero():
+    """All scores zero, half of them -0.0: one tie class, so the closed form of a flat image."""
+    cfg = L.make_cfg(1, 16, 16, "global", 14, 1, 64, 0.4)
+    sc = np.zeros((1, 256))
+    sc[0, ::2] = -0.0
+    dsc = torch.from_numpy(sc).to(DEV)
+    perm = torch.empty((1, 256), dtype=torch.int32, device=DEV)
+    L.sparsesam_perm(cfg, dsc, perm, None, None)
+    torch.cuda.synchronize()
+    assert np.array_equal(perm.cpu().numpy()[0], [4 * k + j for j in range(4) for k in range(64)])
+
+
 # ------------------------------------------------------------------------------------------------
 # S3 attention
 # ------------------------------------------------------------------------------------------------
 def _attn_case(cfg, seed, scale=1.0, heads_check=None, units_check=None):
+    """heads_check / units_check: None (all) or a list of the heads / units the oracle checks."""
     geo = _geo(cfg)
     U, N, H, D = geo.units, geo.unit_tokens, cfg.heads, cfg.head_dim
     g = np.random.default_rng(seed)
@@ -117,11 +165,11 @@ def _attn_case(cfg, seed, scale=1.0, heads_check=None, units_check=None):
     L.sparsesam_attn(cfg, dq, dk, dv, dperm, out, ws, wsb)
     torch.cuda.synchronize()
     got = synth.bf16_to_f64(out)
-    us = slice(None) if units_check is None else slice(0, units_check)
-    hs = slice(None) if heads_check is None else slice(0, heads_check)
-    q64, k64, v64 = (synth.bf16_to_f64(t)[us, :, hs] for t in qkv)
+    us = np.arange(U) if units_check is None else np.asarray(units_check)
+    hs = np.arange(H) if heads_check is None else np.asarray(heads_check)
+    q64, k64, v64 = (synth.bf16_to_f64(t)[us][:, :, hs] for t in qkv)
     want = O.attention(q64, k64, v64, perm[us], cfg.density)
-    _assert_close(got[us, :, hs], want, f"attn {U}x{N}x{H}x{D} d={cfg.density}")
+    _assert_close(got[us][:, :, hs], want, f"attn {U}x{N}x{H}x{D} d={cfg.density}")
     _status_ok()
     return got, want
 
@@ -148,8 +196,12 @@ def test_attention_tiny_workload():
     _attn_case(L.cfg_for(wl), seed=0, scale=wl.qkv_scale)
 
 
+# Full sizes: every unit and head of ViT-B global; elsewhere a spread sample (first, middle and
+# last units; first, middle and last heads), so that an indexing slip past the first unit or head
+# cannot pass.
 @pytest.mark.parametrize("name,heads_check,units_check", [
-    ("vitb_global", None, None), ("vitb_window", None, 8), ("vith_global", 4, 1),
+    ("vitb_global", None, None), ("vitb_window", [0, 5, 11], [0, 1, 49, 50, 98, 99]),
+    ("vith_global", [0, 7, 15], [0, 2, 3]), ("vitl_global", [0, 9, 15], [0, 7]),
 ])
 def test_attention_full_size(name, heads_check, units_check):
     wl = workloads.get(name)
@@ -161,6 +213,8 @@ def test_attention_full_size(name, heads_check, units_check):
 # S4 RC-MLP
 # ------------------------------------------------------------------------------------------------
 def _mlp_case(cfg, C, Hd, seed, bias=True, images_check=None):
+    """images_check: None (all) or a list of the images the oracle checks (the residual rows of
+    every image are checked bit for bit)."""
     B, T = cfg.batch, cfg.grid_h * cfg.grid_w
     g = np.random.default_rng(seed)
     lum = g.random((B, cfg.grid_h, cfg.grid_w)).astype(np.float32)
@@ -173,13 +227,14 @@ def _mlp_case(cfg, C, Hd, seed, bias=True, images_check=None):
     dx = x.to(DEV)
     dev = [None if t is None else t.to(DEV) for t in (w1, b1, w2, b2)]
     dkeep = torch.from_numpy(keep).to(DEV)
-    wsb = L.sparsesam_rcmlp_workspace(cfg, C, Hd)
+    K = keep.shape[1]
+    wsb = L.sparsesam_rcmlp_workspace(cfg, C, Hd, K)
     ws = torch.empty((wsb,), dtype=torch.uint8, device=DEV)
-    L.sparsesam_rcmlp(cfg, dx, C, Hd, dev[0], dev[1], dev[2], dev[3], dkeep, ws, wsb)
+    L.sparsesam_rcmlp(cfg, dx, C, Hd, dev[0], dev[1], dev[2], dev[3], dkeep, K, ws, wsb)
     torch.cuda.synchronize()
     got = synth.bf16_to_f64(dx)
     x64 = synth.bf16_to_f64(x)
-    bs = slice(None) if images_check is None else slice(0, images_check)
+    bs = np.arange(B) if images_check is None else np.asarray(images_check)
     want = O.rcmlp(x64[bs], synth.bf16_to_f64(w1), None if b1 is None else synth.bf16_to_f64(b1),
                    synth.bf16_to_f64(w2), None if b2 is None else synth.bf16_to_f64(b2), keep[bs])
     mask = np.zeros((B, T), bool)
@@ -206,8 +261,8 @@ def test_rcmlp_small(B, H, W, C, Hd, d, bias):
     _mlp_case(cfg, C, Hd, seed=C + Hd, bias=bias)
 
 
-@pytest.mark.parametrize("name,images_check", [("vitb_global", None), ("vitb_window", 1),
-                                               ("vith_global", 1)])
+@pytest.mark.parametrize("name,images_check", [("vitb_global", None), ("vitb_window", [0, 3]),
+                                               ("vith_global", [0, 3]), ("vitl_global", [0, 7])])
 def test_rcmlp_full_size(name, images_check):
     wl = workloads.get(name)
     _mlp_case(L.cfg_for(wl), wl.dim, wl.hidden, seed=wl.seed, images_check=images_check)
