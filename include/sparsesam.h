@@ -11,6 +11,8 @@
  *   sparsesam_block       S1..S4 in one call with one workspace
  *   sparsesam_attn   S3  static block-sparse attention over the permuted sequence
  *   sparsesam_rcmlp  S4  fc1-GELU-fc2 on the kept tokens, added to the residual in place
+ *   sparsesam_random_perm     S2 over random scores (the random-permutation ablation)
+ *   sparsesam_keep_by_update  the keep-set by update magnitude (another keep criterion)
  *
  * Conventions shared by every call
  *   - Pointers marked (device) are device memory owned by the caller; nothing is allocated or
@@ -130,6 +132,26 @@ int sparsesam_perm(const ss_cfg* cfg, const double* score, int32_t* perm, int32_
  * sparsesam_score, both non-NULL; perm, inv, keep as for sparsesam_perm. */
 int sparsesam_score_perm(const ss_cfg* cfg, const float* lum, double* score, int32_t* perm,
                          int32_t* inv, int32_t* keep, void* stream);
+
+/* The random-permutation ablation (the SparseSAM README's registry variant `sparsesam_random`):
+ * S2 over random scores instead of the Sobel ranking. score (device, non-NULL) fp64
+ * [batch, grid_h*grid_w] receives score[b][t] = (X >> 11) * 2^-53, uniform in [0, 1), where X is
+ * output b*grid_h*grid_w + t of the SplitMix64 generator started from state `seed` (Steele, Lea
+ * and Flood, OOPSLA 2014: output n = mix(seed + (n + 1) * 0x9E3779B97F4A7C15)); then
+ * sparsesam_perm(cfg, score, perm, inv, keep) runs on them (perm, inv, keep as there). */
+int sparsesam_random_perm(const ss_cfg* cfg, uint64_t seed, double* score, int32_t* perm,
+                          int32_t* inv, int32_t* keep, void* stream);
+
+/* The keep-set by update magnitude (Dutch summary, "Methodologie" 2, "Selectieve Berekening": the
+ * MLP runs on the top-K tokens with high feature dissimilarity or update magnitude). delta (device)
+ * bf16 [batch, grid_h*grid_w, C], 16-byte aligned, C % 8 == 0: each token's update (e.g. the
+ * block's attention output). mag (device) fp64 [batch, grid_h*grid_w] receives
+ * sum over c = 0..C-1 (in that order, one fp64 rounding per multiply and per add) of
+ * delta[b,t,c]^2; keep (device) int32 [batch, K] the first K tokens of each image's stable
+ * descending ranking by mag (equal magnitudes: lower token first), 0 <= K <= grid_h*grid_w, for
+ * sparsesam_rcmlp(..., keep, K, ...). K = 0 launches nothing. */
+int sparsesam_keep_by_update(const ss_cfg* cfg, const uint16_t* delta, int32_t C, int32_t K,
+                             double* mag, int32_t* keep, void* stream);
 
 /* Bytes of device workspace sparsesam_attn needs for cfg (0 on an invalid cfg). */
 size_t sparsesam_attn_workspace(const ss_cfg* cfg);

@@ -330,6 +330,63 @@ def rcmlp(x, w1, b1, w2, b2, keep) -> np.ndarray:
     return y
 
 
+def keep_top(score: np.ndarray, K: int) -> np.ndarray:
+    """int32 [B, K]: the K first tokens of each image's stable descending ranking by `score`
+    (ties: lower token index first) -- the keep list of any keep criterion given as a score."""
+    B, T = score.shape
+    assert 0 <= K <= T
+    out = np.empty((B, K), dtype=np.int32)
+    for b in range(B):
+        out[b] = ranked_order(score[b])[:K]
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# Variants: the random-permutation ablation and the update-magnitude keep criterion
+# ---------------------------------------------------------------------------------------------
+_GOLDEN_GAMMA = np.uint64(0x9E3779B97F4A7C15)
+
+
+def splitmix64(seed: int, n: np.ndarray) -> np.ndarray:
+    """Output n (n = 0, 1, ...) of the SplitMix64 generator started from state `seed` (Steele,
+    Lea and Flood, "Fast splittable pseudorandom number generators", OOPSLA 2014): the state after
+    n + 1 steps, seed + (n + 1) * gamma, through the generator's output mix. uint64 arithmetic
+    wraps modulo 2^64."""
+    n = np.asarray(n, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        z = np.uint64(seed) + (n + np.uint64(1)) * _GOLDEN_GAMMA
+        z = (z ^ (z >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
+        z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
+        return z ^ (z >> np.uint64(31))
+
+
+def random_scores(batch: int, tokens: int, seed: int) -> np.ndarray:
+    """float64 [B, T] uniform in [0, 1): token t of image b draws output b*T + t of SplitMix64
+    from `seed`, keeps its top 53 bits and scales them by 2^-53.
+
+    Reading of the README's registry variant `sparsesam_random`: the stripe-sort permutation (and
+    keep list) built from a random token order instead of the Sobel ranking -- the same sort,
+    transpose and pattern, over these scores."""
+    idx = np.arange(batch * tokens, dtype=np.uint64)
+    u = splitmix64(seed, idx) >> np.uint64(11)
+    return (u.astype(np.float64) * 2.0 ** -53).reshape(batch, tokens)
+
+
+def update_magnitude(delta) -> np.ndarray:
+    """float64 [B, T]: sum over channels c = 0, 1, ..., C-1, in that order, of delta[b, t, c]^2.
+
+    Reading of the Dutch summary's "Selectieve Berekening" (the MLP runs on the top-K tokens "with
+    high feature dissimilarity or update magnitude"): a token's update magnitude is the squared
+    norm of the update its row receives (e.g. the block's attention output); the keep-set is
+    keep_top(update_magnitude(delta), K). Each square of a bf16 value is exact in float64; the
+    sum is rounded step by step in channel order."""
+    d = np.asarray(delta, dtype=np.float64)
+    acc = np.zeros(d.shape[:2], dtype=np.float64)
+    for c in range(d.shape[2]):
+        acc = acc + d[:, :, c] * d[:, :, c]
+    return acc
+
+
 # ---------------------------------------------------------------------------------------------
 # The whole block, for the smoke check and the CPU baseline
 # ---------------------------------------------------------------------------------------------

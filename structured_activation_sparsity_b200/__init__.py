@@ -18,6 +18,7 @@ _LIB_NAMES = {
     "sparsesam_device_status", "sparsesam_launch_count", "sparsesam_pattern", "sparsesam_perm",
     "sparsesam_rcmlp", "sparsesam_rcmlp_noalloc", "sparsesam_rcmlp_workspace", "sparsesam_score",
     "sparsesam_score_perm", "sparsesam_block", "sparsesam_block_workspace",
+    "sparsesam_random_perm", "sparsesam_keep_by_update",
     "sparsesam_trace_start", "sparsesam_trace_stop", "strerror",
 }
 

@@ -55,6 +55,8 @@ def _load():
         "sparsesam_score": (ctypes.c_int, [cfgp, P, P, VP]),
         "sparsesam_perm": (ctypes.c_int, [cfgp, P, P, P, P, VP]),
         "sparsesam_score_perm": (ctypes.c_int, [cfgp, P, P, P, P, P, VP]),
+        "sparsesam_random_perm": (ctypes.c_int, [cfgp, ctypes.c_uint64, P, P, P, P, VP]),
+        "sparsesam_keep_by_update": (ctypes.c_int, [cfgp, P, I32, I32, P, P, VP]),
         "sparsesam_block_workspace": (SZ, [cfgp, I32, I32]),
         "sparsesam_block": (ctypes.c_int, [cfgp, P, P, P, P, P, I32, I32, P, P, P, P, P, P, P, P,
                                            P, P, SZ, VP]),
@@ -154,6 +156,20 @@ def sparsesam_score_perm(cfg, lum, score, perm, inv, keep, stream=None):
     return _check("sparsesam_score_perm",
                   lib.sparsesam_score_perm(ctypes.byref(cfg), _ptr(lum), _ptr(score), _ptr(perm),
                                            _ptr(inv), _ptr(keep), _stream(stream)))
+
+
+def sparsesam_random_perm(cfg, seed, score, perm, inv, keep, stream=None):
+    """S2 over seeded random scores (the random-permutation ablation)."""
+    return _check("sparsesam_random_perm",
+                  lib.sparsesam_random_perm(ctypes.byref(cfg), int(seed), _ptr(score), _ptr(perm),
+                                            _ptr(inv), _ptr(keep), _stream(stream)))
+
+
+def sparsesam_keep_by_update(cfg, delta, C, K, mag, keep, stream=None):
+    """The keep list of the K tokens with the largest update magnitude sum_c delta[b,t,c]^2."""
+    return _check("sparsesam_keep_by_update",
+                  lib.sparsesam_keep_by_update(ctypes.byref(cfg), _ptr(delta), int(C), int(K),
+                                               _ptr(mag), _ptr(keep), _stream(stream)))
 
 
 def sparsesam_block_workspace(cfg, C, hidden) -> int:

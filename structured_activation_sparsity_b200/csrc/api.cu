@@ -186,13 +186,45 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 
 int cuda_err(cudaError_t e) { return e == cudaSuccess ? SS_OK : SS_ECUDA; }
 
-size_t attn_ws_bytes(const Geo& g, int heads, int dh) {
-  return 3 * align256((size_t)g.U * heads * g.N * dh * 2);
-}
-
-// The GEMM work split is planned for the B200's 148 SMs, so the workspace size does not depend on
-// the device a call runs on; the launch uses min(units, the device's SMs) persistent CTAs.
+// The GEMM and attention work splits are planned for the B200's 148 SMs, so workspace sizes do
+// not depend on the device a call runs on; launches use min(units, the device's SMs) CTAs.
 constexpr int kPlanSMs = 148;
+
+// The attention workspace: the gathered Q, K and V ([U*heads, N, dh] bf16 each); for the pair
+// kernel its permuted output Op (the same layout), and, when it splits pairs into pieces, its
+// per-piece partials and per-pair merge counters.
+struct AttnLayout {
+  AttnParams ap;     // geometry and plan fields filled; perm, out, sms by the launch
+  AttnPlan plan;
+  size_t one;        // bytes of one gathered array (256-byte multiple)
+  size_t operm, partial, counters, total;   // byte offsets, total size
+};
+
+int attn_layout(const ss_cfg* c, const Geo& g, AttnLayout* L) {
+  ss_pattern p;
+  int rc = pattern_of(c, g, &p);
+  if (rc) return rc;
+  AttnParams& ap = L->ap;
+  ap = AttnParams{};
+  ap.U = g.U;
+  ap.N = g.N;
+  ap.heads = c->heads;
+  ap.L = p.L;
+  ap.b = p.b;
+  ap.nb = p.nb;
+  ap.W = p.W;
+  ap.g = p.g;
+  ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c->head_dim));
+  L->plan = attn_plan(ap, c->head_dim, kPlanSMs);
+  ap.whole = L->plan.whole;
+  ap.tail_split = L->plan.tail_split;
+  L->one = align256((size_t)g.U * c->heads * g.N * c->head_dim * 2);
+  L->operm = 3 * L->one;
+  L->partial = L->operm + (L->plan.pair_kernel ? L->one : 0);
+  L->counters = L->partial + align256(L->plan.partial_bytes);
+  L->total = L->counters + align256(L->plan.counter_bytes);
+  return SS_OK;
+}
 
 struct MlpPlan {
   GemmPlan fc1, fc2;
@@ -331,10 +363,52 @@ int sparsesam_score_perm(const ss_cfg* cfg, const float* lum, double* score, int
   return rank_path(cfg, lum, nullptr, score, perm, inv, keep, stream);
 }
 
+int sparsesam_random_perm(const ss_cfg* cfg, uint64_t seed, double* score, int32_t* perm,
+                          int32_t* inv, int32_t* keep, void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  if (!score || (!perm && !inv && !keep)) return SS_EINVAL;
+  if (perm || inv) {
+    ss_pattern p;
+    if ((rc = pattern_of(cfg, g, &p))) return rc;
+  }
+  if (g.N > kMaxRankTokens || g.T > kMaxRankTokens || g.U > 65535) return SS_EUNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = cuda_err(traced("random_score", st, [&] {
+    return launch_random_score(score, (long long)g.B * g.T, seed, st);
+  }));
+  if (rc) return rc;
+  return rank_path(cfg, nullptr, score, nullptr, perm, inv, keep, stream);
+}
+
+int sparsesam_keep_by_update(const ss_cfg* cfg, const uint16_t* delta, int32_t C, int32_t K,
+                             double* mag, int32_t* keep, void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  if (!delta || !mag || !keep || C < 1 || K < 0 || K > g.T) return SS_EINVAL;
+  if (C % 8 != 0) return SS_EUNSUPPORTED;
+  if (!aligned(delta, 16)) return SS_EINVAL;
+  if (g.T > kMaxRankTokens) return SS_EUNSUPPORTED;
+  if (K == 0) return SS_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = cuda_err(traced("update_magnitude", st, [&] {
+    return launch_update_magnitude(delta, mag, (long long)g.B * g.T, C, st);
+  }));
+  if (rc) return rc;
+  return cuda_err(traced("keep_rank", st, [&] {
+    return launch_stripe_rank(mag, nullptr, nullptr, 0, g.B, g.Hg, g.Wg, 0, g.B, g.T, K, nullptr,
+                              nullptr, keep, st);
+  }));
+}
+
 size_t sparsesam_attn_workspace(const ss_cfg* cfg) {
   Geo g;
-  if (geometry(cfg, &g) || cfg->heads < 1 || cfg->head_dim < 1) return 0;
-  return attn_ws_bytes(g, cfg->heads, cfg->head_dim);
+  AttnLayout L;
+  if (geometry(cfg, &g) || cfg->heads < 1 || cfg->head_dim < 1 || attn_layout(cfg, g, &L))
+    return 0;
+  return L.total;
 }
 
 // Argument checks of the attention step (also for the whole-block path); fills the pattern.
@@ -353,39 +427,59 @@ static int attn_check(const ss_cfg* cfg, const Geo& g, const uint16_t* q, const 
   return SS_OK;
 }
 
-// The attention over the gathered Q, K, V in ws (laid out as attn_ws_bytes describes).
-static int attn_launch(const ss_cfg* cfg, const Geo& g, const ss_pattern& p, uint8_t* ws,
+// The Q/K/V gather into ws (laid out as attn_layout describes); it also zeroes the merge counters.
+static int gather_launch(const Geo& g, int heads, int dh, const AttnLayout& L, const uint16_t* q,
+                         const uint16_t* k, const uint16_t* v, const int32_t* perm, uint8_t* ws,
+                         int* status, cudaStream_t st) {
+  return cuda_err(traced("gather_qkv", st, [&] {
+    return launch_gather_qkv(q, k, v, perm, reinterpret_cast<uint16_t*>(ws),
+                             reinterpret_cast<uint16_t*>(ws + L.one),
+                             reinterpret_cast<uint16_t*>(ws + 2 * L.one), g.U, g.N, heads, dh,
+                             L.ap.b, reinterpret_cast<int*>(ws + L.counters),
+                             (int)(L.plan.counter_bytes / sizeof(int)), status, st);
+  }));
+}
+
+// The attention over the gathered Q, K, V in ws (laid out as attn_layout describes).
+static int attn_launch(const ss_cfg* cfg, const Geo& g, const AttnLayout& L, uint8_t* ws,
                        const int32_t* perm, uint16_t* out, int* status, cudaStream_t st) {
   const int heads = cfg->heads, dh = cfg->head_dim;
-  const size_t one = attn_ws_bytes(g, heads, dh) / 3;
   const uint16_t* bufs[3] = {reinterpret_cast<uint16_t*>(ws),
-                             reinterpret_cast<uint16_t*>(ws + one),
-                             reinterpret_cast<uint16_t*>(ws + 2 * one)};
-  CUtensorMap tm[6];
+                             reinterpret_cast<uint16_t*>(ws + L.one),
+                             reinterpret_cast<uint16_t*>(ws + 2 * L.one)};
+  uint16_t* operm = reinterpret_cast<uint16_t*>(ws + L.operm);
+  CUtensorMap tm[7];   // Q, K, V; Q and K tails; Op and its tail (pair kernel)
   const uint64_t mats = (uint64_t)g.U * heads;
-  for (int i = 0; i < 3; ++i) {
+  for (int i = 0; i < 3; ++i)
     if (!encode_bf16(&tm[i], 3, bufs[i], dh, g.N, mats, (uint64_t)dh * 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return SS_ECUDA;
+  for (int i = 0; i < 2; ++i)   // columns 64..79 of Q and K at head dim 80
     if (dh == 80 && !encode_bf16(&tm[3 + i], 3, bufs[i], dh, g.N, mats, (uint64_t)dh * 2, 16, 128,
                                  CU_TENSOR_MAP_SWIZZLE_32B))
       return SS_ECUDA;
+  if (L.plan.pair_kernel) {
+    if (!encode_bf16(&tm[5], 3, operm, dh, g.N, mats, (uint64_t)dh * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return SS_ECUDA;
+    if (dh == 80 && !encode_bf16(&tm[6], 3, operm, dh, g.N, mats, (uint64_t)dh * 2, 16, 128,
+                                 CU_TENSOR_MAP_SWIZZLE_32B))
+      return SS_ECUDA;
   }
-  AttnParams ap;
+  AttnParams ap = L.ap;
   ap.perm = perm;
   ap.out = out;
-  ap.U = g.U;
-  ap.N = g.N;
-  ap.heads = heads;
-  ap.L = p.L;
-  ap.b = p.b;
-  ap.nb = p.nb;
-  ap.W = p.W;
-  ap.g = p.g;
-  ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dh));
   ap.sms = sm_count();
-  return cuda_err(traced("attn", st, [&] {
-    return launch_attn(&tm[0], &tm[1], &tm[2], &tm[3], &tm[4], &tm[5], ap, dh, status, st);
+  ap.partial = reinterpret_cast<float*>(ws + L.partial);
+  ap.counters = reinterpret_cast<int*>(ws + L.counters);
+  ap.operm = operm;
+  int rc = cuda_err(traced("attn", st, [&] {
+    return launch_attn(&tm[0], &tm[1], &tm[2], &tm[3], &tm[4], &tm[5], &tm[6], ap, dh, status,
+                       st);
+  }));
+  if (rc || !L.plan.pair_kernel) return rc;
+  return cuda_err(traced("unpermute_out", st, [&] {
+    return launch_unpermute_out(operm, perm, out, g.U, g.N, heads, dh, ap.b, status, st);
   }));
 }
 
@@ -396,22 +490,16 @@ int sparsesam_attn(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k, cons
   if (rc) return rc;
   ss_pattern p;
   if ((rc = attn_check(cfg, g, q, k, v, perm, out, &p))) return rc;
-  const int heads = cfg->heads, dh = cfg->head_dim;
-  const size_t need = attn_ws_bytes(g, heads, dh);
-  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SS_EWORKSPACE;
+  AttnLayout L;
+  if ((rc = attn_layout(cfg, g, &L))) return rc;
+  if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return SS_EWORKSPACE;
   int* status = status_word();
   if (!status) return SS_ECUDA;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  const size_t one = need / 3;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  rc = cuda_err(traced("gather_qkv", st, [&] {
-    return launch_gather_qkv(q, k, v, perm, reinterpret_cast<uint16_t*>(wsb),
-                             reinterpret_cast<uint16_t*>(wsb + one),
-                             reinterpret_cast<uint16_t*>(wsb + 2 * one), g.U, g.N, heads, dh, p.b,
-                             status, st);
-  }));
-  if (rc) return rc;
-  return attn_launch(cfg, g, p, wsb, perm, out, status, st);
+  if ((rc = gather_launch(g, cfg->heads, cfg->head_dim, L, q, k, v, perm, wsb, status, st)))
+    return rc;
+  return attn_launch(cfg, g, L, wsb, perm, out, status, st);
 }
 
 int sparsesam_attn_gathered(const ss_cfg* cfg, const void* ws, size_t ws_bytes,
@@ -424,11 +512,12 @@ int sparsesam_attn_gathered(const ss_cfg* cfg, const void* ws, size_t ws_bytes,
   if ((rc = attn_check(cfg, g, static_cast<const uint16_t*>(ws), static_cast<const uint16_t*>(ws),
                        static_cast<const uint16_t*>(ws), perm, out, &p)))
     return rc == SS_EINVAL && !ws ? SS_EWORKSPACE : rc;
-  const size_t need = attn_ws_bytes(g, cfg->heads, cfg->head_dim);
-  if (!aligned(ws, 256) || ws_bytes < need) return SS_EWORKSPACE;
+  AttnLayout L;
+  if ((rc = attn_layout(cfg, g, &L))) return rc;
+  if (!aligned(ws, 256) || ws_bytes < L.total) return SS_EWORKSPACE;
   int* status = status_word();
   if (!status) return SS_ECUDA;
-  return attn_launch(cfg, g, p, static_cast<uint8_t*>(const_cast<void*>(ws)), perm, out, status,
+  return attn_launch(cfg, g, L, static_cast<uint8_t*>(const_cast<void*>(ws)), perm, out, status,
                      static_cast<cudaStream_t>(stream));
 }
 
@@ -525,9 +614,11 @@ int sparsesam_rcmlp(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden, c
 
 size_t sparsesam_block_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden) {
   Geo g;
-  if (geometry(cfg, &g) || cfg->heads < 1 || cfg->head_dim < 1 || C < 1 || hidden < 1) return 0;
-  return align256(attn_ws_bytes(g, cfg->heads, cfg->head_dim)) +
-         rcmlp_ws_bytes(g, keep_count(cfg->density, g.T), C, hidden);
+  AttnLayout L;
+  if (geometry(cfg, &g) || cfg->heads < 1 || cfg->head_dim < 1 || C < 1 || hidden < 1 ||
+      attn_layout(cfg, g, &L))
+    return 0;
+  return align256(L.total) + rcmlp_ws_bytes(g, keep_count(cfg->density, g.T), C, hidden);
 }
 
 int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, const uint16_t* k,
@@ -545,7 +636,9 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
   if ((rc = rcmlp_check(g, x, C, hidden, w1, b1, w2, b2, keep, K))) return rc;
   if (g.N > kMaxRankTokens || g.T > kMaxRankTokens) return SS_EUNSUPPORTED;
   const int heads = cfg->heads, dh = cfg->head_dim;
-  const size_t attn_part = align256(attn_ws_bytes(g, heads, dh));
+  AttnLayout L;
+  if ((rc = attn_layout(cfg, g, &L))) return rc;
+  const size_t attn_part = align256(L.total);
   if (!ws || !aligned(ws, 256) || ws_bytes < attn_part + rcmlp_ws_bytes(g, K, C, hidden))
     return SS_EWORKSPACE;
   // out may not overlap x: S4's row gather starts before S3 has finished writing out.
@@ -560,7 +653,6 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
   if (!status) return SS_ECUDA;
   uint8_t* wsa = static_cast<uint8_t*>(ws);
   uint8_t* wsm = wsa + attn_part;
-  const size_t one = attn_ws_bytes(g, heads, dh) / 3;
   const MlpPlan plan = mlp_plan(g, K, C, hidden);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // S1 + S2 in one pass, the attention's gather and the attention, the MLP's gather (which also
@@ -568,14 +660,8 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
   // the two gathers into the ranking launch was measured slower: its 128 ranking CTAs copy the
   // rows less efficiently than the gathers spread over every SM.)
   if ((rc = rank_path(cfg, lum, nullptr, score, perm, inv, keep, stream))) return rc;
-  rc = cuda_err(traced("gather_qkv", st, [&] {
-    return launch_gather_qkv(q, k, v, perm, reinterpret_cast<uint16_t*>(wsa),
-                             reinterpret_cast<uint16_t*>(wsa + one),
-                             reinterpret_cast<uint16_t*>(wsa + 2 * one), g.U, g.N, heads, dh, p.b,
-                             status, st);
-  }));
-  if (rc) return rc;
-  if ((rc = attn_launch(cfg, g, p, wsa, perm, out, status, st))) return rc;
+  if ((rc = gather_launch(g, heads, dh, L, q, k, v, perm, wsa, status, st))) return rc;
+  if ((rc = attn_launch(cfg, g, L, wsa, perm, out, status, st))) return rc;
   // The row gather's inputs are final: keep came from the ranking launch, which the Q/K/V gather
   // and the attention waited for before this launch can start, and x is not written before fc2.
   // Its copy runs in the attention's tail; its dependency wait comes last (late_wait).

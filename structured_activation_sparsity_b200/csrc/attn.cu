@@ -40,9 +40,13 @@ __global__ void __launch_bounds__(256, MINB) k_gather_qkv(const uint16_t* __rest
                                                        uint16_t* __restrict__ qp,
                                                        uint16_t* __restrict__ kp,
                                                        uint16_t* __restrict__ vp, int N,
-                                                       int heads, int b, int L, int* status) {
+                                                       int heads, int b, int L,
+                                                       int* __restrict__ zero, int nzero,
+                                                       int* status) {
   griddep_wait();
   griddep_launch();
+  if (blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
   const int u = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qpos = blockIdx.x * 8 + warp;
@@ -84,13 +88,13 @@ __global__ void __launch_bounds__(256, MINB) k_gather_qkv(const uint16_t* __rest
 
 cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                               const int32_t* perm, uint16_t* qp, uint16_t* kp, uint16_t* vp,
-                              int U, int N, int heads, int dh, int b, int* status,
-                              cudaStream_t st) {
+                              int U, int N, int heads, int dh, int b, int* zero, int nzero,
+                              int* status, cudaStream_t st) {
   dim3 grid((N + 7) / 8, U);
   const int L = N / kStripes;
   auto go = [&](auto kernel) {
     return launch_pdl(kernel, grid, dim3(256), 0, st, q, k, v, perm, qp, kp, vp, N, heads, b, L,
-                      status);
+                      zero, nzero, status);
   };
   const int per_tok = heads * (dh / 8);
   if (dh != 64 && dh != 80) return cudaErrorInvalidValue;
@@ -112,7 +116,6 @@ constexpr int kAttnThreads = 384;     // 12 warps = 3 warpgroups
 constexpr float kLazyRescale = 8.f;   // log2 headroom before O and l are rescaled
 constexpr int kPairTiles = 4;         // items of at most this many key tiles: k_attn_pairs
 constexpr bool kPairInterleave = true;   // k_attn_pairs ring order A_0, B_0, A_1, B_1, ...
-constexpr int kPolyPairs = 0;         // of every 16 exp pairs on full tiles, those on the FMA pipe
 // Register split (launch: 384 threads x 168): producer warpgroup 56, softmax warpgroups 224.
 constexpr uint32_t kRegsProducer = 56, kRegsSoftmax = 224;
 static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= 384 * 168, "register split too large");
@@ -123,30 +126,6 @@ struct AttnTmem {
   static constexpr uint32_t kS = 0, kSStride = 128;
   static constexpr uint32_t kO = 256, kOStride = DH <= 64 ? 64 : 128;
   static constexpr uint32_t kP = kSeparateP ? 384 : 0, kPStride = kSeparateP ? 64 : 128;
-};
-
-template <int DH>
-struct AttnSmem {
-  static constexpr int kTail = DH - 64;                // 0 or 16 columns past the 128B atom
-  static constexpr int kMain = kBM * 128;              // 128 rows x 128 B
-  static constexpr int kTailBytes = kTail ? kBM * kTail * 2 : 0;
-  static constexpr int kTileBytes = ((kMain + kTailBytes + 1023) / 1024) * 1024;
-  static constexpr int kStages = DH == 64 ? 5 : 4;     // depth of the K/V ring
-  static constexpr int kQ = 0;                         // two Q buffers (consecutive items)
-  static constexpr int kK = 2 * kTileBytes;
-  static constexpr int kV = kK + kStages * kTileBytes;
-  // group 0's float m[2 items][128], l[2 items][128]: one item's rows stay intact while the
-  // next item's are written
-  static constexpr int kML = kV + kStages * kTileBytes;
-  // Output staging: 128 rows of DH bf16, padded by 16 bytes so that the 32 rows a warp writes
-  // at once spread over all banks; then the rows' destination tokens.
-  static constexpr int kStageStride = DH * 2 + 16;
-  static constexpr int kStage = kML + 4 * kBM * 4;
-  static constexpr int kDst = kStage + kBM * kStageStride;
-  static constexpr int kBar = kDst + kBM * 4;
-  static constexpr int kBytes = kBar + 512;
-  static constexpr int kAlloc = kBytes + 1024;         // slack to align the base to 1024
-  static_assert(kAlloc <= 227 * 1024, "attention shared memory above the per-CTA limit");
 };
 
 // The key tiles of one query tile, visited from an item-dependent starting point: CTAs that share
@@ -199,29 +178,6 @@ __device__ __forceinline__ uint32_t run_bits(int lo, int hi, int base) {
   return h > l ? (mh & ~ml) : 0u;
 }
 
-// 2^x on the FMA pipe for x in [-125, 8] (Cody-Waite style reduction 2^x = 2^n 2^f, n = round(x),
-// f in [-1/2, 1/2]; 2^f by the cubic that interpolates it at the four Chebyshev nodes of the
-// interval, coefficients from csrc/exp2_poly.py, relative error < 1e-4). Operates on a pair.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
-  constexpr float kMagic = 12582912.f;   // 1.5 * 2^23: adding it rounds to an integer in the low bits
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  const uint64_t x2 = f2_pack(x0, x1);
-  const uint64_t t2 = f2_add(x2, f2_pack(kMagic, kMagic));
-  const uint64_t n2 = f2_add(t2, f2_pack(-kMagic, -kMagic));
-  const uint64_t fr = f2_fma(n2, f2_pack(-1.f, -1.f), x2);
-  uint64_t q = f2_fma(f2_pack(0.05583828315138817f, 0.05583828315138817f), fr,
-                      f2_pack(0.2426394820213318f, 0.2426394820213318f));
-  q = f2_fma(q, fr, f2_pack(0.6931367516517639f, 0.6931367516517639f));
-  q = f2_fma(q, fr, f2_pack(0.9999245405197144f, 0.9999245405197144f));
-  float q0, q1, t0, t1;
-  f2_unpack(q, q0, q1);
-  f2_unpack(t2, t0, t1);
-  // add n to the exponent field: the low mantissa bits of t hold n (two's complement)
-  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
-}
-
 // Destination token of an output row: perm's entry if it lies in the unit, else -1 (the row is
 // not stored) with SS_EINDEX recorded.
 __device__ __forceinline__ int dst_token(int perm_t, int N, int* status) {
@@ -246,84 +202,180 @@ __device__ __forceinline__ Item item_of(int it, int nq, const AttnParams& P) {
   return I;
 }
 
-// Persistent: one CTA per SM walks the items it, it + gridDim.x, ... . The key tiles of an item
-// are split between two softmax warpgroups (tile n goes to group n % 2), so the MMA pipe
-// alternates between them: while one group turns its S tile into probabilities, the tensor core
-// runs the other group's P*V and the next Q*K^T. Each group keeps its own running max m, sum l
-// and accumulator O (in TMEM); at the end of an item the two partial results of every row are
-// merged and scattered. Q is double-buffered, so the next item's Q*K^T starts while this item's
-// last tiles and its epilogue are still running.
-//   warp 0        TMA producer (Q per item; K and V tiles into a ring of stages)
-//   warp 1        TMEM allocator and Q*K^T issuer
-//   warp 2        P*V issuer
-//   warp 3        idle (completes the producer warpgroup for the register split)
-//   warps 4-7     softmax group 0 (one thread per query row = TMEM lane)
-//   warps 8-11    softmax group 1
-// TMEM columns (AttnTmem): S0 [0,128), S1 [128,256); dh 64: O0 [256,320), O1 [320,384),
-// P0 [384,448), P1 [448,512); dh 80: O0 [256,336), O1 [384,464) and P_w over the first 64
-// columns of S_w. P is bf16, two per column: the A operand of P*V. Keeping P apart from S (when
-// it fits) lets Q*K^T of tile n+2 start while P*V of tile n still reads P.
-// Barrier phases count uses across items: every role walks the same items and tiles in order.
+// ---------------------------------------------------------------------------------------------
+// Pair kernel: two query tiles that share their key tiles
+// ---------------------------------------------------------------------------------------------
+// A pair is the query tiles 2k and 2k+1 (rows [256k, 256k + 256)) of one (unit, head). With
+// b = 64 (every 64 x 64-token global block) those 256 rows are one offset block, so both tiles
+// keep exactly the same key tiles; otherwise each row masks the tiles of the pair's union list
+// that it does not keep. Softmax group A owns tile 2k and group B tile 2k+1 for the whole pair:
+// each K/V tile is loaded once and feeds both groups' Q*K^T and P*V, and no partial row is ever
+// merged between the groups.
+// The groups take turns on the exponentials (SFU): group B starts tile n when group A is half way
+// through it, and A starts tile n+1 when B is half way through tile n. Everything else of a
+// group's tile (its S load, row max and exponent arguments, its P*V, the next Q*K^T into S) then
+// runs while the other group exponentiates, so the SFU, the one unit both groups need most, is not
+// left idle by both groups' gaps at once.
+// That also lets the groups share one S buffer in TMEM: the Q*K^T of one group's tile goes into it
+// as soon as the other group has read its own S out.
+// Work is pieces: the pairs of the full rounds of CTAs are whole pieces; the pairs of a partial
+// last round are cut into `tail_split` key ranges each, so that round spreads over every CTA, and
+// each group of such a piece writes (O, m, l) to a global slot; the pair's last piece to finish
+// merges them.
+//   warp 0        TMA producer: Q_A, Q_B per piece; K and V tiles into a ring of stages
+//   warp 1        TMEM allocator and Q*K^T issuer (both groups)
+//   warp 2        P*V issuer (both groups)
+//   warp 3        output storer: each group's normalised rows, staged as a tile in shared
+//                 memory, go by one TMA store to the permuted output Op (block-major, like Q)
+//   warps 4-7     softmax group A (one thread per query row = TMEM lane), and its epilogue
+//   warps 8-11    softmax group B, and its epilogue
+// TMEM columns: S [0,128) (shared), P_A [128,192), P_B [192,256) (64 columns of bf16 pairs each),
+// O_A from 256, O_B from 320 (head dim 64) or 352 (head dim 80).
+// V stays in its gathered [key, dh] layout as the MN-major B operand of P*V: at head dim 80 its
+// tile is two 128-byte-swizzled 64-column atoms, the second loaded from column 64 with the
+// columns past 80 filled with zeros, so one N = 80 MMA per 16 keys covers the whole head.
+constexpr int kMaxSplit = 4;
+
+template <int DH>
+struct PairTmem {
+  static constexpr uint32_t kS = 0;
+  static constexpr uint32_t kP = 128, kPStride = 64;
+  static constexpr uint32_t kO = 256, kOStride = DH <= 64 ? 64 : 96;
+  static_assert(kO + kOStride + DH <= 512, "TMEM columns");
+};
+
+template <int DH>
+struct PairSmem {
+  static constexpr int kTail = DH - 64;                        // 0 or 16 columns
+  static constexpr int kQKMain = kBM * 128;                    // 128 rows x 64 bf16, 128B swizzle
+  static constexpr int kQKTail = kTail ? kBM * kTail * 2 : 0;  // 128 rows x 16 bf16, 32B swizzle
+  static constexpr int kQK = kQKMain + kQKTail;                // one Q or K tile
+  static constexpr int kVAtom = kBN * 128;                     // 128 keys x 64 bf16, 128B swizzle
+  static constexpr int kV = kTail ? 2 * kVAtom : kVAtom;
+  static constexpr int kStageBytes = kQK + kV;
+  static constexpr int kStages = DH == 64 ? 5 : 3;             // depth of the K/V ring
+  static constexpr int kQ = 0;                                 // Q_A, then Q_B
+  static constexpr int kKV = 2 * kQK;
+  // Output staging, used by the groups in turn: one 128-row tile of O in the layout of a Q tile
+  // (128-byte-swizzled 64 columns, then the 32-byte-swizzled tail at head dim 80), the box layout
+  // of the TMA store that writes it.
+  static constexpr int kStage = kKV + kStages * kStageBytes;
+  static constexpr int kBar = kStage + kQK;
+  static constexpr int kBytes = kBar + 512;
+  static constexpr int kAlloc = kBytes + 1024;                 // slack to align the base to 1024
+  static_assert(kQK % 1024 == 0 && kStageBytes % 1024 == 0 && kKV % 1024 == 0,
+                "tiles must stay 1024-byte aligned for the 128-byte swizzle");
+  static_assert(kAlloc <= 227 * 1024, "pair kernel shared memory above the per-CTA limit");
+};
+
+// Piece i: pieces [0, whole) are the whole pairs 0..whole-1; piece whole + v is key range
+// v % tail_split of pair whole + v / tail_split. Pairs are numbered head-major (all pairs of one
+// (unit, head) together), so concurrently running CTAs share K/V in L2.
+struct Piece {
+  int pair, uh, qA, qB, n0, n1;
+  int tail;          // index among the split pieces (their slots), or -1 for a whole pair
+  KeyTiles tiles;
+};
+__host__ __device__ __forceinline__ int pairs_per_head(int N) {
+  return ((N + kBM - 1) / kBM + 1) / 2;
+}
+__device__ __forceinline__ Piece piece_of(int i, int npairs, const AttnParams& P) {
+  Piece c;
+  int j = 0, ns = 1;
+  if (i < P.whole) {
+    c.pair = i;
+    c.tail = -1;
+  } else {
+    c.tail = i - P.whole;
+    c.pair = P.whole + c.tail / P.tail_split;
+    j = c.tail - (c.pair - P.whole) * P.tail_split;
+    ns = P.tail_split;
+  }
+  c.uh = c.pair / npairs;
+  const int pq = c.pair - c.uh * npairs;
+  c.qA = pq * 2 * kBM;
+  c.qB = c.qA + kBM;
+  c.tiles = key_tiles(c.qA, min(c.qA + 2 * kBM, P.N) - 1, pq, c.uh, P);
+  const int nt = c.tiles.count();
+  c.n0 = j * nt / ns;
+  c.n1 = (j + 1) * nt / ns;
+  return c;
+}
+// Every row of the pair keeps every key of the tile: the pair lies in one offset block
+// (4b % 256 == 0) and the tile is whole.
+__device__ __forceinline__ bool pair_tile_full(int c0, const AttnParams& P) {
+  return (P.b * kStripes) % (2 * kBM) == 0 && c0 + kBN <= P.N;
+}
+
+// If the CTA gave up a wait, a bounded pause lets its copies and MMAs still in flight land before
+// its shared memory and TMEM are released.
+__device__ __forceinline__ void abort_drain(volatile int* abort) {
+  if (*abort) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 50000ull) {
+    }
+  }
+}
+
+// Row `row` of O (TMEM, DH fp32 columns at t_o) into registers: every 16-column load issued
+// before the one wait (a TMEM load takes a few hundred cycles; one after another they add up).
+template <int DH>
+__device__ __forceinline__ void load_o_row(uint32_t t_o, uint32_t (&o)[DH]) {
+#pragma unroll
+  for (int cc = 0; cc < DH / 16; ++cc)
+    tmem_ld16_nowait(t_o + cc * 16, *reinterpret_cast<uint32_t(*)[16]>(o + 16 * cc));
+  tmem_ld_wait();
+}
 template <int DH>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    k_attn(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tq_tail,
-           const __grid_constant__ CUtensorMap tk_tail, const __grid_constant__ CUtensorMap tv_tail,
-           const AttnParams P, int* status) {
-  using S = AttnSmem<DH>;
-  using T = AttnTmem<DH>;
+    k_attn_pair(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tq_tail,
+                const __grid_constant__ CUtensorMap tk_tail, const __grid_constant__ CUtensorMap to,
+                const __grid_constant__ CUtensorMap to_tail, const AttnParams P, int* status) {
+  using S = PairSmem<DH>;
+  using T = PairTmem<DH>;
   constexpr int NS = S::kStages;
-  constexpr bool kSplitHandoff = T::kSeparateP;   // P handed to P*V in two halves
   constexpr bool kHasTail = S::kTail > 0;
-  // Epilogue: dh 80 lets group 1 merge and emit each item while group 0 moves on to the next
-  // (measured faster there: ViT-H 284 -> 273 us); dh 64 keeps both groups on the merge (the
-  // one-group form measured slower: ViT-B 52.8 -> 55.2 us).
-  constexpr bool kOneGroupEpi = DH == 80;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  float* s_m = reinterpret_cast<float*>(smem + S::kML);   // [2][128] group 0's, by item parity
-  float* s_l = s_m + 2 * kBM;                              // [2][128]
-  int* s_dst = reinterpret_cast<int*>(smem + S::kDst);     // [128] destination token or -1
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
-  uint64_t* q_full = bars + 0;                 // [2] Q buffer landed
-  uint64_t* q_empty = q_full + 2;              // [2] Q*K^T of the buffer's item done
-  uint64_t* kv_full = q_empty + 2;             // [NS] K and V of a stage landed
-  uint64_t* kv_empty = kv_full + NS;           // [NS] P*V of the stage's tile done (K, V free)
-  uint64_t* s_full = kv_empty + NS;            // [2] S_w computed
-  uint64_t* s_free = s_full + 2;               // [2] S_w read into registers by its group
-  uint64_t* p_full = s_free + 2;               // [2][2] half h of P_w written (O_w rescaled first)
-  uint64_t* o_done = p_full + 4;               // an item's last P*V done
-  // [2] by item parity: group 0's m, l of the item written. Two, so that group 0 (which moves on
-  // to the next item at once) cannot complete a second phase before group 1 has waited the first.
-  uint64_t* ml_ready = o_done + 1;
-  uint64_t* o_free = ml_ready + 2;             // O0, O1 of the item read (next item may reuse them)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 1);
+  uint64_t* q_full = bars + 0;               // [2] Q_g of the piece landed
+  uint64_t* q_empty = q_full + 2;            // [2] the piece's Q*K^T of group g done
+  uint64_t* kv_full = q_empty + 2;           // [NS] K and V of a stage landed
+  uint64_t* kv_empty = kv_full + NS;         // [NS] both groups' P*V of the stage's tile done
+  uint64_t* s_full = kv_empty + NS;          // [2] group g's S computed
+  uint64_t* s_free = s_full + 2;             // S read into registers by the group it was for
+  uint64_t* p_full = s_free + 2;             // [2][2] half h of P_g written (O_g rescaled first)
+  uint64_t* pv_done = p_full + 4;            // [2] P_g * V of a tile done
+  uint64_t* grp_bar = pv_done + 2;           // [2] rendezvous of group g's 128 threads
+  uint64_t* stage_free = grp_bar + 2;        // the staging tile read by its TMA store
+  uint64_t* staged = stage_free + 1;         // a group's rows are in the staging tile
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(staged + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);   // [2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nq = (P.N + kBM - 1) / kBM;
-  const int n_items = nq * P.U * P.heads;
+  const int npairs = pairs_per_head(P.N);
+  const int n_pieces = P.whole + (npairs * P.U * P.heads - P.whole) * P.tail_split;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(q_full + i, 1);
-      mbar_init(q_empty + i, 1);
-      mbar_init(s_full + i, 1);
-      mbar_init(s_free + i, 128);
-      mbar_init(p_full + 2 * i, 128);
-      mbar_init(p_full + 2 * i + 1, 128);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(q_full + g, 1);
+      mbar_init(q_empty + g, 1);
+      mbar_init(s_full + g, 1);
+      if (g == 0) mbar_init(s_free, 128);
+      mbar_init(p_full + 2 * g, 128);
+      mbar_init(p_full + 2 * g + 1, 128);
+      mbar_init(pv_done + g, 1);
+      mbar_init(grp_bar + g, 128);
     }
     for (int i = 0; i < NS; ++i) {
       mbar_init(kv_full + i, 1);
       mbar_init(kv_empty + i, 1);
     }
-    mbar_init(o_done, 1);
-    if constexpr (kOneGroupEpi) {
-      mbar_init(ml_ready, 128);
-      mbar_init(ml_ready + 1, 128);
-      mbar_init(o_free, 128);
-    }
+    mbar_init(stage_free, 1);
+    mbar_init(staged, 128);
     *abort = 0;
     fence_barrier_init();
   }
@@ -332,12 +384,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   cta_sync_converged();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  griddep_wait();   // Q, K, V and perm come from the work before this launch
+  griddep_wait();   // Q, K, V, perm and the merge counters come from the work before this launch
   griddep_launch();
 
-  // An mbarrier wait whose result gates the next instruction costs ~150 cycles even when the
-  // phase has already completed, so the two MMA streams get their own issuing threads: one for
-  // Q*K^T, one for P*V. Their data dependencies all go through the barriers above.
   if (warp < 4) {
     setmaxnreg_dec<kRegsProducer>();
     if (warp == 0 && lane == 0) {
@@ -346,28 +395,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
       bool ok = true;
-      int gn = 0;   // tiles loaded so far (all items)
-      for (int it = blockIdx.x, li = 0; ok && it < n_items; it += gridDim.x, ++li) {
-        const Item I = item_of(it, nq, P);
-        const int qb = li & 1;
-        if (li >= 2 && !(ok = mbar_wait(q_empty + qb, ((li >> 1) - 1) & 1, abort, status))) break;
-        uint8_t* qbuf = smem + S::kQ + qb * S::kTileBytes;
-        mbar_expect_tx(q_full + qb, S::kMain + S::kTailBytes);
-        tma_load_3d(qbuf, &tq, q_full + qb, 0, I.q0, I.uh);
-        if (kHasTail) tma_load_3d(qbuf + S::kMain, &tq_tail, q_full + qb, 64, I.q0, I.uh);
-        const int nt = I.tiles.count();
-        for (int n = 0; n < nt; ++n, ++gn) {
+      int gn = 0;   // tiles loaded so far (all pieces)
+      for (int i = blockIdx.x, li = 0; ok && i < n_pieces; i += gridDim.x, ++li) {
+        const Piece c = piece_of(i, npairs, P);
+        for (int g = 0; g < 2; ++g) {
+          if (li > 0 && !(ok = mbar_wait(q_empty + g, (li - 1) & 1, abort, status))) break;
+          // A pair whose second tile lies past N loads tile A's rows again (never stored).
+          const int q0 = (g == 1 && c.qB < P.N) ? c.qB : c.qA;
+          uint8_t* qb = smem + S::kQ + g * S::kQK;
+          mbar_expect_tx(q_full + g, S::kQK);
+          tma_load_3d(qb, &tq, q_full + g, 0, q0, c.uh);
+          if (kHasTail) tma_load_3d(qb + S::kQKMain, &tq_tail, q_full + g, 64, q0, c.uh);
+        }
+        for (int n = c.n0; ok && n < c.n1; ++n, ++gn) {
           const int st = gn % NS;
-          const int c0 = I.tiles.tile(n) * kBN;
           if (gn >= NS && !(ok = mbar_wait(kv_empty + st, ((gn / NS) - 1) & 1, abort, status)))
             break;
-          uint8_t* kb = smem + S::kK + st * S::kTileBytes;
-          uint8_t* vb = smem + S::kV + st * S::kTileBytes;
-          mbar_expect_tx(kv_full + st, 2 * (S::kMain + S::kTailBytes));
-          tma_load_3d(kb, &tk, kv_full + st, 0, c0, I.uh);
-          if (kHasTail) tma_load_3d(kb + S::kMain, &tk_tail, kv_full + st, 64, c0, I.uh);
-          tma_load_3d(vb, &tv, kv_full + st, 0, c0, I.uh);
-          if (kHasTail) tma_load_3d(vb + S::kMain, &tv_tail, kv_full + st, 64, c0, I.uh);
+          const int c0 = c.tiles.tile(n) * kBN;
+          uint8_t* kb = smem + S::kKV + st * S::kStageBytes;
+          uint8_t* vb = kb + S::kQK;
+          mbar_expect_tx(kv_full + st, S::kStageBytes);
+          tma_load_3d(kb, &tk, kv_full + st, 0, c0, c.uh);
+          if (kHasTail) tma_load_3d(kb + S::kQKMain, &tk_tail, kv_full + st, 64, c0, c.uh);
+          tma_load_3d(vb, &tv, kv_full + st, 0, c0, c.uh);
+          // head dim 80: columns 64..127 of V; 80..127 lie outside the tensor and read as zero
+          if (kHasTail) tma_load_3d(vb + S::kVAtom, &tv, kv_full + st, 64, c0, c.uh);
         }
       }
     } else if (warp == 1 && lane == 0) {
@@ -375,127 +427,131 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
       bool ok = true;
       int gn = 0;
-      int uses[2] = {0, 0};     // tiles computed into S_w so far
-      int last[2] = {0, 0};     // global index of the tile that last used S_w
-      for (int it = blockIdx.x, li = 0; ok && it < n_items; it += gridDim.x, ++li) {
-        const Item I = item_of(it, nq, P);
-        const int qb = li & 1;
-        if (!(ok = mbar_wait(q_full + qb, (li >> 1) & 1, abort, status))) break;
-        const uint32_t q_addr = smem_u32(smem + S::kQ + qb * S::kTileBytes);
-        const int nt = I.tiles.count();
-        for (int n = 0; n < nt; ++n, ++gn) {
-          const int st = gn % NS, w = n & 1;
-          if (uses[w] > 0) {
-            // S_w is reusable once its previous tile's S is in its group's registers (P apart
-            // from S), or once that tile's P*V is done (P over S).
-            if constexpr (T::kSeparateP)
-              ok = mbar_wait(s_free + w, (uses[w] - 1) & 1, abort, status);
-            else
-              ok = mbar_wait(kv_empty + last[w] % NS, (last[w] / NS) & 1, abort, status);
-            if (!ok) break;
-          }
+      for (int i = blockIdx.x, li = 0; ok && i < n_pieces; i += gridDim.x, ++li) {
+        const Piece c = piece_of(i, npairs, P);
+        if (!(ok = mbar_wait(q_full + 0, li & 1, abort, status))) break;
+        if (!(ok = mbar_wait(q_full + 1, li & 1, abort, status))) break;
+        for (int n = c.n0; ok && n < c.n1; ++n, ++gn) {
+          const int st = gn % NS;
           if (!(ok = mbar_wait(kv_full + st, (gn / NS) & 1, abort, status))) break;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(smem + S::kK + st * S::kTileBytes);
-          const uint32_t d = tmem + T::kS + w * T::kSStride;
+          const uint32_t k_addr = smem_u32(smem + S::kKV + st * S::kStageBytes);
+          for (int g = 0; g < 2; ++g) {
+            // S is reusable once the group it last held S for has read it (use 2 * gn + g - 1).
+            const int use = 2 * gn + g;
+            if (use > 0 && !(ok = mbar_wait(s_free, (use - 1) & 1, abort, status))) break;
+            tc_fence_after();
+            const uint32_t q_addr = smem_u32(smem + S::kQ + g * S::kQK);
+            const uint32_t d = tmem + T::kS;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_ss(d, smem_desc(q_addr + kk * 32, 16, 1024, kSwizzle128B),
-                         smem_desc(k_addr + kk * 32, 16, 1024, kSwizzle128B), idesc_qk, kk > 0);
-          if (kHasTail)
-            umma_bf16_ss(d, smem_desc(q_addr + S::kMain, 16, 256, kSwizzle32B),
-                         smem_desc(k_addr + S::kMain, 16, 256, kSwizzle32B), idesc_qk, 1);
-          umma_commit(s_full + w);
-          ++uses[w];
-          last[w] = gn;
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_ss(d, smem_desc(q_addr + kk * 32, 16, 1024, kSwizzle128B),
+                           smem_desc(k_addr + kk * 32, 16, 1024, kSwizzle128B), idesc_qk, kk > 0);
+            if (kHasTail)
+              umma_bf16_ss(d, smem_desc(q_addr + S::kQKMain, 16, 256, kSwizzle32B),
+                           smem_desc(k_addr + S::kQKMain, 16, 256, kSwizzle32B), idesc_qk, 1);
+            umma_commit(s_full + g);
+          }
         }
         if (!ok) break;
-        umma_commit(q_empty + qb);   // the Q buffer is free once this item's Q*K^T are done
+        umma_commit(q_empty + 0);   // the Q buffers are free once the piece's Q*K^T are done
+        umma_commit(q_empty + 1);
       }
     } else if (warp == 2 && lane == 0) {
       // ------------------------------ P*V issuer --------------------------------
-      // P_w of tile n exists only after S of tile n, which followed that stage's K/V landing
-      // (observed by the Q*K^T issuer), so V is ready whenever P is.
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, 64, false, true);
-      constexpr uint32_t idesc_pv_tail = idesc_bf16_f32(kBM, 16, false, true);
+      // P_g of a tile exists only after S_g of it, which followed the stage's K/V landing
+      // (observed by the Q*K^T issuer), so V is ready whenever P is. A piece's first P_g * V
+      // overwrites O_g: its group read the previous piece's O_g before handing over this P.
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, DH, false, true);
       bool ok = true;
       int gn = 0;
-      int uses[2] = {0, 0};   // P_w handed over so far (p_full phases)
-      for (int it = blockIdx.x, li = 0; ok && it < n_items; it += gridDim.x, ++li) {
-        const int nt = item_of(it, nq, P).tiles.count();
-        // The item's first P*V into O_w overwrites it: the previous item's epilogue must have
-        // read O0 and O1.
-        if (kOneGroupEpi && li > 0 && !(ok = mbar_wait(o_free, (li - 1) & 1, abort, status)))
-          break;
-        for (int n = 0; n < nt; ++n, ++gn) {
-          const int st = gn % NS, w = n & 1;
-          const uint32_t v_addr = smem_u32(smem + S::kV + st * S::kTileBytes);
-          const uint32_t a = tmem + T::kP + w * T::kPStride;   // P_w
-          const uint32_t d = tmem + T::kO + w * T::kOStride;
-          // The first tile of each group overwrites O_w: released by o_free above, or (two-group
-          // epilogue) by the group itself, which read the previous item's O before handing over
-          // this P.
-          const uint32_t acc = n >= 2;
-          // P arrives in two halves (keys 0-63, 64-127): the first half's MMAs run while the
-          // softmax still computes the second.
+      for (int i = blockIdx.x; ok && i < n_pieces; i += gridDim.x) {
+        const Piece c = piece_of(i, npairs, P);
+        for (int n = c.n0; ok && n < c.n1; ++n, ++gn) {
+          const int st = gn % NS;
+          const uint32_t v_addr = smem_u32(smem + S::kKV + st * S::kStageBytes + S::kQK);
+          for (int g = 0; ok && g < 2; ++g) {
+            const uint32_t a = tmem + T::kP + g * T::kPStride;
+            const uint32_t d = tmem + T::kO + g * T::kOStride;
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            if (kk % (kBN / 32) == 0) {
-              if (!(ok = mbar_wait(p_full + 2 * w + kk / (kBN / 32), uses[w] & 1, abort, status)))
-                break;
-              tc_fence_after();
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+              if (kk % (kBN / 32) == 0) {
+                // P arrives in two halves (keys 0-63, 64-127): the first half's MMAs run while
+                // the softmax still computes the second.
+                if (!(ok = mbar_wait(p_full + 2 * g + kk / (kBN / 32), gn & 1, abort, status)))
+                  break;
+                tc_fence_after();
+              }
+              umma_bf16_ts(d, a + kk * 8,
+                           smem_desc(v_addr + kk * 2048, S::kVAtom, 1024, kSwizzle128B), idesc_pv,
+                           (n > c.n0 || kk > 0) ? 1u : 0u);
             }
-            umma_bf16_ts(d, a + kk * 8, smem_desc(v_addr + kk * 2048, kBN * 128, 1024, kSwizzle128B),
-                         idesc_pv, acc | (kk > 0));
-            if (kHasTail)
-              umma_bf16_ts(d + 64, a + kk * 8,
-                           smem_desc(v_addr + S::kMain + kk * 512, kBN * 32, 256, kSwizzle32B),
-                           idesc_pv_tail, acc | (kk > 0));
+            if (!ok) break;
+            umma_commit(pv_done + g);
           }
           if (!ok) break;
-          ++uses[w];
-          umma_commit(kv_empty + st);   // Q*K^T of this tile finished before its P existed
+          umma_commit(kv_empty + st);
         }
-        if (!ok) break;
-        umma_commit(o_done);   // phase = the item's parity in this CTA's sequence
       }
+    } else if (warp == 3 && lane == 0) {
+      // ------------------------------ output storer -----------------------------
+      // Each whole piece's staged tiles (group A's, then B's: the order the groups stage them)
+      // go by TMA to rows q0 .. q0+127 of matrix u*heads+h of Op; rows past N are not written.
+      bool ok = true;
+      int use = 0;
+      for (int i = blockIdx.x; ok && i < n_pieces; i += gridDim.x) {
+        const Piece c = piece_of(i, npairs, P);
+        if (c.tail >= 0 && P.tail_split > 1) continue;   // split pieces store their own rows
+        for (int g = 0; ok && g < 2; ++g, ++use) {
+          if (!(ok = mbar_wait(staged, use & 1, abort, status))) break;
+          const int q0 = g ? c.qB : c.qA;
+          if (q0 < P.N) {
+            tma_store_3d(&to, smem + S::kStage, 0, q0, c.uh);
+            if (kHasTail) tma_store_3d(&to_tail, smem + S::kStage + S::kQKMain, 64, q0, c.uh);
+            bulk_commit();
+          }
+          bulk_wait_read();          // the staging tile has been read out
+          mbar_arrive(stage_free);   // it may be rewritten
+        }
+      }
+      bulk_wait_all();   // every store has completed before the CTA exits
     }
   } else {
     setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------ softmax groups ----------------------------
-    const int grp = (warp - 4) >> 2;                    // 0 or 1
+    const int grp = (warp - 4) >> 2;                    // 0: tile A of the pair, 1: tile B
     const int row = 32 * (warp & 3) + lane;             // TMEM lane == query row
+    const int tid = threadIdx.x - 128 * (1 + grp);      // 0..127 within the group
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
-    const uint32_t t_s = tmem + T::kS + grp * T::kSStride + lane_off;
+    const uint32_t t_s = tmem + T::kS + lane_off;
     const uint32_t t_p = tmem + T::kP + grp * T::kPStride + lane_off;
     const uint32_t t_o = tmem + T::kO + grp * T::kOStride + lane_off;
     const int b4 = P.b * kStripes;
     const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
+    constexpr int kSlot = (DH + 2) * kBM;               // floats of one group's partial
+    uint32_t bar_phase = 0;
+    auto grp_sync = [&]() -> bool {                     // bounded rendezvous of the group
+      mbar_arrive(grp_bar + grp);
+      const bool r = mbar_wait(grp_bar + grp, bar_phase, abort, status);
+      bar_phase ^= 1;
+      return r;
+    };
     bool ok = true;
-    int gn0 = 0;           // global index of the item's first tile
-    int uses = 0;          // tiles of this group so far (s_full phases)
+    int gn = 0;            // tiles of this group so far (all pieces): the phase count
     bool s_ready = false;  // the next s_full phase was already seen complete (non-blocking test)
-    int g_last = -1;       // global index of this group's previous tile (any item), -1: none
-    for (int it = blockIdx.x, li = 0; it < n_items; it += gridDim.x, ++li) {
-      const Item I = item_of(it, nq, P);
-      const int nt = I.tiles.count();
-      const int qrow = I.q0 + row;
-      // Destination token of the row: loaded now, used in the epilogue (the load's latency
-      // overlaps the item's tiles).
-      const bool store = qrow < P.N;
-      const int u_i = I.uh / P.heads, h_i = I.uh - u_i * P.heads;
-      const int perm_t =
-          store ? __ldg(P.perm + (size_t)u_i * P.N + blockmajor_to_canonical(qrow, P.b, P.L)) : 0;
+    int stage_uses = 0;    // this group's uses of the staging rows (they alternate with the other's)
+    for (int i = blockIdx.x; ok && i < n_pieces; i += gridDim.x) {
+      const Piece c = piece_of(i, npairs, P);
+      const int u_i = c.uh / P.heads, h_i = c.uh - u_i * P.heads;
+      const int qrow = (grp ? c.qB : c.qA) + row;
       const int a_q = min(qrow, P.N - 1) / b4;
       const int s_q = band_start(a_q, P.W, P.nb);
       const int band_lo = s_q * b4, band_hi = (s_q + P.W) * b4, glob_hi = P.g * b4;
       float m_ref = -INFINITY, l_run = 0.f;
-      int j = 0;
-      for (int n = grp; ok && n < nt; n += 2, ++j) {
+      for (int n = c.n0; ok && n < c.n1; ++n, ++gn) {
+        const int j = n - c.n0;
         // Warp-collective wait: either every lane goes on to the .sync.aligned TMEM ops or none.
         if (!__all_sync(0xffffffffu, s_ready))
-          ok = __all_sync(0xffffffffu, mbar_wait(s_full + grp, uses & 1, abort, status));
-        ++uses;
+          ok = __all_sync(0xffffffffu, mbar_wait(s_full + grp, gn & 1, abort, status));
         if (!ok) break;
         tc_fence_after();
         float sv[kBN];
@@ -503,26 +559,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           uint32_t r[128];
           tmem_ld128(t_s, r);
 #pragma unroll
-          for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(r[i]);
+          for (int k = 0; k < kBN; ++k) sv[k] = __uint_as_float(r[k]);
         }
-        // Has P*V of this group's previous tile (in this item or the last) released P_w? Tested
-        // now, used after the row max, so the test's latency is hidden behind the max.
-        // (With the two-group epilogue both groups waited for the previous item's P*V, so only
-        // this item's earlier tiles count.)
-        int gprev = n >= 2 ? gn0 + n - 2 : -1;
-        if constexpr (kOneGroupEpi) {
-          gprev = g_last;
-          g_last = gn0 + n;
-        }
-        bool prev_pv_done = true;
-        if constexpr (T::kSeparateP) {
-          tc_fence_before();
-          mbar_arrive(s_free + grp);   // S_w may now be overwritten by the next Q*K^T into it
-          if (gprev >= 0) prev_pv_done = mbar_test(kv_empty + gprev % NS, (gprev / NS) & 1);
-        }
-        const int c0 = I.tiles.tile(n) * kBN;
-        const bool full = tile_full(c0, P);
-        if (!full) {
+        tc_fence_before();
+        mbar_arrive(s_free);   // S is in registers: the other group's Q*K^T may overwrite it
+        // Has this group's previous P * V released P_g and O_g? Tested now, waited for below.
+        bool prev_pv_done = gn == 0 || mbar_test(pv_done + grp, (gn - 1) & 1);
+        const int c0 = c.tiles.tile(n) * kBN;
+        if (!pair_tile_full(c0, P)) {
           // The row's kept keys in this tile are two runs, [0, e0) and [s1, e1) relative to c0:
           // turned into four 32-bit column masks, so the per-key test has no branch.
           const int e0 = min(glob_hi, P.N) - c0, s1 = band_lo - c0, e1 = min(band_hi, P.N) - c0;
@@ -530,8 +574,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int k = 0; k < 4; ++k) km[k] = run_bits(0, e0, 32 * k) | run_bits(s1, e1, 32 * k);
 #pragma unroll
-          for (int i = 0; i < kBN; ++i)
-            sv[i] = (km[i >> 5] >> (i & 31)) & 1u ? sv[i] : -INFINITY;
+          for (int k = 0; k < kBN; ++k) sv[k] = (km[k >> 5] >> (k & 31)) & 1u ? sv[k] : -INFINITY;
         }
         // Row max: eight independent chains of 3-input max over elements k, k+8, k+16, ...
         float mx[8];
@@ -547,8 +590,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                   fmaxf(mx[6], mx[7])) *
                             P.scale_log2;
         // Lazy rescale: the reference max moves only when the row max passes it by 2^8, so O in
-        // TMEM is rescaled on few tiles. The decision is warp-wide (TMEM ops are warp-collective);
-        // the rescale itself runs after P is written, when the S registers are free.
+        // TMEM is rescaled on few tiles. The decision is warp-wide (TMEM ops are warp-collective).
         const bool grow = x_max > m_ref + kLazyRescale;
         const bool rescale = __any_sync(0xffffffffu, grow);
         float alpha = 1.f;
@@ -559,250 +601,181 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m_ref = m_new;
         }
         const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
-        const uint64_t nref2 = f2_pack(-ref, -ref);
+        // The exponents x = s*scale - ref, in place (two per packed FMA), before this group's SFU
+        // turn, so that the turn holds little besides the exponentials. Masked keys give -inf.
+        {
+          const uint64_t nref2 = f2_pack(-ref, -ref);
+#pragma unroll
+          for (int k = 0; k < kBN; k += 2)
+            f2_unpack(f2_fma(f2_pack(sv[k], sv[k + 1]), scale2, nref2), sv[k], sv[k + 1]);
+        }
+        // P_g and O_g are free once this group's previous P * V is done.
+        if (gn > 0) {
+          if (!__all_sync(0xffffffffu, prev_pv_done)) {
+            ok = __all_sync(0xffffffffu, mbar_wait(pv_done + grp, (gn - 1) & 1, abort, status));
+            if (!ok) break;
+          }
+          tc_fence_after();
+        }
+        // The SFU turn: A exponentiates tile n once B is half way through tile n-1 (B's first P
+        // half is in), B tile n once A is half way through tile n. The two groups' exponentials
+        // overlap by half a tile, so the SFU has two warps' work then, and the gap a group has
+        // between its tiles stays offset from the other group's.
+        if (grp == 1 || gn > 0) {
+          const int other = 1 - grp, t_other = grp ? gn : gn - 1;
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(p_full + 2 * other, t_other & 1, abort, status));
+          if (!ok) break;
+        }
+        // P as bf16 pairs (column i holds keys 2i, 2i+1), 16 columns at a time; each 64-key half
+        // is handed to the P*V issuer as soon as it is in TMEM. 2^x on the SFU in fp32 (as fast
+        // per value as its packed forms, and exact to fp32 input); ex2(-inf) = 0 for masked keys.
         uint64_t sum2a = 0, sum2b = 0;   // two packed partial sums (bit pattern 0 = +0.0f pair)
-        // The group's previous P*V must be done before P_w is rewritten and O_w rescaled (with P
-        // over S it already is: this S was computed after that P*V).
-        if constexpr (T::kSeparateP) {
-          if (gprev >= 0) {
-            if (!__all_sync(0xffffffffu, prev_pv_done)) {
-              ok = __all_sync(0xffffffffu,
-                              mbar_wait(kv_empty + gprev % NS, (gprev / NS) & 1, abort, status));
-              if (!ok) break;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t pw[16];
+#pragma unroll
+          for (int i2 = 0; i2 < 16; ++i2) {
+            const int k = 32 * cc + 2 * i2;
+            const float p0 = ex2_mufu(sv[k]), p1 = ex2_mufu(sv[k + 1]);
+            if (i2 & 1)
+              sum2b = f2_add(sum2b, f2_pack(p0, p1));
+            else
+              sum2a = f2_add(sum2a, f2_pack(p0, p1));
+            pw[i2] = pack_bf16_pos(p0, p1);   // p >= 0: integer-pipe rounding
+          }
+          tmem_st16_async(t_p + 16 * cc, pw);
+          if (cc == 1 && rescale && j > 0) {
+            // O_g holds the piece's earlier tiles (their P*V completed, above); it is rescaled
+            // before this tile's first P*V accumulates into it.
+#pragma unroll 1
+            for (int oc = 0; oc < DH / 16; ++oc) {
+              uint32_t o[16];
+              tmem_ld16(t_o + oc * 16, o);
+#pragma unroll
+              for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st16_async(t_o + oc * 16, o);
             }
-            tc_fence_after();
+          }
+          if (cc & 1) {
+            tmem_st_wait();   // this half of P (and O) is in TMEM before the arrive releases it
+            tc_fence_before();
+            mbar_arrive(p_full + 2 * grp + (cc >> 1));
           }
         }
-        // P row as bf16 pairs (column i holds keys 2i, 2i+1), written to P_w (its own columns, or
-        // over S_w, whose row is already in registers) in two halves of 32 columns. 2^x runs on
-        // MUFU in f32 (measured faster here than packed-f16 MUFU or the FMA-pipe exp2_poly2, which
-        // full tiles can route kPolyPairs of every 16 pairs to). Masked keys give ex2(-inf) = 0.
-        auto softmax_row = [&](auto poly_tag) {
-          constexpr bool kPoly = decltype(poly_tag)::value;
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t pw[32];
-#pragma unroll
-            for (int i2 = 0; i2 < 32; ++i2) {
-              const int i = 64 * half + 2 * i2;
-              float x0, x1, p0, p1;
-              f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), scale2, nref2), x0, x1);
-              if (kPoly && (i2 & 15) < kPolyPairs) {
-                exp2_poly2(x0, x1, p0, p1);
-              } else {
-                p0 = ex2_mufu(x0);
-                p1 = ex2_mufu(x1);
-              }
-              if (i2 & 1)
-                sum2b = f2_add(sum2b, f2_pack(p0, p1));
-              else
-                sum2a = f2_add(sum2a, f2_pack(p0, p1));
-              pw[i2] = pack_bf16_pos(p0, p1);   // p >= 0: integer-pipe rounding
-            }
-            tmem_st32_async(t_p + 32 * half, pw);
-            if constexpr (kSplitHandoff) {
-              // Each half is handed over as soon as it is written.
-              if (half == 0 && rescale && j > 0) {
-                // O_w holds the group's earlier tiles (their P*V completed: waited above); it is
-                // rescaled before this tile's first P*V accumulates into it.
-#pragma unroll 1
-                for (int c = 0; c < (DH + 31) / 32; ++c) {
-                  uint32_t o[32];
-                  tmem_ld32(t_o + c * 32, o);
-#pragma unroll
-                  for (int i = 0; i < 32; ++i)
-                    o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                  tmem_st32_async(t_o + c * 32, o);
-                }
-              }
-              tmem_st_wait();   // P (and O) complete in TMEM before the arrive releases it
-              tc_fence_before();
-              mbar_arrive(p_full + 2 * grp + half);
-            }
-          }
-        };
-        if (full)
-          softmax_row(std::integral_constant<bool, true>());
-        else
-          softmax_row(std::integral_constant<bool, false>());
+        if (!ok) break;
         // Is S of this group's next tile already there? Tested here, where the result is not
         // needed at once, instead of by a blocking wait at the top of the next iteration.
-        s_ready = mbar_test(s_full + grp, uses & 1);
+        s_ready = mbar_test(s_full + grp, (gn + 1) & 1);
         float sa0, sa1;
         f2_unpack(f2_add(sum2a, sum2b), sa0, sa1);
         l_run += sa0 + sa1;
-        if constexpr (!kSplitHandoff) {
-          // Both halves go together (the split costs the dh 80 variant registers it does not
-          // have): P written, then O_w rescaled if needed (its earlier P*V completed before this
-          // S was committed), then the hand-over.
-          tmem_st_wait();
-          if (rescale && j > 0) {
-#pragma unroll 1
-            for (int c = 0; c < (DH + 31) / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(t_o + c * 32, o);
+      }
+      if (!ok) break;
+      // ---- the piece's rows: O_g is final once the piece's last P_g * V is done ----
+      ok = __all_sync(0xffffffffu, mbar_wait(pv_done + grp, (gn - 1) & 1, abort, status));
+      if (!ok) break;
+      tc_fence_after();
+      if (c.tail < 0 || P.tail_split == 1) {
+        uint32_t o[DH];
+        load_o_row<DH>(t_o, o);
+        tc_fence_before();   // O_g read before the next piece's first P goes to P*V
+        // Normalised row -> the staging tile, once the TMA store of its previous contents (the
+        // other group's rows, or this group's a piece ago) has read them; warp 3 then stores it.
+        const int use = 2 * stage_uses + grp;
+        ++stage_uses;
+        if (use > 0 &&
+            !(ok = __all_sync(0xffffffffu, mbar_wait(stage_free, (use - 1) & 1, abort, status))))
+          break;
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        const uint32_t tile = smem_u32(smem + S::kStage);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st32(t_o + c * 32, o);
-            }
-          }
-          tc_fence_before();
-          mbar_arrive(p_full + 2 * grp);
-          mbar_arrive(p_full + 2 * grp + 1);
+        for (int cc = 0; cc < DH / 8; ++cc) {
+          // 16-byte chunk cc of the row, at its place in the swizzled box: 128-byte rows with the
+          // chunk index XORed with row % 8 (columns 0..63), 32-byte rows with it XORed with
+          // (row / 4) % 2 (the tail, columns 64..79).
+          const uint32_t addr = cc < 8 ? tile + row * 128 + ((cc ^ (row & 7)) << 4)
+                                       : tile + S::kQKMain + row * 32 + (((cc - 8) ^ ((row >> 2) & 1)) << 4);
+          st_shared_v4(addr,
+                       pack_bf16(__uint_as_float(o[8 * cc + 0]) * inv, __uint_as_float(o[8 * cc + 1]) * inv),
+                       pack_bf16(__uint_as_float(o[8 * cc + 2]) * inv, __uint_as_float(o[8 * cc + 3]) * inv),
+                       pack_bf16(__uint_as_float(o[8 * cc + 4]) * inv, __uint_as_float(o[8 * cc + 5]) * inv),
+                       pack_bf16(__uint_as_float(o[8 * cc + 6]) * inv, __uint_as_float(o[8 * cc + 7]) * inv));
         }
+        fence_proxy_async_smem();   // visible to the TMA store
+        mbar_arrive(staged);
+        continue;
       }
-      if constexpr (kOneGroupEpi) {
-        // ---- merge both groups' partial rows and scatter them to out[u, perm[p], h, :] ----
-        // Group 1 merges and emits the item; group 0 hands over its row max and sum and goes on to
-        // the next item at once (its first P*V there waits for o_free, i.e. for group 1 to have
-        // read O0 and O1). Every wait and barrier below is passed also after a failed wait.
-        const int mb = li & 1;   // this item's m, l buffer
-        if (grp == 0) {
-          s_m[mb * kBM + row] = m_ref;
-          s_l[mb * kBM + row] = l_run;
-          mbar_arrive(ml_ready + mb);
-        } else {
-          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ml_ready + mb, (li >> 1) & 1, abort, status));
-          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, li & 1, abort, status));
-          tc_fence_after();
-          const float m0 = s_m[mb * kBM + row], l0 = s_l[mb * kBM + row];
-          const float m1 = m_ref, l1 = l_run;
-          const float mm = fmaxf(m0, m1);
-          const float a0 = (m0 == -INFINITY) ? 0.f : ex2_mufu(m0 - mm);
-          const float a1 = (m1 == -INFINITY) ? 0.f : ex2_mufu(m1 - mm);
-          const float L = l0 * a0 + l1 * a1;
-          const float inv = L > 0.f ? 1.f / L : 0.f;
-          const float f0 = a0 * inv, f1 = a1 * inv;
-          const bool has0 = nt > 0, has1 = nt > 1;   // a group with no tile has a stale O
-          // The previous item's copy-out is finished before the staging rows are rewritten.
-          named_barrier(2, 128);
-          // Normalised row -> shared staging (rows padded by 16 bytes against bank conflicts); then
-          // the group copies whole rows out, so that each warp store covers contiguous rows.
-          const uint32_t stage_row = smem_u32(smem + S::kStage) + row * S::kStageStride;
-          if (ok) {
-            const uint32_t o0 = tmem + T::kO + lane_off;
-            const uint32_t o1 = o0 + T::kOStride;
-            auto emit8 = [&](const uint32_t* u0, const uint32_t* u1, int col) {
-              float v[8];
-  #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                v[i] = (has0 ? __uint_as_float(u0[i]) * f0 : 0.f) +
-                       (has1 ? __uint_as_float(u1[i]) * f1 : 0.f);
-              st_shared_v4(stage_row + col * 2, pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
-                           pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-            };
-  #pragma unroll 1
-            for (int c = 0; c < DH / 32; ++c) {   // 32 columns of O0 and O1 at a time
-              uint32_t x0[32], x1[32];
-              tmem_ld32_pair(o0 + c * 32, o1 + c * 32, x0, x1);
-  #pragma unroll
-              for (int e = 0; e < 4; ++e) emit8(x0 + 8 * e, x1 + 8 * e, c * 32 + 8 * e);
-            }
-            if constexpr (DH % 32) {   // dh 80: columns 64..79
-  #pragma unroll
-              for (int c = (DH / 32) * 32; c < DH; c += 8) {
-                uint32_t x0[8], x1[8];
-                tmem_ld8_pair(o0 + c, o1 + c, x0, x1);
-                emit8(x0, x1, c);
-              }
-            }
-            s_dst[row] = store ? dst_token(perm_t, P.N, status) : -1;
-          }
-          tc_fence_before();
-          mbar_arrive(o_free);   // O0, O1 read: the next item's first P*V may overwrite them
-          named_barrier(2, 128);
-          if (ok) {
-            constexpr int kCpr = DH / 8;                  // 16-byte chunks per row
-            const int tid = threadIdx.x - 256;            // 0..127: group 1
-            const uint32_t stage = smem_u32(smem + S::kStage);
-            uint8_t* out_uh = reinterpret_cast<uint8_t*>(P.out) +
-                              ((size_t)u_i * P.N * P.heads + h_i) * DH * 2;
-  #pragma unroll 2
-            for (int k = 0; k < kBM * kCpr / 128; ++k) {
-              const int q = tid + 128 * k;
-              const int r = q / kCpr, c = q - r * kCpr;
-              const int t = s_dst[r];
-              if (t >= 0) {
-                const uint4 v = ld_shared_v4(stage + r * S::kStageStride + c * 16);
-                *reinterpret_cast<uint4*>(out_uh + (size_t)t * P.heads * DH * 2 + c * 16) = v;
-              }
-            }
-          }
-        }
-      } else {
-        // ---- merge both groups' partial rows and scatter them to out[u, perm[p], h, :] ----
-        // Every softmax thread passes both named barriers once per item, also after a failed wait.
-        s_m[grp * kBM + row] = m_ref;
-        s_l[grp * kBM + row] = l_run;
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, li & 1, abort, status));
-        tc_fence_after();
-        named_barrier(1, 256);
-        constexpr int kCols = DH / 2;   // this group's output columns [grp*kCols, (grp+1)*kCols)
-        uint32_t x0[32], x1[32], y0[8], y1[8];   // columns 0-31 and (dh 80) 32-39 of O0, O1
-        float m0 = 0.f, m1 = 0.f, l0 = 0.f, l1 = 0.f;
-        if (ok) {
-          m0 = s_m[row];
-          m1 = s_m[kBM + row];
-          l0 = s_l[row];
-          l1 = s_l[kBM + row];
-          const uint32_t o0 = tmem + T::kO + lane_off + grp * kCols;
-          const uint32_t o1 = o0 + T::kOStride;
-          tmem_ld32_pair(o0, o1, x0, x1);
-          if constexpr (kCols > 32) tmem_ld8_pair(o0 + 32, o1 + 32, y0, y1);
-        }
-        // Both groups have read O0 and O1 (and m, l) before either hands the next item's first P
-        // to the P*V issuer, whose first MMA into O_w overwrites it.
+      // Row qrow of Op (the permuted output, block-major like Q), unless past N.
+      uint8_t* drow = qrow < P.N ? reinterpret_cast<uint8_t*>(P.operm) +
+                                       ((size_t)c.uh * P.N + qrow) * DH * 2
+                                 : nullptr;
+      // Split pair: this piece's O_g (relative to m) column-major, so that a warp's 32 rows of one
+      // column are one 128-byte line, then m and l; the group's last piece merges every piece's
+      // partial in piece order, so the result does not depend on which finished last.
+      {
+        float* slot = P.partial + ((size_t)c.tail * 2 + grp) * kSlot + row;
+        uint32_t o[DH];
+        load_o_row<DH>(t_o, o);
         tc_fence_before();
-        named_barrier(1, 256);
-        // Normalised half-row -> shared staging; then the 256 threads copy whole rows out, so
-        // that each warp store covers four contiguous 128-byte rows (dh 64) instead of 32 rows.
-        const uint32_t stage_row = smem_u32(smem + S::kStage) + row * S::kStageStride;
-        if (ok) {
-          const float mm = fmaxf(m0, m1);
-          const float a0 = (m0 == -INFINITY) ? 0.f : ex2_mufu(m0 - mm);
-          const float a1 = (m1 == -INFINITY) ? 0.f : ex2_mufu(m1 - mm);
-          const float L = l0 * a0 + l1 * a1;
-          const float inv = L > 0.f ? 1.f / L : 0.f;
-          const float f0 = a0 * inv, f1 = a1 * inv;
-          // A group with no tile in this item has a stale O: select, do not multiply by zero.
-          const bool has0 = nt > 0, has1 = nt > 1;
-  #pragma unroll
-          for (int c = 0; c < kCols / 8; ++c) {
-            float v[8];
-  #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint32_t u0 = c < 4 ? x0[8 * c + i] : y0[i];
-              const uint32_t u1 = c < 4 ? x1[8 * c + i] : y1[i];
-              v[i] = (has0 ? __uint_as_float(u0) * f0 : 0.f) + (has1 ? __uint_as_float(u1) * f1 : 0.f);
-            }
-            st_shared_v4(stage_row + grp * kCols * 2 + c * 16, pack_bf16(v[0], v[1]),
-                         pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-          }
-          if (grp == 0) s_dst[row] = store ? dst_token(perm_t, P.N, status) : -1;
-        }
-        named_barrier(1, 256);
-        if (ok) {
-          constexpr int kCpr = DH / 8;                  // 16-byte chunks per row
-          const int tid = threadIdx.x - 128;            // 0..255
-          const uint32_t stage = smem_u32(smem + S::kStage);
-          uint8_t* out_uh = reinterpret_cast<uint8_t*>(P.out) +
-                            ((size_t)u_i * P.N * P.heads + h_i) * DH * 2;
-  #pragma unroll
-          for (int k = 0; k < kBM * kCpr / 256; ++k) {
-            const int q = tid + 256 * k;
-            const int r = q / kCpr, c = q - r * kCpr;
-            const int t = s_dst[r];
-            if (t >= 0) {
-              const uint4 v = ld_shared_v4(stage + r * S::kStageStride + c * 16);
-              *reinterpret_cast<uint4*>(out_uh + (size_t)t * P.heads * DH * 2 + c * 16) = v;
-            }
-          }
+#pragma unroll
+        for (int e = 0; e < DH; ++e) slot[e * kBM] = __uint_as_float(o[e]);
+        slot[DH * kBM] = m_ref;
+        slot[(DH + 1) * kBM] = l_run;
+      }
+      __threadfence();
+      if (!(ok = grp_sync())) break;
+      const int tp = c.pair - P.whole;   // the pair's index among the split pairs
+      if (tid == 0) s_last[grp] = atomicAdd(P.counters + 2 * tp + grp, 1) == P.tail_split - 1;
+      if (!(ok = grp_sync())) break;
+      const bool last = s_last[grp] != 0;
+      if (!(ok = grp_sync())) break;   // s_last[grp] is rewritten by the next piece
+      if (!last) continue;
+      __threadfence();
+      const float* first = P.partial + ((size_t)tp * P.tail_split * 2 + grp) * kSlot + row;
+      float f[kMaxSplit];
+      float M = -INFINITY;
+#pragma unroll
+      for (int jj = 0; jj < kMaxSplit; ++jj)
+        if (jj < P.tail_split) M = fmaxf(M, __ldcg(first + (size_t)jj * 2 * kSlot + DH * kBM));
+      float Lsum = 0.f;
+#pragma unroll
+      for (int jj = 0; jj < kMaxSplit; ++jj) {
+        f[jj] = 0.f;
+        if (jj < P.tail_split) {
+          const float* sj = first + (size_t)jj * 2 * kSlot;
+          const float mj = __ldcg(sj + DH * kBM);
+          f[jj] = mj == -INFINITY ? 0.f : ex2_mufu(mj - M);
+          Lsum += f[jj] * __ldcg(sj + (DH + 1) * kBM);
         }
       }
-      gn0 += nt;
+      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < DH / 8; ++cc) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < kMaxSplit; ++jj) {
+          if (jj >= P.tail_split) break;
+          const float* sj = first + (size_t)jj * 2 * kSlot + (size_t)cc * 8 * kBM;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] += __ldcg(sj + e * kBM) * f[jj];
+        }
+        if (drow) {
+          uint4 w;
+          w.x = pack_bf16(v[0] * inv, v[1] * inv);
+          w.y = pack_bf16(v[2] * inv, v[3] * inv);
+          w.z = pack_bf16(v[4] * inv, v[5] * inv);
+          w.w = pack_bf16(v[6] * inv, v[7] * inv);
+          reinterpret_cast<uint4*>(drow)[cc] = w;
+        }
+      }
+      if (tid == 0) P.counters[2 * tp + grp] = 0;   // re-armed for the next launch
     }
   }
   tc_fence_before();
+  abort_drain(abort);
   cta_sync_converged();
   if (warp == 1) {
     tc_fence_after();
@@ -1223,21 +1196,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-template <int DH>
-static cudaError_t launch_attn_dh(const CUtensorMap* tq, const CUtensorMap* tk,
-                                  const CUtensorMap* tv, const CUtensorMap* tq_tail,
-                                  const CUtensorMap* tk_tail, const CUtensorMap* tv_tail,
-                                  const AttnParams& p, int* status, cudaStream_t st) {
-  using S = AttnSmem<DH>;
-  cudaError_t e = cudaFuncSetAttribute(k_attn<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       S::kAlloc);
-  if (e != cudaSuccess) return e;
-  const int items = ((p.N + kBM - 1) / kBM) * p.U * p.heads;
-  dim3 grid(std::max(1, std::min(items, p.sms)));
-  return launch_pdl(k_attn<DH>, grid, dim3(kAttnThreads), S::kAlloc, st, *tq, *tk, *tv, *tq_tail,
-                    *tk_tail, *tv_tail, p, status);
-}
-
 static cudaError_t launch_attn_pairs(const CUtensorMap* tq, const CUtensorMap* tk,
                                      const CUtensorMap* tv, const AttnParams& p, int* status,
                                      cudaStream_t st) {
@@ -1251,22 +1209,131 @@ static cudaError_t launch_attn_pairs(const CUtensorMap* tq, const CUtensorMap* t
   return launch_pdl(kernel, grid, dim3(kAttnThreads), S::kAlloc, st, *tq, *tk, *tv, p, status);
 }
 
+template <int DH>
+static cudaError_t launch_attn_pair(const CUtensorMap* tq, const CUtensorMap* tk,
+                                    const CUtensorMap* tv, const CUtensorMap* tq_tail,
+                                    const CUtensorMap* tk_tail, const CUtensorMap* to,
+                                    const CUtensorMap* to_tail, const AttnParams& p, int* status,
+                                    cudaStream_t st) {
+  using S = PairSmem<DH>;
+  cudaError_t e = cudaFuncSetAttribute(k_attn_pair<DH>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc);
+  if (e != cudaSuccess) return e;
+  const int pieces = p.whole + (pairs_per_head(p.N) * p.U * p.heads - p.whole) * p.tail_split;
+  dim3 grid(std::max(1, std::min(pieces, p.sms)));
+  return launch_pdl(k_attn_pair<DH>, grid, dim3(kAttnThreads), S::kAlloc, st, *tq, *tk, *tv,
+                    *tq_tail, *tk_tail, *to, *to_tail, p, status);
+}
+
+// Short items: every query tile has at most kPairTiles key tiles (the windowed blocks).
+static bool short_items(const AttnParams& p) {
+  const int nq = (p.N + kBM - 1) / kBM;
+  int nt_max = 0;
+  for (int qt = 0; qt < nq; ++qt)
+    nt_max = std::max(nt_max, key_tiles(qt * kBM, std::min(qt * kBM + kBM, p.N) - 1, qt, 0, p).count());
+  return nt_max <= kPairTiles;
+}
+
+AttnPlan attn_plan(const AttnParams& p, int dh, int sms) {
+  AttnPlan r = {};
+  r.pair_kernel = !(dh == 64 && short_items(p));
+  if (!r.pair_kernel) return r;
+  const int npairs = pairs_per_head(p.N);
+  r.pairs = npairs * p.U * p.heads;
+  r.whole = r.pairs;
+  r.tail_split = 1;
+  int nt_min = 1 << 30, nt_max = 0;
+  for (int pq = 0; pq < npairs; ++pq) {
+    const int q0 = pq * 2 * kBM;
+    const int nt = key_tiles(q0, std::min(q0 + 2 * kBM, p.N) - 1, pq, 0, p).count();
+    nt_min = std::min(nt_min, nt);
+    nt_max = std::max(nt_max, nt);
+  }
+  // The pairs of a partial last round (r of them) are split into s pieces each, s = how many
+  // times r fits the CTAs (at most kMaxSplit, and every piece keeps a tile), when that shortens
+  // the busiest CTA: full rounds of whole pairs plus one split piece, against one more round of
+  // whole pairs (each piece costs about one tile of pipeline fill and drain; a merge about one).
+  const int rem = r.pairs % sms;
+  if (rem > 0) {
+    const int s = std::min(std::min(kMaxSplit, nt_min), sms / rem);
+    const long long full = r.pairs / sms;
+    const long long cost_whole = (full + 1) * (nt_max + 1);
+    const long long cost_split = full * (nt_max + 1) + (nt_max + s - 1) / s + 2;
+    if (s > 1 && cost_split < cost_whole) {
+      r.whole = r.pairs - rem;
+      r.tail_split = s;
+      r.partial_bytes = (size_t)rem * s * 2 * (dh + 2) * kBM * sizeof(float);
+      r.counter_bytes = (size_t)rem * 2 * sizeof(int);   // one per split pair and group
+    }
+  }
+  return r;
+}
+
 cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                         const CUtensorMap* tq_tail, const CUtensorMap* tk_tail,
-                        const CUtensorMap* tv_tail, const AttnParams& p, int dh, int* status,
-                        cudaStream_t st) {
-  if (dh == 64) {
-    // Short items (at most kPairTiles key tiles per query tile, as in windowed blocks) go to the
-    // whole-item-per-group kernel.
-    const int nq = (p.N + kBM - 1) / kBM;
-    int nt_max = 0;
-    for (int qt = 0; qt < nq; ++qt)
-      nt_max = std::max(nt_max,
-                        key_tiles(qt * kBM, std::min(qt * kBM + kBM, p.N) - 1, qt, 0, p).count());
-    if (nt_max <= kPairTiles) return launch_attn_pairs(tq, tk, tv, p, status, st);
-    return launch_attn_dh<64>(tq, tk, tv, tq, tk, tv, p, status, st);
+                        const CUtensorMap* to, const CUtensorMap* to_tail, const AttnParams& p,
+                        int dh, int* status, cudaStream_t st) {
+  if (dh == 64 && short_items(p)) return launch_attn_pairs(tq, tk, tv, p, status, st);
+  if (dh == 64) return launch_attn_pair<64>(tq, tk, tv, tq, tk, to, to, p, status, st);
+  if (dh == 80) return launch_attn_pair<80>(tq, tk, tv, tq_tail, tk_tail, to, to_tail, p, status, st);
+  return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Un-permute: out[u, perm[p], h, :] = Op[u*heads + h, q(p), :] (the pair kernel's output order)
+// ---------------------------------------------------------------------------------------------
+// One warp per block-major position q of a unit: the warp resolves the token t = perm[u][p(q)],
+// reads the position's row of every head matrix (heads * CPR 16-byte chunks) and writes them as
+// token t's one contiguous heads * dh row of out. All of a lane's loads are in flight before its
+// stores. CPR = 16-byte chunks per head, KPL = chunks per lane.
+template <int CPR, int KPL>
+__global__ void __launch_bounds__(256) k_unpermute_out(const uint16_t* __restrict__ op,
+                                                       const int32_t* __restrict__ perm,
+                                                       uint16_t* __restrict__ out, int N,
+                                                       int heads, int b, int L, int* status) {
+  griddep_wait();
+  griddep_launch();
+  const int u = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qpos = blockIdx.x * 8 + warp;
+  if (qpos >= N) return;
+  const int tok = __ldg(perm + (size_t)u * N + blockmajor_to_canonical(qpos, b, L));
+  if ((unsigned)tok >= (unsigned)N) {   // not a token of this unit: skip the row, report it
+    if (lane == 0) record_bad_index(status);
+    return;
   }
-  if (dh == 80) return launch_attn_dh<80>(tq, tk, tv, tq_tail, tk_tail, tv_tail, p, status, st);
+  const int per_tok = heads * CPR;
+  const size_t plane = (size_t)N * CPR;   // 16-byte chunks per (unit, head) matrix
+  const uint4* src = reinterpret_cast<const uint4*>(op) + (size_t)u * heads * plane +
+                     (size_t)qpos * CPR;
+  uint4* dst = reinterpret_cast<uint4*>(out) + ((size_t)u * N + tok) * per_tok;
+  uint4 buf[KPL];
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int cidx = e * 32 + lane;
+    if (cidx < per_tok) {
+      const int h = cidx / CPR, cc = cidx - h * CPR;
+      buf[e] = __ldg(src + h * plane + cc);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int cidx = e * 32 + lane;
+    if (cidx < per_tok) dst[cidx] = buf[e];
+  }
+}
+
+cudaError_t launch_unpermute_out(const uint16_t* op, const int32_t* perm, uint16_t* out, int U,
+                                 int N, int heads, int dh, int b, int* status, cudaStream_t st) {
+  dim3 grid((N + 7) / 8, U);
+  const int L = N / kStripes;
+  const int per_tok = heads * (dh / 8);
+  if (per_tok > 32 * 10) return cudaErrorInvalidValue;   // heads * dh > 2560
+  auto go = [&](auto kernel) {
+    return launch_pdl(kernel, grid, dim3(256), 0, st, op, perm, out, N, heads, b, L, status);
+  };
+  if (dh == 64) return per_tok <= 32 * 8 ? go(k_unpermute_out<8, 8>) : go(k_unpermute_out<8, 10>);
+  if (dh == 80) return go(k_unpermute_out<10, 10>);
   return cudaErrorInvalidValue;
 }
 

@@ -31,11 +31,19 @@ cudaError_t launch_stripe_rank(const double* score, const float* lum, double* sc
                                int K, int32_t* perm, int32_t* inv, int32_t* keep,
                                cudaStream_t st);
 
-// Gathers q, k, v [U, N, heads, dh] into the block-major permuted layout [U*heads, N, dh].
+// score[i] = SplitMix64 output i from `seed`, as a uniform double in [0, 1), i < n.
+cudaError_t launch_random_score(double* score, long long n, unsigned long long seed,
+                                cudaStream_t st);
+// mag[r] = sum over c in order of delta[r, c]^2 in fp64, for rows r < rows of C bf16 (C % 8 == 0).
+cudaError_t launch_update_magnitude(const uint16_t* delta, double* mag, long long rows, int C,
+                                    cudaStream_t st);
+
+// Gathers q, k, v [U, N, heads, dh] into the block-major permuted layout [U*heads, N, dh];
+// also zeroes zero[0, nzero) (the attention's merge counters).
 cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                               const int32_t* perm, uint16_t* qp, uint16_t* kp, uint16_t* vp,
-                              int U, int N, int heads, int dh, int b, int* status,
-                              cudaStream_t st);
+                              int U, int N, int heads, int dh, int b, int* zero, int nzero,
+                              int* status, cudaStream_t st);
 
 struct AttnParams {
   const int32_t* perm;   // [U, N]
@@ -43,12 +51,31 @@ struct AttnParams {
   int U, N, heads, L, b, nb, W, g;
   float scale_log2;      // log2(e) / sqrt(dh)
   int sms;               // persistent CTAs to launch (one per SM)
+  int whole;             // pair kernel: pairs processed whole (the rest are split)
+  int tail_split;        // pair kernel: pieces per split pair
+  float* partial;        // per split piece and group, fp32 O [dh][128], m [128], l [128]
+  int* counters;         // per split pair and group, finished pieces; zero between launches
+  uint16_t* operm;       // pair kernel output: [U*heads, N, dh] in block-major permuted order
 };
-// Block-sparse attention over the gathered sequences (tensor maps over [U*heads, N, dh]).
+// Which attention kernel a shape takes, and the scratch beyond the gathered Q, K, V it needs
+// (planned for `sms` CTAs).
+struct AttnPlan {
+  bool pair_kernel;      // the pair kernel (else the short-item kernel)
+  int pairs, whole, tail_split;
+  size_t partial_bytes, counter_bytes;
+};
+AttnPlan attn_plan(const AttnParams& p, int dh, int sms);
+// Block-sparse attention over the gathered sequences (tensor maps over [U*heads, N, dh]; the
+// tails cover columns 64..79 at head dim 80). The pair kernel writes its output, permuted, through
+// `to` / `to_tail` (maps over p.operm laid out like Q); launch_unpermute_out then scatters it to
+// p.out. The short-item kernel writes p.out itself.
 cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                         const CUtensorMap* tq_tail, const CUtensorMap* tk_tail,
-                        const CUtensorMap* tv_tail, const AttnParams& p, int dh, int* status,
-                        cudaStream_t st);
+                        const CUtensorMap* to, const CUtensorMap* to_tail, const AttnParams& p,
+                        int dh, int* status, cudaStream_t st);
+// out[u, perm[u][p(q)], h, :] = op[u*heads + h, q, :] for every block-major position q.
+cudaError_t launch_unpermute_out(const uint16_t* op, const int32_t* perm, uint16_t* out, int U,
+                                 int N, int heads, int dh, int b, int* status, cudaStream_t st);
 
 // Gathers the kept rows of x [B, T, C] into xk [B*K, C]; zeroes zero[0, nzero). late_wait: keep
 // and x are known final at launch (see k_gather_rows), the copy need not wait for the previous

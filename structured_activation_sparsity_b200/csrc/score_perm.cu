@@ -243,4 +243,65 @@ cudaError_t launch_stripe_rank(const double* score, const float* lum, double* sc
   return N >= 2048 ? go(k_stripe_rank<32, false>, 32) : go(k_stripe_rank<8, false>, 8);
 }
 
+// ---------------------------------------------------------------------------------------------
+// Variants: random scores (the random-permutation ablation) and update magnitudes (a keep
+// criterion). Both produce scores that the ranking kernel above turns into perm / keep.
+// ---------------------------------------------------------------------------------------------
+// Output n of the SplitMix64 generator (Steele, Lea and Flood, "Fast splittable pseudorandom
+// number generators", OOPSLA 2014) from state `seed`: the state after n + 1 steps of the golden
+// gamma, through the generator's output mix.
+__device__ __forceinline__ unsigned long long splitmix64_at(unsigned long long seed,
+                                                           unsigned long long n) {
+  unsigned long long z = seed + (n + 1ull) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// score[i] = (output i >> 11) * 2^-53, uniform in [0, 1), for i < n (= images * tokens).
+__global__ void __launch_bounds__(256) k_random_score(double* __restrict__ score, long long n,
+                                                      unsigned long long seed) {
+  griddep_wait();
+  griddep_launch();
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) score[i] = (double)(splitmix64_at(seed, (unsigned long long)i) >> 11) * 0x1p-53;
+}
+
+// mag[r] = sum over c = 0..C-1, in that order, of delta[r, c]^2 (one fp64 round-to-nearest
+// operation per multiply and per add, never fused): one thread per token row, 16-byte loads.
+__global__ void __launch_bounds__(128) k_update_magnitude(const uint16_t* __restrict__ delta,
+                                                          double* __restrict__ mag, long long rows,
+                                                          int C) {
+  griddep_wait();
+  griddep_launch();
+  const long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= rows) return;
+  const uint4* src = reinterpret_cast<const uint4*>(delta + r * C);
+  double acc = 0.0;
+  for (int c8 = 0; c8 < C / 8; ++c8) {
+    const uint4 w = __ldg(src + c8);
+    const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const double lo = (double)__uint_as_float(v[e] << 16);
+      const double hi = (double)__uint_as_float(v[e] & 0xFFFF0000u);
+      acc = __dadd_rn(acc, __dmul_rn(lo, lo));
+      acc = __dadd_rn(acc, __dmul_rn(hi, hi));
+    }
+  }
+  mag[r] = acc;
+}
+
+cudaError_t launch_random_score(double* score, long long n, unsigned long long seed,
+                                cudaStream_t st) {
+  return launch_pdl(k_random_score, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, score, n,
+                    seed);
+}
+
+cudaError_t launch_update_magnitude(const uint16_t* delta, double* mag, long long rows, int C,
+                                    cudaStream_t st) {
+  return launch_pdl(k_update_magnitude, dim3((unsigned)((rows + 127) / 128)), dim3(128), 0, st,
+                    delta, mag, rows, C);
+}
+
 }  // namespace ss

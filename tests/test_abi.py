@@ -151,6 +151,15 @@ def test_validation_codes():
     # 51 MB of partials
     extra = L.sparsesam_rcmlp_workspace(vith, 1280, 5120, O.keep_count(0.3, 4096)) - xk_h
     assert 47 * 128 * 256 * 4 <= extra < 8 << 20
+    # variants: missing outputs, K outside [0, T], C not a multiple of 8, misaligned delta
+    assert lib.sparsesam_random_perm(by(good), 1, None, FAKE, None, None, None) == L.SS_EINVAL
+    assert lib.sparsesam_random_perm(by(good), 1, FAKE, None, None, None, None) == L.SS_EINVAL
+    assert lib.sparsesam_keep_by_update(by(good), FAKE, 64, 257, FAKE, FAKE, None) == L.SS_EINVAL
+    assert lib.sparsesam_keep_by_update(by(good), FAKE, 64, -1, FAKE, FAKE, None) == L.SS_EINVAL
+    assert lib.sparsesam_keep_by_update(by(good), FAKE, 60, 10, FAKE, FAKE, None) == L.SS_EUNSUPPORTED
+    assert lib.sparsesam_keep_by_update(by(good), FAKE + 2, 64, 10, FAKE, FAKE, None) == L.SS_EINVAL
+    assert lib.sparsesam_keep_by_update(by(good), None, 64, 10, FAKE, FAKE, None) == L.SS_EINVAL
+    assert lib.sparsesam_keep_by_update(by(good), FAKE, 64, 0, FAKE, FAKE, None) == L.SS_OK
     # blocklist capacity
     rp = (ctypes.c_int32 * 8)()
     ci = (ctypes.c_int32 * 2)()

@@ -403,3 +403,77 @@ def test_mutation_band_off_by_one_caught(monkeypatch):
     with pytest.raises(AssertionError):
         for row in _golden_patterns():
             test_pattern_hand_derived_table(row)
+
+
+# ---- variants: SplitMix64 random scores, update magnitude, keep_top ---------------------------
+def test_splitmix64_published_first_output():
+    # The generator's first output from state 0, as the SplitMix64 reference implementation
+    # (Steele, Lea and Flood, OOPSLA 2014) produces it.
+    assert int(O.splitmix64(0, [0])[0]) == 0xE220A8397B1DCDAF
+
+
+def test_splitmix64_counter_is_the_sequential_stream():
+    # Output n from `seed` is the (n+1)-th step of the sequential generator: stepping the state
+    # by gamma n times first gives the same value as output 0 from the stepped seed.
+    gamma = 0x9E3779B97F4A7C15
+    seed = 123456789
+    for n in (1, 2, 17, 1000):
+        stepped = (seed + n * gamma) % (1 << 64)
+        assert int(O.splitmix64(seed, [n])[0]) == int(O.splitmix64(stepped, [0])[0])
+
+
+def test_random_scores_are_uniform_in_unit_interval():
+    r = O.random_scores(8, 4096, seed=3)
+    assert r.shape == (8, 4096) and r.min() >= 0.0 and r.max() < 1.0
+    assert abs(r.mean() - 0.5) < 0.005
+    counts = np.histogram(r, bins=16, range=(0.0, 1.0))[0]
+    expected = r.size / 16
+    chi2 = float(((counts - expected) ** 2 / expected).sum())
+    assert chi2 < 50.0   # 15 degrees of freedom: far beyond any plausible draw only if broken
+    assert len(np.unique(r)) == r.size
+    assert not np.array_equal(O.random_scores(1, 64, 1), O.random_scores(1, 64, 2))
+
+
+def test_random_permutation_is_a_stripe_sorted_bijection():
+    geo = O.Geometry(2, 16, 16, "global", 14)
+    sc = O.random_scores(2, 256, seed=11)
+    perm, inv = O.stripe_sort(sc, geo)
+    for u in range(2):
+        assert sorted(perm[u]) == list(range(256))
+        assert np.array_equal(inv[u][perm[u]], np.arange(256))
+        ranked = np.argsort(-sc[u], kind="stable")
+        # stripe j holds ranks j, j+4, ...: position j*64 + k is rank 4k + j
+        assert all(perm[u][j * 64 + k] == ranked[4 * k + j] for j in range(4) for k in range(64))
+
+
+def test_update_magnitude_exact_on_small_integers():
+    g = np.random.default_rng(4)
+    d = g.integers(-20, 21, size=(3, 50, 96)).astype(np.float64)
+    got = O.update_magnitude(d)
+    want = np.array([[sum(int(v) * int(v) for v in d[b, t]) for t in range(50)] for b in range(3)])
+    assert np.array_equal(got, want.astype(np.float64))
+    one_hot = np.zeros((1, 4, 8))
+    one_hot[0, 2, 5] = -3.0
+    assert np.array_equal(O.update_magnitude(one_hot), [[0.0, 0.0, 9.0, 0.0]])
+
+
+def test_update_magnitude_sums_in_channel_order():
+    # 1 + 3 * 2^-54: added to 1 one at a time each 2^-54 is below half an ulp of 1 and is lost;
+    # the three summed first (reversed channel order) give 1.5 * 2^-53, which rounds 1 up to
+    # 1 + 2^-52. The oracle's order is channel order.
+    e = 2.0 ** -27   # e^2 = 2^-54 exactly
+    d = np.array([[[1.0, e, e, e]]])
+    assert O.update_magnitude(d)[0, 0] == 1.0
+    assert O.update_magnitude(d[:, :, ::-1])[0, 0] == 1.0 + 2.0 ** -52
+
+
+def test_keep_top_brute_force_with_ties():
+    g = np.random.default_rng(6)
+    sc = g.integers(0, 4, size=(3, 40)).astype(np.float64)
+    for K in (0, 1, 13, 40):
+        keep = O.keep_top(sc, K)
+        assert keep.shape == (3, K)
+        for b in range(3):
+            rank = [int(np.sum(sc[b] > sc[b, t]) + np.sum((sc[b] == sc[b, t]) & (np.arange(40) < t)))
+                    for t in range(40)]
+            assert [int(t) for t in keep[b]] == [rank.index(r) for r in range(K)]
