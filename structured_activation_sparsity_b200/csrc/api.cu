@@ -192,12 +192,12 @@ constexpr int kPlanSMs = 148;
 
 // The attention workspace: the gathered Q, K and V ([U*heads, N, dh] bf16 each); for the pair
 // kernel its permuted output Op (the same layout), and, when it splits pairs into pieces, its
-// per-piece partials and per-pair merge counters.
+// per-piece partials.
 struct AttnLayout {
   AttnParams ap;     // geometry and plan fields filled; perm, out, sms by the launch
   AttnPlan plan;
   size_t one;        // bytes of one gathered array (256-byte multiple)
-  size_t operm, partial, counters, total;   // byte offsets, total size
+  size_t operm, partial, total;   // byte offsets, total size
 };
 
 int attn_layout(const ss_cfg* c, const Geo& g, AttnLayout* L) {
@@ -221,8 +221,7 @@ int attn_layout(const ss_cfg* c, const Geo& g, AttnLayout* L) {
   L->one = align256((size_t)g.U * c->heads * g.N * c->head_dim * 2);
   L->operm = 3 * L->one;
   L->partial = L->operm + (L->plan.pair_kernel ? L->one : 0);
-  L->counters = L->partial + align256(L->plan.partial_bytes);
-  L->total = L->counters + align256(L->plan.counter_bytes);
+  L->total = L->partial + align256(L->plan.partial_bytes);
   return SS_OK;
 }
 
@@ -427,7 +426,7 @@ static int attn_check(const ss_cfg* cfg, const Geo& g, const uint16_t* q, const 
   return SS_OK;
 }
 
-// The Q/K/V gather into ws (laid out as attn_layout describes); it also zeroes the merge counters.
+// The Q/K/V gather into ws (laid out as attn_layout describes).
 static int gather_launch(const Geo& g, int heads, int dh, const AttnLayout& L, const uint16_t* q,
                          const uint16_t* k, const uint16_t* v, const int32_t* perm, uint8_t* ws,
                          int* status, cudaStream_t st) {
@@ -435,8 +434,7 @@ static int gather_launch(const Geo& g, int heads, int dh, const AttnLayout& L, c
     return launch_gather_qkv(q, k, v, perm, reinterpret_cast<uint16_t*>(ws),
                              reinterpret_cast<uint16_t*>(ws + L.one),
                              reinterpret_cast<uint16_t*>(ws + 2 * L.one), g.U, g.N, heads, dh,
-                             L.ap.b, reinterpret_cast<int*>(ws + L.counters),
-                             (int)(L.plan.counter_bytes / sizeof(int)), status, st);
+                             L.ap.b, status, st);
   }));
 }
 
@@ -471,13 +469,15 @@ static int attn_launch(const ss_cfg* cfg, const Geo& g, const AttnLayout& L, uin
   ap.out = out;
   ap.sms = sm_count();
   ap.partial = reinterpret_cast<float*>(ws + L.partial);
-  ap.counters = reinterpret_cast<int*>(ws + L.counters);
   ap.operm = operm;
   int rc = cuda_err(traced("attn", st, [&] {
     return launch_attn(&tm[0], &tm[1], &tm[2], &tm[3], &tm[4], &tm[5], &tm[6], ap, dh, status,
                        st);
   }));
   if (rc || !L.plan.pair_kernel) return rc;
+  if (L.plan.tail_split > 1 &&
+      (rc = cuda_err(traced("merge_pieces", st, [&] { return launch_merge_pieces(ap, dh, st); }))))
+    return rc;
   return cuda_err(traced("unpermute_out", st, [&] {
     return launch_unpermute_out(operm, perm, out, g.U, g.N, heads, dh, ap.b, status, st);
   }));

@@ -41,12 +41,9 @@ __global__ void __launch_bounds__(256, MINB) k_gather_qkv(const uint16_t* __rest
                                                        uint16_t* __restrict__ kp,
                                                        uint16_t* __restrict__ vp, int N,
                                                        int heads, int b, int L,
-                                                       int* __restrict__ zero, int nzero,
                                                        int* status) {
   griddep_wait();
   griddep_launch();
-  if (blockIdx.x == 0 && blockIdx.y == 0)
-    for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
   const int u = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qpos = blockIdx.x * 8 + warp;
@@ -88,13 +85,13 @@ __global__ void __launch_bounds__(256, MINB) k_gather_qkv(const uint16_t* __rest
 
 cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                               const int32_t* perm, uint16_t* qp, uint16_t* kp, uint16_t* vp,
-                              int U, int N, int heads, int dh, int b, int* zero, int nzero,
-                              int* status, cudaStream_t st) {
+                              int U, int N, int heads, int dh, int b, int* status,
+                              cudaStream_t st) {
   dim3 grid((N + 7) / 8, U);
   const int L = N / kStripes;
   auto go = [&](auto kernel) {
     return launch_pdl(kernel, grid, dim3(256), 0, st, q, k, v, perm, qp, kp, vp, N, heads, b, L,
-                      zero, nzero, status);
+                      status);
   };
   const int per_tok = heads * (dh / 8);
   if (dh != 64 && dh != 80) return cudaErrorInvalidValue;
@@ -219,9 +216,8 @@ __device__ __forceinline__ Item item_of(int it, int nq, const AttnParams& P) {
 // That also lets the groups share one S buffer in TMEM: the Q*K^T of one group's tile goes into it
 // as soon as the other group has read its own S out.
 // Work is pieces: the pairs of the full rounds of CTAs are whole pieces; the pairs of a partial
-// last round are cut into `tail_split` key ranges each, so that round spreads over every CTA, and
-// each group of such a piece writes (O, m, l) to a global slot; the pair's last piece to finish
-// merges them.
+// last round are cut into `tail_split` key ranges each, so that round spreads over every CTA; each
+// group of such a piece writes its (O, m, l) to a global slot, and k_merge_pieces combines them.
 //   warp 0        TMA producer: Q_A, Q_B per piece; K and V tiles into a ring of stages
 //   warp 1        TMEM allocator and Q*K^T issuer (both groups)
 //   warp 2        P*V issuer (both groups)
@@ -348,12 +344,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* s_free = s_full + 2;             // S read into registers by the group it was for
   uint64_t* p_full = s_free + 2;             // [2][2] half h of P_g written (O_g rescaled first)
   uint64_t* pv_done = p_full + 4;            // [2] P_g * V of a tile done
-  uint64_t* grp_bar = pv_done + 2;           // [2] rendezvous of group g's 128 threads
-  uint64_t* stage_free = grp_bar + 2;        // the staging tile read by its TMA store
+  uint64_t* stage_free = pv_done + 2;        // the staging tile read by its TMA store
   uint64_t* staged = stage_free + 1;         // a group's rows are in the staging tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(staged + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);   // [2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int npairs = pairs_per_head(P.N);
@@ -368,7 +362,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(p_full + 2 * g, 128);
       mbar_init(p_full + 2 * g + 1, 128);
       mbar_init(pv_done + g, 1);
-      mbar_init(grp_bar + g, 128);
     }
     for (int i = 0; i < NS; ++i) {
       mbar_init(kv_full + i, 1);
@@ -384,7 +377,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   cta_sync_converged();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  griddep_wait();   // Q, K, V, perm and the merge counters come from the work before this launch
+  griddep_wait();   // Q, K, V and perm come from the work before this launch
   griddep_launch();
 
   if (warp < 4) {
@@ -520,7 +513,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ------------------------------ softmax groups ----------------------------
     const int grp = (warp - 4) >> 2;                    // 0: tile A of the pair, 1: tile B
     const int row = 32 * (warp & 3) + lane;             // TMEM lane == query row
-    const int tid = threadIdx.x - 128 * (1 + grp);      // 0..127 within the group
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
     const uint32_t t_s = tmem + T::kS + lane_off;
     const uint32_t t_p = tmem + T::kP + grp * T::kPStride + lane_off;
@@ -528,13 +520,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int b4 = P.b * kStripes;
     const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
     constexpr int kSlot = (DH + 2) * kBM;               // floats of one group's partial
-    uint32_t bar_phase = 0;
-    auto grp_sync = [&]() -> bool {                     // bounded rendezvous of the group
-      mbar_arrive(grp_bar + grp);
-      const bool r = mbar_wait(grp_bar + grp, bar_phase, abort, status);
-      bar_phase ^= 1;
-      return r;
-    };
     bool ok = true;
     int gn = 0;            // tiles of this group so far (all pieces): the phase count
     bool s_ready = false;  // the next s_full phase was already seen complete (non-blocking test)
@@ -706,13 +691,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(staged);
         continue;
       }
-      // Row qrow of Op (the permuted output, block-major like Q), unless past N.
-      uint8_t* drow = qrow < P.N ? reinterpret_cast<uint8_t*>(P.operm) +
-                                       ((size_t)c.uh * P.N + qrow) * DH * 2
-                                 : nullptr;
-      // Split pair: this piece's O_g (relative to m) column-major, so that a warp's 32 rows of one
-      // column are one 128-byte line, then m and l; the group's last piece merges every piece's
-      // partial in piece order, so the result does not depend on which finished last.
+      // Split pair: this piece's O_g (relative to its m) column-major, so that a warp's 32 rows
+      // of one column are one 128-byte line, then m and l; k_merge_pieces combines the pair's
+      // pieces after this launch.
       {
         float* slot = P.partial + ((size_t)c.tail * 2 + grp) * kSlot + row;
         uint32_t o[DH];
@@ -723,55 +704,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         slot[DH * kBM] = m_ref;
         slot[(DH + 1) * kBM] = l_run;
       }
-      __threadfence();
-      if (!(ok = grp_sync())) break;
-      const int tp = c.pair - P.whole;   // the pair's index among the split pairs
-      if (tid == 0) s_last[grp] = atomicAdd(P.counters + 2 * tp + grp, 1) == P.tail_split - 1;
-      if (!(ok = grp_sync())) break;
-      const bool last = s_last[grp] != 0;
-      if (!(ok = grp_sync())) break;   // s_last[grp] is rewritten by the next piece
-      if (!last) continue;
-      __threadfence();
-      const float* first = P.partial + ((size_t)tp * P.tail_split * 2 + grp) * kSlot + row;
-      float f[kMaxSplit];
-      float M = -INFINITY;
-#pragma unroll
-      for (int jj = 0; jj < kMaxSplit; ++jj)
-        if (jj < P.tail_split) M = fmaxf(M, __ldcg(first + (size_t)jj * 2 * kSlot + DH * kBM));
-      float Lsum = 0.f;
-#pragma unroll
-      for (int jj = 0; jj < kMaxSplit; ++jj) {
-        f[jj] = 0.f;
-        if (jj < P.tail_split) {
-          const float* sj = first + (size_t)jj * 2 * kSlot;
-          const float mj = __ldcg(sj + DH * kBM);
-          f[jj] = mj == -INFINITY ? 0.f : ex2_mufu(mj - M);
-          Lsum += f[jj] * __ldcg(sj + (DH + 1) * kBM);
-        }
-      }
-      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-#pragma unroll 1
-      for (int cc = 0; cc < DH / 8; ++cc) {
-        float v[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = 0.f;
-#pragma unroll
-        for (int jj = 0; jj < kMaxSplit; ++jj) {
-          if (jj >= P.tail_split) break;
-          const float* sj = first + (size_t)jj * 2 * kSlot + (size_t)cc * 8 * kBM;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] += __ldcg(sj + e * kBM) * f[jj];
-        }
-        if (drow) {
-          uint4 w;
-          w.x = pack_bf16(v[0] * inv, v[1] * inv);
-          w.y = pack_bf16(v[2] * inv, v[3] * inv);
-          w.z = pack_bf16(v[4] * inv, v[5] * inv);
-          w.w = pack_bf16(v[6] * inv, v[7] * inv);
-          reinterpret_cast<uint4*>(drow)[cc] = w;
-        }
-      }
-      if (tid == 0) P.counters[2 * tp + grp] = 0;   // re-armed for the next launch
     }
   }
   tc_fence_before();
@@ -1252,7 +1184,7 @@ AttnPlan attn_plan(const AttnParams& p, int dh, int sms) {
   // The pairs of a partial last round (r of them) are split into s pieces each, s = how many
   // times r fits the CTAs (at most kMaxSplit, and every piece keeps a tile), when that shortens
   // the busiest CTA: full rounds of whole pairs plus one split piece, against one more round of
-  // whole pairs (each piece costs about one tile of pipeline fill and drain; a merge about one).
+  // whole pairs (each piece costs about one tile of pipeline fill and drain; the merge about one).
   const int rem = r.pairs % sms;
   if (rem > 0) {
     const int s = std::min(std::min(kMaxSplit, nt_min), sms / rem);
@@ -1263,10 +1195,63 @@ AttnPlan attn_plan(const AttnParams& p, int dh, int sms) {
       r.whole = r.pairs - rem;
       r.tail_split = s;
       r.partial_bytes = (size_t)rem * s * 2 * (dh + 2) * kBM * sizeof(float);
-      r.counter_bytes = (size_t)rem * 2 * sizeof(int);   // one per split pair and group
     }
   }
   return r;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Merge of split pairs: the pieces' (O, m, l) of each row, combined in piece order, normalised and
+// written to the row of Op.
+// ---------------------------------------------------------------------------------------------
+// One CTA per (split pair, group, 8-column chunk), one thread per row: O = sum_j 2^(m_j - M) O_j,
+// l = sum_j 2^(m_j - M) l_j with M = max_j m_j; Op row chunk = bf16(O / l). A row whose pieces kept
+// no key (every m_j = -inf) is written as zeros. (A CTA per chunk, rather than per row block, keeps
+// enough loads in flight: one CTA per row block ran latency-bound at a tenth of the L2 bandwidth.)
+template <int DH>
+__global__ void __launch_bounds__(kBM) k_merge_pieces(const float* __restrict__ partial,
+                                                      uint16_t* __restrict__ operm, AttnParams P) {
+  griddep_wait();
+  griddep_launch();
+  constexpr int kSlot = (DH + 2) * kBM;
+  constexpr int kChunks = DH / 8;
+  const int cc = blockIdx.x % kChunks, pg = blockIdx.x / kChunks;
+  const int tp = pg >> 1, grp = pg & 1, row = threadIdx.x;
+  const int pair = P.whole + tp;
+  const int npairs = pairs_per_head(P.N);
+  const int uh = pair / npairs, pq = pair - uh * npairs;
+  const int qrow = pq * 2 * kBM + grp * kBM + row;
+  if (qrow >= P.N) return;
+  const int ns = P.tail_split;
+  const float* first = partial + ((size_t)tp * ns * 2 + grp) * kSlot + row;
+  float m[kMaxSplit], l[kMaxSplit];
+  float M = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kMaxSplit; ++j) {
+    const float* sj = first + (size_t)j * 2 * kSlot;
+    m[j] = j < ns ? __ldg(sj + DH * kBM) : -INFINITY;
+    l[j] = j < ns ? __ldg(sj + (DH + 1) * kBM) : 0.f;
+    M = fmaxf(M, m[j]);
+  }
+  float v[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] = 0.f;
+  float Lsum = 0.f;
+#pragma unroll
+  for (int j = 0; j < kMaxSplit; ++j) {
+    const float f = m[j] == -INFINITY ? 0.f : exp2f(m[j] - M);
+    Lsum += f * l[j];
+    const float* sj = first + (size_t)j * 2 * kSlot + (size_t)cc * 8 * kBM;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] += (j < ns ? __ldg(sj + e * kBM) : 0.f) * f;
+  }
+  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+  uint4 w;
+  w.x = pack_bf16(v[0] * inv, v[1] * inv);
+  w.y = pack_bf16(v[2] * inv, v[3] * inv);
+  w.z = pack_bf16(v[4] * inv, v[5] * inv);
+  w.w = pack_bf16(v[6] * inv, v[7] * inv);
+  reinterpret_cast<uint4*>(operm + ((size_t)uh * P.N + qrow) * DH)[cc] = w;
 }
 
 cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
@@ -1276,6 +1261,15 @@ cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUte
   if (dh == 64 && short_items(p)) return launch_attn_pairs(tq, tk, tv, p, status, st);
   if (dh == 64) return launch_attn_pair<64>(tq, tk, tv, tq, tk, to, to, p, status, st);
   if (dh == 80) return launch_attn_pair<80>(tq, tk, tv, tq_tail, tk_tail, to, to_tail, p, status, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_merge_pieces(const AttnParams& p, int dh, cudaStream_t st) {
+  const int split_pairs = pairs_per_head(p.N) * p.U * p.heads - p.whole;
+  if (p.tail_split <= 1 || split_pairs <= 0) return cudaSuccess;
+  const dim3 grid(2 * split_pairs * (dh / 8));
+  if (dh == 64) return launch_pdl(k_merge_pieces<64>, grid, dim3(kBM), 0, st, p.partial, p.operm, p);
+  if (dh == 80) return launch_pdl(k_merge_pieces<80>, grid, dim3(kBM), 0, st, p.partial, p.operm, p);
   return cudaErrorInvalidValue;
 }
 

@@ -38,12 +38,11 @@ cudaError_t launch_random_score(double* score, long long n, unsigned long long s
 cudaError_t launch_update_magnitude(const uint16_t* delta, double* mag, long long rows, int C,
                                     cudaStream_t st);
 
-// Gathers q, k, v [U, N, heads, dh] into the block-major permuted layout [U*heads, N, dh];
-// also zeroes zero[0, nzero) (the attention's merge counters).
+// Gathers q, k, v [U, N, heads, dh] into the block-major permuted layout [U*heads, N, dh].
 cudaError_t launch_gather_qkv(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                               const int32_t* perm, uint16_t* qp, uint16_t* kp, uint16_t* vp,
-                              int U, int N, int heads, int dh, int b, int* zero, int nzero,
-                              int* status, cudaStream_t st);
+                              int U, int N, int heads, int dh, int b, int* status,
+                              cudaStream_t st);
 
 struct AttnParams {
   const int32_t* perm;   // [U, N]
@@ -54,7 +53,6 @@ struct AttnParams {
   int whole;             // pair kernel: pairs processed whole (the rest are split)
   int tail_split;        // pair kernel: pieces per split pair
   float* partial;        // per split piece and group, fp32 O [dh][128], m [128], l [128]
-  int* counters;         // per split pair and group, finished pieces; zero between launches
   uint16_t* operm;       // pair kernel output: [U*heads, N, dh] in block-major permuted order
 };
 // Which attention kernel a shape takes, and the scratch beyond the gathered Q, K, V it needs
@@ -62,17 +60,21 @@ struct AttnParams {
 struct AttnPlan {
   bool pair_kernel;      // the pair kernel (else the short-item kernel)
   int pairs, whole, tail_split;
-  size_t partial_bytes, counter_bytes;
+  size_t partial_bytes;
 };
 AttnPlan attn_plan(const AttnParams& p, int dh, int sms);
 // Block-sparse attention over the gathered sequences (tensor maps over [U*heads, N, dh]; the
 // tails cover columns 64..79 at head dim 80). The pair kernel writes its output, permuted, through
-// `to` / `to_tail` (maps over p.operm laid out like Q); launch_unpermute_out then scatters it to
+// `to` / `to_tail` (maps over p.operm laid out like Q), except the rows of split pairs, which
+// launch_merge_pieces writes from the pieces' partials; launch_unpermute_out then scatters Op to
 // p.out. The short-item kernel writes p.out itself.
 cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                         const CUtensorMap* tq_tail, const CUtensorMap* tk_tail,
                         const CUtensorMap* to, const CUtensorMap* to_tail, const AttnParams& p,
                         int dh, int* status, cudaStream_t st);
+// Rows of Op for the split pairs: the pieces' (O, m, l) in p.partial combined and normalised
+// (nothing when the plan splits no pair).
+cudaError_t launch_merge_pieces(const AttnParams& p, int dh, cudaStream_t st);
 // out[u, perm[u][p(q)], h, :] = op[u*heads + h, q, :] for every block-major position q.
 cudaError_t launch_unpermute_out(const uint16_t* op, const int32_t* perm, uint16_t* out, int U,
                                  int N, int heads, int dh, int b, int* status, cudaStream_t st);
