@@ -388,6 +388,120 @@ def update_magnitude(delta) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------------------------
+# The full encoder block around S3 and S4, and the encoder stack
+# ---------------------------------------------------------------------------------------------
+# The pages patch SparseSAM into SAM's image encoder without retraining (README, "SparseSAM":
+# "patched on top of the original checkpoints"), so the block around S3 and S4 is SAM's ViT block
+# (Kirillov et al., "Segment Anything", 2023, image encoder: a ViT with 14x14 windowed blocks and a
+# few global blocks): pre-norm, x = x + proj(attn(LN1(x))), x = x + MLP(LN2(x)). Readings of what
+# the pages leave open: LayerNorm eps 1e-6 (SAM's encoder); the windowed blocks pad the normalised
+# grid bottom/right with zero rows up to a multiple of the window and crop the attention branch
+# back before the residual add; the qkv projection's 3C output columns are ordered (q|k|v, head,
+# channel); the relative-position bias is left out (it is a separate row); the RC-MLP keeps its
+# residual rows exactly (Dutch summary, "Residual-Consistency MLP"), so the MLP branch, LN2
+# included, runs on the kept rows only.
+LN_EPS = 1e-6
+
+
+def layer_norm(x, weight, bias, eps: float = LN_EPS) -> np.ndarray:
+    """LayerNorm over the last axis in float64: (x - mean) / sqrt(var + eps) * weight + bias, with
+    the mean and the (biased) variance of each row."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * np.asarray(weight, np.float64) + np.asarray(bias, np.float64)
+
+
+def to_units(x: np.ndarray, geo: Geometry) -> np.ndarray:
+    """[B, T, C] -> [U, N, C]: each attention unit's rows in enumeration order (unit_members); a
+    pad token's row is zero."""
+    out = np.zeros((geo.units, geo.unit_tokens, x.shape[-1]), dtype=np.float64)
+    for u, (b, ids) in enumerate(unit_members(geo)):
+        real = ids >= 0
+        out[u, real] = x[b, ids[real]]
+    return out
+
+
+def from_units(a: np.ndarray, geo: Geometry) -> np.ndarray:
+    """[U, N, C] -> [B, T, C]: the rows of real tokens back at their image positions (pads
+    dropped)."""
+    out = np.zeros((geo.batch, geo.grid_h * geo.grid_w, a.shape[-1]), dtype=np.float64)
+    for u, (b, ids) in enumerate(unit_members(geo)):
+        real = ids >= 0
+        out[b, ids[real]] = a[u, real]
+    return out
+
+
+@dataclass
+class BlockParams:
+    """One encoder block's weights (torch Linear convention: w [out, in]). Biases may be None."""
+    ln1_w: np.ndarray
+    ln1_b: np.ndarray
+    w_qkv: np.ndarray      # [3C, C]
+    b_qkv: np.ndarray
+    w_proj: np.ndarray     # [C, C]
+    b_proj: np.ndarray
+    ln2_w: np.ndarray
+    ln2_b: np.ndarray
+    w1: np.ndarray         # [hidden, C]
+    b1: np.ndarray
+    w2: np.ndarray         # [C, hidden]
+    b2: np.ndarray
+
+
+def _lin(x, w, b):
+    y = x @ np.asarray(w, np.float64).T
+    return y if b is None else y + np.asarray(b, np.float64)
+
+
+def encoder_block(x, prm: BlockParams, perm, keep, geo: Geometry, heads: int,
+                  density: float) -> np.ndarray:
+    """One SparseSAM encoder block, float64 [B, T, C]:
+        a  = Stripe-Sort attention (S3) of qkv(LN1(x)) over the block's units,
+        x1 = x + proj(a)                      (pad rows cropped),
+        y  = x1; y[t] = x1[t] + MLP(LN2(x1[t])) for t in keep (S4's keep-set).
+    perm: [U, N] of the block's geometry (window or global); keep: [B, K]."""
+    x = np.asarray(x, dtype=np.float64)
+    C = x.shape[-1]
+    dh = C // heads
+    xu = to_units(layer_norm(x, prm.ln1_w, prm.ln1_b), geo)
+    qkv = _lin(xu, prm.w_qkv, prm.b_qkv)                                 # [U, N, 3C]
+    U, N, _ = qkv.shape
+    q, k, v = (qkv[..., i * C:(i + 1) * C].reshape(U, N, heads, dh) for i in range(3))
+    a = attention(q, k, v, perm, density).reshape(U, N, C)
+    x1 = x + from_units(_lin(a, prm.w_proj, prm.b_proj), geo)
+    y = x1.copy()
+    for b in range(x.shape[0]):
+        rows = np.asarray(keep[b], dtype=np.int64)
+        if rows.size == 0:
+            continue
+        h = gelu(_lin(layer_norm(x1[b, rows], prm.ln2_w, prm.ln2_b), prm.w1, prm.b1))
+        y[b, rows] = x1[b, rows] + _lin(h, prm.w2, prm.b2)
+    return y
+
+
+def encoder_stack(x, blocks, lum, grid_window: int, global_blocks, heads: int,
+                  density: float) -> np.ndarray:
+    """The encoder's blocks in order over x [B, T, C]. One Sobel score per image ranks its tokens
+    once (S1); the global blocks take the image's stripe-sort permutation, the windowed blocks the
+    per-window permutations of the same scores, and every block the same keep-set (S2, S4).
+    global_blocks: indices of the global-attention blocks; the others are windowed."""
+    B, Hg, Wg = np.asarray(lum).shape
+    score = sobel_score(lum)
+    geo_g = Geometry(B, Hg, Wg, "global", grid_window)
+    geo_w = Geometry(B, Hg, Wg, "window", grid_window)
+    perm_g, _ = stripe_sort(score, geo_g)
+    perm_w, _ = stripe_sort(score, geo_w)
+    keep = keep_list(score, density)
+    y = np.asarray(x, dtype=np.float64)
+    for i, prm in enumerate(blocks):
+        g = i in global_blocks
+        y = encoder_block(y, prm, perm_g if g else perm_w, keep, geo_g if g else geo_w, heads,
+                          density)
+    return y
+
+
+# ---------------------------------------------------------------------------------------------
 # The whole block, for the smoke check and the CPU baseline
 # ---------------------------------------------------------------------------------------------
 def hot_path(lum, q, k, v, x, w1, b1, w2, b2, geo: Geometry, density: float):

@@ -10,7 +10,10 @@ Recipe:
     regions with edges, like a natural image's luminance at token resolution.
   * q, k, v ~ N(0,1) · qkv_scale, layout [U, N, heads, dh].
   * x ~ N(0,1) [B, Hg·Wg, C]; W1 [hidden, C] and W2 [C, hidden] ~ N(0, 0.02); biases 0 unless asked.
-Every tensor has its own stream: numpy PCG64 seeded with (workload seed, tensor tag).
+  * full encoder blocks (block_params): every Linear weight [out, in] ~ N(0, 1/in) (so that each
+    branch of the block adds O(1) values to the residual stream), its bias ~ N(0, 0.1^2); LayerNorm
+    weights ~ 1 + N(0, 0.1^2), LayerNorm biases ~ N(0, 0.1^2).
+Every tensor has its own stream: numpy PCG64 seeded with (workload seed, tensor tag[, block]).
 """
 from __future__ import annotations
 
@@ -19,11 +22,14 @@ import torch
 
 from .workloads import Workload
 
-_TAGS = {"lum": 1, "q": 2, "k": 3, "v": 4, "x": 5, "w1": 6, "b1": 7, "w2": 8, "b2": 9}
+_TAGS = {"lum": 1, "q": 2, "k": 3, "v": 4, "x": 5, "w1": 6, "b1": 7, "w2": 8, "b2": 9,
+         "ln1_w": 10, "ln1_b": 11, "w_qkv": 12, "b_qkv": 13, "w_proj": 14, "b_proj": 15,
+         "ln2_w": 16, "ln2_b": 17}
 
 
-def rng(seed: int, tag: str) -> np.random.Generator:
-    return np.random.default_rng([int(seed), _TAGS[tag]])
+def rng(seed: int, tag: str, block: int | None = None) -> np.random.Generator:
+    key = [int(seed), _TAGS[tag]] + ([] if block is None else [int(block)])
+    return np.random.default_rng(key)
 
 
 def luminance(wl: Workload, seed: int | None = None, discs: int = 12, noise: float = 0.05) -> np.ndarray:
@@ -71,6 +77,29 @@ def mlp_params(wl: Workload, seed: int | None = None, bias_scale: float = 0.0):
         b1 = np.zeros((wl.hidden,), np.float32)
         b2 = np.zeros((wl.dim,), np.float32)
     return x, w1, b1, w2, b2
+
+
+BLOCK_PARAM_NAMES = ("ln1_w", "ln1_b", "w_qkv", "b_qkv", "w_proj", "b_proj", "ln2_w", "ln2_b",
+                     "w1", "b1", "w2", "b2")
+
+
+def block_params(dim: int, hidden: int, seed: int, block: int) -> dict:
+    """One encoder block's weights as fp32 arrays, keyed by BLOCK_PARAM_NAMES (Linear weights in
+    the [out, in] convention; w_qkv's 3*dim rows are ordered q, k, v)."""
+    shapes = {"w_qkv": (3 * dim, dim), "w_proj": (dim, dim), "w1": (hidden, dim), "w2": (dim, hidden)}
+    out = {}
+    for name in BLOCK_PARAM_NAMES:
+        g = rng(seed, name, block)
+        if name in shapes:
+            shp = shapes[name]
+            a = g.standard_normal(size=shp, dtype=np.float32) * np.float32(1.0 / np.sqrt(shp[1]))
+        else:
+            n = {"b_qkv": 3 * dim, "b1": hidden}.get(name, dim)
+            a = g.standard_normal(size=(n,), dtype=np.float32) * np.float32(0.1)
+            if name.endswith("_w"):
+                a = a + np.float32(1.0)
+        out[name] = a.astype(np.float32)
+    return out
 
 
 def to_bf16(a: np.ndarray) -> torch.Tensor:
