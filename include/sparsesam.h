@@ -9,6 +9,8 @@
  *   sparsesam_perm   S2  stable sort by score + stripe transpose -> permutation; top-K keep list
  *   sparsesam_score_perm  S1 + S2 in one pass (the same results, one launch fewer)
  *   sparsesam_block       S1..S4 in one call with one workspace
+ *   sparsesam_encoder_block  a full encoder block: LN1, qkv, S3, proj, residual, LN2 + S4
+ *   sparsesam_encoder_stack  the encoder's blocks in order over one ranking of the tokens
  *   sparsesam_attn   S3  static block-sparse attention over the permuted sequence
  *   sparsesam_rcmlp  S4  fc1-GELU-fc2 on the kept tokens, added to the residual in place
  *   sparsesam_random_perm     S2 over random scores (the random-permutation ablation)
@@ -213,6 +215,67 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
                     const uint16_t* b1, const uint16_t* w2, const uint16_t* b2, double* score,
                     int32_t* perm, int32_t* inv, int32_t* keep, uint16_t* out, void* ws,
                     size_t ws_bytes, void* stream);
+
+/* One encoder block's weights (device pointers, bf16, 16-byte aligned; Linear weights in the
+ * PyTorch nn.Linear [out, in] layout, row-major). The Linear biases may be NULL (zero); the
+ * LayerNorm weight and bias may not. */
+typedef struct {
+  const uint16_t* ln1_w;    /* [C]        LayerNorm before the attention */
+  const uint16_t* ln1_b;    /* [C] */
+  const uint16_t* w_qkv;    /* [3C, C]    rows: q (C), k (C), v (C); within each, head-major */
+  const uint16_t* b_qkv;    /* [3C] */
+  const uint16_t* w_proj;   /* [C, C]     the attention's output projection */
+  const uint16_t* b_proj;   /* [C] */
+  const uint16_t* ln2_w;    /* [C]        LayerNorm before the MLP */
+  const uint16_t* ln2_b;    /* [C] */
+  const uint16_t* w1;       /* [hidden, C] */
+  const uint16_t* b1;       /* [hidden] */
+  const uint16_t* w2;       /* [C, hidden] */
+  const uint16_t* b2;       /* [C] */
+} ss_block_weights;
+
+/* Bytes of device workspace sparsesam_encoder_block needs for K kept tokens per image (0 on
+ * invalid arguments). */
+size_t sparsesam_encoder_block_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden, int32_t K);
+
+/* One full SparseSAM encoder block, in place on x (device) bf16 [batch, grid_h*grid_w, C]. The
+ * pages patch SparseSAM into SAM's image encoder (README, "SparseSAM": on top of the original
+ * checkpoints), so the block is SAM's pre-norm ViT block with S3 as its attention and S4 as its MLP:
+ *   a  = S3 attention of qkv(LN1(x)) over the cfg's units (window mode: the normalised grid padded
+ *        bottom/right with zero rows to whole windows), heads = cfg->heads, head_dim = C / heads;
+ *   x1 = x + proj(a)   (rows of pad tokens dropped);
+ *   x  = x1, and for each kept token t of image b: x[b,t] = x1[b,t] + fc2(GELU(fc1(LN2(x1[b,t])))).
+ * LayerNorm: (v - mean) / sqrt(var + 1e-6) * weight + bias with the biased variance, fp32
+ * statistics. perm, inv (device) int32 [U, N]: the cfg's stripe-sort permutation and its inverse
+ * (sparsesam_score_perm with the same cfg); keep (device) int32 [batch, K], 0 <= K <=
+ * grid_h*grid_w, as for sparsesam_rcmlp. C = heads * head_dim (head_dim 64 or 80), C and hidden
+ * multiples of 64. bf16 operands and activations between the steps (LN outputs, q/k/v, the
+ * attention output, x1, the MLP's hidden activation), fp32 accumulation and softmax. ws (device,
+ * 256-byte aligned) >= sparsesam_encoder_block_workspace(cfg, C, hidden, K) bytes; its contents on
+ * entry do not matter. Errors: SS_EINVAL (NULL or misaligned pointer, C != heads*head_dim, K out
+ * of range), SS_EUNSUPPORTED (head_dim, C or hidden not a multiple of 64, N % 4, sizes beyond the
+ * launch limits), SS_EWORKSPACE; a perm/inv/keep entry out of range records SS_EINDEX and skips
+ * that row. */
+int sparsesam_encoder_block(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden,
+                            const ss_block_weights* w, const int32_t* perm, const int32_t* inv,
+                            const int32_t* keep, int32_t K, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* Bytes of device workspace sparsesam_encoder_stack needs (0 on invalid arguments). */
+size_t sparsesam_encoder_stack_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden);
+
+/* The encoder's n_blocks blocks in order, in place on x (device) bf16 [batch, grid_h*grid_w, C].
+ * The tokens are ranked once (Dutch summary, "Methodologie": one precomputed permutation set is
+ * reused by every layer; here S1 + S2 of lum): the global blocks (is_global[i] != 0) use the whole-image stripe-sort permutation, the
+ * windowed blocks the per-window permutations (window = cfg->window) of the same scores, and every
+ * block the keep-set of K = ceil(density * grid_h*grid_w) tokens per image. cfg->mode is ignored.
+ * w (host) [n_blocks] and is_global (host) [n_blocks]; each block as sparsesam_encoder_block.
+ * ws (device, 256-byte aligned) >= sparsesam_encoder_stack_workspace(cfg, C, hidden) bytes; it
+ * holds the scores, both permutations, the keep list and one block's workspace, reused by every
+ * block. Errors as for sparsesam_encoder_block, for either geometry. */
+int sparsesam_encoder_stack(const ss_cfg* cfg, const float* lum, uint16_t* x, int32_t C,
+                            int32_t hidden, int32_t n_blocks, const ss_block_weights* w,
+                            const uint8_t* is_global, void* ws, size_t ws_bytes, void* stream);
 
 /* S4 without a caller-provided workspace. The SparseSAM pages have no counterpart to this call;
  * it exists for callers that cannot allocate device memory where they run the block: code inside

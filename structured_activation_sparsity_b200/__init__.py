@@ -1,7 +1,8 @@
 """SparseSAM encoder-block hot path on B200 (sm_100a).
 
 The four steps -- Sobel score, stripe-sort permutation, Stripe-Sort block-sparse attention and the
-Residual-Consistency MLP -- run in the C-ABI library libsparsesam.so (include/sparsesam.h). This
+Residual-Consistency MLP -- run in the C-ABI library libsparsesam.so (include/sparsesam.h), as
+separate calls, as one call per block, and inside full SAM encoder blocks and the encoder stack. This
 package is its thin Python binding (`_lib`), plus the synthetic workload shapes and input
 generators used by the tests and the benchmark.
 
@@ -18,7 +19,9 @@ _LIB_NAMES = {
     "sparsesam_device_status", "sparsesam_launch_count", "sparsesam_pattern", "sparsesam_perm",
     "sparsesam_rcmlp", "sparsesam_rcmlp_noalloc", "sparsesam_rcmlp_workspace", "sparsesam_score",
     "sparsesam_score_perm", "sparsesam_block", "sparsesam_block_workspace",
-    "sparsesam_random_perm", "sparsesam_keep_by_update",
+    "sparsesam_random_perm", "sparsesam_keep_by_update", "SsBlockWeights", "block_weights",
+    "sparsesam_encoder_block", "sparsesam_encoder_block_workspace", "sparsesam_encoder_stack",
+    "sparsesam_encoder_stack_workspace",
     "sparsesam_trace_start", "sparsesam_trace_stop", "strerror",
 }
 

@@ -36,6 +36,14 @@ class SsPattern(ctypes.Structure):
                 ("nnz", ctypes.c_int32), ("keep", ctypes.c_int32), ("rho", ctypes.c_double)]
 
 
+BLOCK_WEIGHT_FIELDS = ("ln1_w", "ln1_b", "w_qkv", "b_qkv", "w_proj", "b_proj", "ln2_w", "ln2_b",
+                       "w1", "b1", "w2", "b2")
+
+
+class SsBlockWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in BLOCK_WEIGHT_FIELDS]
+
+
 class SparseSAMError(RuntimeError):
     def __init__(self, fn: str, code: int):
         self.code = code
@@ -66,6 +74,12 @@ def _load():
         "sparsesam_rcmlp_workspace": (SZ, [cfgp, I32, I32, I32]),
         "sparsesam_rcmlp": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, I32, P, SZ, VP]),
         "sparsesam_rcmlp_noalloc": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, I32, VP]),
+        "sparsesam_encoder_block_workspace": (SZ, [cfgp, I32, I32, I32]),
+        "sparsesam_encoder_block": (ctypes.c_int, [cfgp, P, I32, I32, ctypes.POINTER(SsBlockWeights),
+                                                   P, P, P, I32, P, SZ, VP]),
+        "sparsesam_encoder_stack_workspace": (SZ, [cfgp, I32, I32]),
+        "sparsesam_encoder_stack": (ctypes.c_int, [cfgp, P, P, I32, I32, I32,
+                                                   ctypes.POINTER(SsBlockWeights), P, P, SZ, VP]),
         "sparsesam_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
         "sparsesam_wait_selftest": (ctypes.c_int, [I32, VP]),
         "sparsesam_device_status": (ctypes.c_int, [ctypes.POINTER(I32), VP]),
@@ -220,6 +234,46 @@ def sparsesam_rcmlp_noalloc(cfg, x, C, hidden, w1, b1, w2, b2, keep, K, stream=N
                   lib.sparsesam_rcmlp_noalloc(ctypes.byref(cfg), _ptr(x), int(C), int(hidden),
                                               _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(keep),
                                               int(K), _stream(stream)))
+
+
+def block_weights(w) -> SsBlockWeights:
+    """An ss_block_weights of device pointers from a mapping name -> tensor (or None / address)."""
+    return SsBlockWeights(**{n: _ptr(w.get(n)) for n in BLOCK_WEIGHT_FIELDS})
+
+
+def sparsesam_encoder_block_workspace(cfg, C, hidden, K) -> int:
+    return int(lib.sparsesam_encoder_block_workspace(ctypes.byref(cfg), int(C), int(hidden), int(K)))
+
+
+def sparsesam_encoder_block(cfg, x, C, hidden, weights, perm, inv, keep, K, ws, ws_bytes,
+                            stream=None):
+    """One full encoder block in place on x; weights: an SsBlockWeights or a mapping name ->
+    tensor."""
+    w = weights if isinstance(weights, SsBlockWeights) else block_weights(weights)
+    return _check("sparsesam_encoder_block",
+                  lib.sparsesam_encoder_block(ctypes.byref(cfg), _ptr(x), int(C), int(hidden),
+                                              ctypes.byref(w), _ptr(perm), _ptr(inv), _ptr(keep),
+                                              int(K), _ptr(ws), int(ws_bytes), _stream(stream)))
+
+
+def sparsesam_encoder_stack_workspace(cfg, C, hidden) -> int:
+    return int(lib.sparsesam_encoder_stack_workspace(ctypes.byref(cfg), int(C), int(hidden)))
+
+
+def sparsesam_encoder_stack(cfg, lum, x, C, hidden, weights, is_global, ws, ws_bytes,
+                            stream=None):
+    """The encoder's blocks in order over x; weights: a list of SsBlockWeights or mappings,
+    is_global: one flag per block."""
+    n = len(weights)
+    if len(is_global) != n:
+        raise ValueError("one is_global flag per block")
+    arr = (SsBlockWeights * max(n, 1))(*[w if isinstance(w, SsBlockWeights) else block_weights(w)
+                                          for w in weights])
+    flags = (ctypes.c_uint8 * max(n, 1))(*[1 if g else 0 for g in is_global])
+    return _check("sparsesam_encoder_stack",
+                  lib.sparsesam_encoder_stack(ctypes.byref(cfg), _ptr(lum), _ptr(x), int(C),
+                                              int(hidden), n, arr, ctypes.addressof(flags),
+                                              _ptr(ws), int(ws_bytes), _stream(stream)))
 
 
 def sparsesam_set_wait_limit_ns(ns: int):

@@ -675,6 +675,252 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
   return rcmlp_launch(g, K, x, C, hidden, w1, b1, w2, b2, keep, wsm, status, st);
 }
 
+// ---- the full encoder block -----------------------------------------------------------------
+
+static UnitRows unit_rows_of(const Geo& g) {
+  UnitRows r;
+  r.N = g.N;
+  r.T = g.T;
+  r.grid_w = g.Wg;
+  r.grid_h = g.Hg;
+  r.window = g.window_mode ? g.ws : 0;
+  r.win_per_row = g.wpr;
+  r.windows = g.windows;
+  return r;
+}
+
+// The encoder block's workspace: LN1's output over the units [U*N, C] (later the attention's
+// output, which the projection reads), the attention's workspace (the qkv GEMM writes the gathered
+// Q, K, V into it), the qkv and proj GEMMs' k-split scratch, then the RC-MLP's workspace.
+struct EncLayout {
+  AttnLayout L;
+  GemmPlan qkv, proj;
+  MlpPlan mlp;
+  size_t attn, gemm_partial, gemm_counters, mlp_base, total;   // byte offsets, total size
+};
+
+static int enc_layout(const ss_cfg* cfg, const Geo& g, int C, int hidden, int K, EncLayout* E) {
+  int rc = attn_layout(cfg, g, &E->L);
+  if (rc) return rc;
+  const long long M = (long long)g.U * g.N;
+  E->qkv = gemm_plan((int)M, 3 * C, C, kPlanSMs);
+  E->proj = gemm_plan((int)M, C, C, kPlanSMs);
+  const size_t p1 = gemm_partial_bytes(E->qkv), p2 = gemm_partial_bytes(E->proj);
+  const size_t part = align256(p1 > p2 ? p1 : p2);
+  const int t1 = E->qkv.m_tiles * E->qkv.n_tiles, t2 = E->proj.m_tiles * E->proj.n_tiles;
+  const size_t cnt = part ? align256((size_t)(t1 > t2 ? t1 : t2) * 2 * 4) : 0;
+  E->mlp = mlp_plan(g, K, C, hidden);
+  E->attn = align256((size_t)M * C * 2);
+  E->gemm_partial = E->attn + align256(E->L.total);
+  E->gemm_counters = E->gemm_partial + part;
+  E->mlp_base = E->gemm_counters + cnt;
+  E->total = E->mlp_base + (K > 0 ? E->mlp.total : 0);
+  return SS_OK;
+}
+
+static int enc_check(const ss_cfg* cfg, const Geo& g, const uint16_t* x, int32_t C,
+                     int32_t hidden, const ss_block_weights* w, const int32_t* perm,
+                     const int32_t* inv, const int32_t* keep, int32_t K) {
+  if (cfg->heads < 1 || cfg->head_dim < 1 || C < 1 || hidden < 1) return SS_EINVAL;
+  if (cfg->head_dim != 64 && cfg->head_dim != 80) return SS_EUNSUPPORTED;
+  if ((int64_t)cfg->heads * cfg->head_dim != C) return SS_EINVAL;
+  if (C % 64 != 0 || hidden % 64 != 0) return SS_EUNSUPPORTED;
+  if (!x || !w || !perm || !inv || K < 0 || K > g.T || (K > 0 && !keep)) return SS_EINVAL;
+  if (!w->ln1_w || !w->ln1_b || !w->w_qkv || !w->w_proj || !w->ln2_w || !w->ln2_b || !w->w1 ||
+      !w->w2)
+    return SS_EINVAL;
+  const void* al[] = {x, w->ln1_w, w->ln1_b, w->w_qkv, w->b_qkv, w->w_proj, w->b_proj,
+                      w->ln2_w, w->ln2_b, w->w1, w->b1, w->w2, w->b2};
+  for (const void* a : al)
+    if (!aligned(a, 16)) return SS_EINVAL;
+  ss_pattern p;
+  int rc = pattern_of(cfg, g, &p);
+  if (rc) return rc;
+  const int64_t M = (int64_t)g.U * g.N, Mk = (int64_t)g.B * K;
+  if ((int64_t)g.U * cfg->heads > 65535) return SS_EUNSUPPORTED;
+  if (M * 3 * C >= ((int64_t)1 << 31) || (M + 127) / 128 > 65535) return SS_EUNSUPPORTED;
+  if (Mk * (hidden > C ? hidden : C) >= ((int64_t)1 << 31) || (Mk + 127) / 128 > 65535)
+    return SS_EUNSUPPORTED;
+  if ((int64_t)g.B * g.T * C >= ((int64_t)1 << 31)) return SS_EUNSUPPORTED;
+  return SS_OK;
+}
+
+// LN1 -> qkv GEMM (straight into the gathered layout) -> attention -> proj GEMM (+ residual, pads
+// dropped) -> LN2 over the kept rows -> fc1 -> fc2 (+ residual). ws laid out as enc_layout says.
+static int enc_launch(const ss_cfg* cfg, const Geo& g, const EncLayout& E, uint16_t* x, int C,
+                      int hidden, const ss_block_weights* w, const int32_t* perm,
+                      const int32_t* inv, const int32_t* keep, int K, uint8_t* ws, int* status,
+                      cudaStream_t st) {
+  const long long M = (long long)g.U * g.N;
+  const UnitRows ur = unit_rows_of(g);
+  uint16_t* xn = reinterpret_cast<uint16_t*>(ws);
+  uint8_t* wsa = ws + E.attn;
+  float* partial = reinterpret_cast<float*>(ws + E.gemm_partial);
+  int* counters = reinterpret_cast<int*>(ws + E.gemm_counters);
+  const int n_counters = (int)((E.mlp_base - E.gemm_counters) / sizeof(int));
+  const int sms = sm_count();
+  int rc = cuda_err(traced("ln1", st, [&] {
+    return launch_ln_rows(x, w->ln1_w, w->ln1_b, xn, M, C, ur, nullptr, 0, counters, n_counters,
+                          status, st);
+  }));
+  if (rc) return rc;
+  CUtensorMap ta, tb, tp;
+  if (!encode_bf16(&ta, 2, xn, C, M, 1, (uint64_t)C * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16(&tb, 2, w->w_qkv, C, 3 * C, 1, (uint64_t)C * 2, 64, E.qkv.bn,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16(&tp, 2, w->w_proj, C, C, 1, (uint64_t)C * 2, 64, E.proj.bn,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return SS_ECUDA;
+  GemmEpilogue eq = {};
+  eq.kind = 2;
+  eq.bias = w->b_qkv;
+  eq.out = reinterpret_cast<uint16_t*>(wsa);
+  eq.inv = inv;
+  eq.which_stride = (long long)(E.L.one / 2);
+  eq.heads = cfg->heads;
+  eq.dh = cfg->head_dim;
+  eq.C = C;
+  eq.b = E.L.ap.b;
+  eq.L = E.L.ap.L;
+  eq.ur = ur;
+  rc = cuda_err(traced("qkv", st, [&] {
+    return launch_gemm(&ta, &tb, E.qkv, (int)M, 3 * C, C, eq, partial, counters, sms, status, st);
+  }));
+  if (rc) return rc;
+  // The attention writes its [U, N, heads, dh] output over LN1's rows, which the qkv GEMM has
+  // finished reading: each launch of the chain starts its work only after the previous one has
+  // completed.
+  if ((rc = attn_launch(cfg, g, E.L, wsa, perm, xn, status, st))) return rc;
+  GemmEpilogue ep = {};
+  ep.kind = 3;
+  ep.bias = w->b_proj;
+  ep.x = x;
+  ep.ur = ur;
+  rc = cuda_err(traced("proj", st, [&] {
+    return launch_gemm(&ta, &tp, E.proj, (int)M, C, C, ep, partial, counters, sms, status, st);
+  }));
+  if (rc || K == 0) return rc;
+  uint8_t* wsm = ws + E.mlp_base;
+  const int n_mlp_counters = (int)((E.mlp.total - E.mlp.counters) / sizeof(int));
+  rc = cuda_err(traced("ln2_rows", st, [&] {
+    return launch_ln_rows(x, w->ln2_w, w->ln2_b, reinterpret_cast<uint16_t*>(wsm + E.mlp.xk),
+                          (long long)g.B * K, C, ur, keep, K,
+                          reinterpret_cast<int*>(wsm + E.mlp.counters), n_mlp_counters, status,
+                          st);
+  }));
+  if (rc) return rc;
+  return rcmlp_launch(g, K, x, C, hidden, w->w1, w->b1, w->w2, w->b2, keep, wsm, status, st);
+}
+
+size_t sparsesam_encoder_block_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden, int32_t K) {
+  Geo g;
+  EncLayout E;
+  if (geometry(cfg, &g) || cfg->heads < 1 || cfg->head_dim < 1 || C < 1 || hidden < 1 || K < 0 ||
+      K > g.T || enc_layout(cfg, g, C, hidden, K, &E))
+    return 0;
+  return E.total;
+}
+
+int sparsesam_encoder_block(const ss_cfg* cfg, uint16_t* x, int32_t C, int32_t hidden,
+                            const ss_block_weights* w, const int32_t* perm, const int32_t* inv,
+                            const int32_t* keep, int32_t K, void* ws, size_t ws_bytes,
+                            void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  if ((rc = enc_check(cfg, g, x, C, hidden, w, perm, inv, keep, K))) return rc;
+  EncLayout E;
+  if ((rc = enc_layout(cfg, g, C, hidden, K, &E))) return rc;
+  if (!ws || !aligned(ws, 256) || ws_bytes < E.total) return SS_EWORKSPACE;
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+  return enc_launch(cfg, g, E, x, C, hidden, w, perm, inv, keep, K, static_cast<uint8_t*>(ws),
+                    status, static_cast<cudaStream_t>(stream));
+}
+
+// ---- the encoder stack ------------------------------------------------------------------------
+
+// The stack's workspace: scores, both permutations with their inverses, the keep list, then one
+// encoder block's workspace (the larger of the two geometries'), reused by every block.
+struct StackLayout {
+  ss_cfg cg, cw;       // the global and the windowed blocks' cfg
+  Geo gg, gw;
+  EncLayout eg, ew;
+  int K;
+  size_t score, perm_g, inv_g, perm_w, inv_w, keep, block, total;
+};
+
+static int stack_layout(const ss_cfg* cfg, int C, int hidden, StackLayout* S) {
+  if (!cfg) return SS_EINVAL;
+  S->cg = *cfg;
+  S->cg.mode = SS_GLOBAL;
+  S->cw = *cfg;
+  S->cw.mode = SS_WINDOW;
+  int rc = geometry(&S->cg, &S->gg);
+  if (rc || (rc = geometry(&S->cw, &S->gw))) return rc;
+  if (cfg->heads < 1 || cfg->head_dim < 1 || C < 1 || hidden < 1) return SS_EINVAL;
+  S->K = keep_count(cfg->density, S->gg.T);
+  if ((rc = enc_layout(&S->cg, S->gg, C, hidden, S->K, &S->eg)) ||
+      (rc = enc_layout(&S->cw, S->gw, C, hidden, S->K, &S->ew)))
+    return rc;
+  const size_t BT = (size_t)S->gg.B * S->gg.T, UNw = (size_t)S->gw.U * S->gw.N;
+  S->score = 0;
+  S->perm_g = align256(BT * 8);
+  S->inv_g = S->perm_g + align256(BT * 4);
+  S->perm_w = S->inv_g + align256(BT * 4);
+  S->inv_w = S->perm_w + align256(UNw * 4);
+  S->keep = S->inv_w + align256(UNw * 4);
+  S->block = S->keep + align256((size_t)S->gg.B * (S->K > 0 ? S->K : 1) * 4);
+  S->total = S->block + (S->eg.total > S->ew.total ? S->eg.total : S->ew.total);
+  return SS_OK;
+}
+
+size_t sparsesam_encoder_stack_workspace(const ss_cfg* cfg, int32_t C, int32_t hidden) {
+  StackLayout S;
+  return stack_layout(cfg, C, hidden, &S) ? 0 : S.total;
+}
+
+int sparsesam_encoder_stack(const ss_cfg* cfg, const float* lum, uint16_t* x, int32_t C,
+                            int32_t hidden, int32_t n_blocks, const ss_block_weights* w,
+                            const uint8_t* is_global, void* ws, size_t ws_bytes, void* stream) {
+  StackLayout S;
+  int rc = stack_layout(cfg, C, hidden, &S);
+  if (rc) return rc;
+  if (!lum || n_blocks < 0 || (n_blocks > 0 && (!w || !is_global))) return SS_EINVAL;
+  if (S.gg.T > kMaxRankTokens || S.gw.N > kMaxRankTokens || S.gw.U > 65535 || S.gg.U > 65535)
+    return SS_EUNSUPPORTED;
+  if (!ws || !aligned(ws, 256) || ws_bytes < S.total) return SS_EWORKSPACE;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  double* score = reinterpret_cast<double*>(wsb + S.score);
+  int32_t* perm_g = reinterpret_cast<int32_t*>(wsb + S.perm_g);
+  int32_t* inv_g = reinterpret_cast<int32_t*>(wsb + S.inv_g);
+  int32_t* perm_w = reinterpret_cast<int32_t*>(wsb + S.perm_w);
+  int32_t* inv_w = reinterpret_cast<int32_t*>(wsb + S.inv_w);
+  int32_t* keep = reinterpret_cast<int32_t*>(wsb + S.keep);
+  // Every block's arguments are checked before the first launch.
+  for (int i = 0; i < n_blocks; ++i) {
+    const bool glob = is_global[i] != 0;
+    rc = enc_check(glob ? &S.cg : &S.cw, glob ? S.gg : S.gw, x, C, hidden, &w[i],
+                   glob ? perm_g : perm_w, glob ? inv_g : inv_w, keep, S.K);
+    if (rc) return rc;
+  }
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = rank_path(&S.cg, lum, nullptr, score, perm_g, inv_g, S.K > 0 ? keep : nullptr,
+                      stream)))
+    return rc;
+  if ((rc = rank_path(&S.cw, nullptr, score, nullptr, perm_w, inv_w, nullptr, stream))) return rc;
+  for (int i = 0; i < n_blocks; ++i) {
+    const bool glob = is_global[i] != 0;
+    rc = enc_launch(glob ? &S.cg : &S.cw, glob ? S.gg : S.gw, glob ? S.eg : S.ew, x, C, hidden,
+                    &w[i], glob ? perm_g : perm_w, glob ? inv_g : inv_w, keep, S.K,
+                    wsb + S.block, status, st);
+    if (rc) return rc;
+  }
+  return SS_OK;
+}
+
 int sparsesam_device_status(int32_t* out, void* stream) {
   if (!out) return SS_EINVAL;
   int* status = status_word();

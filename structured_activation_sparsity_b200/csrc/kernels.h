@@ -86,14 +86,56 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* keep, uint16_t*
                                int K, int C, int* zero, int nzero, int* status, cudaStream_t st,
                                bool late_wait = false);
 
+// Rows of an encoder block's attention units: row m = u*N + i is token i (enumeration order) of
+// unit u. Global blocks: unit u is image u, in raster order. Windowed blocks: the grid is padded
+// bottom/right to whole windows of `window` x `window`, unit u = b*windows + w is window w (row-major
+// over the padded grid) of image b, its tokens row-major; a token in the padding has no image row.
+struct UnitRows {
+  int N, T;               // tokens per unit, tokens per image
+  int grid_w, grid_h;
+  int window;             // 0: global
+  int win_per_row, windows;
+};
+// The image row b*T + t of unit row m, or -1 for a pad token.
+__host__ __device__ inline long long unit_row_src(const UnitRows& r, long long m) {
+  const long long u = m / r.N;
+  const int i = (int)(m - u * r.N);
+  if (!r.window) return u * r.T + i;
+  const long long b = u / r.windows;
+  const int w = (int)(u - b * r.windows);
+  const int y = (w / r.win_per_row) * r.window + i / r.window;
+  const int x = (w % r.win_per_row) * r.window + i % r.window;
+  if (y >= r.grid_h || x >= r.grid_w) return -1;
+  return b * r.T + (long long)y * r.grid_w + x;
+}
+
+// LayerNorm of rows, bf16 in and out, fp32 statistics: out[m] = (x[src] - mean) / sqrt(var + eps)
+// * w + b over the C channels of the source row, or zeros where there is none. keep == null: the
+// source of row m < rows is unit_row_src(ur, m) (a block's LN1 over its units, pads zero); else
+// it is image m / K's token keep[m] (LN2 over the kept rows; an entry outside the image records
+// SS_EINDEX and its row is left unwritten). CTA 0 also zeroes zero[0, nzero).
+cudaError_t launch_ln_rows(const uint16_t* x, const uint16_t* w, const uint16_t* b, uint16_t* out,
+                           long long rows, int C, const UnitRows& ur, const int32_t* keep, int K,
+                           int* zero, int nzero, int* status, cudaStream_t st);
+
 struct GemmEpilogue {
   int kind;                 // 0: out = bf16(GELU(acc + bias)) into out[M, N]
                             // 1: x[b, keep[m], n] = bf16(x + acc + bias)
+                            // 2: the q|k|v columns of unit row m into the block-major permuted
+                            //    layout: out[which][(u*heads + h)*N + q(inv[m]), d] =
+                            //    bf16(acc + bias), q(p) the block-major position of permuted
+                            //    position p (pattern block size b, stripe length L)
+                            // 3: x[unit_row_src(ur, m), n] = bf16(x + acc + bias), pad rows skipped
   const uint16_t* bias;     // [N] or null
-  uint16_t* out;            // kind 0
-  uint16_t* x;              // kind 1: [B, T, N]
+  uint16_t* out;            // kind 0; kind 2: gathered Q (K and V follow at which_stride)
+  uint16_t* x;              // kind 1: [B, T, N]; kind 3: [B*T, N]
   const int32_t* keep;      // kind 1: [B*K]
   int K_per_image, T;       // kind 1
+  const int32_t* inv;       // kind 2: [U*N] permuted position of each unit row
+  long long which_stride;   // kind 2: elements from the gathered Q to K (and K to V)
+  int heads, dh, C;         // kind 2: C = heads*dh columns per q, k, v
+  int b, L;                 // kind 2: the pattern's block size and stripe length
+  UnitRows ur;              // kinds 2 (N) and 3
 };
 // Tile width and k-split of C[M, N] = A[M, Kd] * B[N, Kd]^T for `sms` persistent CTAs.
 // tail: without a k-split, the tiles of a last, partial round of units that are each split in two

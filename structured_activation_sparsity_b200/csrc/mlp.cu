@@ -142,10 +142,25 @@ struct GemmShape {
 // kind 1, the keep lookup behind it) is resolved once per unit; a chunk's bias and residual words
 // are loaded before its accumulator values are needed, so their latency overlaps those reads.
 // Kind 1: a keep entry outside the image gives no row (nullptr: the row is skipped) and records
-// SS_EINDEX.
+// SS_EINDEX; so does, for kind 2, a permuted position outside the unit. Kind 2's row is the unit
+// row's (block-major) place in the gathered Q at head 0; kind 3's a pad token has no row (skipped, no error).
 __device__ __forceinline__ uint16_t* epi_row(const GemmEpilogue& ep, const GemmShape& g, int m,
                                              int* status) {
   if (ep.kind == 0) return ep.out + (size_t)m * g.N;
+  if (ep.kind == 2) {
+    const int N = ep.ur.N;
+    const int u = m / N;
+    const int p = __ldg(ep.inv + m);
+    if ((unsigned)p >= (unsigned)N) {
+      record_bad_index(status);
+      return nullptr;
+    }
+    return ep.out + ((size_t)u * ep.heads * N + canonical_to_blockmajor(p, ep.b, ep.L)) * ep.dh;
+  }
+  if (ep.kind == 3) {
+    const long long src = unit_row_src(ep.ur, m);
+    return src < 0 ? nullptr : ep.x + (size_t)src * g.N;
+  }
   const int b = m / ep.K_per_image;
   const int t = __ldg(ep.keep + m);
   if ((unsigned)t >= (unsigned)ep.T) {
@@ -164,7 +179,7 @@ __device__ __forceinline__ void epi_load(const GemmEpilogue& ep, const uint16_t*
 #pragma unroll
     for (int q = 0; q < 4; ++q) in.b[q] = __ldg(bp + q);
   }
-  if (ep.kind == 1) {
+  if (ep.kind == 1 || ep.kind == 3) {
     const uint4* xp = reinterpret_cast<const uint4*>(row + n);
 #pragma unroll
     for (int q = 0; q < 4; ++q) in.x[q] = xp[q];
@@ -174,7 +189,8 @@ __device__ __forceinline__ void epi_load(const GemmEpilogue& ep, const uint16_t*
 __device__ __forceinline__ void f2_add_bf16(float& v0, float& v1, uint32_t w) {
   f2_unpack(f2_add(f2_pack(v0, v1), f2_pack(bf16_lo(w), bf16_hi(w))), v0, v1);
 }
-// Kind 0: row[n..n+32) = bf16(GELU(v + bias)). Kind 1: row[n..n+32) = bf16(x + v + bias).
+// Kind 0: row[n..n+32) = bf16(GELU(v + bias)). Kinds 1, 3: row[n..n+32) = bf16(x + v + bias).
+// Kind 2: bf16(v + bias), each 16 columns (within one head: dh is a multiple of 16) to its place.
 __device__ __forceinline__ void epi_store(const GemmEpilogue& ep, uint16_t* row, int n,
                                           const Epi32In& in, float (&v)[32]) {
   if (ep.bias) {
@@ -184,6 +200,26 @@ __device__ __forceinline__ void epi_store(const GemmEpilogue& ep, uint16_t* row,
 #pragma unroll
       for (int e = 0; e < 4; ++e) f2_add_bf16(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1], w[e]);
     }
+  }
+  if (ep.kind == 2) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int c = n + 16 * j;
+      const int which = c / ep.C, r = c - which * ep.C, h = r / ep.dh, d = r - h * ep.dh;
+      uint4* dst = reinterpret_cast<uint4*>(row + which * ep.which_stride +
+                                            (size_t)h * ep.ur.N * ep.dh + d);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const float* f = v + 16 * j + 8 * q;
+        uint4 w;
+        w.x = pack_bf16(f[0], f[1]);
+        w.y = pack_bf16(f[2], f[3]);
+        w.z = pack_bf16(f[4], f[5]);
+        w.w = pack_bf16(f[6], f[7]);
+        dst[q] = w;
+      }
+    }
+    return;
   }
   if (ep.kind == 0) {
 #pragma unroll

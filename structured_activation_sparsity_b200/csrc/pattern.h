@@ -90,4 +90,13 @@ SS_HD int blockmajor_to_canonical(int q, int b, int L) {
   return j * L + a * b + r;
 }
 
+// The inverse: canonical permuted position p -> block-major position q.
+SS_HD int canonical_to_blockmajor(int p, int b, int L) {
+  int j = p / L;
+  int rem = p - j * L;
+  int a = rem / b;
+  int r = rem - a * b;
+  return a * (b * kStripes) + j * b + r;
+}
+
 }  // namespace ss

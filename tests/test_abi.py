@@ -170,6 +170,60 @@ def test_validation_codes():
     assert L.sparsesam_launch_count() == 0
 
 
+def test_encoder_block_and_stack_validation():
+    lib = L.lib
+    by = ctypes.byref
+    cfg = L.make_cfg(1, 16, 16, "global", 14, 2, 64, 0.4)        # C = 128
+    K = O.keep_count(0.4, 256)
+    need = L.sparsesam_encoder_block_workspace(cfg, 128, 512, K)
+    # LN1 rows + the attention's workspace + the RC-MLP's workspace at least
+    assert need >= 256 * 128 * 2 + L.sparsesam_attn_workspace(cfg) + L.sparsesam_rcmlp_workspace(cfg, 128, 512, K)
+    assert L.sparsesam_encoder_block_workspace(cfg, 128, 512, 0) < need
+    assert L.sparsesam_encoder_block_workspace(cfg, 128, 512, 257) == 0
+    w = L.SsBlockWeights(**{n: FAKE for n in L.BLOCK_WEIGHT_FIELDS})
+
+    def call(c=cfg, x=FAKE, C=128, hidden=512, wt=w, perm=FAKE, inv=FAKE, keep=FAKE, k=K, ws=FAKE,
+             nbytes=1):
+        return lib.sparsesam_encoder_block(by(c), x, C, hidden, by(wt), perm, inv, keep, k, ws,
+                                           nbytes, None)
+    assert call() == L.SS_EWORKSPACE                               # 1 byte of workspace
+    assert call(ws=FAKE + 16, nbytes=1 << 30) == L.SS_EWORKSPACE   # misaligned workspace
+    assert call(C=192) == L.SS_EINVAL                              # C != heads * head_dim
+    assert call(hidden=500) == L.SS_EUNSUPPORTED
+    assert call(c=L.make_cfg(1, 16, 16, "global", 14, 2, 96, 0.4), C=192) == L.SS_EUNSUPPORTED
+    assert call(c=L.make_cfg(1, 16, 16, "global", 14, 3, 80, 0.4), C=240) == L.SS_EUNSUPPORTED
+    assert call(x=None) == L.SS_EINVAL
+    assert call(x=FAKE + 2) == L.SS_EINVAL
+    assert call(perm=None) == L.SS_EINVAL
+    assert call(inv=None) == L.SS_EINVAL
+    assert call(keep=None) == L.SS_EINVAL
+    assert call(k=-1) == L.SS_EINVAL and call(k=257) == L.SS_EINVAL
+    for n in ("ln1_w", "ln1_b", "w_qkv", "w_proj", "ln2_w", "ln2_b", "w1", "w2"):
+        bad = L.SsBlockWeights(**{f: (None if f == n else FAKE) for f in L.BLOCK_WEIGHT_FIELDS})
+        assert call(wt=bad) == L.SS_EINVAL, n
+    for n in ("b_qkv", "b_proj", "b1", "b2"):                      # Linear biases are optional
+        nob = L.SsBlockWeights(**{f: (None if f == n else FAKE) for f in L.BLOCK_WEIGHT_FIELDS})
+        assert call(wt=nob) == L.SS_EWORKSPACE, n
+        mis = L.SsBlockWeights(**{f: (FAKE + 8 if f == n else FAKE) for f in L.BLOCK_WEIGHT_FIELDS})
+        assert call(wt=mis) == L.SS_EINVAL, n
+    # the stack: its workspace holds both geometries' rankings and the larger block workspace
+    sw = L.sparsesam_encoder_stack_workspace(cfg, 128, 512)
+    cw = L.make_cfg(1, 16, 16, "window", 14, 2, 64, 0.4)           # 2 x 2 windows of 196
+    assert sw > max(need, L.sparsesam_encoder_block_workspace(cw, 128, 512, K))
+    arr = (L.SsBlockWeights * 2)(w, w)
+    flags = (ctypes.c_uint8 * 2)(0, 1)
+
+    def stack(lum=FAKE, n=2, ws=FAKE, nbytes=1 << 40, warr=arr):
+        return lib.sparsesam_encoder_stack(by(cfg), lum, FAKE, 128, 512, n, warr,
+                                           ctypes.addressof(flags), ws, nbytes, None)
+    assert stack(nbytes=sw - 1) == L.SS_EWORKSPACE
+    assert stack(lum=None) == L.SS_EINVAL
+    assert stack(n=-1) == L.SS_EINVAL
+    bad = L.SsBlockWeights(**{f: (None if f == "w_proj" else FAKE) for f in L.BLOCK_WEIGHT_FIELDS})
+    assert stack(warr=(L.SsBlockWeights * 2)(w, bad)) == L.SS_EINVAL   # checked before any launch
+    assert L.sparsesam_launch_count() == 0
+
+
 def test_binding_raises_on_error():
     with pytest.raises(L.SparseSAMError) as e:
         L.sparsesam_pattern(L.make_cfg(1, 5, 5, density=0.4))
