@@ -467,6 +467,13 @@ def run_ours(args, wl, rank, world, local_rank, dist):
         del m2
         torch.cuda.empty_cache()
 
+    # ---- the ViT-L encoder stack of full blocks at the density sweep (extra key) --------------
+    stack = None
+    if not args.no_stack:
+        stack = {"model": "vitl_24_blocks", "batch": VITL_STACK["batch"],
+                 "sweep": measure_stack(args, dev, stream, (1.0, 0.5, 0.4, 0.3),
+                                        max(5, min(args.steps, 20)), args.warmup)}
+
     if rank != 0:
         return
     line = {
@@ -487,6 +494,7 @@ def run_ours(args, wl, rank, world, local_rank, dist):
                   "effective_tflops": dense_flops * args.steps * world / td / 1e12,
                   "sparse_speedup": value / dense_value},
         "also": also,
+        "stack": stack,
     }
     if world == 1:
         step_s, desc, cores, _ = cpu_sample(wl)
@@ -523,62 +531,125 @@ def run_kernel_loop(args, wl, local_rank):
                       "note": "inputs stay resident in L2 across calls"}), flush=True)
 
 
-def run_stack(args, local_rank):
-    """The ViT-L encoder stack (24 blocks: global at 5, 11, 17, 23, the rest 14x14 windowed;
-    8 images of 64x64 tokens, 16 heads x 64, MLP 1024->4096) at each density of the sweep, as the
-    sum of its blocks' steps: S1+S2 once per image for each of the two geometries (the permutation
-    depends on the image only), then S3 and S4 for every block. One JSON line per density."""
+VITL_STACK = {"batch": 8, "grid": 64, "dim": 1024, "heads": 16, "head_dim": 64, "hidden": 4096,
+              "blocks": 24, "global_blocks": (5, 11, 17, 23), "window": 14}
+
+
+def stack_flops(cfg_pattern_g, cfg_pattern_w, K):
+    """Algorithmic flops of one pass of the ViT-L stack: per block the qkv and proj GEMMs over its
+    attention units' rows (pad rows of windowed blocks included: they are computed), the attention
+    on its kept blocks and the MLP on the kept rows."""
+    S = VITL_STACK
+    B, C, Hd, T = S["batch"], S["dim"], S["hidden"], S["grid"] ** 2
+    total = 0.0
+    for i in range(S["blocks"]):
+        pat = cfg_pattern_g if i in S["global_blocks"] else cfg_pattern_w
+        rows = pat.units * pat.unit_tokens
+        total += 2.0 * rows * C * 3 * C + 2.0 * rows * C * C
+        total += workloads.attn_flops(pat.units, pat.unit_tokens, S["heads"], S["head_dim"], pat.rho)
+        total += workloads.mlp_flops(B * K, C, Hd)
+    return total, B * T
+
+
+def measure_stack(args, dev, stream, densities, steps, warmup):
+    """The ViT-L encoder stack through sparsesam_encoder_stack (24 full blocks: LN, qkv, attention,
+    proj, LN2 + RC-MLP; global at 5, 11, 17, 23, the rest 14x14 windowed; 8 images of 64x64 tokens;
+    one ranking of the tokens per pass) at each density: random-init weights drawn on the device,
+    x updated in place pass after pass (each pass streams 0.6 GB of weights, well over L2)."""
     import torch
 
     from structured_activation_sparsity_b200 import _lib as L
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    stream = torch.cuda.Stream(device=dev)
-    wg, ww = workloads.get("vitl_global"), workloads.get("vitl_window")
-    n_global, n_window = 4, 20
+    S = VITL_STACK
+    B, G, C, Hd = S["batch"], S["grid"], S["dim"], S["hidden"]
+    flags = [i in S["global_blocks"] for i in range(S["blocks"])]
     bf16_peak = peaks()[0]
-    for d in (1.0, 0.5, 0.4, 0.3):
-        hg = make_sets(wg, 1, dev, density=d)[0][0]
-        hw = make_sets(ww, 1, dev, density=d)[0][0]
+    out = []
+    for d in densities:
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(4)
 
-        def stack_step():
-            hg.score_perm_step(stream)
-            hw.score_perm_step(stream)
-            for i in range(n_global + n_window):
-                h = hg if i % 6 == 5 else hw   # blocks 5, 11, 17, 23 are global
-                h.attn_step(stream)
-                h.mlp_step(stream)
+        def rnd(*shape, scale=1.0, shift=0.0):
+            t_ = torch.randn(*shape, generator=gen, device=dev, dtype=torch.float32)
+            return (t_ * scale + shift).to(torch.bfloat16)
+        blocks = []
+        for _ in range(S["blocks"]):
+            blocks.append({
+                "ln1_w": rnd(C, scale=0.1, shift=1.0), "ln1_b": rnd(C, scale=0.1),
+                "w_qkv": rnd(3 * C, C, scale=C ** -0.5), "b_qkv": rnd(3 * C, scale=0.1),
+                "w_proj": rnd(C, C, scale=C ** -0.5), "b_proj": rnd(C, scale=0.1),
+                "ln2_w": rnd(C, scale=0.1, shift=1.0), "ln2_b": rnd(C, scale=0.1),
+                "w1": rnd(Hd, C, scale=C ** -0.5), "b1": rnd(Hd, scale=0.1),
+                "w2": rnd(C, Hd, scale=Hd ** -0.5), "b2": rnd(C, scale=0.1)})
+        weight_bytes = torch.cuda.memory_allocated(dev) - base
+        wts = [L.block_weights(b) for b in blocks]
+        x = rnd(B, G * G, C)
+        lum = torch.rand(B, G, G, generator=gen, device=dev, dtype=torch.float32)
+        cfg = L.make_cfg(B, G, G, "global", S["window"], S["heads"], S["head_dim"], d)
+        wsb = L.sparsesam_encoder_stack_workspace(cfg, C, Hd)
+        ws = torch.empty((wsb,), dtype=torch.uint8, device=dev)
+
+        def one():
+            L.sparsesam_encoder_stack(cfg, lum, x, C, Hd, wts, flags, ws, wsb, stream)
 
         with torch.cuda.stream(stream):
-            for _ in range(args.warmup):
-                stack_step()
+            for _ in range(warmup):
+                one()
         torch.cuda.synchronize()
+        n0 = L.sparsesam_launch_count()
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev0.record(stream)
         with torch.cuda.stream(stream):
-            for _ in range(args.steps):
-                stack_step()
+            for _ in range(steps):
+                one()
         ev1.record(stream)
         torch.cuda.synchronize()
-        t = ev0.elapsed_time(ev1) / 1e3 / args.steps
+        launches = (L.sparsesam_launch_count() - n0) // steps
+        t = ev0.elapsed_time(ev1) / 1e3 / steps
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        # one traced pass: each launch's CUDA-event time, summed per kernel over the pass
+        L.sparsesam_trace_start(4096)
+        with torch.cuda.stream(stream):
+            one()
+        recs = L.sparsesam_trace_stop()
+        per = {}
+        for name, ms in recs:
+            per[name] = per.get(name, 0.0) + ms * 1e3
         if L.sparsesam_device_status(stream) != L.SS_OK:
-            raise RuntimeError("a device wait timed out during timing")
-        flops = 0.0
-        for h, w, n in ((hg, wg, n_global), (hw, ww, n_window)):
-            pat = h.pattern
-            flops += n * (workloads.attn_flops(w.units, w.unit_tokens, w.heads, w.head_dim, pat.rho)
-                          + workloads.mlp_flops(w.batch * pat.keep, w.dim, w.hidden))
-        tokens = wg.batch * wg.grid_h * wg.grid_w
-        print(json.dumps({"stack": "vitl_24_blocks", "density": d, "ms_per_stack": t * 1e3,
-                          "tokens_per_s": tokens / t, "effective_tflops": flops / t / 1e12,
-                          "frac_bf16_peak": flops / t / 1e12 / bf16_peak,
-                          "global_rho": hg.pattern.rho, "window_rho": hw.pattern.rho,
-                          "steps": args.steps, "warmup": args.warmup,
-                          "note": "sum of block steps; the full block (LN, projections) is not in "
-                                  "the hot path"}), flush=True)
-        del hg, hw
-        torch.cuda.empty_cache()
+            raise RuntimeError("a device wait timed out during the stack")
+        pg = L.sparsesam_pattern(cfg)
+        pw = L.sparsesam_pattern(L.make_cfg(B, G, G, "window", S["window"], S["heads"],
+                                            S["head_dim"], d))
+        flops, tokens = stack_flops(pg, pw, pg.keep)
+        out.append({"density": d, "ms_per_stack": t * 1e3, "tokens_per_s": tokens / t,
+                    "tokens_per_s_per_block": tokens * S["blocks"] / t,
+                    "effective_tflops": flops / t / 1e12,
+                    "frac_bf16_peak": flops / t / 1e12 / bf16_peak,
+                    "global_rho": pg.rho, "window_rho": pw.rho, "kept_tokens_per_image": pg.keep,
+                    "gpu_launches_per_stack": int(launches),
+                    "peak_memory_bytes": int(peak), "weight_bytes": int(weight_bytes),
+                    "workspace_bytes": int(wsb),
+                    "traced_us_per_kernel": {k: round(v, 1) for k, v in
+                                             sorted(per.items(), key=lambda kv: -kv[1])},
+                    "steps": steps, "warmup": warmup})
+        del blocks, wts, x, lum, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_stack(args, local_rank):
+    """The ViT-L stack alone at the density sweep, one JSON line per density (no bench line)."""
+    import torch
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    for r in measure_stack(args, dev, stream, (1.0, 0.5, 0.4, 0.3), args.steps, args.warmup):
+        print(json.dumps({"stack": "vitl_24_blocks", **r}), flush=True)
 
 
 def main():
@@ -596,6 +667,8 @@ def main():
                     help="run only this library call in a loop (profiling aid; no bench line)")
     ap.add_argument("--stack", action="store_true",
                     help="time the ViT-L 24-block stack at densities 1.0/0.5/0.4/0.3 (no bench line)")
+    ap.add_argument("--no-stack", action="store_true",
+                    help="leave the ViT-L stack sweep out of the bench line")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = workloads.get(args.workload)

@@ -9,10 +9,11 @@ single block come from the oracle too.
 Tolerance. The GPU rounds to bf16 between steps (LN outputs, q/k/v, the attention output, the
 MLP's hidden activation, P before P*V) and, above all, stores the residual stream x in bf16 twice
 per block (after the attention branch and after the MLP branch): each store is off by up to half
-an ulp, 2^-9 |x|. With this recipe's O(1) branches (|x| up to about 6 after a few blocks) the
-measured error stays below 0.4 of the bound used here, |gpu - oracle| <= n * (0.03 + 2^-7 |oracle|)
-for n blocks: per block, the two residual roundings (2 * 2^-9 |x| = 2^-8 |x|, doubled for what the
-next steps carry forward) plus 0.03 for the branches' own bf16 rounding."""
+an ulp, 2^-9 |x|. The bound used here is |gpu - oracle| <= n * (0.03 + 2^-7 |oracle|) for n blocks:
+per block, the two residual roundings (2 * 2^-9 |x| = 2^-8 |x|, doubled for what the next steps
+carry forward) plus 0.03 for the branches' own bf16 rounding. With this recipe's O(1) branches
+(|x| up to about 6 after a few blocks) the worst element measured on a B200 reached 0.28 to 0.43 of
+it (max-abs 0.019 to 0.025 and mean-abs about 0.002 per block)."""
 import numpy as np
 import pytest
 import torch
@@ -28,6 +29,14 @@ f64 = synth.bf16_to_f64
 
 def _bound(ref, n_blocks):
     return n_blocks * (0.03 + 2.0 ** -7 * np.abs(ref))
+
+
+def _report(y, ref, n_blocks):
+    """Prints the error against the bound (pytest -s shows it) and returns the worst ratio."""
+    err = np.abs(y - ref)
+    r = float((err / _bound(ref, n_blocks)).max())
+    print(f"max-abs {err.max():.4g} mean-abs {err.mean():.4g} worst err/bound {r:.3f}")
+    return r
 
 
 def _lum(B, Hg, Wg, seed):
@@ -75,6 +84,7 @@ def _block_case(B, Hg, Wg, mode, heads, dh, hidden, density, seed):
 ])
 def test_encoder_block_matches_oracle(B, Hg, Wg, mode, heads, dh, hidden, d):
     y, ref, x0, keep = _block_case(B, Hg, Wg, mode, heads, dh, hidden, d, seed=Hg * 7 + heads)
+    _report(y, ref, 1)
     err = np.abs(y - ref)
     assert (err <= _bound(ref, 1)).all(), (err.max(), np.unravel_index(err.argmax(), err.shape))
     # both branches moved every row (the attention branch reaches every real token)
@@ -123,6 +133,7 @@ def _stack_case(B, Hg, Wg, heads, dh, hidden, density, flags, seed, images=None)
 def test_encoder_stack_matches_oracle():
     flags = [False, True, False]
     y, ref = _stack_case(2, 20, 20, 2, 64, 256, 0.4, flags, seed=11)
+    _report(y, ref, len(flags))
     err = np.abs(y - ref)
     assert (err <= _bound(ref, len(flags))).all(), err.max()
 
@@ -130,6 +141,7 @@ def test_encoder_stack_matches_oracle():
 def test_encoder_stack_head_dim_80_matches_oracle():
     flags = [True, False]
     y, ref = _stack_case(1, 28, 28, 4, 80, 640, 0.3, flags, seed=12)
+    _report(y, ref, len(flags))
     assert (np.abs(y - ref) <= _bound(ref, len(flags))).all()
 
 
@@ -139,5 +151,6 @@ def test_vitl_blocks_full_size_sampled_images():
     and 7 (images are independent)."""
     flags = [False, True, False]
     y, ref = _stack_case(8, 64, 64, 16, 64, 4096, 0.4, flags, seed=4, images=[2, 7])
+    _report(y, ref, len(flags))
     err = np.abs(y - ref)
     assert (err <= _bound(ref, len(flags))).all(), err.max()
