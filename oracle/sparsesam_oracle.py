@@ -388,6 +388,85 @@ def update_magnitude(delta) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------------------------
+# The partial-token-count variant: prefix tokens + patch tokens, 2-D RoPE
+# ---------------------------------------------------------------------------------------------
+# SparseSAM README, "Zero-shot CLIP on ImageNet-1k": the Perception Encoder is patched with
+# `sparsesam_partial` (group_size=4); its "kernels/" directory fuses RoPE into the attention.
+# Readings of what the pages leave open: the sequence is `prefix` extra tokens (the class token)
+# followed by the patch tokens in raster order; the stripe-sort pattern covers the patch tokens
+# only; patch queries also attend every prefix key, prefix queries attend every key; the RoPE is
+# axial 2-D (Su et al., "RoFormer", 2021, extended per axis): the first half of a head's channels
+# rotates with the token's row, the second half with its column, pair i of a half at frequency
+# base^(-i / (dh/4)); prefix tokens are not rotated.
+
+
+def rope_2d(x, grid_h: int, grid_w: int, base: float) -> np.ndarray:
+    """x [U, T, heads, dh] of patch tokens in raster order, rotated (float64): channels (d, d+1),
+    d = half*dh/2 + 2i, turn by pos * base^(-i/(dh/4)), pos = row (half 0) or column (half 1)."""
+    x = np.asarray(x, dtype=np.float64)
+    U, T, H, D = x.shape
+    assert T == grid_h * grid_w and D % 4 == 0
+    half, quart = D // 2, D // 4
+    pos = (np.arange(T) // grid_w, np.arange(T) % grid_w)
+    out = x.copy()
+    for axis in (0, 1):
+        for i in range(quart):
+            d = axis * half + 2 * i
+            phi = pos[axis] * float(base) ** (-i / quart)
+            c, s = np.cos(phi)[None, :, None], np.sin(phi)[None, :, None]
+            a, b = x[:, :, :, d], x[:, :, :, d + 1]
+            out[:, :, :, d] = a * c - b * s
+            out[:, :, :, d + 1] = a * s + b * c
+    return out
+
+
+def attention_partial(q, k, v, perm, density: float, prefix: int, grid_h: int, grid_w: int,
+                      rope_base: float) -> np.ndarray:
+    """Stripe-Sort attention over prefix + patch sequences, float64 [U, prefix + T, heads, dh].
+
+    Patch queries: softmax over their kept patch keys (the pattern over the T patch tokens, perm
+    [U, T] their stripe-sort permutation) and every prefix key. Prefix queries: softmax over all
+    keys. q and k of patch tokens are rotated by rope_2d first (rope_base 0: no rotation)."""
+    q = np.asarray(q, dtype=np.float64).copy()
+    k = np.asarray(k, dtype=np.float64).copy()
+    v = np.asarray(v, dtype=np.float64)
+    U, NT, H, D = q.shape
+    T = NT - prefix
+    if rope_base:
+        q[:, prefix:] = rope_2d(q[:, prefix:], grid_h, grid_w, rope_base)
+        k[:, prefix:] = rope_2d(k[:, prefix:], grid_h, grid_w, rope_base)
+    pat = pattern(T, density)
+    blk = position_offset_block(T, pat.b)
+    scale = 1.0 / math.sqrt(D)
+
+    def softmax_rows(s):
+        s = s - s.max(axis=-1, keepdims=True)
+        e = np.exp(s)
+        return e / e.sum(axis=-1, keepdims=True)
+
+    out = np.empty((U, NT, H, D), dtype=np.float64)
+    for u in range(U):
+        pm = np.asarray(perm[u], dtype=np.int64)
+        qp = q[u, prefix + pm].transpose(1, 0, 2)          # [H, T, D]
+        kp = k[u, prefix + pm].transpose(1, 0, 2)
+        vp = v[u, prefix + pm].transpose(1, 0, 2)
+        kx = k[u, :prefix].transpose(1, 0, 2)              # [H, prefix, D]
+        vx = v[u, :prefix].transpose(1, 0, 2)
+        for a in range(pat.nb):
+            rows = np.nonzero(blk == a)[0]
+            kept = pat.col_idx[pat.row_ptr[a]:pat.row_ptr[a + 1]]
+            keys = np.nonzero(np.isin(blk, kept))[0]
+            kk = np.concatenate([kp[:, keys], kx], axis=1)
+            vv = np.concatenate([vp[:, keys], vx], axis=1)
+            p = softmax_rows(np.matmul(qp[:, rows], kk.transpose(0, 2, 1)) * scale)
+            out[u, prefix + pm[rows]] = np.matmul(p, vv).transpose(1, 0, 2)
+        for j in range(prefix):
+            s = np.einsum("hd,thd->ht", q[u, j], k[u]) * scale   # [H, NT]
+            out[u, j] = np.einsum("ht,thd->hd", softmax_rows(s), v[u])
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
 # The full encoder block around S3 and S4, and the encoder stack
 # ---------------------------------------------------------------------------------------------
 # The pages patch SparseSAM into SAM's image encoder without retraining (README, "SparseSAM":
