@@ -12,6 +12,7 @@
  *   sparsesam_encoder_block  a full encoder block: LN1, qkv, S3, proj, residual, LN2 + S4
  *   sparsesam_encoder_stack  the encoder's blocks in order over one ranking of the tokens
  *   sparsesam_attn   S3  static block-sparse attention over the permuted sequence
+ *   sparsesam_attn_partial   S3 for prefix + patch sequences with 2-D RoPE (PE-style encoders)
  *   sparsesam_rcmlp  S4  fc1-GELU-fc2 on the kept tokens, added to the residual in place
  *   sparsesam_random_perm     S2 over random scores (the random-permutation ablation)
  *   sparsesam_keep_by_update  the keep-set by update magnitude (another keep criterion)
@@ -177,6 +178,31 @@ int sparsesam_attn(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k, cons
  * operands (and timing the kernel by itself). */
 int sparsesam_attn_gathered(const ss_cfg* cfg, const void* ws, size_t ws_bytes,
                             const int32_t* perm, uint16_t* out, void* stream);
+
+/* Bytes of device workspace sparsesam_attn_partial needs (0 on invalid arguments). */
+size_t sparsesam_attn_partial_workspace(const ss_cfg* cfg, int32_t prefix);
+
+/* S3 for Perception-Encoder-style sequences: the SparseSAM README's `sparsesam_partial` variant
+ * ("Zero-shot CLIP on ImageNet-1k": apply_pe(model.visual, "sparsesam_partial", ratio,
+ * group_size=4, ...), with the RoPE of its "kernels/" directory fused). A unit's sequence is
+ * `prefix` extra tokens (e.g. the class token; 0 <= prefix <= 4) followed by the grid_h x grid_w
+ * patch tokens in raster order: q, k, v, out (device) bf16 [batch, prefix + grid_h*grid_w, heads,
+ * head_dim]. cfg must be in global mode; perm (device) int32 [batch, grid_h*grid_w] is the patch
+ * tokens' stripe-sort permutation (sparsesam_perm of the patch grid's scores).
+ *   - RoPE (rope_base > 1; 0 = none): q and k of patch token (y, x) are rotated pairwise: channels
+ *     (d, d+1) of a head, d even, by the angle pos * rope_base^(-i/(head_dim/4)), where
+ *     i = (d mod head_dim/2) / 2 and pos = y for d < head_dim/2, x otherwise (an axial 2-D RoPE:
+ *     the first half of the channels encodes the row, the second the column). Prefix tokens are
+ *     not rotated. Rotation in fp32 from the bf16 inputs, rounded to bf16.
+ *   - Patch query rows: softmax of (q.k)/sqrt(head_dim) over their kept patch keys (the static
+ *     pattern over the patch tokens, as sparsesam_attn) and every prefix key.
+ *   - Prefix query rows: softmax over every key of the unit (dense).
+ * fp32 softmax; ws (device, 256-byte aligned) >= sparsesam_attn_partial_workspace(cfg, prefix)
+ * bytes. Errors: as sparsesam_attn; SS_EUNSUPPORTED for window mode, more than 32 heads or more
+ * than 16384 tokens; SS_EINVAL for prefix or rope_base out of range. */
+int sparsesam_attn_partial(const ss_cfg* cfg, int32_t prefix, float rope_base, const uint16_t* q,
+                           const uint16_t* k, const uint16_t* v, const int32_t* perm,
+                           uint16_t* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of device workspace sparsesam_rcmlp needs for K kept tokens per image (0 on invalid
  * arguments). */

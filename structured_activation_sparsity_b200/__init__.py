@@ -21,7 +21,8 @@ _LIB_NAMES = {
     "sparsesam_score_perm", "sparsesam_block", "sparsesam_block_workspace",
     "sparsesam_random_perm", "sparsesam_keep_by_update", "SsBlockWeights", "block_weights",
     "sparsesam_encoder_block", "sparsesam_encoder_block_workspace", "sparsesam_encoder_stack",
-    "sparsesam_encoder_stack_workspace",
+    "sparsesam_encoder_stack_workspace", "sparsesam_attn_partial",
+    "sparsesam_attn_partial_workspace",
     "sparsesam_trace_start", "sparsesam_trace_stop", "strerror",
 }
 

@@ -74,6 +74,9 @@ def _load():
         "sparsesam_rcmlp_workspace": (SZ, [cfgp, I32, I32, I32]),
         "sparsesam_rcmlp": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, I32, P, SZ, VP]),
         "sparsesam_rcmlp_noalloc": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, I32, VP]),
+        "sparsesam_attn_partial_workspace": (SZ, [cfgp, I32]),
+        "sparsesam_attn_partial": (ctypes.c_int, [cfgp, I32, ctypes.c_float, P, P, P, P, P, P, SZ,
+                                                  VP]),
         "sparsesam_encoder_block_workspace": (SZ, [cfgp, I32, I32, I32]),
         "sparsesam_encoder_block": (ctypes.c_int, [cfgp, P, I32, I32, ctypes.POINTER(SsBlockWeights),
                                                    P, P, P, I32, P, SZ, VP]),
@@ -234,6 +237,18 @@ def sparsesam_rcmlp_noalloc(cfg, x, C, hidden, w1, b1, w2, b2, keep, K, stream=N
                   lib.sparsesam_rcmlp_noalloc(ctypes.byref(cfg), _ptr(x), int(C), int(hidden),
                                               _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(keep),
                                               int(K), _stream(stream)))
+
+
+def sparsesam_attn_partial_workspace(cfg, prefix) -> int:
+    return int(lib.sparsesam_attn_partial_workspace(ctypes.byref(cfg), int(prefix)))
+
+
+def sparsesam_attn_partial(cfg, prefix, rope_base, q, k, v, perm, out, ws, ws_bytes, stream=None):
+    """S3 over prefix + patch tokens with 2-D RoPE on the patch tokens (rope_base 0: none)."""
+    return _check("sparsesam_attn_partial",
+                  lib.sparsesam_attn_partial(ctypes.byref(cfg), int(prefix), float(rope_base),
+                                             _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _ptr(out),
+                                             _ptr(ws), int(ws_bytes), _stream(stream)))
 
 
 def block_weights(w) -> SsBlockWeights:

@@ -440,7 +440,8 @@ static int gather_launch(const Geo& g, int heads, int dh, const AttnLayout& L, c
 
 // The attention over the gathered Q, K, V in ws (laid out as attn_layout describes).
 static int attn_launch(const ss_cfg* cfg, const Geo& g, const AttnLayout& L, uint8_t* ws,
-                       const int32_t* perm, uint16_t* out, int* status, cudaStream_t st) {
+                       const int32_t* perm, uint16_t* out, int* status, cudaStream_t st,
+                       float2* ml = nullptr) {
   const int heads = cfg->heads, dh = cfg->head_dim;
   const uint16_t* bufs[3] = {reinterpret_cast<uint16_t*>(ws),
                              reinterpret_cast<uint16_t*>(ws + L.one),
@@ -470,6 +471,7 @@ static int attn_launch(const ss_cfg* cfg, const Geo& g, const AttnLayout& L, uin
   ap.sms = sm_count();
   ap.partial = reinterpret_cast<float*>(ws + L.partial);
   ap.operm = operm;
+  ap.ml = ml;
   int rc = cuda_err(traced("attn", st, [&] {
     return launch_attn(&tm[0], &tm[1], &tm[2], &tm[3], &tm[4], &tm[5], &tm[6], ap, dh, status,
                        st);
@@ -673,6 +675,82 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
   }));
   if (rc) return rc;
   return rcmlp_launch(g, K, x, C, hidden, w1, b1, w2, b2, keep, wsm, status, st);
+}
+
+// ---- the partial-token-count variant (prefix tokens, RoPE) -------------------------------------
+
+// Workspace: the attention's (gathered and rotated Q, K, V; ...), then the patch rows' attention
+// output in token order [U, N, heads, dh] and their (m, l) [U*heads, N].
+struct PartialLayout {
+  AttnLayout L;
+  size_t po, ml, total;
+};
+
+static int partial_layout(const ss_cfg* cfg, const Geo& g, PartialLayout* P) {
+  int rc = attn_layout(cfg, g, &P->L);
+  if (rc) return rc;
+  const size_t rows = (size_t)g.U * cfg->heads * g.N;
+  P->po = align256(P->L.total);
+  P->ml = P->po + align256(rows * cfg->head_dim * 2);
+  P->total = P->ml + align256(rows * 8);
+  return SS_OK;
+}
+
+size_t sparsesam_attn_partial_workspace(const ss_cfg* cfg, int32_t prefix) {
+  Geo g;
+  PartialLayout P;
+  if (geometry(cfg, &g) || cfg->heads < 1 || cfg->head_dim < 1 || prefix < 0 ||
+      prefix > kMaxPrefix || partial_layout(cfg, g, &P))
+    return 0;
+  return P.total;
+}
+
+int sparsesam_attn_partial(const ss_cfg* cfg, int32_t prefix, float rope_base, const uint16_t* q,
+                           const uint16_t* k, const uint16_t* v, const int32_t* perm,
+                           uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  if (g.window_mode) return SS_EUNSUPPORTED;
+  if (prefix < 0 || prefix > kMaxPrefix) return SS_EINVAL;
+  if (!(rope_base == 0.f || (rope_base > 1.f && rope_base < INFINITY))) return SS_EINVAL;
+  ss_pattern p;
+  if ((rc = attn_check(cfg, g, q, k, v, perm, out, &p))) return rc;
+  if (cfg->heads > kMaxPrefixHeads) return SS_EUNSUPPORTED;
+  if ((size_t)(prefix + g.N) * sizeof(float) > kMaxPrefixRowsSmem) return SS_EUNSUPPORTED;
+  if ((int64_t)g.U * (g.N + prefix) * cfg->heads * (cfg->head_dim / 8) >= (int64_t)1 << 31)
+    return SS_EUNSUPPORTED;
+  PartialLayout P;
+  if ((rc = partial_layout(cfg, g, &P))) return rc;
+  if (!ws || !aligned(ws, 256) || ws_bytes < P.total) return SS_EWORKSPACE;
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+  const int heads = cfg->heads, dh = cfg->head_dim;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint16_t* qp = reinterpret_cast<uint16_t*>(wsb);
+  uint16_t* kp = reinterpret_cast<uint16_t*>(wsb + P.L.one);
+  uint16_t* vp = reinterpret_cast<uint16_t*>(wsb + 2 * P.L.one);
+  uint16_t* po = reinterpret_cast<uint16_t*>(wsb + P.po);
+  float2* ml = reinterpret_cast<float2*>(wsb + P.ml);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float log2_base = rope_base == 0.f ? 0.f : (float)log2((double)rope_base);
+  rc = cuda_err(traced("gather_rope", st, [&] {
+    return launch_gather_rope(q, k, v, perm, qp, kp, vp, g.U, g.N, heads, dh, p.b, prefix, g.Wg,
+                              log2_base, status, st);
+  }));
+  if (rc) return rc;
+  // Without prefix tokens the patch rows are the output itself.
+  if ((rc = attn_launch(cfg, g, P.L, wsb, perm, prefix ? po : out, status, st, ml))) return rc;
+  if (prefix == 0) return SS_OK;
+  rc = cuda_err(traced("prefix_merge", st, [&] {
+    return launch_prefix_merge(po, ml, qp, k, v, perm, out, g.U, g.N, heads, dh, p.b, prefix,
+                               P.L.ap.scale_log2, status, st);
+  }));
+  if (rc) return rc;
+  return cuda_err(traced("prefix_rows", st, [&] {
+    return launch_prefix_rows(q, k, v, kp, vp, out, g.U, g.N, heads, dh, prefix,
+                              P.L.ap.scale_log2, st);
+  }));
 }
 
 // ---- the full encoder block -----------------------------------------------------------------

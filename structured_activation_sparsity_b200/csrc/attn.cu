@@ -673,6 +673,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             !(ok = __all_sync(0xffffffffu, mbar_wait(stage_free, (use - 1) & 1, abort, status))))
           break;
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        if (P.ml && qrow < P.N) P.ml[(size_t)c.uh * P.N + qrow] = make_float2(m_ref, l_run);
         const uint32_t tile = smem_u32(smem + S::kStage);
 #pragma unroll
         for (int cc = 0; cc < DH / 8; ++cc) {
@@ -1085,6 +1086,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       named_barrier(bar, 128);   // the group's previous copy-out is done with the staging rows
       if (ok) {
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        if (P.ml && store) P.ml[(size_t)I.uh * P.N + qrow] = make_float2(m_ref, l_run);
         uint32_t x0[32], x1[32];
         tmem_ld32_pair(t_o, t_o + 32, x0, x1);
 #pragma unroll
@@ -1252,6 +1254,7 @@ __global__ void __launch_bounds__(kBM) k_merge_pieces(const float* __restrict__ 
   w.z = pack_bf16(v[4] * inv, v[5] * inv);
   w.w = pack_bf16(v[6] * inv, v[7] * inv);
   reinterpret_cast<uint4*>(operm + ((size_t)uh * P.N + qrow) * DH)[cc] = w;
+  if (P.ml && cc == 0) P.ml[(size_t)uh * P.N + qrow] = make_float2(M, Lsum);
 }
 
 cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,

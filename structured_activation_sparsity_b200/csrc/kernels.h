@@ -54,6 +54,8 @@ struct AttnParams {
   int tail_split;        // pair kernel: pieces per split pair
   float* partial;        // per split piece and group, fp32 O [dh][128], m [128], l [128]
   uint16_t* operm;       // pair kernel output: [U*heads, N, dh] in block-major permuted order
+  float2* ml;            // null, or [U*heads, N] (block-major): each row's running max m and
+                         // sum l of 2^(s*scale_log2 - m) over its kept keys, s = q.k
 };
 // Which attention kernel a shape takes, and the scratch beyond the gathered Q, K, V it needs
 // (planned for `sms` CTAs).
@@ -78,6 +80,28 @@ cudaError_t launch_merge_pieces(const AttnParams& p, int dh, cudaStream_t st);
 // out[u, perm[u][p(q)], h, :] = op[u*heads + h, q, :] for every block-major position q.
 cudaError_t launch_unpermute_out(const uint16_t* op, const int32_t* perm, uint16_t* out, int U,
                                  int N, int heads, int dh, int b, int* status, cudaStream_t st);
+
+// The partial-token-count variant (prefix tokens before the patch tokens, 2-D RoPE on the patch
+// tokens' q and k). q, k, v, out: [U, prefix + N, heads, dh].
+constexpr int kMaxPrefix = 4;            // prefix (class) tokens per unit
+constexpr int kMaxPrefixHeads = 32;
+constexpr size_t kMaxPrefixRowsSmem = 64 * 1024;   // scores of one dense prefix row: prefix + N <= 16384
+// Patch tokens (rows prefix + perm[u][p]) into the gathered layout, q and k rotated
+// (rope_log2_base = log2 of the RoPE base; 0: none).
+cudaError_t launch_gather_rope(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               const int32_t* perm, uint16_t* qp, uint16_t* kp, uint16_t* vp,
+                               int U, int N, int heads, int dh, int b, int prefix, int grid_w,
+                               float rope_log2_base, int* status, cudaStream_t st);
+// Patch rows: po [U, N, heads, dh] (attention over the kept patch keys, token order) with its
+// (m, l) in ml (block-major) merged with the prefix keys, written to out rows prefix + tok.
+cudaError_t launch_prefix_merge(const uint16_t* po, const float2* ml, const uint16_t* qp,
+                                const uint16_t* k, const uint16_t* v, const int32_t* perm,
+                                uint16_t* out, int U, int N, int heads, int dh, int b, int prefix,
+                                float scale_log2, int* status, cudaStream_t st);
+// Prefix rows: dense attention of each prefix query over all prefix + N keys.
+cudaError_t launch_prefix_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               const uint16_t* kp, const uint16_t* vp, uint16_t* out, int U, int N,
+                               int heads, int dh, int prefix, float scale_log2, cudaStream_t st);
 
 // Gathers the kept rows of x [B, T, C] into xk [B*K, C]; zeroes zero[0, nzero). late_wait: keep
 // and x are known final at launch (see k_gather_rows), the copy need not wait for the previous
