@@ -47,7 +47,11 @@ L2_BYTES = 126 * 1024 * 1024
 # dram__bytes_read.sum + dram__bytes_write.sum of one attention launch per workload, from an ncu
 # capture of the current attention kernel on that workload (profiles/ names the capture). A
 # workload is absent (traffic null) until its capture is taken again after a kernel change.
-ATTN_TRAFFIC_BYTES = {}
+ATTN_TRAFFIC_BYTES = {
+    "vith_global": 125_914_368 + 21_509_376,    # k_attn_pair<80>: profiles/attn_pair_vith_global.md
+    "vitb_global": 18_953_984 + 0,              # k_attn_pair<64>: profiles/attn_pair_vitb_global.md
+    "vitb_window": 90_458_880 + 9_328_384,      # k_attn_pairs: profiles/attn_pairs_vitb_window.md
+}
 
 
 def peaks():
@@ -515,8 +519,9 @@ def run_kernel_loop(args, wl, local_rank):
         hp.score_step(stream)
         hp.perm_step(stream)
     hp.attn_step(stream)   # leaves the permuted Q, K, V in the workspace for attn_kernel
-    fn = {"score": hp.score_step, "perm": hp.perm_step, "attn": hp.attn_step,
-          "attn_kernel": hp.attn_kernel_step, "rcmlp": hp.mlp_step}[args.kernel_loop]
+    fn = {"score": hp.score_step, "perm": hp.perm_step, "score_perm": hp.score_perm_step,
+          "attn": hp.attn_step, "attn_kernel": hp.attn_kernel_step,
+          "rcmlp": hp.mlp_step}[args.kernel_loop]
     for _ in range(args.warmup):
         fn(stream)
     torch.cuda.synchronize()
@@ -663,7 +668,7 @@ def main():
                          "(comma-separated; empty for none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--kernel-loop", default=None,
-                    choices=["score", "perm", "attn", "attn_kernel", "rcmlp"],
+                    choices=["score", "perm", "score_perm", "attn", "attn_kernel", "rcmlp"],
                     help="run only this library call in a loop (profiling aid; no bench line)")
     ap.add_argument("--stack", action="store_true",
                     help="time the ViT-L 24-block stack at densities 1.0/0.5/0.4/0.3 (no bench line)")
