@@ -388,6 +388,72 @@ def update_magnitude(delta) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------------------------
+# Decomposed relative-position bias (SAM's attention), fused into S3
+# ---------------------------------------------------------------------------------------------
+# SparseSAM README, folder layout: "kernels/ fused cutlass-DSL CUDA kernels (FA2 + rel-pos / RoPE)".
+# SAM's image-encoder attention (Kirillov et al., "Segment Anything", 2023, following MViTv2's
+# decomposed relative positions) adds to the scaled score of query token (qh, qw) and key token
+# (kh, kw) of a Hu x Wu unit grid the bias q . Rh[qh - kh + Hu - 1] + q . Rw[qw - kw + Wu - 1],
+# with q unscaled and tables Rh [2Hu - 1, dh], Rw [2Wu - 1, dh] of the unit's size. Readings: the
+# unit grid is the image (global blocks) or the window (windowed blocks; pad tokens have window
+# coordinates like any other); the bias applies to the kept keys of the pattern only.
+
+
+def unit_grid(geo: Geometry):
+    """(Hu, Wu): the grid of one attention unit, whose tokens enumerate row-major."""
+    return (geo.grid_h, geo.grid_w) if geo.mode == "global" else (geo.window, geo.window)
+
+
+def relpos_bias(q, rel_h, rel_w, Hu: int, Wu: int) -> np.ndarray:
+    """float64 [U, heads, N, N]: bias[u, h, i, j] of query token i and key token j (unit-local
+    enumeration order) = q[u,i,h] . rel_h[yi - yj + Hu - 1] + q[u,i,h] . rel_w[xi - xj + Wu - 1]."""
+    q = np.asarray(q, dtype=np.float64)
+    rh = np.asarray(rel_h, dtype=np.float64)
+    rw = np.asarray(rel_w, dtype=np.float64)
+    U, N, H, D = q.shape
+    assert N == Hu * Wu and rh.shape == (2 * Hu - 1, D) and rw.shape == (2 * Wu - 1, D)
+    y, x = np.arange(N) // Wu, np.arange(N) % Wu
+    qh = np.einsum("unhd,rd->uhnr", q, rh)                 # q . rel_h[r] for every r
+    qw = np.einsum("unhd,rd->uhnr", q, rw)
+    ridx_h = y[:, None] - y[None, :] + Hu - 1               # [N (query), N (key)]
+    ridx_w = x[:, None] - x[None, :] + Wu - 1
+    rows = np.arange(N)[:, None]
+    return qh[:, :, rows, ridx_h] + qw[:, :, rows, ridx_w]
+
+
+def attention_relpos(q, k, v, perm, density: float, geo: Geometry, rel_h, rel_w) -> np.ndarray:
+    """Stripe-Sort attention with the decomposed relative-position bias, float64 [U, N, heads, dh]:
+    each permuted query row's softmax over its kept keys of q.k/sqrt(dh) + bias (relpos_bias)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    U, N, H, D = q.shape
+    Hu, Wu = unit_grid(geo)
+    bias = relpos_bias(q, rel_h, rel_w, Hu, Wu)             # [U, H, N, N], token order
+    pat = pattern(N, density)
+    blk = position_offset_block(N, pat.b)
+    scale = 1.0 / math.sqrt(D)
+    out = np.empty((U, N, H, D), dtype=np.float64)
+    for u in range(U):
+        pm = np.asarray(perm[u], dtype=np.int64)
+        qp = q[u][pm].transpose(1, 0, 2)
+        kp = k[u][pm].transpose(1, 0, 2)
+        vp = v[u][pm].transpose(1, 0, 2)
+        bp = bias[u][:, pm][:, :, pm]                       # permuted rows and columns
+        for a in range(pat.nb):
+            rows = np.nonzero(blk == a)[0]
+            kept = pat.col_idx[pat.row_ptr[a]:pat.row_ptr[a + 1]]
+            keys = np.nonzero(np.isin(blk, kept))[0]
+            s = np.matmul(qp[:, rows], kp[:, keys].transpose(0, 2, 1)) * scale
+            s = s + bp[:, rows][:, :, keys]
+            s = s - s.max(axis=2, keepdims=True)
+            e = np.exp(s)
+            o = np.matmul(e / e.sum(axis=2, keepdims=True), vp[:, keys])
+            out[u, pm[rows]] = o.transpose(1, 0, 2)
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
 # The partial-token-count variant: prefix tokens + patch tokens, 2-D RoPE
 # ---------------------------------------------------------------------------------------------
 # SparseSAM README, "Zero-shot CLIP on ImageNet-1k": the Perception Encoder is patched with
