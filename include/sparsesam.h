@@ -12,6 +12,7 @@
  *   sparsesam_encoder_block  a full encoder block: LN1, qkv, S3, proj, residual, LN2 + S4
  *   sparsesam_encoder_stack  the encoder's blocks in order over one ranking of the tokens
  *   sparsesam_attn   S3  static block-sparse attention over the permuted sequence
+ *   sparsesam_attn_relpos    S3 with SAM's decomposed relative-position bias fused
  *   sparsesam_attn_partial   S3 for prefix + patch sequences with 2-D RoPE (PE-style encoders)
  *   sparsesam_rcmlp  S4  fc1-GELU-fc2 on the kept tokens, added to the residual in place
  *   sparsesam_random_perm     S2 over random scores (the random-permutation ablation)
@@ -178,6 +179,25 @@ int sparsesam_attn(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k, cons
  * operands (and timing the kernel by itself). */
 int sparsesam_attn_gathered(const ss_cfg* cfg, const void* ws, size_t ws_bytes,
                             const int32_t* perm, uint16_t* out, void* stream);
+
+/* Bytes of device workspace sparsesam_attn_relpos needs (0 on an invalid cfg). */
+size_t sparsesam_attn_relpos_workspace(const ss_cfg* cfg);
+
+/* S3 with SAM's decomposed relative-position bias fused (SparseSAM README, folder layout:
+ * "kernels/ ... FA2 + rel-pos"): the score of query token (qh, qw) and key token (kh, kw) of a
+ * unit is q.k/sqrt(head_dim) + q.rel_h[qh-kh+Hu-1] + q.rel_w[qw-kw+Wu-1] (q unscaled), over the
+ * same kept keys as sparsesam_attn. The unit grid Hu x Wu is grid_h x grid_w (global mode) or
+ * window x window (window mode; pad tokens have window coordinates). rel_h (device) bf16
+ * [2*Hu-1, head_dim], rel_w (device) bf16 [2*Wu-1, head_dim], 16-byte aligned, shared by the
+ * heads. Everything else as sparsesam_attn. The products q.rel_h[r] and q.rel_w[r] are computed
+ * on the tensor cores in fp32 and kept in fp16 (scaled by log2(e)); the bias is added to the fp32
+ * score. Head dim 64 only and Hu + Wu <= 128 (SS_EUNSUPPORTED otherwise): each query row keeps
+ * its Hu + Wu bias values in shared memory next to a three-stage K/V ring. ws (device, 256-byte
+ * aligned) >= sparsesam_attn_relpos_workspace(cfg) bytes. */
+int sparsesam_attn_relpos(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int32_t* perm, const uint16_t* rel_h,
+                          const uint16_t* rel_w, uint16_t* out, void* ws, size_t ws_bytes,
+                          void* stream);
 
 /* Bytes of device workspace sparsesam_attn_partial needs (0 on invalid arguments). */
 size_t sparsesam_attn_partial_workspace(const ss_cfg* cfg, int32_t prefix);

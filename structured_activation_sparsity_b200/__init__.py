@@ -22,7 +22,7 @@ _LIB_NAMES = {
     "sparsesam_random_perm", "sparsesam_keep_by_update", "SsBlockWeights", "block_weights",
     "sparsesam_encoder_block", "sparsesam_encoder_block_workspace", "sparsesam_encoder_stack",
     "sparsesam_encoder_stack_workspace", "sparsesam_attn_partial",
-    "sparsesam_attn_partial_workspace",
+    "sparsesam_attn_partial_workspace", "sparsesam_attn_relpos", "sparsesam_attn_relpos_workspace",
     "sparsesam_trace_start", "sparsesam_trace_stop", "strerror",
 }
 

@@ -74,6 +74,8 @@ def _load():
         "sparsesam_rcmlp_workspace": (SZ, [cfgp, I32, I32, I32]),
         "sparsesam_rcmlp": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, I32, P, SZ, VP]),
         "sparsesam_rcmlp_noalloc": (ctypes.c_int, [cfgp, P, I32, I32, P, P, P, P, P, I32, VP]),
+        "sparsesam_attn_relpos_workspace": (SZ, [cfgp]),
+        "sparsesam_attn_relpos": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, SZ, VP]),
         "sparsesam_attn_partial_workspace": (SZ, [cfgp, I32]),
         "sparsesam_attn_partial": (ctypes.c_int, [cfgp, I32, ctypes.c_float, P, P, P, P, P, P, SZ,
                                                   VP]),
@@ -237,6 +239,18 @@ def sparsesam_rcmlp_noalloc(cfg, x, C, hidden, w1, b1, w2, b2, keep, K, stream=N
                   lib.sparsesam_rcmlp_noalloc(ctypes.byref(cfg), _ptr(x), int(C), int(hidden),
                                               _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(keep),
                                               int(K), _stream(stream)))
+
+
+def sparsesam_attn_relpos_workspace(cfg) -> int:
+    return int(lib.sparsesam_attn_relpos_workspace(ctypes.byref(cfg)))
+
+
+def sparsesam_attn_relpos(cfg, q, k, v, perm, rel_h, rel_w, out, ws, ws_bytes, stream=None):
+    """S3 with SAM's decomposed relative-position bias (rel_h [2Hu-1, dh], rel_w [2Wu-1, dh])."""
+    return _check("sparsesam_attn_relpos",
+                  lib.sparsesam_attn_relpos(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(perm), _ptr(rel_h), _ptr(rel_w), _ptr(out),
+                                            _ptr(ws), int(ws_bytes), _stream(stream)))
 
 
 def sparsesam_attn_partial_workspace(cfg, prefix) -> int:

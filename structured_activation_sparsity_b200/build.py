@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsparsesam.so")
-SOURCES = ["score_perm.cu", "attn.cu", "mlp.cu", "block.cu", "partial.cu", "api.cu", "noalloc.cu"]
+SOURCES = ["score_perm.cu", "attn.cu", "mlp.cu", "block.cu", "partial.cu", "relpos.cu", "api.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h", "pattern.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -200,7 +200,7 @@ struct AttnLayout {
   size_t operm, partial, total;   // byte offsets, total size
 };
 
-int attn_layout(const ss_cfg* c, const Geo& g, AttnLayout* L) {
+int attn_layout(const ss_cfg* c, const Geo& g, AttnLayout* L, bool force_pair = false) {
   ss_pattern p;
   int rc = pattern_of(c, g, &p);
   if (rc) return rc;
@@ -215,7 +215,7 @@ int attn_layout(const ss_cfg* c, const Geo& g, AttnLayout* L) {
   ap.W = p.W;
   ap.g = p.g;
   ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c->head_dim));
-  L->plan = attn_plan(ap, c->head_dim, kPlanSMs);
+  L->plan = attn_plan(ap, c->head_dim, kPlanSMs, force_pair);
   ap.whole = L->plan.whole;
   ap.tail_split = L->plan.tail_split;
   L->one = align256((size_t)g.U * c->heads * g.N * c->head_dim * 2);
@@ -439,9 +439,10 @@ static int gather_launch(const Geo& g, int heads, int dh, const AttnLayout& L, c
 }
 
 // The attention over the gathered Q, K, V in ws (laid out as attn_layout describes).
+// rel: the relative-position fields of AttnParams (null: none).
 static int attn_launch(const ss_cfg* cfg, const Geo& g, const AttnLayout& L, uint8_t* ws,
                        const int32_t* perm, uint16_t* out, int* status, cudaStream_t st,
-                       float2* ml = nullptr) {
+                       float2* ml = nullptr, const AttnParams* rel = nullptr) {
   const int heads = cfg->heads, dh = cfg->head_dim;
   const uint16_t* bufs[3] = {reinterpret_cast<uint16_t*>(ws),
                              reinterpret_cast<uint16_t*>(ws + L.one),
@@ -472,6 +473,14 @@ static int attn_launch(const ss_cfg* cfg, const Geo& g, const AttnLayout& L, uin
   ap.partial = reinterpret_cast<float*>(ws + L.partial);
   ap.operm = operm;
   ap.ml = ml;
+  if (rel) {
+    ap.rel_tab = rel->rel_tab;
+    ap.rel_ld = rel->rel_ld;
+    ap.rel_h = rel->rel_h;
+    ap.rel_w = rel->rel_w;
+    ap.rel_npad = rel->rel_npad;
+    ap.rel_keyoff = rel->rel_keyoff;
+  }
   int rc = cuda_err(traced("attn", st, [&] {
     return launch_attn(&tm[0], &tm[1], &tm[2], &tm[3], &tm[4], &tm[5], &tm[6], ap, dh, status,
                        st);
@@ -675,6 +684,99 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
   }));
   if (rc) return rc;
   return rcmlp_launch(g, K, x, C, hidden, w1, b1, w2, b2, keep, wsm, status, st);
+}
+
+// ---- the relative-position variant ------------------------------------------------------------
+
+// Workspace: the attention's (pair kernel), then the stacked tables rpack [nr, dh], the bias
+// products [U*heads*N, nr] fp16 and the key offsets [U, npad].
+struct RelLayout {
+  AttnLayout L;
+  GemmPlan gp;
+  int Hu, Wu, nr, npad;
+  size_t rpack, tab, keyoff, total;
+};
+
+static int rel_layout(const ss_cfg* cfg, const Geo& g, RelLayout* R) {
+  int rc = attn_layout(cfg, g, &R->L, /*force_pair=*/true);
+  if (rc) return rc;
+  R->Hu = g.window_mode ? g.ws : g.Hg;
+  R->Wu = g.window_mode ? g.ws : g.Wg;
+  R->nr = (2 * R->Hu - 1 + 2 * R->Wu - 1 + 63) / 64 * 64;
+  R->npad = (g.N + 127) / 128 * 128;
+  const long long M = (long long)g.U * cfg->heads * g.N;
+  R->gp = gemm_plan((int)M, R->nr, cfg->head_dim, kPlanSMs);
+  R->rpack = align256(R->L.total);
+  R->tab = R->rpack + align256((size_t)R->nr * cfg->head_dim * 2);
+  R->keyoff = R->tab + align256((size_t)M * R->nr * 2);
+  R->total = R->keyoff + align256((size_t)g.U * R->npad * 2);
+  return SS_OK;
+}
+
+size_t sparsesam_attn_relpos_workspace(const ss_cfg* cfg) {
+  Geo g;
+  RelLayout R;
+  if (geometry(cfg, &g) || cfg->heads < 1 || cfg->head_dim < 1 || rel_layout(cfg, g, &R))
+    return 0;
+  return R.total;
+}
+
+int sparsesam_attn_relpos(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int32_t* perm, const uint16_t* rel_h,
+                          const uint16_t* rel_w, uint16_t* out, void* ws, size_t ws_bytes,
+                          void* stream) {
+  Geo g;
+  int rc = geometry(cfg, &g);
+  if (rc) return rc;
+  ss_pattern p;
+  if ((rc = attn_check(cfg, g, q, k, v, perm, out, &p))) return rc;
+  if (!rel_h || !rel_w || !aligned(rel_h, 16) || !aligned(rel_w, 16)) return SS_EINVAL;
+  if (cfg->head_dim != 64) return SS_EUNSUPPORTED;
+  RelLayout R;
+  if ((rc = rel_layout(cfg, g, &R))) return rc;
+  // The key offsets are bytes into a row of Hu + Wu fp16 slices (at most 2 * kRelPosRowWords).
+  if (R.Hu + R.Wu > 128) return SS_EUNSUPPORTED;
+  if ((long long)g.U * cfg->heads * g.N * R.nr >= (1ll << 31) ||
+      ((long long)g.U * cfg->heads * g.N + 127) / 128 > 65535)
+    return SS_EUNSUPPORTED;
+  if (!ws || !aligned(ws, 256) || ws_bytes < R.total) return SS_EWORKSPACE;
+  int* status = status_word();
+  if (!status) return SS_ECUDA;
+  const int heads = cfg->heads, dh = cfg->head_dim;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint16_t* rpack = reinterpret_cast<uint16_t*>(wsb + R.rpack);
+  uint16_t* tab = reinterpret_cast<uint16_t*>(wsb + R.tab);
+  uint16_t* keyoff = reinterpret_cast<uint16_t*>(wsb + R.keyoff);
+  if ((rc = gather_launch(g, heads, dh, R.L, q, k, v, perm, wsb, status, st))) return rc;
+  rc = cuda_err(traced("relpos_prep", st, [&] {
+    return launch_relpos_prep(rel_h, rel_w, rpack, dh, R.nr, perm, keyoff, g.U, g.N, R.npad, R.Hu,
+                              R.Wu, R.L.ap.b, status, st);
+  }));
+  if (rc) return rc;
+  const long long M = (long long)g.U * heads * g.N;
+  CUtensorMap ta, tb;
+  if (!encode_bf16(&ta, 2, wsb, dh, M, 1, (uint64_t)dh * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16(&tb, 2, rpack, dh, R.nr, 1, (uint64_t)dh * 2, 64, R.gp.bn,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return SS_ECUDA;
+  GemmEpilogue e = {};
+  e.kind = 4;
+  e.out = tab;
+  e.scale = 1.4426950408889634f;   // log2(e): the kernel's scores are in base-2 units
+  rc = cuda_err(traced("relpos_gemm", st, [&] {
+    return launch_gemm(&ta, &tb, R.gp, (int)M, R.nr, dh, e, nullptr, nullptr, sm_count(), status,
+                       st);
+  }));
+  if (rc) return rc;
+  AttnParams rel = {};
+  rel.rel_tab = tab;
+  rel.rel_ld = R.nr;
+  rel.rel_h = R.Hu;
+  rel.rel_w = R.Wu;
+  rel.rel_npad = R.npad;
+  rel.rel_keyoff = keyoff;
+  return attn_launch(cfg, g, R.L, wsb, perm, out, status, st, nullptr, &rel);
 }
 
 // ---- the partial-token-count variant (prefix tokens, RoPE) -------------------------------------

@@ -240,7 +240,12 @@ struct PairTmem {
   static_assert(kO + kOStride + DH <= 512, "TMEM columns");
 };
 
-template <int DH>
+// kRelPos: the decomposed relative-position variant. Its softmax threads keep their row's bias
+// slices (fp16, Hu + Wu values, an odd number of 32-bit words per row so that the 32 rows a warp
+// reads at one column fall in 32 different banks) in shared memory, for which the K/V ring is
+// three stages deep.
+constexpr int kRelPosRowWords = 65;                            // (64 + 64) / 2 rounded up to odd
+template <int DH, bool kRelPos = false>
 struct PairSmem {
   static constexpr int kTail = DH - 64;                        // 0 or 16 columns
   static constexpr int kQKMain = kBM * 128;                    // 128 rows x 64 bf16, 128B swizzle
@@ -249,7 +254,7 @@ struct PairSmem {
   static constexpr int kVAtom = kBN * 128;                     // 128 keys x 64 bf16, 128B swizzle
   static constexpr int kV = kTail ? 2 * kVAtom : kVAtom;
   static constexpr int kStageBytes = kQK + kV;
-  static constexpr int kStages = DH == 64 ? 5 : 3;             // depth of the K/V ring
+  static constexpr int kStages = kRelPos ? 3 : (DH == 64 ? 5 : 3);   // depth of the K/V ring
   static constexpr int kQ = 0;                                 // Q_A, then Q_B
   static constexpr int kKV = 2 * kQK;
   // Output staging, used by the groups in turn: one 128-row tile of O in the layout of a Q tile
@@ -257,7 +262,8 @@ struct PairSmem {
   // of the TMA store that writes it.
   static constexpr int kStage = kKV + kStages * kStageBytes;
   static constexpr int kBar = kStage + kQK;
-  static constexpr int kBytes = kBar + 512;
+  static constexpr int kTab = kBar + 512;                      // kRelPos: 2 x 128 bias rows
+  static constexpr int kBytes = kTab + (kRelPos ? 2 * kBM * kRelPosRowWords * 4 : 0);
   static constexpr int kAlloc = kBytes + 1024;                 // slack to align the base to 1024
   static_assert(kQK % 1024 == 0 && kStageBytes % 1024 == 0 && kKV % 1024 == 0,
                 "tiles must stay 1024-byte aligned for the 128-byte swizzle");
@@ -322,16 +328,17 @@ __device__ __forceinline__ void load_o_row(uint32_t t_o, uint32_t (&o)[DH]) {
     tmem_ld16_nowait(t_o + cc * 16, *reinterpret_cast<uint32_t(*)[16]>(o + 16 * cc));
   tmem_ld_wait();
 }
-template <int DH>
+template <int DH, bool kRelPos>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn_pair(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tq_tail,
                 const __grid_constant__ CUtensorMap tk_tail, const __grid_constant__ CUtensorMap to,
                 const __grid_constant__ CUtensorMap to_tail, const AttnParams P, int* status) {
-  using S = PairSmem<DH>;
+  using S = PairSmem<DH, kRelPos>;
   using T = PairTmem<DH>;
   constexpr int NS = S::kStages;
   constexpr bool kHasTail = S::kTail > 0;
+  static_assert(!(kRelPos && kHasTail), "the relative-position variant is built for head dim 64");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -518,7 +525,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t t_p = tmem + T::kP + grp * T::kPStride + lane_off;
     const uint32_t t_o = tmem + T::kO + grp * T::kOStride + lane_off;
     const int b4 = P.b * kStripes;
-    const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
+    // The relative-position variant scales S (and adds the bias) before the row max; the
+    // exponents are then x - ref.
+    const float max_scale = kRelPos ? 1.f : P.scale_log2;
+    const uint64_t scale2 = kRelPos ? f2_pack(1.f, 1.f) : f2_pack(P.scale_log2, P.scale_log2);
+    const uint32_t tab_row =
+        smem_u32(smem + S::kTab) + uint32_t((grp * kBM + row) * kRelPosRowWords * 4);
     constexpr int kSlot = (DH + 2) * kBM;               // floats of one group's partial
     bool ok = true;
     int gn = 0;            // tiles of this group so far (all pieces): the phase count
@@ -532,6 +544,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int s_q = band_start(a_q, P.W, P.nb);
       const int band_lo = s_q * b4, band_hi = (s_q + P.W) * b4, glob_hi = P.g * b4;
       float m_ref = -INFINITY, l_run = 0.f;
+      if constexpr (kRelPos) {
+        // This row's bias slices: entries qh .. qh+Hu-1 of its Rh products, then qw .. qw+Wu-1
+        // of its Rw products (the row of the bias GEMM), so that key (kh, kw) finds its terms
+        // at Hu-1-kh and Hu+Wu-1-kw.
+        const int qr = min(qrow, P.N - 1);
+        const int tok = __ldg(P.perm + (size_t)u_i * P.N + blockmajor_to_canonical(qr, P.b, P.L));
+        const int t = (unsigned)tok < (unsigned)P.N ? tok : 0;
+        const int qh = t / P.rel_w, qw = t - qh * P.rel_w;
+        const uint16_t* g = P.rel_tab + ((size_t)c.uh * P.N + qr) * P.rel_ld;
+        for (int e = 0; e < P.rel_h; ++e)
+          st_shared_u16(tab_row + 2 * e, __ldg(g + qh + e));
+        for (int e = 0; e < P.rel_w; ++e)
+          st_shared_u16(tab_row + 2 * (P.rel_h + e), __ldg(g + 2 * P.rel_h - 1 + qw + e));
+      }
       for (int n = c.n0; ok && n < c.n1; ++n, ++gn) {
         const int j = n - c.n0;
         // Warp-collective wait: either every lane goes on to the .sync.aligned TMEM ops or none.
@@ -551,6 +577,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // Has this group's previous P * V released P_g and O_g? Tested now, waited for below.
         bool prev_pv_done = gn == 0 || mbar_test(pv_done + grp, (gn - 1) & 1);
         const int c0 = c.tiles.tile(n) * kBN;
+        if constexpr (kRelPos) {
+          // s*scale_log2 + bias: key k's two byte offsets into this row's slices, 8 keys per load
+          // (the same addresses for every lane).
+          const uint4* ko =
+              reinterpret_cast<const uint4*>(P.rel_keyoff + (size_t)u_i * P.rel_npad + c0);
+#pragma unroll
+          for (int k8 = 0; k8 < kBN / 8; ++k8) {
+            const uint4 w = __ldg(ko + k8);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t off = (ww[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu;
+              const float bias = ld_shared_f16(tab_row + (off & 0xFFu)) +
+                                 ld_shared_f16(tab_row + (off >> 8));
+              sv[8 * k8 + e] = fmaf(sv[8 * k8 + e], P.scale_log2, bias);
+            }
+          }
+        }
         if (!pair_tile_full(c0, P)) {
           // The row's kept keys in this tile are two runs, [0, e0) and [s1, e1) relative to c0:
           // turned into four 32-bit column masks, so the per-key test has no branch.
@@ -573,7 +617,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], sv[k + 8 * 15]);
         const float x_max = fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])),
                                   fmaxf(mx[6], mx[7])) *
-                            P.scale_log2;
+                            max_scale;
         // Lazy rescale: the reference max moves only when the row max passes it by 2^8, so O in
         // TMEM is rescaled on few tiles. The decision is warp-wide (TMEM ops are warp-collective).
         const bool grow = x_max > m_ref + kLazyRescale;
@@ -1143,20 +1187,21 @@ static cudaError_t launch_attn_pairs(const CUtensorMap* tq, const CUtensorMap* t
   return launch_pdl(kernel, grid, dim3(kAttnThreads), S::kAlloc, st, *tq, *tk, *tv, p, status);
 }
 
-template <int DH>
+template <int DH, bool kRelPos = false>
 static cudaError_t launch_attn_pair(const CUtensorMap* tq, const CUtensorMap* tk,
                                     const CUtensorMap* tv, const CUtensorMap* tq_tail,
                                     const CUtensorMap* tk_tail, const CUtensorMap* to,
                                     const CUtensorMap* to_tail, const AttnParams& p, int* status,
                                     cudaStream_t st) {
-  using S = PairSmem<DH>;
-  cudaError_t e = cudaFuncSetAttribute(k_attn_pair<DH>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc);
+  using S = PairSmem<DH, kRelPos>;
+  auto kernel = k_attn_pair<DH, kRelPos>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       S::kAlloc);
   if (e != cudaSuccess) return e;
   const int pieces = p.whole + (pairs_per_head(p.N) * p.U * p.heads - p.whole) * p.tail_split;
   dim3 grid(std::max(1, std::min(pieces, p.sms)));
-  return launch_pdl(k_attn_pair<DH>, grid, dim3(kAttnThreads), S::kAlloc, st, *tq, *tk, *tv,
-                    *tq_tail, *tk_tail, *to, *to_tail, p, status);
+  return launch_pdl(kernel, grid, dim3(kAttnThreads), S::kAlloc, st, *tq, *tk, *tv, *tq_tail,
+                    *tk_tail, *to, *to_tail, p, status);
 }
 
 // Short items: every query tile has at most kPairTiles key tiles (the windowed blocks).
@@ -1168,9 +1213,9 @@ static bool short_items(const AttnParams& p) {
   return nt_max <= kPairTiles;
 }
 
-AttnPlan attn_plan(const AttnParams& p, int dh, int sms) {
+AttnPlan attn_plan(const AttnParams& p, int dh, int sms, bool force_pair) {
   AttnPlan r = {};
-  r.pair_kernel = !(dh == 64 && short_items(p));
+  r.pair_kernel = force_pair || p.rel_tab != nullptr || !(dh == 64 && short_items(p));
   if (!r.pair_kernel) return r;
   const int npairs = pairs_per_head(p.N);
   r.pairs = npairs * p.U * p.heads;
@@ -1261,6 +1306,10 @@ cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUte
                         const CUtensorMap* tq_tail, const CUtensorMap* tk_tail,
                         const CUtensorMap* to, const CUtensorMap* to_tail, const AttnParams& p,
                         int dh, int* status, cudaStream_t st) {
+  if (p.rel_tab) {
+    if (dh != 64) return cudaErrorInvalidValue;
+    return launch_attn_pair<64, true>(tq, tk, tv, tq, tk, to, to, p, status, st);
+  }
   if (dh == 64 && short_items(p)) return launch_attn_pairs(tq, tk, tv, p, status, st);
   if (dh == 64) return launch_attn_pair<64>(tq, tk, tv, tq, tk, to, to, p, status, st);
   if (dh == 80) return launch_attn_pair<80>(tq, tk, tv, tq_tail, tk_tail, to, to_tail, p, status, st);

@@ -56,6 +56,13 @@ struct AttnParams {
   uint16_t* operm;       // pair kernel output: [U*heads, N, dh] in block-major permuted order
   float2* ml;            // null, or [U*heads, N] (block-major): each row's running max m and
                          // sum l of 2^(s*scale_log2 - m) over its kept keys, s = q.k
+  // Decomposed relative-position bias (null rel_tab: none). rel_tab [U*heads*N, rel_ld] fp16 in
+  // block-major row order: the row's q . Rh[r] * log2(e) at column r < 2*rel_h - 1, then q . Rw[r]
+  // * log2(e) from column 2*rel_h - 1; rel_h x rel_w is the unit grid. rel_keyoff [U, rel_npad]
+  // (block-major key order): byte offsets (rel_h-1-kh)*2 | ((rel_h+rel_w-1-kw)*2) << 8.
+  const uint16_t* rel_tab;
+  int rel_ld, rel_h, rel_w, rel_npad;
+  const uint16_t* rel_keyoff;
 };
 // Which attention kernel a shape takes, and the scratch beyond the gathered Q, K, V it needs
 // (planned for `sms` CTAs).
@@ -64,7 +71,12 @@ struct AttnPlan {
   int pairs, whole, tail_split;
   size_t partial_bytes;
 };
-AttnPlan attn_plan(const AttnParams& p, int dh, int sms);
+AttnPlan attn_plan(const AttnParams& p, int dh, int sms, bool force_pair = false);
+// The relative-position variant's inputs: the tables stacked into rpack [nr, dh] (the bias GEMM's
+// B operand) and the key offsets keyoff [U, npad] of AttnParams::rel_keyoff.
+cudaError_t launch_relpos_prep(const uint16_t* rel_h, const uint16_t* rel_w, uint16_t* rpack,
+                               int dh, int nr, const int32_t* perm, uint16_t* keyoff, int U, int N,
+                               int npad, int Hu, int Wu, int b, int* status, cudaStream_t st);
 // Block-sparse attention over the gathered sequences (tensor maps over [U*heads, N, dh]; the
 // tails cover columns 64..79 at head dim 80). The pair kernel writes its output, permuted, through
 // `to` / `to_tail` (maps over p.operm laid out like Q), except the rows of split pairs, which
@@ -150,6 +162,7 @@ struct GemmEpilogue {
                             //    bf16(acc + bias), q(p) the block-major position of permuted
                             //    position p (pattern block size b, stripe length L)
                             // 3: x[unit_row_src(ur, m), n] = bf16(x + acc + bias), pad rows skipped
+                            // 4: out[M, N] = fp16(acc * scale) (the relative-position products)
   const uint16_t* bias;     // [N] or null
   uint16_t* out;            // kind 0; kind 2: gathered Q (K and V follow at which_stride)
   uint16_t* x;              // kind 1: [B, T, N]; kind 3: [B*T, N]
@@ -159,6 +172,7 @@ struct GemmEpilogue {
   long long which_stride;   // kind 2: elements from the gathered Q to K (and K to V)
   int heads, dh, C;         // kind 2: C = heads*dh columns per q, k, v
   int b, L;                 // kind 2: the pattern's block size and stripe length
+  float scale;              // kind 4
   UnitRows ur;              // kinds 2 (N) and 3
 };
 // Tile width and k-split of C[M, N] = A[M, Kd] * B[N, Kd]^T for `sms` persistent CTAs.

@@ -146,7 +146,7 @@ struct GemmShape {
 // row's (block-major) place in the gathered Q at head 0; kind 3's a pad token has no row (skipped, no error).
 __device__ __forceinline__ uint16_t* epi_row(const GemmEpilogue& ep, const GemmShape& g, int m,
                                              int* status) {
-  if (ep.kind == 0) return ep.out + (size_t)m * g.N;
+  if (ep.kind == 0 || ep.kind == 4) return ep.out + (size_t)m * g.N;
   if (ep.kind == 2) {
     const int N = ep.ur.N;
     const int u = m / N;
@@ -191,8 +191,23 @@ __device__ __forceinline__ void f2_add_bf16(float& v0, float& v1, uint32_t w) {
 }
 // Kind 0: row[n..n+32) = bf16(GELU(v + bias)). Kinds 1, 3: row[n..n+32) = bf16(x + v + bias).
 // Kind 2: bf16(v + bias), each 16 columns (within one head: dh is a multiple of 16) to its place.
+// Kind 4: row[n..n+32) = fp16(v * scale).
 __device__ __forceinline__ void epi_store(const GemmEpilogue& ep, uint16_t* row, int n,
                                           const Epi32In& in, float (&v)[32]) {
+  if (ep.kind == 4) {
+    uint4* d = reinterpret_cast<uint4*>(row + n);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __half2 h = __floats2half2_rn(v[q * 8 + 2 * e] * ep.scale, v[q * 8 + 2 * e + 1] * ep.scale);
+        w[e] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      d[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return;
+  }
   if (ep.bias) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {

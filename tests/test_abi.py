@@ -224,6 +224,36 @@ def test_encoder_block_and_stack_validation():
     assert L.sparsesam_launch_count() == 0
 
 
+def test_relpos_and_partial_validation():
+    lib = L.lib
+    by = ctypes.byref
+    g = L.make_cfg(1, 16, 16, "global", 14, 2, 64, 0.4)
+    need = L.sparsesam_attn_relpos_workspace(g)
+    # the pair kernel's workspace, the stacked tables, the bias products (fp16, 2*(31+31)->64
+    # columns per row), the key offsets
+    assert need >= L.sparsesam_attn_workspace(g) + 2 * 256 * 64 * 2
+
+    def rel(cfg=g, rh=FAKE, rw=FAKE, nbytes=1 << 40):
+        return lib.sparsesam_attn_relpos(by(cfg), FAKE, FAKE, FAKE, FAKE, rh, rw, FAKE, FAKE,
+                                         nbytes, None)
+    assert rel(nbytes=need - 1) == L.SS_EWORKSPACE
+    assert rel(rh=None) == L.SS_EINVAL and rel(rw=FAKE + 2) == L.SS_EINVAL
+    assert rel(cfg=L.make_cfg(1, 16, 16, "global", 14, 2, 80, 0.4)) == L.SS_EUNSUPPORTED
+    assert rel(cfg=L.make_cfg(1, 80, 64, "global", 14, 2, 64, 0.4)) == L.SS_EUNSUPPORTED   # 80 + 64 > 128
+
+    def part(cfg=g, prefix=1, base=10000.0, nbytes=1 << 40):
+        return lib.sparsesam_attn_partial(by(cfg), prefix, base, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                          nbytes, None)
+    pneed = L.sparsesam_attn_partial_workspace(g, 1)
+    assert pneed > L.sparsesam_attn_workspace(g)
+    assert part(nbytes=pneed - 1) == L.SS_EWORKSPACE
+    assert part(prefix=-1) == L.SS_EINVAL and part(prefix=5) == L.SS_EINVAL
+    assert part(base=0.5) == L.SS_EINVAL and part(base=float("inf")) == L.SS_EINVAL
+    assert part(cfg=L.make_cfg(1, 16, 16, "window", 14, 2, 64, 0.4)) == L.SS_EUNSUPPORTED
+    assert part(cfg=L.make_cfg(1, 16, 16, "global", 14, 33, 64, 0.4)) == L.SS_EUNSUPPORTED
+    assert L.sparsesam_launch_count() == 0
+
+
 def test_binding_raises_on_error():
     with pytest.raises(L.SparseSAMError) as e:
         L.sparsesam_pattern(L.make_cfg(1, 5, 5, density=0.4))
