@@ -471,6 +471,11 @@ def run_ours(args, wl, rank, world, local_rank, dist):
         del m2
         torch.cuda.empty_cache()
 
+    # ---- the variants (attention only), measured the same way (extra key) --------------------
+    variants = None if args.no_stack else measure_variants(args, dev, stream,
+                                                           max(10, min(args.steps, 50)),
+                                                           args.warmup)
+
     # ---- the ViT-L encoder stack of full blocks at the density sweep (extra key) --------------
     stack = None
     if not args.no_stack:
@@ -499,6 +504,7 @@ def run_ours(args, wl, rank, world, local_rank, dist):
                   "sparse_speedup": value / dense_value},
         "also": also,
         "stack": stack,
+        "variants": variants,
     }
     if world == 1:
         step_s, desc, cores, _ = cpu_sample(wl)
@@ -646,6 +652,116 @@ def measure_stack(args, dev, stream, densities, steps, warmup):
     return out
 
 
+def measure_variants(args, dev, stream, steps, warmup):
+    """Attention-only timings of the variants, each over rotating input sets (> 3x L2 in total):
+    Stripe-Sort attention with SAM's relative-position bias (ViT-B global and windowed shapes),
+    the PE-style partial attention with 2-D RoPE (PE-Core-L14-336: 128 images of 1 class token +
+    24 x 24 patches, 16 heads x 64, density 0.5), and plain attention only (the attention-only
+    registry variant) on the ViT-B global block. Per call: CUDA events around `steps` calls."""
+    import torch
+
+    from structured_activation_sparsity_b200 import _lib as L
+
+    bf16_peak = peaks()[0]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+
+    def bf(*shape, scale=1.0):
+        return (torch.randn(*shape, generator=gen, device=dev) * scale).to(torch.bfloat16)
+
+    def perm_of(cfg, U, N):
+        lum = torch.rand(cfg.batch, cfg.grid_h, cfg.grid_w, generator=gen, device=dev)
+        score = torch.empty(cfg.batch, cfg.grid_h * cfg.grid_w, dtype=torch.float64, device=dev)
+        perm = torch.empty(U, N, dtype=torch.int32, device=dev)
+        L.sparsesam_score_perm(cfg, lum, score, perm, None, None, stream)
+        return perm
+
+    def timed(calls):
+        with torch.cuda.stream(stream):
+            for i in range(warmup):
+                calls[i % len(calls)]()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        with torch.cuda.stream(stream):
+            for i in range(steps):
+                calls[i % len(calls)]()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if L.sparsesam_device_status(stream) != L.SS_OK:
+            raise RuntimeError("a device wait timed out in a variant")
+        t = ev0.elapsed_time(ev1) / 1e3 / steps
+        L.sparsesam_trace_start(64)    # one traced call: each launch's CUDA-event time
+        with torch.cuda.stream(stream):
+            calls[0]()
+        per = {}
+        for n_, ms in L.sparsesam_trace_stop():
+            per[n_] = round(per.get(n_, 0.0) + ms * 1e3, 1)
+        traced[0] = per
+        return t
+
+    out = {}
+    traced = [None]
+    for name, wl_name in (("relpos_vitb_global", "vitb_global"), ("relpos_vitb_window", "vitb_window"),
+                          ("attn_only_vitb_global", "vitb_global")):
+        wl = workloads.get(wl_name)
+        cfg = L.cfg_for(wl)
+        U, N = wl.units, wl.unit_tokens
+        pat = L.sparsesam_pattern(cfg)
+        Hu, Wu = (wl.window, wl.window) if wl.mode == "window" else (wl.grid_h, wl.grid_w)
+        relpos = name.startswith("relpos")
+        wsb = (L.sparsesam_attn_relpos_workspace(cfg) if relpos else L.sparsesam_attn_workspace(cfg))
+        per_set = 4 * U * N * wl.heads * wl.head_dim * 2 + wsb
+        n_sets = max(2, math.ceil(3 * L2_BYTES / per_set))
+        calls = []
+        for _ in range(n_sets):
+            q, k, v, o = (bf(U, N, wl.heads, wl.head_dim) for _ in range(4))
+            perm = perm_of(cfg, U, N)
+            ws = torch.empty((wsb,), dtype=torch.uint8, device=dev)
+            if relpos:
+                rh, rw = bf(2 * Hu - 1, wl.head_dim, scale=0.1), bf(2 * Wu - 1, wl.head_dim, scale=0.1)
+                calls.append(lambda q=q, k=k, v=v, o=o, perm=perm, ws=ws, rh=rh, rw=rw:
+                             L.sparsesam_attn_relpos(cfg, q, k, v, perm, rh, rw, o, ws, wsb, stream))
+            else:
+                calls.append(lambda q=q, k=k, v=v, o=o, perm=perm, ws=ws:
+                             L.sparsesam_attn(cfg, q, k, v, perm, o, ws, wsb, stream))
+        t = timed(calls)
+        flops = workloads.attn_flops(U, N, wl.heads, wl.head_dim, pat.rho)
+        out[name] = {"us_per_call": t * 1e6, "tokens_per_s": wl.batch * wl.tokens_per_image / t,
+                     "attn_tflops": flops / t / 1e12, "frac_bf16_peak": flops / t / 1e12 / bf16_peak,
+                     "traced_us": traced[0],
+                     "note": "gather + (bias GEMM) + attention + un-permute per call"}
+        del calls
+        torch.cuda.empty_cache()
+    # PE-Core-L14-336 partial attention with RoPE
+    B, G, P_, H, D, d = 128, 24, 1, 16, 64, 0.5
+    cfg = L.make_cfg(B, G, G, "global", 14, H, D, d)
+    pat = L.sparsesam_pattern(cfg)
+    wsb = L.sparsesam_attn_partial_workspace(cfg, P_)
+    NT = P_ + G * G
+    calls = []
+    n_sets = max(2, math.ceil(3 * L2_BYTES / (4 * B * NT * H * D * 2 + wsb)))
+    for _ in range(n_sets):
+        q, k, v, o = (bf(B, NT, H, D) for _ in range(4))
+        perm = perm_of(cfg, B, G * G)
+        ws = torch.empty((wsb,), dtype=torch.uint8, device=dev)
+        calls.append(lambda q=q, k=k, v=v, o=o, perm=perm, ws=ws:
+                     L.sparsesam_attn_partial(cfg, P_, 10000.0, q, k, v, perm, o, ws, wsb, stream))
+    t = timed(calls)
+    flops = workloads.attn_flops(B, G * G, H, D, pat.rho) + 4.0 * B * H * D * (
+        2 * P_ * NT - P_ * P_)   # prefix rows and the prefix keys of the patch rows
+    out["partial_pe_core_l14_336"] = {
+        "us_per_call": t * 1e6, "tokens_per_s": B * NT / t, "attn_tflops": flops / t / 1e12,
+        "frac_bf16_peak": flops / t / 1e12 / bf16_peak,
+        "config": {"images": B, "prefix": P_, "grid": f"{G}x{G}", "heads": H, "head_dim": D,
+                   "density": d, "rope_base": 10000.0, "realised_density": pat.rho},
+        "traced_us": traced[0],
+        "note": "RoPE gather + attention + prefix merge + prefix rows per call"}
+    del calls
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_stack(args, local_rank):
     """The ViT-L stack alone at the density sweep, one JSON line per density (no bench line)."""
     import torch
@@ -673,7 +789,9 @@ def main():
     ap.add_argument("--stack", action="store_true",
                     help="time the ViT-L 24-block stack at densities 1.0/0.5/0.4/0.3 (no bench line)")
     ap.add_argument("--no-stack", action="store_true",
-                    help="leave the ViT-L stack sweep out of the bench line")
+                    help="leave the ViT-L stack sweep and the variants out of the bench line")
+    ap.add_argument("--variants", action="store_true",
+                    help="time the attention variants only (no bench line)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = workloads.get(args.workload)
@@ -689,6 +807,13 @@ def main():
         return
     if args.stack:
         run_stack(args, local_rank)
+        return
+    if args.variants:
+        import torch
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        print(json.dumps(measure_variants(args, dev, torch.cuda.Stream(device=dev), args.steps,
+                                          args.warmup)), flush=True)
         return
     dist = None
     if world > 1:
