@@ -190,10 +190,11 @@ size_t sparsesam_attn_relpos_workspace(const ss_cfg* cfg);
  * window x window (window mode; pad tokens have window coordinates). rel_h (device) bf16
  * [2*Hu-1, head_dim], rel_w (device) bf16 [2*Wu-1, head_dim], 16-byte aligned, shared by the
  * heads. Everything else as sparsesam_attn. The products q.rel_h[r] and q.rel_w[r] are computed
- * on the tensor cores in fp32 and kept in fp16 (scaled by log2(e)); the bias is added to the fp32
- * score. Head dim 64 only and Hu + Wu <= 128 (SS_EUNSUPPORTED otherwise): each query row keeps
- * its Hu + Wu bias values in shared memory next to a three-stage K/V ring. ws (device, 256-byte
- * aligned) >= sparsesam_attn_relpos_workspace(cfg) bytes. */
+ * on the tensor cores in fp32 and kept in fp16 (scaled by sqrt(head_dim)); the attention adds a
+ * key's two terms to its fp32 score with one more tensor-core product (the row's bias values
+ * times the key tile's one-hot matrix). Head dim 64 only and Hu + Wu <= 128 (SS_EUNSUPPORTED
+ * otherwise): a query row's bias values fill its group's 64 spare TMEM columns. ws (device,
+ * 256-byte aligned) >= sparsesam_attn_relpos_workspace(cfg) bytes. */
 int sparsesam_attn_relpos(const ss_cfg* cfg, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int32_t* perm, const uint16_t* rel_h,
                           const uint16_t* rel_w, uint16_t* out, void* ws, size_t ws_bytes,

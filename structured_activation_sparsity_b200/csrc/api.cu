@@ -442,7 +442,8 @@ static int gather_launch(const Geo& g, int heads, int dh, const AttnLayout& L, c
 // rel: the relative-position fields of AttnParams (null: none).
 static int attn_launch(const ss_cfg* cfg, const Geo& g, const AttnLayout& L, uint8_t* ws,
                        const int32_t* perm, uint16_t* out, int* status, cudaStream_t st,
-                       float2* ml = nullptr, const AttnParams* rel = nullptr) {
+                       float2* ml = nullptr, const AttnParams* rel = nullptr,
+                       const CUtensorMap* te = nullptr) {
   const int heads = cfg->heads, dh = cfg->head_dim;
   const uint16_t* bufs[3] = {reinterpret_cast<uint16_t*>(ws),
                              reinterpret_cast<uint16_t*>(ws + L.one),
@@ -478,12 +479,11 @@ static int attn_launch(const ss_cfg* cfg, const Geo& g, const AttnLayout& L, uin
     ap.rel_ld = rel->rel_ld;
     ap.rel_h = rel->rel_h;
     ap.rel_w = rel->rel_w;
-    ap.rel_npad = rel->rel_npad;
-    ap.rel_keyoff = rel->rel_keyoff;
+    ap.rel_ksteps = rel->rel_ksteps;
   }
   int rc = cuda_err(traced("attn", st, [&] {
     return launch_attn(&tm[0], &tm[1], &tm[2], &tm[3], &tm[4], &tm[5], &tm[6], ap, dh, status,
-                       st);
+                       st, te);
   }));
   if (rc || !L.plan.pair_kernel) return rc;
   if (L.plan.tail_split > 1 &&
@@ -689,12 +689,12 @@ int sparsesam_block(const ss_cfg* cfg, const float* lum, const uint16_t* q, cons
 // ---- the relative-position variant ------------------------------------------------------------
 
 // Workspace: the attention's (pair kernel), then the stacked tables rpack [nr, dh], the bias
-// products [U*heads*N, nr] fp16 and the key offsets [U, npad].
+// products [U*heads*N, nr] fp16 and the one-hot rows [U, npad, 128] fp16.
 struct RelLayout {
   AttnLayout L;
   GemmPlan gp;
   int Hu, Wu, nr, npad;
-  size_t rpack, tab, keyoff, total;
+  size_t rpack, tab, onehot, total;
 };
 
 static int rel_layout(const ss_cfg* cfg, const Geo& g, RelLayout* R) {
@@ -708,8 +708,8 @@ static int rel_layout(const ss_cfg* cfg, const Geo& g, RelLayout* R) {
   R->gp = gemm_plan((int)M, R->nr, cfg->head_dim, kPlanSMs);
   R->rpack = align256(R->L.total);
   R->tab = R->rpack + align256((size_t)R->nr * cfg->head_dim * 2);
-  R->keyoff = R->tab + align256((size_t)M * R->nr * 2);
-  R->total = R->keyoff + align256((size_t)g.U * R->npad * 2);
+  R->onehot = R->tab + align256((size_t)M * R->nr * 2);
+  R->total = R->onehot + align256((size_t)g.U * R->npad * kRelPosOneHotCols * 2);
   return SS_OK;
 }
 
@@ -734,8 +734,8 @@ int sparsesam_attn_relpos(const ss_cfg* cfg, const uint16_t* q, const uint16_t* 
   if (cfg->head_dim != 64) return SS_EUNSUPPORTED;
   RelLayout R;
   if ((rc = rel_layout(cfg, g, &R))) return rc;
-  // The key offsets are bytes into a row of Hu + Wu fp16 slices (at most 2 * kRelPosRowWords).
-  if (R.Hu + R.Wu > 128) return SS_EUNSUPPORTED;
+  // A query row's bias slices (Hu + Wu fp16 values) fill at most the 64 TMEM columns of its group.
+  if (R.Hu + R.Wu > kRelPosOneHotCols) return SS_EUNSUPPORTED;
   if ((long long)g.U * cfg->heads * g.N * R.nr >= (1ll << 31) ||
       ((long long)g.U * cfg->heads * g.N + 127) / 128 > 65535)
     return SS_EUNSUPPORTED;
@@ -747,23 +747,28 @@ int sparsesam_attn_relpos(const ss_cfg* cfg, const uint16_t* q, const uint16_t* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint16_t* rpack = reinterpret_cast<uint16_t*>(wsb + R.rpack);
   uint16_t* tab = reinterpret_cast<uint16_t*>(wsb + R.tab);
-  uint16_t* keyoff = reinterpret_cast<uint16_t*>(wsb + R.keyoff);
+  uint16_t* onehot = reinterpret_cast<uint16_t*>(wsb + R.onehot);
   if ((rc = gather_launch(g, heads, dh, R.L, q, k, v, perm, wsb, status, st))) return rc;
   rc = cuda_err(traced("relpos_prep", st, [&] {
-    return launch_relpos_prep(rel_h, rel_w, rpack, dh, R.nr, perm, keyoff, g.U, g.N, R.npad, R.Hu,
+    return launch_relpos_prep(rel_h, rel_w, rpack, dh, R.nr, perm, onehot, g.U, g.N, R.npad, R.Hu,
                               R.Wu, R.L.ap.b, status, st);
   }));
   if (rc) return rc;
   const long long M = (long long)g.U * heads * g.N;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, te;
   if (!encode_bf16(&ta, 2, wsb, dh, M, 1, (uint64_t)dh * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_bf16(&tb, 2, rpack, dh, R.nr, 1, (uint64_t)dh * 2, 64, R.gp.bn,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      // the one-hot rows as [U][npad][128] 16-bit values: 64-column boxes of 128 rows (the
+      // layout of a K tile); TMA moves bytes, so the bf16 encoding serves the fp16 data
+      !encode_bf16(&te, 3, onehot, kRelPosOneHotCols, R.npad, g.U,
+                   (uint64_t)kRelPosOneHotCols * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return SS_ECUDA;
   GemmEpilogue e = {};
   e.kind = 4;
   e.out = tab;
-  e.scale = 1.4426950408889634f;   // log2(e): the kernel's scores are in base-2 units
+  // sqrt(dh): the attention scales S = q.k + bias * sqrt(dh) by 1/sqrt(dh) (and log2 e) as a whole
+  e.scale = (float)sqrt((double)dh);
   rc = cuda_err(traced("relpos_gemm", st, [&] {
     return launch_gemm(&ta, &tb, R.gp, (int)M, R.nr, dh, e, nullptr, nullptr, sm_count(), status,
                        st);
@@ -774,9 +779,8 @@ int sparsesam_attn_relpos(const ss_cfg* cfg, const uint16_t* q, const uint16_t* 
   rel.rel_ld = R.nr;
   rel.rel_h = R.Hu;
   rel.rel_w = R.Wu;
-  rel.rel_npad = R.npad;
-  rel.rel_keyoff = keyoff;
-  return attn_launch(cfg, g, R.L, wsb, perm, out, status, st, nullptr, &rel);
+  rel.rel_ksteps = (R.Hu + R.Wu + 15) / 16;
+  return attn_launch(cfg, g, R.L, wsb, perm, out, status, st, nullptr, &rel, &te);
 }
 
 // ---- the partial-token-count variant (prefix tokens, RoPE) -------------------------------------

@@ -237,14 +237,16 @@ struct PairTmem {
   static constexpr uint32_t kS = 0;
   static constexpr uint32_t kP = 128, kPStride = 64;
   static constexpr uint32_t kO = 256, kOStride = DH <= 64 ? 64 : 96;
+  static constexpr uint32_t kBq = 384;   // relative-position variant: A of the bias MMA, 64 per group
   static_assert(kO + kOStride + DH <= 512, "TMEM columns");
 };
 
-// kRelPos: the decomposed relative-position variant. Its softmax threads keep their row's bias
-// slices (fp16, Hu + Wu values, an odd number of 32-bit words per row so that the 32 rows a warp
-// reads at one column fall in 32 different banks) in shared memory, for which the K/V ring is
-// three stages deep.
-constexpr int kRelPosRowWords = 65;                            // (64 + 64) / 2 rounded up to odd
+// kRelPos: the decomposed relative-position variant (head dim 64). The bias is one more MMA into
+// S per tile and group: A = the group's per-row bias slices (Hu + Wu fp16 values per row, in TMEM
+// columns 384 + 64g), B = the key tile's one-hot matrix E [128 keys x 128] (fp16 1.0 at columns
+// Hu-1-kh and Hu+Wu-1-kw of key (kh, kw)), loaded by TMA with K and V. E makes the stage 64 KB, so
+// the ring is two stages deep.
+constexpr int kRelPosCols = 128;                               // E columns (Hu + Wu <= 128)
 template <int DH, bool kRelPos = false>
 struct PairSmem {
   static constexpr int kTail = DH - 64;                        // 0 or 16 columns
@@ -253,8 +255,9 @@ struct PairSmem {
   static constexpr int kQK = kQKMain + kQKTail;                // one Q or K tile
   static constexpr int kVAtom = kBN * 128;                     // 128 keys x 64 bf16, 128B swizzle
   static constexpr int kV = kTail ? 2 * kVAtom : kVAtom;
-  static constexpr int kStageBytes = kQK + kV;
-  static constexpr int kStages = kRelPos ? 3 : (DH == 64 ? 5 : 3);   // depth of the K/V ring
+  static constexpr int kE = kRelPos ? kBN * kRelPosCols * 2 : 0;   // two 128B-swizzled atoms
+  static constexpr int kStageBytes = kQK + kV + kE;
+  static constexpr int kStages = kRelPos ? 2 : (DH == 64 ? 5 : 3);   // depth of the K/V ring
   static constexpr int kQ = 0;                                 // Q_A, then Q_B
   static constexpr int kKV = 2 * kQK;
   // Output staging, used by the groups in turn: one 128-row tile of O in the layout of a Q tile
@@ -262,8 +265,7 @@ struct PairSmem {
   // of the TMA store that writes it.
   static constexpr int kStage = kKV + kStages * kStageBytes;
   static constexpr int kBar = kStage + kQK;
-  static constexpr int kTab = kBar + 512;                      // kRelPos: 2 x 128 bias rows
-  static constexpr int kBytes = kTab + (kRelPos ? 2 * kBM * kRelPosRowWords * 4 : 0);
+  static constexpr int kBytes = kBar + 512;
   static constexpr int kAlloc = kBytes + 1024;                 // slack to align the base to 1024
   static_assert(kQK % 1024 == 0 && kStageBytes % 1024 == 0 && kKV % 1024 == 0,
                 "tiles must stay 1024-byte aligned for the 128-byte swizzle");
@@ -333,12 +335,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn_pair(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tq_tail,
                 const __grid_constant__ CUtensorMap tk_tail, const __grid_constant__ CUtensorMap to,
-                const __grid_constant__ CUtensorMap to_tail, const AttnParams P, int* status) {
+                const __grid_constant__ CUtensorMap to_tail, const __grid_constant__ CUtensorMap te,
+                const AttnParams P, int* status) {
   using S = PairSmem<DH, kRelPos>;
   using T = PairTmem<DH>;
   constexpr int NS = S::kStages;
   constexpr bool kHasTail = S::kTail > 0;
   static_assert(!(kRelPos && kHasTail), "the relative-position variant is built for head dim 64");
+  static_assert(!kRelPos || T::kBq == T::kO + 2 * T::kOStride, "bias columns follow O_B");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -353,7 +357,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* pv_done = p_full + 4;            // [2] P_g * V of a tile done
   uint64_t* stage_free = pv_done + 2;        // the staging tile read by its TMA store
   uint64_t* staged = stage_free + 1;         // a group's rows are in the staging tile
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(staged + 1);
+  uint64_t* bq_full = staged + 1;            // [2] relative-position variant: group g's bias rows
+                                             // of the piece are in TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bq_full + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -376,6 +382,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     mbar_init(stage_free, 1);
     mbar_init(staged, 128);
+    mbar_init(bq_full + 0, 128);
+    mbar_init(bq_full + 1, 128);
     *abort = 0;
     fence_barrier_init();
   }
@@ -420,6 +428,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tma_load_3d(vb, &tv, kv_full + st, 0, c0, c.uh);
           // head dim 80: columns 64..127 of V; 80..127 lie outside the tensor and read as zero
           if (kHasTail) tma_load_3d(vb + S::kVAtom, &tv, kv_full + st, 64, c0, c.uh);
+          if constexpr (kRelPos) {   // the key tile's one-hot matrix (per unit, not per head)
+            uint8_t* eb = vb + S::kV;
+            const int u_c = c.uh / P.heads;
+            tma_load_3d(eb, &te, kv_full + st, 0, c0, u_c);
+            tma_load_3d(eb + kBN * 128, &te, kv_full + st, 64, c0, u_c);
+          }
         }
       }
     } else if (warp == 1 && lane == 0) {
@@ -431,6 +445,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const Piece c = piece_of(i, npairs, P);
         if (!(ok = mbar_wait(q_full + 0, li & 1, abort, status))) break;
         if (!(ok = mbar_wait(q_full + 1, li & 1, abort, status))) break;
+        if constexpr (kRelPos) {   // both groups' bias rows of this piece are in TMEM
+          if (!(ok = mbar_wait(bq_full + 0, li & 1, abort, status))) break;
+          if (!(ok = mbar_wait(bq_full + 1, li & 1, abort, status))) break;
+          tc_fence_after();
+        }
         for (int n = c.n0; ok && n < c.n1; ++n, ++gn) {
           const int st = gn % NS;
           if (!(ok = mbar_wait(kv_full + st, (gn / NS) & 1, abort, status))) break;
@@ -449,6 +468,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (kHasTail)
               umma_bf16_ss(d, smem_desc(q_addr + S::kQKMain, 16, 256, kSwizzle32B),
                            smem_desc(k_addr + S::kQKMain, 16, 256, kSwizzle32B), idesc_qk, 1);
+            if constexpr (kRelPos) {
+              // S += Bq_g E^T: each key's two bias terms, summed by the tensor core (fp16 x 1.0).
+              const uint32_t e_addr = k_addr + S::kQK + S::kV;
+              for (int kk = 0; kk < P.rel_ksteps; ++kk)
+                umma_bf16_ts(d, tmem + T::kBq + g * 64 + kk * 8,
+                             smem_desc(e_addr + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024,
+                                       kSwizzle128B),
+                             idesc_f16_f32(kBM, kBN, false, false), 1u);
+            }
             umma_commit(s_full + g);
           }
         }
@@ -525,12 +553,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t t_p = tmem + T::kP + grp * T::kPStride + lane_off;
     const uint32_t t_o = tmem + T::kO + grp * T::kOStride + lane_off;
     const int b4 = P.b * kStripes;
-    // The relative-position variant scales S (and adds the bias) before the row max; the
-    // exponents are then x - ref.
-    const float max_scale = kRelPos ? 1.f : P.scale_log2;
-    const uint64_t scale2 = kRelPos ? f2_pack(1.f, 1.f) : f2_pack(P.scale_log2, P.scale_log2);
-    const uint32_t tab_row =
-        smem_u32(smem + S::kTab) + uint32_t((grp * kBM + row) * kRelPosRowWords * 4);
+    const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
     constexpr int kSlot = (DH + 2) * kBM;               // floats of one group's partial
     bool ok = true;
     int gn = 0;            // tiles of this group so far (all pieces): the phase count
@@ -545,18 +568,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int band_lo = s_q * b4, band_hi = (s_q + P.W) * b4, glob_hi = P.g * b4;
       float m_ref = -INFINITY, l_run = 0.f;
       if constexpr (kRelPos) {
-        // This row's bias slices: entries qh .. qh+Hu-1 of its Rh products, then qw .. qw+Wu-1
-        // of its Rw products (the row of the bias GEMM), so that key (kh, kw) finds its terms
-        // at Hu-1-kh and Hu+Wu-1-kw.
+        // This row's bias slices into TMEM (A of the bias MMA): entries qh .. qh+Hu-1 of its Rh
+        // products, then qw .. qw+Wu-1 of its Rw products (the row of the bias GEMM), so that key
+        // (kh, kw) meets them at columns Hu-1-kh and Hu+Wu-1-kw of E. The previous piece's bias
+        // MMAs of this group are complete: this thread has read every S they fed.
         const int qr = min(qrow, P.N - 1);
         const int tok = __ldg(P.perm + (size_t)u_i * P.N + blockmajor_to_canonical(qr, P.b, P.L));
         const int t = (unsigned)tok < (unsigned)P.N ? tok : 0;
         const int qh = t / P.rel_w, qw = t - qh * P.rel_w;
         const uint16_t* g = P.rel_tab + ((size_t)c.uh * P.N + qr) * P.rel_ld;
-        for (int e = 0; e < P.rel_h; ++e)
-          st_shared_u16(tab_row + 2 * e, __ldg(g + qh + e));
-        for (int e = 0; e < P.rel_w; ++e)
-          st_shared_u16(tab_row + 2 * (P.rel_h + e), __ldg(g + 2 * P.rel_h - 1 + qw + e));
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          uint32_t w[32];
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) {
+            uint32_t lohi[2];
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) {
+              const int e = 64 * half + 2 * e2 + s2;
+              uint16_t h = 0;
+              if (e < P.rel_h) h = __ldg(g + qh + e);
+              else if (e < P.rel_h + P.rel_w) h = __ldg(g + 2 * P.rel_h - 1 + qw + (e - P.rel_h));
+              lohi[s2] = h;
+            }
+            w[e2] = lohi[0] | (lohi[1] << 16);
+          }
+          tmem_st32_async(tmem + T::kBq + grp * 64 + half * 32 + lane_off, w);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bq_full + grp);
       }
       for (int n = c.n0; ok && n < c.n1; ++n, ++gn) {
         const int j = n - c.n0;
@@ -577,24 +618,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // Has this group's previous P * V released P_g and O_g? Tested now, waited for below.
         bool prev_pv_done = gn == 0 || mbar_test(pv_done + grp, (gn - 1) & 1);
         const int c0 = c.tiles.tile(n) * kBN;
-        if constexpr (kRelPos) {
-          // s*scale_log2 + bias: key k's two byte offsets into this row's slices, 8 keys per load
-          // (the same addresses for every lane).
-          const uint4* ko =
-              reinterpret_cast<const uint4*>(P.rel_keyoff + (size_t)u_i * P.rel_npad + c0);
-#pragma unroll
-          for (int k8 = 0; k8 < kBN / 8; ++k8) {
-            const uint4 w = __ldg(ko + k8);
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint32_t off = (ww[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu;
-              const float bias = ld_shared_f16(tab_row + (off & 0xFFu)) +
-                                 ld_shared_f16(tab_row + (off >> 8));
-              sv[8 * k8 + e] = fmaf(sv[8 * k8 + e], P.scale_log2, bias);
-            }
-          }
-        }
         if (!pair_tile_full(c0, P)) {
           // The row's kept keys in this tile are two runs, [0, e0) and [s1, e1) relative to c0:
           // turned into four 32-bit column masks, so the per-key test has no branch.
@@ -617,7 +640,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], sv[k + 8 * 15]);
         const float x_max = fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])),
                                   fmaxf(mx[6], mx[7])) *
-                            max_scale;
+                            P.scale_log2;
         // Lazy rescale: the reference max moves only when the row max passes it by 2^8, so O in
         // TMEM is rescaled on few tiles. The decision is warp-wide (TMEM ops are warp-collective).
         const bool grow = x_max > m_ref + kLazyRescale;
@@ -1191,8 +1214,8 @@ template <int DH, bool kRelPos = false>
 static cudaError_t launch_attn_pair(const CUtensorMap* tq, const CUtensorMap* tk,
                                     const CUtensorMap* tv, const CUtensorMap* tq_tail,
                                     const CUtensorMap* tk_tail, const CUtensorMap* to,
-                                    const CUtensorMap* to_tail, const AttnParams& p, int* status,
-                                    cudaStream_t st) {
+                                    const CUtensorMap* to_tail, const CUtensorMap* te,
+                                    const AttnParams& p, int* status, cudaStream_t st) {
   using S = PairSmem<DH, kRelPos>;
   auto kernel = k_attn_pair<DH, kRelPos>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1201,7 +1224,7 @@ static cudaError_t launch_attn_pair(const CUtensorMap* tq, const CUtensorMap* tk
   const int pieces = p.whole + (pairs_per_head(p.N) * p.U * p.heads - p.whole) * p.tail_split;
   dim3 grid(std::max(1, std::min(pieces, p.sms)));
   return launch_pdl(kernel, grid, dim3(kAttnThreads), S::kAlloc, st, *tq, *tk, *tv, *tq_tail,
-                    *tk_tail, *to, *to_tail, p, status);
+                    *tk_tail, *to, *to_tail, *te, p, status);
 }
 
 // Short items: every query tile has at most kPairTiles key tiles (the windowed blocks).
@@ -1305,14 +1328,15 @@ __global__ void __launch_bounds__(kBM) k_merge_pieces(const float* __restrict__ 
 cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                         const CUtensorMap* tq_tail, const CUtensorMap* tk_tail,
                         const CUtensorMap* to, const CUtensorMap* to_tail, const AttnParams& p,
-                        int dh, int* status, cudaStream_t st) {
+                        int dh, int* status, cudaStream_t st, const CUtensorMap* te) {
   if (p.rel_tab) {
-    if (dh != 64) return cudaErrorInvalidValue;
-    return launch_attn_pair<64, true>(tq, tk, tv, tq, tk, to, to, p, status, st);
+    if (dh != 64 || !te) return cudaErrorInvalidValue;
+    return launch_attn_pair<64, true>(tq, tk, tv, tq, tk, to, to, te, p, status, st);
   }
   if (dh == 64 && short_items(p)) return launch_attn_pairs(tq, tk, tv, p, status, st);
-  if (dh == 64) return launch_attn_pair<64>(tq, tk, tv, tq, tk, to, to, p, status, st);
-  if (dh == 80) return launch_attn_pair<80>(tq, tk, tv, tq_tail, tk_tail, to, to_tail, p, status, st);
+  if (dh == 64) return launch_attn_pair<64>(tq, tk, tv, tq, tk, to, to, tq, p, status, st);
+  if (dh == 80)
+    return launch_attn_pair<80>(tq, tk, tv, tq_tail, tk_tail, to, to_tail, tq, p, status, st);
   return cudaErrorInvalidValue;
 }
 

@@ -56,13 +56,13 @@ struct AttnParams {
   uint16_t* operm;       // pair kernel output: [U*heads, N, dh] in block-major permuted order
   float2* ml;            // null, or [U*heads, N] (block-major): each row's running max m and
                          // sum l of 2^(s*scale_log2 - m) over its kept keys, s = q.k
-  // Decomposed relative-position bias (null rel_tab: none). rel_tab [U*heads*N, rel_ld] fp16 in
-  // block-major row order: the row's q . Rh[r] * log2(e) at column r < 2*rel_h - 1, then q . Rw[r]
-  // * log2(e) from column 2*rel_h - 1; rel_h x rel_w is the unit grid. rel_keyoff [U, rel_npad]
-  // (block-major key order): byte offsets (rel_h-1-kh)*2 | ((rel_h+rel_w-1-kw)*2) << 8.
+  // Decomposed relative-position bias (null rel_tab: none; head dim 64). rel_tab [U*heads*N,
+  // rel_ld] fp16 in block-major row order: the row's q . Rh[r] * sqrt(dh) at column r <
+  // 2*rel_h - 1, then q . Rw[r] * sqrt(dh) from column 2*rel_h - 1 (rel_h x rel_w: the unit
+  // grid); the key tiles' one-hot matrices come by the launch's `te` map over [U, npad, 128] fp16;
+  // rel_ksteps = the bias MMA's K steps of 16 columns, ceil((rel_h + rel_w) / 16).
   const uint16_t* rel_tab;
-  int rel_ld, rel_h, rel_w, rel_npad;
-  const uint16_t* rel_keyoff;
+  int rel_ld, rel_h, rel_w, rel_ksteps;
 };
 // Which attention kernel a shape takes, and the scratch beyond the gathered Q, K, V it needs
 // (planned for `sms` CTAs).
@@ -72,10 +72,12 @@ struct AttnPlan {
   size_t partial_bytes;
 };
 AttnPlan attn_plan(const AttnParams& p, int dh, int sms, bool force_pair = false);
+constexpr int kRelPosOneHotCols = 128;   // columns of a one-hot row (Hu + Wu <= 128)
 // The relative-position variant's inputs: the tables stacked into rpack [nr, dh] (the bias GEMM's
-// B operand) and the key offsets keyoff [U, npad] of AttnParams::rel_keyoff.
+// B operand) and every key position's one-hot row of E [U, npad, 128] fp16 (1.0 at columns
+// Hu-1-kh and Hu+Wu-1-kw; zero rows past N).
 cudaError_t launch_relpos_prep(const uint16_t* rel_h, const uint16_t* rel_w, uint16_t* rpack,
-                               int dh, int nr, const int32_t* perm, uint16_t* keyoff, int U, int N,
+                               int dh, int nr, const int32_t* perm, uint16_t* onehot, int U, int N,
                                int npad, int Hu, int Wu, int b, int* status, cudaStream_t st);
 // Block-sparse attention over the gathered sequences (tensor maps over [U*heads, N, dh]; the
 // tails cover columns 64..79 at head dim 80). The pair kernel writes its output, permuted, through
@@ -85,7 +87,7 @@ cudaError_t launch_relpos_prep(const uint16_t* rel_h, const uint16_t* rel_w, uin
 cudaError_t launch_attn(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                         const CUtensorMap* tq_tail, const CUtensorMap* tk_tail,
                         const CUtensorMap* to, const CUtensorMap* to_tail, const AttnParams& p,
-                        int dh, int* status, cudaStream_t st);
+                        int dh, int* status, cudaStream_t st, const CUtensorMap* te = nullptr);
 // Rows of Op for the split pairs: the pieces' (O, m, l) in p.partial combined and normalised
 // (nothing when the plan splits no pair).
 cudaError_t launch_merge_pieces(const AttnParams& p, int dh, cudaStream_t st);

@@ -1,7 +1,8 @@
 """sparsesam_attn_relpos (SAM's decomposed relative-position bias fused into the attention) against
 the oracle. Same bar as the other attention outputs: max-abs 2e-2, mean-abs 2e-3. The bias products
 q.R are computed on the tensor cores in fp32 and kept in fp16 (relative rounding 2^-11), below the
-bf16 rounding of q and k that every score already carries. The permutation is the oracle's."""
+bf16 rounding of q and k that every score already carries; the attention sums them into the score
+exactly (fp16 times a one-hot 1.0). The permutation is the oracle's."""
 import numpy as np
 import pytest
 import torch
