@@ -748,12 +748,15 @@ int sparsesam_attn_relpos(const ss_cfg* cfg, const uint16_t* q, const uint16_t* 
   uint16_t* rpack = reinterpret_cast<uint16_t*>(wsb + R.rpack);
   uint16_t* tab = reinterpret_cast<uint16_t*>(wsb + R.tab);
   uint16_t* onehot = reinterpret_cast<uint16_t*>(wsb + R.onehot);
-  if ((rc = gather_launch(g, heads, dh, R.L, q, k, v, perm, wsb, status, st))) return rc;
+  // The packed tables are the bias GEMM's B operand, whose first tiles it requests before its
+  // dependency wait: they come from the launch before the gather (which completes before the
+  // gather lets the GEMM start).
   rc = cuda_err(traced("relpos_prep", st, [&] {
     return launch_relpos_prep(rel_h, rel_w, rpack, dh, R.nr, perm, onehot, g.U, g.N, R.npad, R.Hu,
                               R.Wu, R.L.ap.b, status, st);
   }));
   if (rc) return rc;
+  if ((rc = gather_launch(g, heads, dh, R.L, q, k, v, perm, wsb, status, st))) return rc;
   const long long M = (long long)g.U * heads * g.N;
   CUtensorMap ta, tb, te;
   if (!encode_bf16(&ta, 2, wsb, dh, M, 1, (uint64_t)dh * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||

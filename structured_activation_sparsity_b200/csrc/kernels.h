@@ -189,7 +189,8 @@ int gemm_tail(int tiles, int kb, int sms);
 // fp32 partial-tile bytes the plan needs (0 without a k-split); plus one int counter per tile.
 size_t gemm_partial_bytes(const GemmPlan& p);
 // C = A B^T on tcgen05 with the given epilogue. partial / counters: workspace for k-splits
-// (counters zero on entry).
+// (counters zero on entry). B must not be written by the launch directly before this one: its
+// first tiles are requested before the kernel's dependency wait (weights are the caller's).
 cudaError_t launch_gemm(const CUtensorMap* ta, const CUtensorMap* tb, const GemmPlan& p, int M,
                         int N, int Kd, const GemmEpilogue& ep, float* partial, int* counters,
                         int sms, int* status, cudaStream_t st);
