@@ -95,13 +95,14 @@ struct UnitMap {
   }
 };
 
-// grid (ceil(N/32), units), block 32 * WARPS, dynamic smem N * 8 bytes (16-byte aligned).
-// Each CTA ranks 32 target tokens; its WARPS warps split the unit's keys and count, for all 32
-// targets at once, the keys that come before each target.
+// grid (ceil(N/(32*TG)), units), block 32 * WARPS, dynamic smem N * 8 bytes (16-byte aligned).
+// Each CTA ranks TG groups of 32 target tokens; its WARPS warps split the unit's keys and count,
+// for the 32 targets of a group at once, the keys that come before each target. More groups per
+// CTA mean fewer CTAs filling the same keys (worth it once the grid exceeds a couple of waves).
 // FROM_LUM: the keys are the Sobel scores computed here from `lum` (S1 fused into S2); each CTA
-// also stores the scores of its 32 target tokens into `score_out`, so every real token's score is
+// also stores the scores of its target tokens into `score_out`, so every real token's score is
 // written once.
-template <int WARPS, bool FROM_LUM>
+template <int WARPS, bool FROM_LUM, int TG = 1>
 __global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __restrict__ score,
                                                             const float* __restrict__ lum,
                                                             double* __restrict__ score_out,
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __rest
                                                             int32_t* __restrict__ inv,
                                                             int32_t* __restrict__ keep) {
   extern __shared__ __align__(16) unsigned long long s_key[];
-  __shared__ int s_cnt[WARPS][32];
+  __shared__ int s_cnt[TG][WARPS][32];
   griddep_wait();
   griddep_launch();
   const int u = blockIdx.y;
@@ -159,51 +160,57 @@ __global__ void __launch_bounds__(32 * WARPS) k_stripe_rank(const double* __rest
   cta_sync_converged();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 32 + lane;
-  const int tt = t < N ? t : N - 1;
-  const unsigned long long kt = s_key[tt];
   const int chunk = (((N + WARPS - 1) / WARPS) + 1) & ~1;   // even: pairs stay 16-byte aligned
   const int lo = min(N, warp * chunk), hi = min(N, lo + chunk);
   const ulonglong2* s_pair = reinterpret_cast<const ulonglong2*>(s_key);
-  // Tokens before tt count when their key is >= kt (ties broken by the lower index), tokens
-  // after it only when strictly greater: two runs, no per-element index compare. Keys are read
-  // in pairs (one 16-byte shared load, the same address across the warp: a broadcast); four
-  // independent counters keep the compare chains short.
-  const int mid = max(lo, min(hi, tt));
-  int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
-  int o = lo;
-  for (; o + 4 <= mid; o += 4) {
-    const ulonglong2 p = s_pair[o >> 1], q = s_pair[(o >> 1) + 1];
-    c0 += p.x >= kt;
-    c1 += p.y >= kt;
-    c2 += q.x >= kt;
-    c3 += q.y >= kt;
+#pragma unroll 1
+  for (int gi = 0; gi < TG; ++gi) {
+    const int t = (blockIdx.x * TG + gi) * 32 + lane;
+    const int tt = t < N ? t : N - 1;
+    const unsigned long long kt = s_key[tt];
+    // Tokens before tt count when their key is >= kt (ties broken by the lower index), tokens
+    // after it only when strictly greater: two runs, no per-element index compare. Keys are read
+    // in pairs (one 16-byte shared load, the same address across the warp: a broadcast); four
+    // independent counters keep the compare chains short.
+    const int mid = max(lo, min(hi, tt));
+    int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+    int o = lo;
+    for (; o + 4 <= mid; o += 4) {
+      const ulonglong2 p = s_pair[o >> 1], q = s_pair[(o >> 1) + 1];
+      c0 += p.x >= kt;
+      c1 += p.y >= kt;
+      c2 += q.x >= kt;
+      c3 += q.y >= kt;
+    }
+    for (; o < mid; ++o) c0 += s_key[o] >= kt;
+    if ((o & 1) && o < hi) c1 += s_key[o++] > kt;   // back to an even index
+    for (; o + 4 <= hi; o += 4) {
+      const ulonglong2 p = s_pair[o >> 1], q = s_pair[(o >> 1) + 1];
+      c0 += p.x > kt;
+      c1 += p.y > kt;
+      c2 += q.x > kt;
+      c3 += q.y > kt;
+    }
+    for (; o < hi; ++o) c0 += s_key[o] > kt;
+    s_cnt[gi][warp][lane] = (c0 + c1) + (c2 + c3);
   }
-  for (; o < mid; ++o) c0 += s_key[o] >= kt;
-  if ((o & 1) && o < hi) c1 += s_key[o++] > kt;   // back to an even index
-  for (; o + 4 <= hi; o += 4) {
-    const ulonglong2 p = s_pair[o >> 1], q = s_pair[(o >> 1) + 1];
-    c0 += p.x > kt;
-    c1 += p.y > kt;
-    c2 += q.x > kt;
-    c3 += q.y > kt;
-  }
-  for (; o < hi; ++o) c0 += s_key[o] > kt;
-  const int cnt = (c0 + c1) + (c2 + c3);
-  s_cnt[warp][lane] = cnt;
   cta_sync_converged();
-  if (warp == 0 && t < N) {
-    int r = 0;
+  if (warp < TG) {
+    const int t = (blockIdx.x * TG + warp) * 32 + lane;
+    if (t < N) {
+      const unsigned long long kt = s_key[t];
+      int r = 0;
 #pragma unroll
-    for (int w = 0; w < WARPS; ++w) r += s_cnt[w][lane];
-    const int L = N / kStripes;
-    const int pos = (r % kStripes) * L + r / kStripes;   // stripe transpose
-    if (perm) perm[(size_t)u * N + pos] = t;
-    if (inv) inv[(size_t)u * N + t] = pos;
-    if (keep && r < K) keep[(size_t)u * K + r] = t;
-    if (FROM_LUM && score_out) {
-      int b, y, x;
-      if (m.locate(u, t, b, y, x)) score_out[((size_t)b * m.Hg + y) * m.Wg + x] = key_value(kt);
+      for (int w = 0; w < WARPS; ++w) r += s_cnt[warp][w][lane];
+      const int L = N / kStripes;
+      const int pos = (r % kStripes) * L + r / kStripes;   // stripe transpose
+      if (perm) perm[(size_t)u * N + pos] = t;
+      if (inv) inv[(size_t)u * N + t] = pos;
+      if (keep && r < K) keep[(size_t)u * K + r] = t;
+      if (FROM_LUM && score_out) {
+        int b, y, x;
+        if (m.locate(u, t, b, y, x)) score_out[((size_t)b * m.Hg + y) * m.Wg + x] = key_value(kt);
+      }
     }
   }
 }
@@ -226,21 +233,23 @@ cudaError_t launch_stripe_rank(const double* score, const float* lum, double* sc
   m.wpr = window_mode ? (Wg + ws - 1) / ws : 1;
   m.nwin = window_mode ? m.wpr * ((Hg + ws - 1) / ws) : 1;
   size_t smem = (size_t)N * sizeof(unsigned long long);
-  dim3 grid((N + 31) / 32, units);
   // Long units split their keys over 32 warps per CTA (a shorter count per warp), short ones
-  // over 8 (more CTAs per SM).
-  auto go = [&](auto kernel, int warps) -> cudaError_t {
-    if (smem > 48 * 1024) {
-      cudaError_t e =
-          cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-    }
+  // over 8 (more CTAs per SM). When one group of 32 targets per CTA would take more than one wave
+  // of CTAs (two per SM at 32 warps), each CTA ranks four groups against the keys it filled once.
+  const bool big = (long long)units * ((N + 31) / 32) > 2LL * 148;
+  auto go = [&](auto kernel, int warps, int tg) -> cudaError_t {
+    cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((N + 32 * tg - 1) / (32 * tg), units);
     return launch_pdl(kernel, grid, dim3(32 * warps), smem, st, score, lum, score_out, m, N, K,
                       perm, inv, keep);
   };
+  if (N >= 2048 && big)
+    return lum ? go(k_stripe_rank<32, true, 4>, 32, 4) : go(k_stripe_rank<32, false, 4>, 32, 4);
   if (lum)
-    return N >= 2048 ? go(k_stripe_rank<32, true>, 32) : go(k_stripe_rank<8, true>, 8);
-  return N >= 2048 ? go(k_stripe_rank<32, false>, 32) : go(k_stripe_rank<8, false>, 8);
+    return N >= 2048 ? go(k_stripe_rank<32, true>, 32, 1) : go(k_stripe_rank<8, true>, 8, 1);
+  return N >= 2048 ? go(k_stripe_rank<32, false>, 32, 1) : go(k_stripe_rank<8, false>, 8, 1);
 }
 
 // ---------------------------------------------------------------------------------------------
