@@ -39,6 +39,7 @@ __global__ void __launch_bounds__(256) k_gather_rope(const uint16_t* __restrict_
   griddep_wait();
   griddep_launch();
   constexpr int DH = CPR * 8, HALF = DH / 2, QUART = DH / 4;
+  __shared__ float2 s_rot[8][DH / 2];   // per warp: (cos, sin) of the token's dh/2 channel pairs
   const int u = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qpos = blockIdx.x * 8 + warp;
@@ -67,23 +68,31 @@ __global__ void __launch_bounds__(256) k_gather_rope(const uint16_t* __restrict_
       if (c < per_tok) buf[t][e] = __ldg(src[t] + c);
     }
   const int y = tok / grid_w, x = tok - y * grid_w;
-#pragma unroll
-  for (int e = 0; e < KPL; ++e) {
-    const int c = e * 32 + lane;
-    if (c >= per_tok || rope_log2_base == 0.f) continue;
-    const int cc = c % CPR;
-    uint32_t* wq = reinterpret_cast<uint32_t*>(&buf[0][e]);
-    uint32_t* wk = reinterpret_cast<uint32_t*>(&buf[1][e]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int d = cc * 8 + 2 * j;
+  if (rope_log2_base != 0.f) {
+    // The token's dh/2 angles (the same for every head), one or two per lane, shared by the warp.
+    for (int pr = lane; pr < DH / 2; pr += 32) {
+      const int d = 2 * pr;
       const bool col = d >= HALF;
       const int i = (d - (col ? HALF : 0)) >> 1;
       const float theta = exp2f(-(float)i * rope_log2_base / (float)QUART);
       float sn, cs;
       sincosf((float)(col ? x : y) * theta, &sn, &cs);
-      wq[j] = rope_pair(wq[j], cs, sn);
-      wk[j] = rope_pair(wk[j], cs, sn);
+      s_rot[warp][pr] = make_float2(cs, sn);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+      const int c = e * 32 + lane;
+      if (c >= per_tok) continue;
+      const int cc = c % CPR;
+      uint32_t* wq = reinterpret_cast<uint32_t*>(&buf[0][e]);
+      uint32_t* wk = reinterpret_cast<uint32_t*>(&buf[1][e]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 r = s_rot[warp][cc * 4 + j];
+        wq[j] = rope_pair(wq[j], r.x, r.y);
+        wk[j] = rope_pair(wk[j], r.x, r.y);
+      }
     }
   }
 #pragma unroll
@@ -120,8 +129,9 @@ cudaError_t launch_gather_rope(const uint16_t* q, const uint16_t* k, const uint1
 // k[u, j]) are combined in one more online-softmax step, with s_j = q_rot . k_j:
 //   M = max(m, s_j * scale_log2), a = l * 2^(m - M), c_j = 2^(s_j * scale_log2 - M),
 //   out[u, prefix + tok] = (po * a + sum_j c_j v_j) / (a + sum_j c_j).
-// The dot products are summed per head through shared memory (a head's chunks may span two of a
-// lane's chunk slots).
+// The dot products are summed per head by shuffles at head dim 64 (a head's 8 chunks sit in 8
+// adjacent lanes of one slot), through shared memory at head dim 80 (a head's 10 chunks may span
+// two of a lane's slots).
 template <int CPR, int KPL>
 __global__ void __launch_bounds__(256) k_prefix_merge(const uint16_t* __restrict__ po,
                                                       const float2* __restrict__ ml,
@@ -156,20 +166,38 @@ __global__ void __launch_bounds__(256) k_prefix_merge(const uint16_t* __restrict
   const uint4* vbase = reinterpret_cast<const uint4*>(v) + (size_t)u * (N + prefix) * per_tok;
 #pragma unroll
   for (int e = 0; e < KPL; ++e) {
+    // Every lane takes part in every iteration (the shuffles below need the whole warp); lanes
+    // past the row's chunks contribute zeros and write nothing.
     const int c = e * 32 + lane;
-    if (c >= per_tok) continue;
-    const int h = c / CPR, cc = c - h * CPR;
-    const uint4 qv = __ldg(qrow + h * plane + cc);
-    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+    const bool active = c < per_tok;
+    const int h = active ? c / CPR : 0, cc = active ? c - h * CPR : 0;
+    uint32_t qw[4] = {0u, 0u, 0u, 0u};
+    if (active) {
+      const uint4 qv = __ldg(qrow + h * plane + cc);
+      qw[0] = qv.x;
+      qw[1] = qv.y;
+      qw[2] = qv.z;
+      qw[3] = qv.w;
+    }
     for (int j = 0; j < prefix; ++j) {
-      const uint4 kv = __ldg(kbase + (size_t)j * per_tok + c);
-      const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
       float d = 0.f;
+      if (active) {
+        const uint4 kv = __ldg(kbase + (size_t)j * per_tok + c);
+        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-      for (int t = 0; t < 4; ++t)
-        d += __uint_as_float(qw[t] << 16) * __uint_as_float(kw[t] << 16) +
-             __uint_as_float(qw[t] & 0xFFFF0000u) * __uint_as_float(kw[t] & 0xFFFF0000u);
-      atomicAdd(&s_dot[warp][h][j], d);
+        for (int t = 0; t < 4; ++t)
+          d += __uint_as_float(qw[t] << 16) * __uint_as_float(kw[t] << 16) +
+               __uint_as_float(qw[t] & 0xFFFF0000u) * __uint_as_float(kw[t] & 0xFFFF0000u);
+      }
+      if constexpr (CPR == 8) {
+        // a head's 8 chunks sit in 8 adjacent lanes of this slot: reduce among them
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        d += __shfl_xor_sync(0xffffffffu, d, 2);
+        d += __shfl_xor_sync(0xffffffffu, d, 4);
+        if (active && (lane & 7) == 0) s_dot[warp][h][j] = d;
+      } else {
+        if (active) atomicAdd(&s_dot[warp][h][j], d);
+      }
     }
   }
   __syncwarp();
@@ -245,7 +273,7 @@ __global__ void __launch_bounds__(256) k_prefix_rows(const uint16_t* __restrict_
   extern __shared__ float s_score[];                  // [prefix + N]
   __shared__ float s_q[DH];
   __shared__ float s_red[8];
-  __shared__ float s_acc[256 / DH][DH];
+  __shared__ float2 s_acc[8][DH / 2];
   const int j = blockIdx.x % prefix, uh = blockIdx.x / prefix;
   const int u = uh / heads, h = uh - u * heads;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -293,21 +321,36 @@ __global__ void __launch_bounds__(256) k_prefix_rows(const uint16_t* __restrict_
   __syncthreads();
   float Ls = 0.f;
   for (int w = 0; w < 8; ++w) Ls += s_red[w];
-  // Output: thread (r, d) sums p_t v_t[d] over the keys t = r, r + R, ... (R = 256 / DH groups).
-  constexpr int R = 256 / DH;
-  const int r = tid / DH, d = tid - r * DH;
-  if (r < R) {
-    float acc = 0.f;
-    for (int t = r; t < n_keys; t += R) acc += s_score[t] * __uint_as_float(uint32_t(key_row(v, vp, t)[d]) << 16);
-    s_acc[r][d] = acc;
+  // Output: warp w sums p_t v_t over the keys t = w, w + 8, ...; lane l holds the channel pairs
+  // l and l + 32 (one coalesced 4-byte load per pair and key); the 8 warps' sums then meet.
+  constexpr int DP = DH / 2;
+  float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  for (int t = warp; t < n_keys; t += 8) {
+    const float pt = s_score[t];
+    const uint32_t* vr = reinterpret_cast<const uint32_t*>(key_row(v, vp, t));
+#pragma unroll
+    for (int r2 = 0; r2 < 2; ++r2) {
+      const int pr = lane + 32 * r2;
+      if (pr < DP) {
+        const uint32_t w = __ldg(vr + pr);
+        acc[r2].x += pt * __uint_as_float(w << 16);
+        acc[r2].y += pt * __uint_as_float(w & 0xFFFF0000u);
+      }
+    }
   }
+#pragma unroll
+  for (int r2 = 0; r2 < 2; ++r2)
+    if (lane + 32 * r2 < DP) s_acc[warp][lane + 32 * r2] = acc[r2];
   __syncthreads();
-  if (tid < DH) {
-    float acc = 0.f;
-    for (int rr = 0; rr < R; ++rr) acc += s_acc[rr][tid];
-    const float o = Ls > 0.f ? acc / Ls : 0.f;
-    out[((size_t)u * n_keys + j) * tok_stride + (size_t)h * DH + tid] =
-        (uint16_t)(pack_bf16(o, 0.f) & 0xFFFFu);
+  if (tid < DP) {
+    float2 a = make_float2(0.f, 0.f);
+    for (int w = 0; w < 8; ++w) {
+      a.x += s_acc[w][tid].x;
+      a.y += s_acc[w][tid].y;
+    }
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+    reinterpret_cast<uint32_t*>(out + ((size_t)u * n_keys + j) * tok_stride + (size_t)h * DH)[tid] =
+        pack_bf16(a.x * inv, a.y * inv);
   }
 }
 
