@@ -48,8 +48,7 @@ L2_BYTES = 126 * 1024 * 1024
 # capture of the current attention kernel on that workload (profiles/ names the capture). A
 # workload is absent (traffic null) until its capture is taken again after a kernel change.
 ATTN_TRAFFIC_BYTES = {
-    "vith_global": 125_914_368 + 21_509_376,    # k_attn_pair<80>: profiles/attn_pair_vith_global.md
-    "vitb_global": 18_953_984 + 0,              # k_attn_pair<64>: profiles/attn_pair_vitb_global.md
+    "vith_global": 125_915_648 + 21_010_176,    # k_attn_pair<80>: profiles/attn_pair_vith_global.md
     "vitb_window": 90_458_880 + 9_328_384,      # k_attn_pairs: profiles/attn_pairs_vitb_window.md
 }
 
