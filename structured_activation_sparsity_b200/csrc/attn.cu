@@ -208,13 +208,11 @@ __device__ __forceinline__ Item item_of(int it, int nq, const AttnParams& P) {
 // that it does not keep. Softmax group A owns tile 2k and group B tile 2k+1 for the whole pair:
 // each K/V tile is loaded once and feeds both groups' Q*K^T and P*V, and no partial row is ever
 // merged between the groups.
-// The groups take turns on the exponentials (SFU): group B starts tile n when group A is half way
-// through it, and A starts tile n+1 when B is half way through tile n. Everything else of a
-// group's tile (its S load, row max and exponent arguments, its P*V, the next Q*K^T into S) then
-// runs while the other group exponentiates, so the SFU, the one unit both groups need most, is not
-// left idle by both groups' gaps at once.
-// That also lets the groups share one S buffer in TMEM: the Q*K^T of one group's tile goes into it
-// as soon as the other group has read its own S out.
+// The groups run unsynchronised with each other: each exponentiates as soon as its own S is read
+// and its previous P*V is done. (Making them take turns on the SFU, B starting a tile's
+// exponentials when A was half way through them, measured 4% slower at ViT-H: the waits cost more
+// than the contention they avoid.) The shared S buffer in TMEM orders them loosely: the Q*K^T of
+// one group's tile goes into it as soon as the other group has read its own S out.
 // Work is pieces: the pairs of the full rounds of CTAs are whole pieces; the pairs of a partial
 // last round are cut into `tail_split` key ranges each, so that round spreads over every CTA; each
 // group of such a piece writes its (O, m, l) to a global slot, and k_merge_pieces combines them.
@@ -653,8 +651,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m_ref = m_new;
         }
         const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // The exponents x = s*scale - ref, in place (two per packed FMA), before this group's SFU
-        // turn, so that the turn holds little besides the exponentials. Masked keys give -inf.
+        // The exponents x = s*scale - ref, in place (two per packed FMA), so that the loop below
+        // holds little besides the exponentials. Masked keys give -inf.
         {
           const uint64_t nref2 = f2_pack(-ref, -ref);
 #pragma unroll
@@ -668,16 +666,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (!ok) break;
           }
           tc_fence_after();
-        }
-        // The SFU turn: A exponentiates tile n once B is half way through tile n-1 (B's first P
-        // half is in), B tile n once A is half way through tile n. The two groups' exponentials
-        // overlap by half a tile, so the SFU has two warps' work then, and the gap a group has
-        // between its tiles stays offset from the other group's.
-        if (grp == 1 || gn > 0) {
-          const int other = 1 - grp, t_other = grp ? gn : gn - 1;
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(p_full + 2 * other, t_other & 1, abort, status));
-          if (!ok) break;
         }
         // P as bf16 pairs (column i holds keys 2i, 2i+1), 16 columns at a time; each 64-key half
         // is handed to the P*V issuer as soon as it is in TMEM. 2^x on the SFU in fp32 (as fast
