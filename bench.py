@@ -49,6 +49,7 @@ L2_BYTES = 126 * 1024 * 1024
 # workload is absent (traffic null) until its capture is taken again after a kernel change.
 ATTN_TRAFFIC_BYTES = {
     "vith_global": 125_934_848 + 21_374_464,    # k_attn_pair<80>: profiles/attn_pair_vith_global.md
+    "vitb_global": 18_952_960 + 0,              # k_attn_pair<64>: profiles/attn_pair_vitb_global.md
     "vitb_window": 90_458_880 + 9_328_384,      # k_attn_pairs: profiles/attn_pairs_vitb_window.md
 }
 
