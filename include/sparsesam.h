@@ -325,10 +325,9 @@ int sparsesam_encoder_stack(const ss_cfg* cfg, const float* lum, uint16_t* x, in
                             const uint8_t* is_global, void* ws, size_t ws_bytes, void* stream);
 
 /* S4 without a caller-provided workspace. The SparseSAM pages have no counterpart to this call;
- * it exists for callers that cannot allocate device memory where they run the block: code inside
- * another runtime's stream capture (cudaMalloc is not allowed there), hosts whose allocator owns
- * all device memory and gives plug-ins none, and latency-bound loops that must not pay cudaMalloc's
- * implicit device-wide synchronisation. Same arguments, semantics and results as sparsesam_rcmlp,
+ * it exists for callers that cannot allocate device memory where they run the block: hosts whose
+ * allocator owns all device memory and gives plug-ins none, and latency-bound loops that must not
+ * pay cudaMalloc's implicit device-wide synchronisation. Same arguments, semantics and results as sparsesam_rcmlp,
  * minus ws/ws_bytes: the scratch lives in a 32 MiB array inside this library (a file-scope
  * __device__ array that every GPU loading the library holds until the process exits).
  *   - Arguments are checked as sparsesam_rcmlp checks them (same codes); then, before any CUDA
@@ -336,7 +335,7 @@ int sparsesam_encoder_stack(const ss_cfg* cfg, const float* lum, uint16_t* x, in
  *     the SAM ViT-B global block, 28 MB, fits; batch 4 does not).
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
- *     that device current); make that first call before any stream capture. The address is kept
+ *     that device current). The address is kept
  *     for the process; after a cudaDeviceReset of that device it is stale (so is the status
  *     word's address that every call looks up the same way), and the library must not be used on
  *     that device again.

@@ -1,10 +1,9 @@
 // sparsesam_rcmlp_noalloc: the Residual-Consistency MLP with its scratch in a fixed, library-owned
 // device array instead of a caller-provided workspace.
 //
-// Some callers cannot allocate device memory at the point where they run the block: code running
-// under another runtime's stream capture (where cudaMalloc is not allowed), hosts whose allocator
-// owns all device memory and hands none to plug-ins, and latency-bound loops that must not pay
-// cudaMalloc's implicit device-wide synchronisation. For them this entry point takes only inputs
+// Some callers cannot allocate device memory at the point where they run the block: hosts whose
+// allocator owns all device memory and hands none to plug-ins, and latency-bound loops that must not
+// pay cudaMalloc's implicit device-wide synchronisation. For them this entry point takes only inputs
 // and outputs; the two scratch buffers the MLP needs (the gathered kept rows and the hidden
 // activation) live in `g_rcmlp_scratch` below.
 //

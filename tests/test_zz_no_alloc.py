@@ -1,6 +1,6 @@
 """sparsesam_rcmlp_noalloc: the RC-MLP for callers that cannot allocate device memory at the point
-where they run the block (code inside another runtime's stream capture, hosts whose allocator owns
-all device memory, loops that must avoid cudaMalloc's device-wide synchronisation). Its scratch is a
+where they run the block (hosts whose allocator owns all device memory, loops that must avoid
+cudaMalloc's device-wide synchronisation). Its scratch is a
 fixed 32 MiB array inside the library, so it takes no workspace argument.
 
 It runs the same launches as sparsesam_rcmlp with the same plan, only over other scratch memory,
